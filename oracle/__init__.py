@@ -1,0 +1,201 @@
+"""The oracle: a plain, slow CPU restatement of the extreme-low-bit linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and
+the benchmark's CPU-baseline / reference leg may import this package.  The
+product path (``bit_weight_linear_b200``) never imports it and shares no code
+with it.
+
+The arithmetic lives in ``oref.c`` (scalar C, IEEE fp32 without contraction,
+fp64 where the pages fix no precision); this module only marshals numpy arrays
+through ctypes.  ``build()`` compiles ``liboref.so`` next to this file.
+
+Pages followed (cited by title and section):
+
+* BitNet b1.58 -- "微软、国科大开启1Bit时代：大模型转三进制，速度快4倍能耗降至1/41",
+  section "BitNet b1.58 介绍" (ternary weights, per-token symmetric int8
+  activations, no zero point, no bias), "内存和延迟" (2-bit kernel).
+* OneBit -- "清华、哈工大把大模型压缩到了1bit，把大模型放在手机里跑的愿望就快要实现了！",
+  sections "1. 新的 1bit 结构" (+-1 matrix, FP16 value vectors g and h, the
+  4096x4096 storage example), "2. 基于 SVID 初始化量化模型" (sign times a rank-1
+  approximation of |W|; order swap), "3. 通过知识蒸馏迁移原模型能力" (save the
+  post-Sign() parameters).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liboref.so")
+_SRC = os.path.join(_HERE, "oref.c")
+
+OREF_OK, OREF_ERR_SHAPE, OREF_ERR_VALUE, OREF_ERR_ALLOC = 0, -1, -2, -3
+
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+          "-fno-unsafe-math-optimizations", "-Wall"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oref.c`` into ``liboref.so`` (gcc); returns the library path."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= max(os.path.getmtime(_SRC),
+                                                   os.path.getmtime(os.path.join(_HERE, "oref.h")))):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"], cwd=_HERE)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        L.oref_half_to_double.argtypes = [ctypes.c_uint16]
+        L.oref_half_to_double.restype = ctypes.c_double
+        L.oref_double_to_half.argtypes = [ctypes.c_double]
+        L.oref_double_to_half.restype = ctypes.c_uint16
+        L.oref_float_to_half.argtypes = [ctypes.c_float]
+        L.oref_float_to_half.restype = ctypes.c_uint16
+        L.oref_pack_ternary.argtypes = [P, I, I, P]
+        L.oref_pack_sign.argtypes = [P, I, I, P]
+        L.oref_quant_act.argtypes = [P, I, I, P, P]
+        L.oref_ternary_linear.argtypes = [P, I, I, I, P, ctypes.c_float, P, P]
+        L.oref_ob_linear.argtypes = [P, I, I, I, P, P, P, P, P]
+        L.oref_svid.argtypes = [P, I, I, P, P, P, P, I, ctypes.c_double]
+        L.oref_onebit_bits.argtypes = [ctypes.c_int64, ctypes.c_int64]
+        L.oref_onebit_bits.restype = ctypes.c_int64
+        L.oref_onebit_params.argtypes = [ctypes.c_int64, ctypes.c_int64]
+        L.oref_onebit_params.restype = ctypes.c_int64
+        for f in ("oref_pack_ternary", "oref_pack_sign", "oref_quant_act",
+                  "oref_ternary_linear", "oref_ob_linear", "oref_svid"):
+            getattr(L, f).restype = I
+        _lib = L
+    return _lib
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _check(rc: int, what: str) -> int:
+    if rc < 0:
+        raise OracleError(f"{what}: oracle error {rc}")
+    return rc
+
+
+def _half_bits(x) -> np.ndarray:
+    x = np.asarray(x)
+    if x.dtype == np.float16:
+        return _c(x.view(np.uint16), np.uint16)
+    if x.dtype == np.uint16:
+        return _c(x, np.uint16)
+    raise TypeError("expected float16 (or its uint16 bit pattern)")
+
+
+def half_to_double(bits: int) -> float:
+    return lib().oref_half_to_double(int(bits))
+
+
+def double_to_half(v: float) -> int:
+    return lib().oref_double_to_half(float(v))
+
+
+def float_to_half(v: float) -> int:
+    return lib().oref_float_to_half(float(v))
+
+
+def pack_ternary(w: np.ndarray) -> np.ndarray:
+    """int8 [N,K] in {-1,0,1} -> uint32 [N, K/16] (2-bit codes t+1)."""
+    w = _c(w, np.int8)
+    N, K = w.shape
+    out = np.zeros((N, K // 16), dtype=np.uint32)
+    _check(lib().oref_pack_ternary(_p(w), N, K, _p(out)), "pack_ternary")
+    return out
+
+
+def pack_sign(w: np.ndarray) -> np.ndarray:
+    """fp16 [N,K] -> uint32 [N, K/32]; bit set iff w >= 0 (sign(0) = +1)."""
+    wb = _half_bits(w)
+    N, K = wb.shape
+    out = np.zeros((N, K // 32), dtype=np.uint32)
+    _check(lib().oref_pack_sign(_p(wb), N, K, _p(out)), "pack_sign")
+    return out
+
+
+def quant_act(x: np.ndarray):
+    """fp16 [M,K] -> (q int8 [M,K], s fp32 [M])."""
+    xb = _half_bits(x)
+    M, K = xb.shape
+    q = np.zeros((M, K), dtype=np.int8)
+    s = np.zeros((M,), dtype=np.float32)
+    _check(lib().oref_quant_act(_p(xb), M, K, _p(q), _p(s)), "quant_act")
+    return q, s
+
+
+def ternary_linear(x: np.ndarray, w2: np.ndarray, w_scale: float):
+    """BitLinear forward: returns (y fp16 [M,N], acc int32 [M,N])."""
+    xb = _half_bits(x)
+    w2 = _c(w2, np.uint32)
+    M, K = xb.shape
+    N = w2.shape[0]
+    assert w2.shape[1] * 16 == K
+    y = np.zeros((M, N), dtype=np.uint16)
+    acc = np.zeros((M, N), dtype=np.int32)
+    _check(lib().oref_ternary_linear(_p(xb), M, K, N, _p(w2), float(w_scale), _p(y), _p(acc)),
+           "ternary_linear")
+    return y.view(np.float16), acc
+
+
+def ob_linear(x: np.ndarray, s1: np.ndarray, g: np.ndarray, h: np.ndarray):
+    """OneBit forward: returns (y fp16 [M,N], z fp64 [M,N] before fp16 rounding)."""
+    xb = _half_bits(x)
+    s1 = _c(s1, np.uint32)
+    gb = _half_bits(g)
+    hb = _half_bits(h)
+    M, K = xb.shape
+    N = s1.shape[0]
+    assert s1.shape[1] * 32 == K and gb.shape == (K,) and hb.shape == (N,)
+    y = np.zeros((M, N), dtype=np.uint16)
+    z = np.zeros((M, N), dtype=np.float64)
+    _check(lib().oref_ob_linear(_p(xb), M, K, N, _p(s1), _p(gb), _p(hb), _p(y), _p(z)),
+           "ob_linear")
+    return y.view(np.float16), z
+
+
+def svid(W: np.ndarray, max_iter: int = 1000, tol: float = 1e-12):
+    """SVID of fp32 W [N,K]: returns (S int8 +-1, a fp64 [N], b fp64 [K], sigma, iters)."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    S = np.zeros((N, K), dtype=np.int8)
+    a = np.zeros((N,), dtype=np.float64)
+    b = np.zeros((K,), dtype=np.float64)
+    sig = ctypes.c_double(0.0)
+    it = _check(lib().oref_svid(_p(W), N, K, _p(S), _p(a), _p(b), ctypes.byref(sig),
+                                int(max_iter), float(tol)), "svid")
+    return S, a, b, sig.value, it
+
+
+def onebit_bits(N: int, K: int) -> int:
+    return lib().oref_onebit_bits(N, K)
+
+
+def onebit_params(N: int, K: int) -> int:
+    return lib().oref_onebit_params(N, K)
