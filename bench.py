@@ -1,0 +1,441 @@
+#!/usr/bin/env python
+"""Benchmark of the extreme-low-bit linear layer forward on B200.
+
+Headline workload (one "step"): the M=1 decode pass over a LLaMA-7B-shaped
+stack of ternary BitLinear layers -- 32 blocks x (q, k, v, o: 4096->4096;
+gate, up: 4096->11008; down: 11008->4096) = 224 calls of ``bl_ternary_linear``,
+each quantising its own fp16 input token to int8 and contracting it with
+2-bit packed weights (1,619,001,344 weight bytes per step, far above the
+126 MB L2, so no flush is needed between steps).  The step is captured once
+as a CUDA graph and replayed.
+
+Metric: effective packed-weight GB/s at M=1 (and, in the ``prefill`` object,
+int8 TOPS at M=512 on LLaMA-70B-shaped layers), each with its roofline
+fraction.  The ``onebit_decode`` object repeats the headline workload with the
+OneBit layer (1-bit signs, fp16 g and h).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Multi-GPU (torchrun): independent replicas, no collective on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+LLAMA7B_BLOCK = [("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
+                 ("gate", 4096, 11008), ("up", 4096, 11008), ("down", 11008, 4096)]  # (name, K, N)
+LLAMA7B_LAYERS = 32
+LLAMA70B_PREFILL = [("qkvo-like", 8192, 8192), ("gate/up", 8192, 28672), ("down", 28672, 8192)]
+PREFILL_M = 512
+W_SCALE = 0.02
+METRIC = "1.58/1-bit linear: weight GB/s at M=1 & int8 TOPS at M=512, % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+# ------------------------------------------------------------ clocks ------
+
+class ClockSampler:
+    """nvidia-smi sampling (200 ms) of SM clock and throttle reasons."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.t_start = self.t_stop = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self._reader = threading.Thread(target=self._read, daemon=True)
+        self._reader.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        setattr(self, "t_" + which, time.time())
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((ts, float(parts[1]), float(parts[2]), parts))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        inside = [r for r in rows if self.t_start and self.t_stop
+                  and self.t_start - 0.1 <= r[0] <= self.t_stop + 0.1]
+        window = "timed"
+        if len(inside) < 1:
+            inside, window = rows, "warmup+timed"
+        mhz = sorted(r[1] for r in inside)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in inside:
+            for i, n in enumerate(names):
+                if r[3][5 + i].lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": inside[0][2],
+                "reasons": sorted(reasons), "samples": len(inside), "window": window}
+
+
+# ----------------------------------------------------------- workloads ----
+
+def decode_stack(blw, synth, dev, form: str, M: int = 1, layers: int = LLAMA7B_LAYERS):
+    """Allocate and pack the 7B-shaped stack.  Every call's input and output are
+    views into one contiguous device buffer each (so an end-to-end step is one
+    host->device copy, the graph, and one device->host copy)."""
+    shapes = [(layer, j, K, N) for layer in range(layers) for j, (_, K, N) in enumerate(LLAMA7B_BLOCK)]
+    x_all = torch.empty((sum(M * K for _, _, K, _ in shapes),), dtype=torch.float16, device=dev)
+    y_all = torch.empty((sum(M * N for _, _, _, N in shapes),), dtype=torch.float16, device=dev)
+    calls = []
+    wbytes = 0
+    xo = yo = 0
+    for layer, j, K, N in shapes:
+        seed = 2_000_000 + layer * 16 + j
+        x = x_all[xo:xo + M * K].view(M, K)
+        x.copy_(synth.activations(M, K, seed=seed, device=dev))
+        y = y_all[yo:yo + M * N].view(M, N)
+        xo += M * K
+        yo += M * N
+        if form == "ternary":
+            w = synth.ternary_weights(N, K, seed=seed + 7, device=dev)
+            packed = blw.bl_pack_ternary(w)
+            del w
+            ws = torch.empty((blw.bl_ternary_workspace_bytes(M, K, N),), dtype=torch.uint8, device=dev)
+            calls.append(dict(x=x, w=packed, y=y, ws=ws, K=K, N=N))
+        else:
+            w = synth.sign_weights(N, K, seed=seed + 7, device=dev)
+            packed = blw.ob_pack_sign(w)
+            del w
+            g = synth.value_vector(K, seed=seed + 8, device=dev)
+            h = synth.value_vector(N, seed=seed + 9, device=dev)
+            ws = torch.empty((blw.ob_workspace_bytes(M, K, N),), dtype=torch.uint8, device=dev)
+            calls.append(dict(x=x, w=packed, y=y, ws=ws, g=g, h=h, K=K, N=N))
+            wbytes += 2 * (K + N)
+        wbytes += packed.numel() * 4
+    torch.cuda.synchronize()
+    return calls, wbytes, x_all, y_all
+
+
+def run_calls(blw, calls, form):
+    if form == "ternary":
+        for c in calls:
+            blw.bl_ternary_linear(c["x"], c["w"], W_SCALE, workspace=c["ws"], out=c["y"])
+    else:
+        for c in calls:
+            blw.ob_linear(c["x"], c["w"], c["g"], c["h"], workspace=c["ws"], out=c["y"])
+
+
+def capture(fn):
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm the path once outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def barrier(dist_on):
+    if dist_on:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, dist_on: bool, dev) -> float:
+    if not dist_on:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_replays(g, steps, warmup, dist_on, dev, clocks=None):
+    for _ in range(warmup):
+        g.replay()
+    barrier(dist_on)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if clocks:
+        clocks.mark("start")
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.mark("stop")
+    barrier(dist_on)
+    ms = e0.elapsed_time(e1)
+    return max_over_ranks(ms, dist_on, dev) / steps
+
+
+# ------------------------------------------------------------- oracle -----
+
+def oracle_decode_sample(synth, form: str, budget_s: float = 12.0):
+    """Time the oracle on a bounded sample of the decode stack (whole layers,
+    M=1), packing the sampled weights itself.  Returns (GB/s, sample text, s)."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    total_bytes = 0
+    t_total = 0.0
+    done = []
+    layer = 0
+    while t_total < budget_s and layer < LLAMA7B_LAYERS:
+        for j, (name, K, N) in enumerate(LLAMA7B_BLOCK):
+            seed = 2_000_000 + layer * 16 + j
+            x = synth.activations(1, K, seed=seed).numpy()
+            if form == "ternary":
+                w2 = oracle.pack_ternary(synth.ternary_weights(N, K, seed=seed + 7).numpy())
+                t0 = time.perf_counter()
+                oracle.ternary_linear(x, w2, W_SCALE)
+                t_total += time.perf_counter() - t0
+                total_bytes += w2.nbytes
+            else:
+                s1 = oracle.pack_sign(synth.sign_weights(N, K, seed=seed + 7).numpy())
+                g = synth.value_vector(K, seed=seed + 8).numpy()
+                h = synth.value_vector(N, seed=seed + 9).numpy()
+                t0 = time.perf_counter()
+                oracle.ob_linear(x, s1, g, h)
+                t_total += time.perf_counter() - t0
+                total_bytes += s1.nbytes + 2 * (K + N)
+            done.append(name)
+        layer += 1
+    return total_bytes / t_total / 1e9, f"{layer} of 32 blocks (x7 linears, M=1), CPU-generated seeds", t_total
+
+
+# --------------------------------------------------------------- main -----
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-extras", action="store_true", help="headline workload only")
+    ap.add_argument("--layers", type=int, default=LLAMA7B_LAYERS,
+                    help="blocks in the decode stack (fewer = a small profiling case)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from bit_weight_linear_b200 import synth
+
+    if args.impl == "reference":
+        # The oracle (scalar C on the host cores) is this workload's reference arm.
+        if rank != 0:
+            return 0
+        gbs, sample, secs = oracle_decode_sample(synth, "ternary", budget_s=max(3.0, 0.05 * args.steps))
+        wbytes_step = sum(N * K // 4 for _, K, N in LLAMA7B_BLOCK) * LLAMA7B_LAYERS
+        ms = wbytes_step / (gbs * 1e9) * 1e3
+        line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "s8", "data": "synthetic",
+                "config": {"workload": "llama7b-decode-M1-ternary-bitlinear-32x7",
+                           "M": 1, "layers": LLAMA7B_LAYERS, "parallelism": "replicas"},
+                "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+
+    import bit_weight_linear_b200 as blw
+    from bit_weight_linear_b200 import build
+    build.build()
+    peaks = load_peaks()
+
+    # ---- headline: ternary decode stack, M=1
+    calls, wbytes, x_all, y_all = decode_stack(blw, synth, dev, "ternary", layers=args.layers)
+    in_b, out_b = x_all.numel() * 2, y_all.numel() * 2
+    g = capture(lambda: run_calls(blw, calls, "ternary"))
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ms = time_replays(g, args.steps, args.warmup, dist_on, dev, clocks)
+    time.sleep(0.3)
+    clocks.stop()
+    n_calls = len(calls)
+    value = wbytes * world / (ms * 1e-3) / 1e9
+
+    # roofline of the dominant kernel: the packed-weight decode contraction
+    alg_bytes_per_launch = (wbytes + in_b + out_b) / n_calls
+    launch_ms = ms / n_calls          # upper bound: includes the per-call activation quant
+    achieved = alg_bytes_per_launch / (launch_ms * 1e-3) / 1e9
+    roofline = {"kernel": "ternary decode contraction (skinny_kernel<0,1>)", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "peak_source": peaks["_source"],
+                "note": "launch duration = timed region / launches (includes activation-quant kernel and gaps)"}
+
+    # ---- e2e: host buffers, H2D of every call's input and D2H of every output inside the timed region
+    xin = x_all.cpu().pin_memory()
+    yout = torch.empty(y_all.shape, dtype=torch.float16).pin_memory()
+
+    def e2e_step():
+        x_all.copy_(xin, non_blocking=True)
+        g.replay()
+        yout.copy_(y_all, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier(dist_on)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(10, args.steps // 4)
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(dist_on)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist_on, dev) / e2e_steps
+    e2e = {"value": round(wbytes * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+           "h2d_bytes_per_step": xin.numel() * 2, "d2h_bytes_per_step": yout.numel() * 2,
+           "ms_per_step": round(e2e_ms, 4)}
+    del g, calls, x_all, y_all
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    extras = {}
+    if not args.no_extras:
+        # ---- OneBit decode stack, M=1
+        ocalls, owbytes, _ox, _oy = decode_stack(blw, synth, dev, "onebit", layers=args.layers)
+        og = capture(lambda: run_calls(blw, ocalls, "onebit"))
+        oms = time_replays(og, max(10, args.steps // 2), args.warmup, dist_on, dev)
+        oval = owbytes * world / (oms * 1e-3) / 1e9
+        extras["onebit_decode"] = {
+            "workload": "llama7b-decode-M1-onebit-32x7", "value": round(oval, 2), "unit": "GB/s",
+            "ms_per_step": round(oms, 4), "weight_bytes_per_step": owbytes,
+            "roofline": {"bound": "hbm", "achieved": round(oval / world, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(oval / world / peaks["hbm_gbs"], 4)}}
+        del og, ocalls, _ox, _oy
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+        # ---- prefill M=512, 70B-shaped ternary layers
+        pcalls = []
+        flops = 0
+        for j, (name, K, N) in enumerate(LLAMA70B_PREFILL):
+            seed = 3_000_000 + j
+            x = synth.activations(PREFILL_M, K, seed=seed, device=dev, outlier_frac=0.01)
+            w = synth.ternary_weights(N, K, seed=seed + 7, device=dev)
+            w2 = blw.bl_pack_ternary(w)
+            del w
+            ws = torch.empty((blw.bl_ternary_workspace_bytes(PREFILL_M, K, N),), dtype=torch.uint8,
+                             device=dev)
+            pcalls.append(dict(x=x, w=w2, y=torch.empty((PREFILL_M, N), dtype=torch.float16,
+                                                       device=dev), ws=ws, K=K, N=N))
+            flops += 2 * PREFILL_M * K * N
+        pg = capture(lambda: run_calls(blw, pcalls, "ternary"))
+        pms = time_replays(pg, max(5, args.steps // 20), args.warmup, dist_on, dev)
+        tops = flops * world / (pms * 1e-3) / 1e12
+        i8_peak = 2.0 * peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        extras["prefill"] = {
+            "workload": "llama70b-prefill-M512-ternary (8192x8192, 8192x28672, 28672x8192; 1% outlier channels x20)",
+            "value": round(tops, 2), "unit": "TOPS", "ms_per_step": round(pms, 4),
+            "roofline": {"bound": "tensor", "achieved": round(tops / world, 2), "peak": round(i8_peak, 1),
+                         "unit": "TOPS", "frac": round(tops / world / i8_peak, 4),
+                         "peak_source": "2 x measured sustained bf16 (nominal int8/bf16 ratio)"}}
+        del pg, pcalls
+        torch.cuda.synchronize()
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8",
+        "data": "synthetic",
+        "config": {"workload": "llama7b-decode-M1-ternary-bitlinear-32x7", "M": 1,
+                   "layers": args.layers, "shapes_KxN": [[K, N] for _, K, N in LLAMA7B_BLOCK],
+                   "weight_bytes_per_step": wbytes, "w_scale": W_SCALE,
+                   "l2": "inputs larger than L2 (1.62 GB packed weights per step, 126 MB L2)",
+                   "parallelism": f"replicas x{world}", "graph": "CUDA graph of 224 calls"},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": args.steps * n_calls * 2,
+        "clocks": clocks.summary(),
+    }
+    line.update(extras)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, sample, secs = oracle_decode_sample(synth, "ternary")
+        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                "sample": sample, "seconds": round(secs, 2)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

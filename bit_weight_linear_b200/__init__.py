@@ -1,0 +1,184 @@
+"""bit_weight_linear_b200 -- B200-native extreme-low-bit linear layers.
+
+Two forward forms that replace ``nn.Linear``:
+
+* BitLinear (BitNet b1.58): ternary weights packed 2 bits each, activations
+  quantised per token to int8 (absmax, Q_b = 127, no zero point), exact int32
+  contraction, fp16 output -- ``bl_pack_ternary``, ``bl_quant_act``,
+  ``bl_ternary_linear``.
+* OneBit: y = ((x * g) S^T) * h with a 1-bit sign matrix S and fp16 value
+  vectors g, h -- ``ob_pack_sign``, ``ob_linear``.
+
+This module is argument marshalling only: every step runs in the CUDA kernels
+of ``libbitlinear.so`` (C ABI declared in ``include/bitlinear.h``), called
+through ctypes on torch's current stream.  torch supplies device memory and
+streams.  There is no CPU fallback: if the library is missing or no CUDA
+device is present, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
+
+BL_OK = 0
+STATUS_NAMES = {0: "BL_OK", 1: "BL_ERR_NULL", 2: "BL_ERR_SHAPE", 3: "BL_ERR_ALIGN",
+                4: "BL_ERR_INVALID_VALUE", 5: "BL_ERR_CUDA", 6: "BL_ERR_TIMEOUT",
+                7: "BL_ERR_WORKSPACE"}
+
+# Entry points declared in include/bitlinear.h: name -> (argtypes, restype)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+ABI = {
+    "bl_status_string": ([_I], ctypes.c_char_p),
+    "bl_abi_version": ([], _I),
+    "bl_pack_ternary": ([_P, _I, _I, _P, _P], _I),
+    "ob_pack_sign": ([_P, _I, _I, _P, _P], _I),
+    "bl_quant_act": ([_P, _I, _I, _P, _P, _P], _I),
+    "bl_ternary_workspace_bytes": ([_I, _I, _I], _SZ),
+    "bl_ternary_linear": ([_P, _I, _I, _I, _P, ctypes.c_float, _P, _P, _P, _SZ, _P], _I),
+    "ob_workspace_bytes": ([_I, _I, _I], _SZ),
+    "ob_linear": ([_P, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "bl_device_status": ([_P], _I),
+}
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbitlinear.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libbitlinear.so not built at {LIB_PATH}; run "
+                              "`python -m bit_weight_linear_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in ABI.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != BL_OK:
+        raise BitLinearError(fn, status)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(*ts: torch.Tensor):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("bit_weight_linear_b200 runs on CUDA tensors only (no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous (row-major)")
+
+
+def bl_pack_ternary(w: torch.Tensor) -> torch.Tensor:
+    """int8 [N,K] in {-1,0,1} (CUDA) -> packed words [N, K/16] (int32 storage of uint32)."""
+    _need_cuda(w)
+    assert w.dtype == torch.int8 and w.dim() == 2
+    N, K = w.shape
+    w2 = torch.empty((N, K // 16), dtype=torch.int32, device=w.device)
+    _check("bl_pack_ternary", lib().bl_pack_ternary(_ptr(w), N, K, _ptr(w2), _stream()))
+    return w2
+
+
+def ob_pack_sign(w: torch.Tensor) -> torch.Tensor:
+    """fp16 [N,K] (CUDA) -> packed sign bits [N, K/32] (int32 storage of uint32)."""
+    _need_cuda(w)
+    assert w.dtype == torch.float16 and w.dim() == 2
+    N, K = w.shape
+    s1 = torch.empty((N, K // 32), dtype=torch.int32, device=w.device)
+    _check("ob_pack_sign", lib().ob_pack_sign(_ptr(w), N, K, _ptr(s1), _stream()))
+    return s1
+
+
+def bl_quant_act(x: torch.Tensor):
+    """fp16 [M,K] -> (q int8 [M,K], scale fp32 [M]) by per-token absmax (Q_b = 127)."""
+    _need_cuda(x)
+    assert x.dtype == torch.float16 and x.dim() == 2
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check("bl_quant_act", lib().bl_quant_act(_ptr(x), M, K, _ptr(q), _ptr(s), _stream()))
+    return q, s
+
+
+def bl_ternary_workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(lib().bl_ternary_workspace_bytes(M, K, N))
+
+
+def ob_workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(lib().ob_workspace_bytes(M, K, N))
+
+
+def _workspace(nbytes: int, device, workspace: torch.Tensor | None) -> torch.Tensor:
+    if workspace is not None:
+        return workspace
+    return torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=device)
+
+
+def bl_ternary_linear(x: torch.Tensor, w2: torch.Tensor, w_scale: float, *,
+                      return_acc: bool = False, workspace: torch.Tensor | None = None,
+                      out: torch.Tensor | None = None):
+    """BitLinear forward: fp16 x [M,K], packed w2 [N,K/16] -> fp16 y [M,N] (and int32 acc)."""
+    _need_cuda(x, w2)
+    M, K = x.shape
+    N = w2.shape[0]
+    if w2.shape[1] * 16 != K:
+        raise ValueError("w2 must be [N, K/16]")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
+    acc = torch.empty((M, N), dtype=torch.int32, device=x.device) if return_acc else None
+    nbytes = bl_ternary_workspace_bytes(M, K, N)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = lib().bl_ternary_linear(_ptr(x), M, K, N, _ptr(w2), float(w_scale), _ptr(y), _ptr(acc),
+                                 _ptr(ws), ws.numel() * ws.element_size(), _stream())
+    _check("bl_ternary_linear", st)
+    return (y, acc) if return_acc else y
+
+
+def ob_linear(x: torch.Tensor, s1: torch.Tensor, g: torch.Tensor, h: torch.Tensor, *,
+              workspace: torch.Tensor | None = None, out: torch.Tensor | None = None):
+    """OneBit forward: y = ((x * g) S^T) * h, fp16 in/out, packed S [N, K/32]."""
+    _need_cuda(x, s1, g, h)
+    M, K = x.shape
+    N = s1.shape[0]
+    if s1.shape[1] * 32 != K or g.shape != (K,) or h.shape != (N,):
+        raise ValueError("shapes: s1 [N,K/32], g [K], h [N]")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
+    nbytes = ob_workspace_bytes(M, K, N)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = lib().ob_linear(_ptr(x), M, K, N, _ptr(s1), _ptr(g), _ptr(h), _ptr(y), _ptr(ws),
+                         ws.numel() * ws.element_size(), _stream())
+    _check("ob_linear", st)
+    return y
+
+
+def bl_device_status() -> int:
+    return int(lib().bl_device_status(_stream()))
+
+
+__all__ = ["bl_pack_ternary", "ob_pack_sign", "bl_quant_act", "bl_ternary_linear",
+           "ob_linear", "bl_ternary_workspace_bytes", "ob_workspace_bytes",
+           "bl_device_status", "BitLinearError", "lib", "ABI"]

@@ -1,0 +1,197 @@
+// api.cu -- the C ABI (include/bitlinear.h): argument validation, workspace
+// layout and shape dispatch.  No allocation happens here; all buffers are the
+// caller's.
+#include <cstdlib>
+#include <cstring>
+
+#include "../../include/bitlinear.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bl {
+__device__ unsigned int g_device_flags = 0;
+// Error word of the packers (one per device; packer calls must not overlap).
+__device__ unsigned int g_pack_error = 0;
+}  // namespace bl
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+inline bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+inline cudaStream_t cs(bl_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bl_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BL_OK : BL_ERR_CUDA; }
+
+// Shape rules shared by every entry point.  Sizes are also capped so that
+// M*K, N*K and M*N byte counts stay far inside size_t and int32 indexing of
+// rows.
+bl_status check_mk(int M, int K) {
+    if (M < 0 || K <= 0 || K % 128 != 0) return BL_ERR_SHAPE;
+    if (K > (1 << 20) || M > (1 << 24)) return BL_ERR_SHAPE;
+    return BL_OK;
+}
+
+bl_status check_nk(int N, int K) {
+    if (N < 0 || N % 16 != 0 || K <= 0 || K % 128 != 0) return BL_ERR_SHAPE;
+    if (K > (1 << 20) || N > (1 << 24)) return BL_ERR_SHAPE;
+    return BL_OK;
+}
+
+// Workspace layouts (offsets in bytes, each region 256-byte aligned):
+//   ternary: [0] permuted q  M*K int8 | scale M fp32 | row sums M int32
+//   onebit : [0] limb planes 2*M*K int8 | step M fp32 | row sums M int32
+struct WsLayout {
+    size_t act, scale, rsum, total;
+};
+
+WsLayout ws_layout(int M, int K, int planes) {
+    WsLayout l;
+    l.act = 0;
+    l.scale = align_up((size_t)M * (size_t)K * (size_t)planes);
+    l.rsum = l.scale + align_up((size_t)M * sizeof(float));
+    l.total = l.rsum + align_up((size_t)M * sizeof(int32_t));
+    return l;
+}
+
+bl_status pack_finish(cudaError_t launch_err, cudaStream_t s) {
+    if (launch_err != cudaSuccess) return BL_ERR_CUDA;
+    unsigned int host_err = 0;
+    if (cudaMemcpyFromSymbolAsync(&host_err, bl::g_pack_error, sizeof(host_err), 0,
+                                  cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return BL_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
+    return host_err ? BL_ERR_INVALID_VALUE : BL_OK;
+}
+
+bl_status pack_begin(unsigned int** flag, cudaStream_t s) {
+    static const unsigned int zero = 0;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(flag), bl::g_pack_error) != cudaSuccess)
+        return BL_ERR_CUDA;
+    if (cudaMemcpyToSymbolAsync(bl::g_pack_error, &zero, sizeof(zero), 0,
+                                cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return BL_ERR_CUDA;
+    return BL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bl_status_string(int status) {
+    switch (status) {
+        case BL_OK: return "BL_OK";
+        case BL_ERR_NULL: return "BL_ERR_NULL: a required pointer is NULL";
+        case BL_ERR_SHAPE: return "BL_ERR_SHAPE: M, N or K violates the shape rules";
+        case BL_ERR_ALIGN: return "BL_ERR_ALIGN: a pointer is not 16-byte aligned";
+        case BL_ERR_INVALID_VALUE: return "BL_ERR_INVALID_VALUE: an input value the format cannot hold";
+        case BL_ERR_CUDA: return "BL_ERR_CUDA: a CUDA call or kernel launch failed";
+        case BL_ERR_TIMEOUT: return "BL_ERR_TIMEOUT: a bounded device-side wait expired";
+        case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE: workspace missing or too small";
+        default: return "unknown bl_status";
+    }
+}
+
+int bl_abi_version(void) { return 100; }
+
+bl_status bl_pack_ternary(const int8_t* w, int N, int K, uint32_t* w2, bl_stream_t stream) {
+    if (bl_status st = check_nk(N, K)) return st;
+    if (N == 0) return BL_OK;
+    if (!w || !w2) return BL_ERR_NULL;
+    if (misaligned(w) || misaligned(w2)) return BL_ERR_ALIGN;
+    unsigned int* flag = nullptr;
+    if (bl_status st = pack_begin(&flag, cs(stream))) return st;
+    return pack_finish(bl::launch_pack_ternary(w, N, K, w2, flag, cs(stream)), cs(stream));
+}
+
+bl_status ob_pack_sign(const uint16_t* w, int N, int K, uint32_t* s1, bl_stream_t stream) {
+    if (bl_status st = check_nk(N, K)) return st;
+    if (N == 0) return BL_OK;
+    if (!w || !s1) return BL_ERR_NULL;
+    if (misaligned(w) || misaligned(s1)) return BL_ERR_ALIGN;
+    unsigned int* flag = nullptr;
+    if (bl_status st = pack_begin(&flag, cs(stream))) return st;
+    return pack_finish(bl::launch_pack_sign(w, N, K, s1, flag, cs(stream)), cs(stream));
+}
+
+bl_status bl_quant_act(const uint16_t* x, int M, int K, int8_t* q, float* scale,
+                       bl_stream_t stream) {
+    if (bl_status st = check_mk(M, K)) return st;
+    if (M == 0) return BL_OK;
+    if (!x || !q || !scale) return BL_ERR_NULL;
+    if (misaligned(x) || misaligned(q) || misaligned(scale)) return BL_ERR_ALIGN;
+    return from_cuda(bl::launch_quant_plain(x, M, K, q, scale, cs(stream)));
+}
+
+size_t bl_ternary_workspace_bytes(int M, int K, int N) {
+    (void)N;
+    if (check_mk(M, K) != BL_OK) return 0;
+    return ws_layout(M, K, 1).total;
+}
+
+bl_status bl_ternary_linear(const uint16_t* x, int M, int K, int N, const uint32_t* w2,
+                            float w_scale, uint16_t* y, int32_t* acc_out, void* workspace,
+                            size_t workspace_bytes, bl_stream_t stream) {
+    if (bl_status st = check_mk(M, K)) return st;
+    if (bl_status st = check_nk(N, K)) return st;
+    if (M == 0 || N == 0) return BL_OK;
+    if (!x || !w2 || !y) return BL_ERR_NULL;
+    if (misaligned(x) || misaligned(w2) || misaligned(y) || misaligned(acc_out))
+        return BL_ERR_ALIGN;
+    const WsLayout l = ws_layout(M, K, 1);
+    if (!workspace || workspace_bytes < l.total) return BL_ERR_WORKSPACE;
+    if (misaligned(workspace)) return BL_ERR_ALIGN;
+    char* ws = static_cast<char*>(workspace);
+    int8_t* qp = reinterpret_cast<int8_t*>(ws + l.act);
+    float* sc = reinterpret_cast<float*>(ws + l.scale);
+    int32_t* qs = reinterpret_cast<int32_t*>(ws + l.rsum);
+    cudaError_t e = bl::launch_quant_ternary_perm(x, M, K, qp, sc, qs, cs(stream));
+    if (e != cudaSuccess) return BL_ERR_CUDA;
+    e = bl::launch_ternary_skinny(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, cs(stream));
+    return from_cuda(e);
+}
+
+size_t ob_workspace_bytes(int M, int K, int N) {
+    (void)N;
+    if (check_mk(M, K) != BL_OK || K > 65536) return 0;
+    return ws_layout(M, K, 2).total;
+}
+
+bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
+                    const uint16_t* g, const uint16_t* h, uint16_t* y, void* workspace,
+                    size_t workspace_bytes, bl_stream_t stream) {
+    if (bl_status st = check_mk(M, K)) return st;
+    if (bl_status st = check_nk(N, K)) return st;
+    if (K > 65536) return BL_ERR_SHAPE;
+    if (M == 0 || N == 0) return BL_OK;
+    if (!x || !s1 || !g || !h || !y) return BL_ERR_NULL;
+    if (misaligned(x) || misaligned(s1) || misaligned(g) || misaligned(h) || misaligned(y))
+        return BL_ERR_ALIGN;
+    const WsLayout l = ws_layout(M, K, 2);
+    if (!workspace || workspace_bytes < l.total) return BL_ERR_WORKSPACE;
+    if (misaligned(workspace)) return BL_ERR_ALIGN;
+    char* ws = static_cast<char*>(workspace);
+    int8_t* planes = reinterpret_cast<int8_t*>(ws + l.act);
+    float* step = reinterpret_cast<float*>(ws + l.scale);
+    int32_t* ts = reinterpret_cast<int32_t*>(ws + l.rsum);
+    cudaError_t e = bl::launch_prep_onebit(x, g, M, K, planes, step, ts, cs(stream));
+    if (e != cudaSuccess) return BL_ERR_CUDA;
+    e = bl::launch_onebit_skinny(s1, planes, step, ts, h, M, K, N, y, cs(stream));
+    return from_cuda(e);
+}
+
+bl_status bl_device_status(bl_stream_t stream) {
+    if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return BL_ERR_CUDA;
+    unsigned int flags = 0;
+    static const unsigned int zero = 0;
+    if (cudaMemcpyFromSymbol(&flags, bl::g_device_flags, sizeof(flags)) != cudaSuccess)
+        return BL_ERR_CUDA;
+    if (flags && cudaMemcpyToSymbol(bl::g_device_flags, &zero, sizeof(zero)) != cudaSuccess)
+        return BL_ERR_CUDA;
+    return (flags & bl::kFlagTimeout) ? BL_ERR_TIMEOUT : BL_OK;
+}
+
+}  // extern "C"

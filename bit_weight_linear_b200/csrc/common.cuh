@@ -1,0 +1,60 @@
+// common.cuh -- device helpers shared by the library's kernels (sm_100a).
+// Hand-written inline PTX for the legacy warp-level integer MMA and for
+// streaming loads; no generated code is embedded here.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace bl {
+
+// Bits of the per-device condition word that bl_device_status() reads and
+// clears (kernels receive its address as an argument).
+constexpr unsigned int kFlagTimeout = 1u;
+
+// D = A * B + D for one m16n8k32 tile: A is u8 [16 x 32] (row), B is s8
+// [32 x 8] (col), D is s32 [16 x 8].  Fragment layout per the PTX ISA:
+//   a0: row g,   k 4t..4t+3      a1: row g+8, k 4t..4t+3
+//   a2: row g,   k 16+4t..+3     a3: row g+8, k 16+4t..+3
+//   b0: col g,   k 4t..4t+3      b1: col g,   k 16+4t..+3
+//   d0,d1: row g, cols 2t,2t+1   d2,d3: row g+8, cols 2t,2t+1
+// with g = lane/4 and t = lane%4.
+__device__ __forceinline__ void mma_u8s8_16832(int (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 16-byte load that bypasses L1 allocation: packed weights are read exactly
+// once per launch, so they should not evict the reused activations.
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// 16-byte read-only load through L1 (activations, reused by many CTAs).
+__device__ __forceinline__ uint4 ld_ro_v4(const void* p) {
+    return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+}  // namespace bl

@@ -1,0 +1,38 @@
+// kernels.h -- internal launchers behind the C ABI (host side, no validation:
+// the ABI layer in api.cu checks shapes, pointers and workspace first).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace bl {
+
+// Packers (pack.cu).  Each ORs a nonzero value into *err_flag (device) when it
+// meets an input value the format cannot hold.
+cudaError_t launch_pack_ternary(const int8_t* w, int N, int K, uint32_t* w2,
+                                unsigned int* err_flag, cudaStream_t s);
+cudaError_t launch_pack_sign(const uint16_t* w, int N, int K, uint32_t* s1,
+                             unsigned int* err_flag, cudaStream_t s);
+
+// Activation preparation (quant.cu).
+//   plain   : q [M][K] in natural k order, scale [M]          (bl_quant_act)
+//   ternary : q [M][K] in the decode kernel's permuted order, scale, row sum
+//   onebit  : 16-bit fixed-point image of x*g split into two int8 limb planes
+//             [M][2][K] (permuted), fixed-point step [M], row sum of the image
+cudaError_t launch_quant_plain(const uint16_t* x, int M, int K, int8_t* q, float* scale,
+                               cudaStream_t s);
+cudaError_t launch_quant_ternary_perm(const uint16_t* x, int M, int K, int8_t* qp,
+                                      float* scale, int32_t* qsum, cudaStream_t s);
+cudaError_t launch_prep_onebit(const uint16_t* x, const uint16_t* g, int M, int K,
+                               int8_t* planes, float* step, int32_t* tsum, cudaStream_t s);
+
+// Decode-shaped (small M) packed-weight kernels on warp-level int8 MMA (skinny.cu).
+cudaError_t launch_ternary_skinny(const uint32_t* w2, const int8_t* qp, const float* scale,
+                                  const int32_t* qsum, int M, int K, int N, float w_scale,
+                                  uint16_t* y, int32_t* acc_out, cudaStream_t s);
+cudaError_t launch_onebit_skinny(const uint32_t* s1, const int8_t* planes, const float* step,
+                                 const int32_t* tsum, const uint16_t* h, int M, int K, int N,
+                                 uint16_t* y, cudaStream_t s);
+
+}  // namespace bl

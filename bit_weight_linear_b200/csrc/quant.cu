@@ -1,0 +1,221 @@
+// quant.cu -- per-token activation preparation kernels.
+//
+// BitLinear: BitNet b1.58 page ("微软、国科大开启1Bit时代…"), "BitNet b1.58 介绍":
+// activations are quantised per token to [-Qb, Qb], Qb = 127, with no zero
+// point.  Exact fp32 sequence (shared with the ABI's statement of the op):
+//   amax = max_k |x|, inv = 127 / amax (IEEE division), q = rne(x * inv)
+//   clamped to +-127, scale = amax / 127; an all-zero token gives 0, 0.
+//
+// OneBit: OneBit page ("清华、哈工大把大模型压缩到了1bit…"), "1. 新的 1bit 结构":
+// the input-side value vector g multiplies x before the sign contraction.  The
+// product x*g (exact in fp32: two 11-bit significands) is turned into a
+// per-token 16-bit fixed-point image X = rne(x*g * 32639 / amax'), split into
+// two signed bytes X = 256*hi + lo (hi = floor((X+128)/256), lo in [-128,127]),
+// so that the contraction with the 0/1 sign bits runs exactly in int8 MMA.
+//
+// One CTA per token, two passes over the token (the second hits L1/L2).
+// HBM-bound: the plain/ternary kernels read 2 B and write 1 B per element.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bl {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+// max over the block of a non-negative float carried as its bit pattern
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    uint32_t r = red[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) r = max(r, red[w]);
+    __syncthreads();
+    return r;
+}
+
+__device__ __forceinline__ int block_sum_i32(int v, int* red) {
+    v = warp_sum(v);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    int r = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) r += red[w];
+    return r;
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint32_t bits) {
+    return __half2float(__ushort_as_half((unsigned short)(bits & 0xffffu)));
+}
+
+__device__ __forceinline__ int quant127(float xv, float inv) {
+    int r = __float2int_rn(__fmul_rn(xv, inv));
+    return min(127, max(-127, r));
+}
+
+// Layout 0: natural order.  Layout 1: the decode kernel's order, a 4x4 byte
+// transpose inside every 16-byte group (byte 4j+b holds element 4b+j), which
+// matches the byte order the 2-bit unpack (w >> 2j) & 0x03030303 produces.
+template <int LAYOUT>
+__global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t* __restrict__ x,
+                                                             int K, int8_t* __restrict__ q,
+                                                             float* __restrict__ scale,
+                                                             int32_t* __restrict__ qsum) {
+    __shared__ uint32_t redu[kWarps];
+    __shared__ int redi[kWarps];
+    const int m = blockIdx.x;
+    const uint16_t* row = x + (size_t)m * K;
+
+    // pass 1: amax as the max of |x| bit patterns (monotone for finite halves)
+    uint32_t mx = 0;
+    for (int c = threadIdx.x; c < K / 8; c += kThreads) {
+        uint4 v = ld_ro_v4(row + 8 * c);
+        mx = __vmaxu2(mx, v.x & 0x7fff7fffu);
+        mx = __vmaxu2(mx, v.y & 0x7fff7fffu);
+        mx = __vmaxu2(mx, v.z & 0x7fff7fffu);
+        mx = __vmaxu2(mx, v.w & 0x7fff7fffu);
+    }
+    mx = max(mx & 0xffffu, mx >> 16);
+    const float amax = half_bits_to_float(block_max_u32(mx, redu));
+    const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+
+    // pass 2: quantise 16 elements per step, store 16 bytes
+    int sum = 0;
+    int8_t* qrow = q + (size_t)m * K;
+    for (int c = threadIdx.x; c < K / 16; c += kThreads) {
+        uint4 a = ld_ro_v4(row + 16 * c);
+        uint4 b = ld_ro_v4(row + 16 * c + 8);
+        uint32_t hv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        int qv[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            qv[e] = quant127(half_bits_to_float(hv[e >> 1] >> (16 * (e & 1))), inv);
+            sum += qv[e];
+        }
+        uint32_t out[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t wv = 0;
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                int src = LAYOUT == 0 ? 4 * j + bb : 4 * bb + j;
+                wv |= ((uint32_t)qv[src] & 0xffu) << (8 * bb);
+            }
+            out[j] = wv;
+        }
+        *reinterpret_cast<uint4*>(qrow + 16 * c) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+    if (LAYOUT == 1) {
+        int tot = block_sum_i32(sum, redi);
+        if (threadIdx.x == 0) qsum[m] = tot;
+    }
+    if (threadIdx.x == 0) scale[m] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
+}
+
+constexpr int kFixMax = 32639;  // |X| <= 32639 keeps hi = floor((X+128)/256) in int8
+
+__global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* __restrict__ x,
+                                                               const uint16_t* __restrict__ g,
+                                                               int K, int8_t* __restrict__ planes,
+                                                               float* __restrict__ step,
+                                                               int32_t* __restrict__ tsum) {
+    __shared__ uint32_t redu[kWarps];
+    __shared__ int redi[kWarps];
+    const int m = blockIdx.x;
+    const uint16_t* row = x + (size_t)m * K;
+
+    float mx = 0.f;
+    for (int c = threadIdx.x; c < K / 8; c += kThreads) {
+        uint4 v = ld_ro_v4(row + 8 * c);
+        uint4 gv = ld_ro_v4(g + 8 * c);
+        uint32_t xs[4] = {v.x, v.y, v.z, v.w}, gs[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float p = __fmul_rn(half_bits_to_float(xs[e >> 1] >> (16 * (e & 1))),
+                                half_bits_to_float(gs[e >> 1] >> (16 * (e & 1))));
+            mx = fmaxf(mx, fabsf(p));
+        }
+    }
+    const float amax = __uint_as_float(block_max_u32(__float_as_uint(mx), redu));
+    const float inv = amax > 0.f ? __fdiv_rn((float)kFixMax, amax) : 0.f;
+
+    int sum = 0;
+    int8_t* hi_row = planes + (size_t)m * 2 * K;
+    int8_t* lo_row = hi_row + K;
+    for (int c = threadIdx.x; c < K / 32; c += kThreads) {
+        int hv[32], lv[32];
+#pragma unroll
+        for (int part = 0; part < 4; ++part) {
+            uint4 v = ld_ro_v4(row + 32 * c + 8 * part);
+            uint4 gv = ld_ro_v4(g + 32 * c + 8 * part);
+            uint32_t xs[4] = {v.x, v.y, v.z, v.w}, gs[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float p = __fmul_rn(half_bits_to_float(xs[e >> 1] >> (16 * (e & 1))),
+                                    half_bits_to_float(gs[e >> 1] >> (16 * (e & 1))));
+                int X = __float2int_rn(__fmul_rn(p, inv));
+                X = min(kFixMax, max(-kFixMax, X));
+                int hi = (X + 128) >> 8;  // arithmetic shift = floor
+                hv[8 * part + e] = hi;
+                lv[8 * part + e] = X - 256 * hi;
+                sum += X;
+            }
+        }
+        // byte 4j+b of the 32-byte group holds element 8b+j, the order the
+        // 1-bit unpack (w >> j) & 0x01010101 produces
+        uint32_t ho[8], lo[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            uint32_t a = 0, b = 0;
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                a |= ((uint32_t)hv[8 * bb + j] & 0xffu) << (8 * bb);
+                b |= ((uint32_t)lv[8 * bb + j] & 0xffu) << (8 * bb);
+            }
+            ho[j] = a;
+            lo[j] = b;
+        }
+        uint4* hd = reinterpret_cast<uint4*>(hi_row + 32 * c);
+        uint4* ld = reinterpret_cast<uint4*>(lo_row + 32 * c);
+        hd[0] = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+        hd[1] = make_uint4(ho[4], ho[5], ho[6], ho[7]);
+        ld[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        ld[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+    }
+    int tot = block_sum_i32(sum, redi);
+    if (threadIdx.x == 0) {
+        tsum[m] = tot;
+        step[m] = amax > 0.f ? __fdiv_rn(amax, (float)kFixMax) : 0.f;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_quant_plain(const uint16_t* x, int M, int K, int8_t* q, float* scale,
+                               cudaStream_t s) {
+    if (M == 0) return cudaSuccess;
+    quant_act_kernel<0><<<M, kThreads, 0, s>>>(x, K, q, scale, nullptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_ternary_perm(const uint16_t* x, int M, int K, int8_t* qp,
+                                      float* scale, int32_t* qsum, cudaStream_t s) {
+    if (M == 0) return cudaSuccess;
+    quant_act_kernel<1><<<M, kThreads, 0, s>>>(x, K, qp, scale, qsum);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prep_onebit(const uint16_t* x, const uint16_t* g, int M, int K,
+                               int8_t* planes, float* step, int32_t* tsum, cudaStream_t s) {
+    if (M == 0) return cudaSuccess;
+    prep_onebit_kernel<<<M, kThreads, 0, s>>>(x, g, K, planes, step, tsum);
+    return cudaGetLastError();
+}
+
+}  // namespace bl

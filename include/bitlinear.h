@@ -1,0 +1,165 @@
+/*
+ * bitlinear.h -- C ABI of libbitlinear.so: the forward pass of the two
+ * extreme-low-bit linear layers that replace nn.Linear, on NVIDIA B200
+ * (sm_100a).
+ *
+ *   BitLinear (BitNet b1.58 page, "微软、国科大开启1Bit时代：大模型转三进制，速度快4倍能耗降至1/41",
+ *   section "BitNet b1.58 介绍"): ternary weights {-1, 0, +1}, activations
+ *   quantised per token to 8 bits over the symmetric range [-127, 127] (no
+ *   zero point), no bias.  The contraction is integer add/subtract
+ *   (section "能耗"); the weights are stored 2 bits each (section "内存和延迟").
+ *
+ *   OneBit linear (OneBit page, "清华、哈工大把大模型压缩到了1bit，把大模型放在手机里跑的愿望就快要实现了！",
+ *   section "1. 新的 1bit 结构"): a +-1 sign matrix S and two fp16 value
+ *   vectors g (input side, length K) and h (output side, length N):
+ *       y = ((x (.) g) . S^T) (.) h
+ *   stored as one bit per sign (section "讨论与分析 / 1. 效率").
+ *
+ * Conventions for every entry point:
+ *   - Tensors are row-major.  x is [M, K], y is [M, N], weights are [N, K]
+ *     (nn.Linear orientation: y = x W^T).  fp16 values are passed as their
+ *     IEEE binary16 bit patterns (uint16_t).
+ *   - Every pointer is caller-owned DEVICE memory (cudaMalloc or torch),
+ *     16-byte aligned.  The library allocates and frees nothing.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream)
+ *     except the two packers, which synchronise `stream` to report invalid
+ *     input values.
+ *   - Shapes: M >= 0 and N >= 0 (0 is a no-op returning BL_OK); N % 16 == 0;
+ *     K > 0 and K % 128 == 0.  Anything else returns BL_ERR_SHAPE without
+ *     touching memory.
+ *   - Errors are returned, never raised on the device: validation errors are
+ *     detected before any launch; a failed launch returns BL_ERR_CUDA.
+ *
+ * Packed weight formats (bit-exact ABI; little-endian 32-bit words):
+ *   w2 (ternary): uint32 [N][K/16]; weight (n,k) is the 2-bit field at bits
+ *       2*(k%16) .. 2*(k%16)+1 of word [n][k/16], holding t+1
+ *       (0 -> -1, 1 -> 0, 2 -> +1; 3 is never written).
+ *   s1 (sign):    uint32 [N][K/32]; bit k%32 of word [n][k/32] is 1 iff
+ *       sign(w[n][k]) = +1, with sign(+0) = sign(-0) = +1.
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *bl_stream_t;
+
+typedef enum {
+    BL_OK = 0,
+    BL_ERR_NULL = 1,          /* a required pointer is NULL */
+    BL_ERR_SHAPE = 2,         /* M, N or K outside the rules above */
+    BL_ERR_ALIGN = 3,         /* a pointer is not 16-byte aligned */
+    BL_ERR_INVALID_VALUE = 4, /* an input value outside the format (packers) */
+    BL_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
+    BL_ERR_TIMEOUT = 6,       /* a bounded device-side wait expired */
+    BL_ERR_WORKSPACE = 7      /* workspace missing or smaller than required */
+} bl_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *bl_status_string(int status);
+
+/* ABI version of this header (major * 100 + minor). */
+int bl_abi_version(void);
+
+/*
+ * bl_pack_ternary -- pack ternary weights into the 2-bit w2 format above.
+ * BitNet b1.58 page, "BitNet b1.58 介绍" (weights in {-1,0,1}) and "内存和延迟"
+ * (2-bit storage).
+ *   w  : int8 [N, K], each value in {-1, 0, 1}
+ *   w2 : uint32 [N, K/16] output
+ * Synchronises `stream`.  Any value outside {-1,0,1} -> BL_ERR_INVALID_VALUE
+ * (w2 contents are then unspecified).  Concurrent packer calls on one device
+ * share one error word: do not overlap them.
+ */
+bl_status bl_pack_ternary(const int8_t *w, int N, int K, uint32_t *w2, bl_stream_t stream);
+
+/*
+ * ob_pack_sign -- pack sign(W) into the 1-bit s1 format above.
+ * OneBit page, "3. 通过知识蒸馏迁移原模型能力": after training, the parameters
+ * after Sign() are saved and used directly at inference.
+ *   w  : fp16 [N, K] (any finite values; +-0 packs as +1)
+ *   s1 : uint32 [N, K/32] output
+ * Synchronises `stream`.  A NaN input -> BL_ERR_INVALID_VALUE.
+ */
+bl_status ob_pack_sign(const uint16_t *w, int N, int K, uint32_t *s1, bl_stream_t stream);
+
+/*
+ * bl_quant_act -- per-token absmax activation quantisation.
+ * BitNet b1.58 page, "BitNet b1.58 介绍": each token's activations are scaled
+ * into [-Qb, Qb] (Qb = 127), removing the zero point.  Per token m, in IEEE
+ * fp32 with round-to-nearest-even:
+ *     amax = max_k |x[m,k]|;  inv = 127 / amax;
+ *     q[m,k] = clamp(rne(x[m,k] * inv), -127, 127);  scale[m] = amax / 127
+ * An all-zero token gives q = 0 and scale 0.  Non-finite inputs are
+ * undefined.
+ *   x     : fp16 [M, K]
+ *   q     : int8 [M, K] output
+ *   scale : fp32 [M] output
+ */
+bl_status bl_quant_act(const uint16_t *x, int M, int K, int8_t *q, float *scale,
+                       bl_stream_t stream);
+
+/* Workspace bytes bl_ternary_linear needs for this shape (a multiple of 256). */
+size_t bl_ternary_workspace_bytes(int M, int K, int N);
+
+/*
+ * bl_ternary_linear -- BitLinear forward, y = BitLinear(x; W, w_scale).
+ * BitNet b1.58 page, "BitNet b1.58 介绍" (8-bit per-token activations, ternary
+ * weights, no bias) and "能耗" (the contraction is INT8 additions):
+ *     (q, s) = bl_quant_act(x)
+ *     acc[m,n] = sum_k q[m,k] * t[n,k]                 (exact int32)
+ *     y[m,n]   = fp16_rne( ((float)acc[m,n] * s[m]) * w_scale )
+ *   x         : fp16 [M, K]
+ *   w2        : packed ternary weights, uint32 [N, K/16]
+ *   w_scale   : per-tensor weight scale (fp32, host value)
+ *   y         : fp16 [M, N] output
+ *   acc_out   : optional int32 [M, N] output of the accumulators (NULL = skip)
+ *   workspace : device scratch of at least bl_ternary_workspace_bytes(M,K,N)
+ *               bytes, used only during the call (stream-ordered); calls that
+ *               overlap on the GPU need separate workspaces.
+ * Invalid codes (3) in w2 are undefined behaviour (bl_pack_ternary never
+ * writes them).
+ */
+bl_status bl_ternary_linear(const uint16_t *x, int M, int K, int N, const uint32_t *w2,
+                            float w_scale, uint16_t *y, int32_t *acc_out,
+                            void *workspace, size_t workspace_bytes, bl_stream_t stream);
+
+/* Workspace bytes ob_linear needs for this shape (a multiple of 256). */
+size_t ob_workspace_bytes(int M, int K, int N);
+
+/*
+ * ob_linear -- OneBit linear forward.
+ * OneBit page, "1. 新的 1bit 结构": y = ((x (.) g) . S^T) (.) h, with S = +-1
+ * (packed s1) and fp16 value vectors g [K] and h [N].
+ * The contraction is accumulated exactly in integers on a 16-bit per-token
+ * fixed-point image of x (.) g (relative error of that image <= 2^-16 of the
+ * token's max |x (.) g|), then scaled in fp32 and rounded once to fp16.
+ * K <= 65536.
+ *   x, y      : fp16 [M, K] in, fp16 [M, N] out
+ *   s1        : packed signs, uint32 [N, K/32]
+ *   g, h      : fp16 [K], fp16 [N]
+ *   workspace : device scratch of at least ob_workspace_bytes(M,K,N) bytes
+ *               (stream-ordered; overlapping calls need separate workspaces)
+ */
+bl_status ob_linear(const uint16_t *x, int M, int K, int N, const uint32_t *s1,
+                    const uint16_t *g, const uint16_t *h, uint16_t *y,
+                    void *workspace, size_t workspace_bytes, bl_stream_t stream);
+
+/*
+ * bl_device_status -- synchronise `stream` and report (then clear) any
+ * device-side condition the library's kernels recorded since the last call:
+ * BL_ERR_TIMEOUT if a bounded wait inside a kernel gave up, else BL_OK
+ * (or BL_ERR_CUDA if the synchronisation itself failed).
+ */
+bl_status bl_device_status(bl_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BITLINEAR_H */

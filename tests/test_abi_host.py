@@ -1,0 +1,103 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+entry point include/bitlinear.h declares, and rejects bad arguments before any
+CUDA call is made."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_weight_linear_b200 import build as b
+    b.build()
+    import bit_weight_linear_b200 as blw
+    return blw.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b((?:bl|ob)_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_five_calls():
+    names = declared_functions()
+    for n in ["bl_pack_ternary", "ob_pack_sign", "bl_quant_act", "bl_ternary_linear", "ob_linear"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    import bit_weight_linear_b200 as blw
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert name in blw.ABI, f"binding lacks {name}"
+
+
+def test_status_strings(L):
+    assert L.bl_status_string(0) == b"BL_OK"
+    assert L.bl_status_string(2).startswith(b"BL_ERR_SHAPE")
+    assert L.bl_status_string(99) == b"unknown bl_status"
+    assert L.bl_abi_version() == 100
+
+
+def test_workspace_sizes(L):
+    assert L.bl_ternary_workspace_bytes(1, 4096, 4096) == 4096 + 256 + 256
+    assert L.bl_ternary_workspace_bytes(8, 4096, 4096) == 8 * 4096 + 256 + 256
+    assert L.ob_workspace_bytes(16, 4096, 4096) == 2 * 16 * 4096 + 256 + 256
+    assert L.bl_ternary_workspace_bytes(1, 100, 16) == 0       # bad K
+    assert L.ob_workspace_bytes(1, 65536 + 128, 16) == 0        # OneBit K limit
+    for v in (L.bl_ternary_workspace_bytes(3, 384, 16), L.ob_workspace_bytes(5, 640, 32)):
+        assert v % 256 == 0
+
+
+A = ctypes.c_void_p(0x10000)       # aligned fake device address (never dereferenced)
+MIS = ctypes.c_void_p(0x10004)     # misaligned
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 100, 16), (1, 0, 16), (1, 128, 15), (-1, 128, 16),
+                                   (1, 128, -16), (1, 64, 16)])
+def test_shape_rules(L, M, K, N):
+    assert L.bl_ternary_linear(A, M, K, N, A, 1.0, A, None, A, 1 << 30, None) == 2
+    assert L.ob_linear(A, M, K, N, A, A, A, A, A, 1 << 30, None) == 2
+
+
+def test_shape_checks_of_packers_and_quant(L):
+    assert L.bl_pack_ternary(A, 16, 100, A, None) == 2
+    assert L.ob_pack_sign(A, 17, 128, A, None) == 2
+    assert L.bl_quant_act(A, 1, 96, A, A, None) == 2
+
+
+def test_empty_inputs_are_noops(L):
+    assert L.bl_ternary_linear(None, 0, 128, 16, None, 1.0, None, None, None, 0, None) == 0
+    assert L.bl_ternary_linear(None, 4, 128, 0, None, 1.0, None, None, None, 0, None) == 0
+    assert L.ob_linear(None, 0, 128, 16, None, None, None, None, None, 0, None) == 0
+    assert L.bl_quant_act(None, 0, 128, None, None, None) == 0
+    assert L.bl_pack_ternary(None, 0, 128, None, None) == 0
+
+
+def test_null_alignment_and_workspace(L):
+    assert L.bl_ternary_linear(None, 1, 128, 16, A, 1.0, A, None, A, 1 << 20, None) == 1
+    assert L.bl_ternary_linear(MIS, 1, 128, 16, A, 1.0, A, None, A, 1 << 20, None) == 3
+    assert L.bl_ternary_linear(A, 1, 128, 16, A, 1.0, A, MIS, A, 1 << 20, None) == 3
+    assert L.bl_ternary_linear(A, 1, 128, 16, A, 1.0, A, None, None, 1 << 20, None) == 7
+    need = L.bl_ternary_workspace_bytes(1, 128, 16)
+    assert L.bl_ternary_linear(A, 1, 128, 16, A, 1.0, A, None, A, need - 1, None) == 7
+    assert L.bl_ternary_linear(A, 1, 128, 16, A, 1.0, A, None, MIS, need, None) == 3
+    assert L.ob_linear(A, 1, 128, 16, A, None, A, A, A, 1 << 20, None) == 1
+    assert L.ob_linear(A, 1, 128, 16, A, A, MIS, A, A, 1 << 20, None) == 3
+    assert L.ob_linear(A, 1, 128, 16, A, A, A, A, A, 10, None) == 7
+    assert L.ob_linear(A, 1, 65536 + 128, 16, A, A, A, A, A, 1 << 30, None) == 2
+    assert L.bl_quant_act(A, 1, 128, None, A, None) == 1
+    assert L.bl_pack_ternary(A, 16, 128, MIS, None) == 3
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    import bit_weight_linear_b200 as blw
+    with pytest.raises(ValueError):
+        blw.bl_quant_act(torch.zeros((1, 128), dtype=torch.float16))

@@ -1,0 +1,200 @@
+"""GPU parity: the CUDA path (through the C ABI) against the oracle on the same
+seeded inputs.
+
+Bars (from the statement of the two layer forms):
+* packed bytes, int8 activations, fp32 token scales and int32 accumulators:
+  bit-exact;
+* BitLinear fp16 output: max|y_gpu - y_ref| / max|y_ref| <= 1e-3 (the GPU
+  evaluates the same fp32 sequence, so it is also checked bit-exact);
+* OneBit fp16 output: max|y_gpu - y_ref| / max|y_ref| <= 2e-3 against the fp64
+  oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bit_weight_linear_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+BL_TOL = 1e-3
+OB_TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def blw():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from bit_weight_linear_b200 import build
+    build.build()
+    import bit_weight_linear_b200 as m
+    return m
+
+
+def _np_u32(t):
+    return t.cpu().numpy().view(np.uint32)
+
+
+def _rel_err(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    den = np.max(np.abs(b))
+    return float(np.max(np.abs(a - b)) / (den if den > 0 else 1.0))
+
+
+# ------------------------------------------------------------- packers -----
+
+@pytest.mark.parametrize("N,K", [(16, 128), (48, 384), (272, 640), (4096, 4096)])
+def test_pack_ternary_bytes_identical(blw, oref, N, K):
+    w = synth.ternary_weights(N, K, seed=N + K)
+    w2 = blw.bl_pack_ternary(w.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(_np_u32(w2), oref.pack_ternary(w.numpy()))
+
+
+def test_pack_ternary_rejects_invalid(blw):
+    w = torch.zeros((16, 128), dtype=torch.int8)
+    w[7, 33] = 2
+    with pytest.raises(blw.BitLinearError) as e:
+        blw.bl_pack_ternary(w.cuda())
+    assert e.value.status == 4
+    w[7, 33] = -128
+    with pytest.raises(blw.BitLinearError):
+        blw.bl_pack_ternary(w.cuda())
+    w[7, 33] = 1
+    blw.bl_pack_ternary(w.cuda())   # the error word is cleared per call
+
+
+@pytest.mark.parametrize("N,K", [(16, 128), (48, 384), (4096, 4096)])
+def test_pack_sign_bytes_identical(blw, oref, N, K):
+    w = synth.svid_weights(N, K, seed=3).to(torch.float16)
+    w[0, :40] = 0.0
+    w[1, :40] = -0.0
+    s1 = blw.ob_pack_sign(w.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(_np_u32(s1), oref.pack_sign(w.numpy()))
+
+
+def test_pack_sign_rejects_nan(blw):
+    w = torch.ones((16, 128), dtype=torch.float16)
+    w[3, 3] = float("nan")
+    with pytest.raises(blw.BitLinearError) as e:
+        blw.ob_pack_sign(w.cuda())
+    assert e.value.status == 4
+
+
+# ------------------------------------------------------ activation quant ---
+
+@pytest.mark.parametrize("M,K", [(1, 128), (3, 384), (77, 4096), (5, 28672)])
+def test_quant_act_bit_exact(blw, oref, M, K):
+    x = synth.activations(M, K, seed=M * 7 + K, outlier_frac=0.01)
+    if M > 2:
+        x[1] = 0.0                       # all-zero token
+        x[2, 5] = -60000.0               # dominant negative outlier
+    q, s = blw.bl_quant_act(x.cuda())
+    torch.cuda.synchronize()
+    q_ref, s_ref = oref.quant_act(x.numpy())
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+# ----------------------------------------------------------- BitLinear -----
+
+TERNARY_SHAPES = [
+    (1, 128, 16), (1, 384, 48), (3, 640, 272), (8, 4096, 4096),      # the M=8 4096^2 layer
+    (9, 384, 64), (17, 1152, 96), (40, 256, 32), (100, 768, 48), (1, 11008, 64),
+]
+
+
+@pytest.mark.parametrize("M,K,N", TERNARY_SHAPES)
+def test_ternary_linear_parity(blw, oref, M, K, N):
+    x = synth.activations(M, K, seed=11 + M + K + N)
+    w = synth.ternary_weights(N, K, seed=12 + M + K + N)
+    w2 = oref.pack_ternary(w.numpy())
+    y, acc = blw.bl_ternary_linear(x.cuda(), torch.from_numpy(w2.view(np.int32)).cuda(), 0.02,
+                                   return_acc=True)
+    torch.cuda.synchronize()
+    y_ref, acc_ref = oref.ternary_linear(x.numpy(), w2, 0.02)
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    yg = y.cpu().numpy()
+    assert _rel_err(yg, y_ref) <= BL_TOL
+    assert np.array_equal(yg.view(np.uint16), y_ref.view(np.uint16))
+
+
+def test_ternary_linear_special_weights_and_zero_token(blw, oref):
+    M, K, N = 4, 512, 48
+    x = synth.activations(M, K, seed=21)
+    x[2] = 0.0
+    w = torch.zeros((N, K), dtype=torch.int8)
+    w[:16] = 1
+    w[16:32] = -1
+    w2 = blw.bl_pack_ternary(w.cuda())
+    y, acc = blw.bl_ternary_linear(x.cuda(), w2, 0.5, return_acc=True)
+    torch.cuda.synchronize()
+    q_ref, _ = oref.quant_act(x.numpy())
+    rs = q_ref.astype(np.int64).sum(axis=1)
+    a = acc.cpu().numpy()
+    assert np.array_equal(a[:, :16], np.repeat(rs[:, None], 16, axis=1))
+    assert np.array_equal(a[:, 16:32], -np.repeat(rs[:, None], 16, axis=1))
+    assert np.all(a[:, 32:] == 0)
+    assert np.all(y.cpu().numpy()[2] == 0)
+
+
+def test_ternary_linear_deterministic(blw):
+    M, K, N = 8, 4096, 512
+    x = synth.activations(M, K, seed=31).cuda()
+    w2 = blw.bl_pack_ternary(synth.ternary_weights(N, K, seed=32).cuda())
+    y1, a1 = blw.bl_ternary_linear(x, w2, 0.02, return_acc=True)
+    y2, a2 = blw.bl_ternary_linear(x, w2, 0.02, return_acc=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a1, a2) and torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+# --------------------------------------------------------------- OneBit ----
+
+ONEBIT_SHAPES = [
+    (1, 128, 16), (1, 384, 48), (3, 640, 272), (1, 4096, 4096), (16, 4096, 4096),
+    (5, 1152, 96), (9, 256, 32), (33, 768, 48), (1, 13824, 64),
+]
+
+
+def _onebit_inputs(M, K, N, seed):
+    x = synth.activations(M, K, seed=seed)
+    ws = synth.sign_weights(N, K, seed=seed + 1)
+    g = synth.value_vector(K, seed=seed + 2)
+    h = synth.value_vector(N, seed=seed + 3)
+    return x, ws, g, h
+
+
+@pytest.mark.parametrize("M,K,N", ONEBIT_SHAPES)
+def test_ob_linear_parity(blw, oref, M, K, N):
+    x, ws, g, h = _onebit_inputs(M, K, N, seed=41 + M + K + N)
+    s1 = oref.pack_sign(ws.numpy())
+    y = blw.ob_linear(x.cuda(), torch.from_numpy(s1.view(np.int32)).cuda(), g.cuda(), h.cuda())
+    torch.cuda.synchronize()
+    y_ref, z_ref = oref.ob_linear(x.numpy(), s1, g.numpy(), h.numpy())
+    assert _rel_err(y.cpu().numpy(), z_ref) <= OB_TOL
+
+
+def test_ob_linear_svid_initialised_layer(blw, oref):
+    """A OneBit layer initialised by SVID (sign of W, rank-1 factors of |W| as h
+    and g) gives the oracle's output through the CUDA path."""
+    N, K, M = 256, 512, 4
+    W = synth.svid_weights(N, K, seed=51).numpy()
+    S, a, b, sigma, _ = oref.svid(W)
+    g = torch.from_numpy(b.astype(np.float16))
+    h = torch.from_numpy(a.astype(np.float16))
+    x = synth.activations(M, K, seed=52)
+    s1 = blw.ob_pack_sign(torch.from_numpy(W).to(torch.float16).cuda())
+    y = blw.ob_linear(x.cuda(), s1, g.cuda(), h.cuda())
+    torch.cuda.synchronize()
+    _, z_ref = oref.ob_linear(x.numpy(), oref.pack_sign(W.astype(np.float16)), g.numpy(), h.numpy())
+    assert _rel_err(y.cpu().numpy(), z_ref) <= OB_TOL
+
+
+def test_ob_linear_zero_token(blw):
+    M, K, N = 3, 256, 32
+    x, ws, g, h = _onebit_inputs(M, K, N, seed=61)
+    x[1] = 0
+    y = blw.ob_linear(x.cuda(), blw.ob_pack_sign(ws.cuda()), g.cuda(), h.cuda())
+    torch.cuda.synchronize()
+    assert torch.all(y[1] == 0)
