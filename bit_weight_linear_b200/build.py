@@ -14,8 +14,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libbitlinear.so")
-SOURCES = ["api.cu", "pack.cu", "quant.cu", "skinny.cu"]
-HEADERS = ["common.cuh", "kernels.h"]
+SOURCES = ["api.cu", "pack.cu", "quant.cu", "skinny.cu", "prefill.cu"]
+HEADERS = ["common.cuh", "kernels.h", "tc_prims.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

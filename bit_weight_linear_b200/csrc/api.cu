@@ -67,6 +67,13 @@ bl_status pack_finish(cudaError_t launch_err, cudaStream_t s) {
     return host_err ? BL_ERR_INVALID_VALUE : BL_OK;
 }
 
+unsigned int* device_flags() {
+    unsigned int* p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), bl::g_device_flags) != cudaSuccess)
+        return nullptr;
+    return p;
+}
+
 bl_status pack_begin(unsigned int** flag, cudaStream_t s) {
     static const unsigned int zero = 0;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(flag), bl::g_pack_error) != cudaSuccess)
@@ -150,7 +157,14 @@ bl_status bl_ternary_linear(const uint16_t* x, int M, int K, int N, const uint32
     int32_t* qs = reinterpret_cast<int32_t*>(ws + l.rsum);
     cudaError_t e = bl::launch_quant_ternary_perm(x, M, K, qp, sc, qs, cs(stream));
     if (e != cudaSuccess) return BL_ERR_CUDA;
-    e = bl::launch_ternary_skinny(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, cs(stream));
+    if (M >= bl::kTernaryPrefillMinM) {
+        unsigned int* flags = device_flags();
+        if (!flags) return BL_ERR_CUDA;
+        e = bl::launch_ternary_prefill(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, flags,
+                                       cs(stream));
+    } else {
+        e = bl::launch_ternary_skinny(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, cs(stream));
+    }
     return from_cuda(e);
 }
 
@@ -179,7 +193,13 @@ bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
     int32_t* ts = reinterpret_cast<int32_t*>(ws + l.rsum);
     cudaError_t e = bl::launch_prep_onebit(x, g, M, K, planes, step, ts, cs(stream));
     if (e != cudaSuccess) return BL_ERR_CUDA;
-    e = bl::launch_onebit_skinny(s1, planes, step, ts, h, M, K, N, y, cs(stream));
+    if (M >= bl::kOnebitPrefillMinM) {
+        unsigned int* flags = device_flags();
+        if (!flags) return BL_ERR_CUDA;
+        e = bl::launch_onebit_prefill(s1, planes, step, ts, h, M, K, N, y, flags, cs(stream));
+    } else {
+        e = bl::launch_onebit_skinny(s1, planes, step, ts, h, M, K, N, y, cs(stream));
+    }
     return from_cuda(e);
 }
 

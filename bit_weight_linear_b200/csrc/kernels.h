@@ -35,4 +35,19 @@ cudaError_t launch_onebit_skinny(const uint32_t* s1, const int8_t* planes, const
                                  const int32_t* tsum, const uint16_t* h, int M, int K, int N,
                                  uint16_t* y, cudaStream_t s);
 
+// Prefill-shaped (large M) GEMM on tcgen05 int8 tensor cores with TMEM
+// accumulators (prefill.cu).  `flags` is the device condition word that bounded
+// waits mark on timeout.
+cudaError_t launch_ternary_prefill(const uint32_t* w2, const int8_t* qp, const float* scale,
+                                   const int32_t* qsum, int M, int K, int N, float w_scale,
+                                   uint16_t* y, int32_t* acc_out, unsigned int* flags,
+                                   cudaStream_t s);
+cudaError_t launch_onebit_prefill(const uint32_t* s1, const int8_t* planes, const float* step,
+                                  const int32_t* tsum, const uint16_t* h, int M, int K, int N,
+                                  uint16_t* y, unsigned int* flags, cudaStream_t s);
+
+// Token counts at or above which the tensor-core prefill kernel is used.
+constexpr int kTernaryPrefillMinM = 33;
+constexpr int kOnebitPrefillMinM = 17;
+
 }  // namespace bl

@@ -198,3 +198,82 @@ def test_ob_linear_zero_token(blw):
     y = blw.ob_linear(x.cuda(), blw.ob_pack_sign(ws.cuda()), g.cuda(), h.cuda())
     torch.cuda.synchronize()
     assert torch.all(y[1] == 0)
+
+
+# ------------------------------------------------- tensor-core prefill ------
+
+PREFILL_TERNARY = [(33, 128, 16), (128, 4096, 512), (200, 384, 272), (512, 1024, 1024),
+                   (77, 11008, 256), (300, 640, 48)]
+
+
+@pytest.mark.parametrize("M,K,N", PREFILL_TERNARY)
+def test_ternary_prefill_parity(blw, oref, M, K, N):
+    x = synth.activations(M, K, seed=71 + M + K + N, outlier_frac=0.01)
+    w = synth.ternary_weights(N, K, seed=72 + M + K + N)
+    w2 = oref.pack_ternary(w.numpy())
+    y, acc = blw.bl_ternary_linear(x.cuda(), torch.from_numpy(w2.view(np.int32)).cuda(), 0.02,
+                                   return_acc=True)
+    torch.cuda.synchronize()
+    assert blw.bl_device_status() == 0
+    y_ref, acc_ref = oref.ternary_linear(x.numpy(), w2, 0.02)
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    yg = y.cpu().numpy()
+    assert _rel_err(yg, y_ref) <= BL_TOL
+    assert np.array_equal(yg.view(np.uint16), y_ref.view(np.uint16))
+
+
+PREFILL_ONEBIT = [(17, 128, 16), (64, 4096, 512), (150, 640, 272), (256, 1024, 1024)]
+
+
+@pytest.mark.parametrize("M,K,N", PREFILL_ONEBIT)
+def test_onebit_prefill_parity(blw, oref, M, K, N):
+    x, ws, g, h = _onebit_inputs(M, K, N, seed=81 + M + K + N)
+    s1 = oref.pack_sign(ws.numpy())
+    y = blw.ob_linear(x.cuda(), torch.from_numpy(s1.view(np.int32)).cuda(), g.cuda(), h.cuda())
+    torch.cuda.synchronize()
+    assert blw.bl_device_status() == 0
+    _, z_ref = oref.ob_linear(x.numpy(), s1, g.numpy(), h.numpy())
+    assert _rel_err(y.cpu().numpy(), z_ref) <= OB_TOL
+
+
+def test_ternary_prefill_70b_full_size_sampled_rows(blw, oref):
+    """The 70B-shaped gate/up layer (K=8192, N=28672) at M=512 with 1% outlier
+    channels, run whole on the GPU; the oracle recomputes 96 sampled weight rows
+    for all 512 tokens (rows are independent)."""
+    M, K, N = 512, 8192, 28672
+    x = synth.activations(M, K, seed=3_000_001, outlier_frac=0.01)
+    w = synth.ternary_weights(N, K, seed=3_000_008)
+    y, acc = blw.bl_ternary_linear(x.cuda(), blw.bl_pack_ternary(w.cuda()), 0.02, return_acc=True)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(5).choice(N, size=96, replace=False))
+    rows[-1] = N - 1
+    w2s = oref.pack_ternary(w.numpy()[rows])
+    y_ref, acc_ref = oref.ternary_linear(x.numpy(), w2s, 0.02)
+    assert np.array_equal(acc.cpu().numpy()[:, rows], acc_ref)
+    assert np.array_equal(y.cpu().numpy()[:, rows].view(np.uint16), y_ref.view(np.uint16))
+
+
+def test_onebit_prefill_13b_full_size_sampled_rows(blw, oref):
+    """The 13B-shaped down layer (K=13824, N=5120) at M=256, sampled rows."""
+    M, K, N = 256, 13824, 5120
+    x, ws, g, h = _onebit_inputs(M, K, N, seed=4_000_000)
+    y = blw.ob_linear(x.cuda(), blw.ob_pack_sign(ws.cuda()), g.cuda(), h.cuda())
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(6).choice(N, size=64, replace=False))
+    s1s = oref.pack_sign(ws.numpy()[rows])
+    _, z_ref = oref.ob_linear(x.numpy(), s1s, g.numpy(), h.numpy()[rows])
+    assert _rel_err(y.cpu().numpy()[:, rows], z_ref) <= OB_TOL
+
+
+def test_decode_full_size_layers(blw, oref):
+    """Whole 7B down-projection (K=11008, N=4096) at M=1 and the 13B up layer
+    (K=5120, N=13824) at M=4 against the oracle."""
+    for (M, K, N, seed) in [(1, 11008, 4096, 91), (4, 5120, 13824, 92)]:
+        x = synth.activations(M, K, seed=seed)
+        w = synth.ternary_weights(N, K, seed=seed + 1)
+        w2 = oref.pack_ternary(w.numpy())
+        y, acc = blw.bl_ternary_linear(x.cuda(), torch.from_numpy(w2.view(np.int32)).cuda(), 0.02,
+                                       return_acc=True)
+        torch.cuda.synchronize()
+        y_ref, acc_ref = oref.ternary_linear(x.numpy(), w2, 0.02)
+        assert np.array_equal(acc.cpu().numpy(), acc_ref)
