@@ -329,11 +329,11 @@ def main():
     alg_bytes_per_launch = (wbytes + in_b + out_b) / n_calls
     launch_ms = ms / n_calls          # upper bound: includes the per-call activation quant
     achieved = alg_bytes_per_launch / (launch_ms * 1e-3) / 1e9
-    roofline = {"kernel": "ternary decode contraction (skinny_kernel<0,1>)", "bound": "hbm",
+    roofline = {"kernel": "fused ternary decode (decode_kernel<0,1>)", "bound": "hbm",
                 "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
                 "peak_source": peaks["_source"],
-                "note": "launch duration = timed region / launches (includes activation-quant kernel and gaps)"}
+                "note": "launch duration = timed region / launches (one kernel per call; includes launch gaps)"}
 
     # ---- e2e: host buffers, H2D of every call's input and D2H of every output inside the timed region
     xin = x_all.cpu().pin_memory()
@@ -420,7 +420,7 @@ def main():
                    "parallelism": f"replicas x{world}", "graph": "CUDA graph of 224 calls"},
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": args.steps * n_calls * 2,
+        "gpu_launches": args.steps * n_calls,
         "clocks": clocks.summary(),
     }
     line.update(extras)

@@ -151,6 +151,11 @@ bl_status bl_ternary_linear(const uint16_t* x, int M, int K, int N, const uint32
     const WsLayout l = ws_layout(M, K, 1);
     if (!workspace || workspace_bytes < l.total) return BL_ERR_WORKSPACE;
     if (misaligned(workspace)) return BL_ERR_ALIGN;
+    unsigned int* flags = device_flags();
+    if (!flags) return BL_ERR_CUDA;
+    if (M < bl::kTernaryPrefillMinM && bl::decode_fused_fits(0, M, K))
+        return from_cuda(
+            bl::launch_ternary_decode(x, w2, M, K, N, w_scale, y, acc_out, flags, cs(stream)));
     char* ws = static_cast<char*>(workspace);
     int8_t* qp = reinterpret_cast<int8_t*>(ws + l.act);
     float* sc = reinterpret_cast<float*>(ws + l.scale);
@@ -158,8 +163,6 @@ bl_status bl_ternary_linear(const uint16_t* x, int M, int K, int N, const uint32
     cudaError_t e = bl::launch_quant_ternary_perm(x, M, K, qp, sc, qs, cs(stream));
     if (e != cudaSuccess) return BL_ERR_CUDA;
     if (M >= bl::kTernaryPrefillMinM) {
-        unsigned int* flags = device_flags();
-        if (!flags) return BL_ERR_CUDA;
         e = bl::launch_ternary_prefill(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, flags,
                                        cs(stream));
     } else {
@@ -187,6 +190,10 @@ bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
     const WsLayout l = ws_layout(M, K, 2);
     if (!workspace || workspace_bytes < l.total) return BL_ERR_WORKSPACE;
     if (misaligned(workspace)) return BL_ERR_ALIGN;
+    unsigned int* flags = device_flags();
+    if (!flags) return BL_ERR_CUDA;
+    if (M < bl::kOnebitPrefillMinM && bl::decode_fused_fits(1, M, K))
+        return from_cuda(bl::launch_onebit_decode(x, g, h, s1, M, K, N, y, flags, cs(stream)));
     char* ws = static_cast<char*>(workspace);
     int8_t* planes = reinterpret_cast<int8_t*>(ws + l.act);
     float* step = reinterpret_cast<float*>(ws + l.scale);
@@ -194,8 +201,6 @@ bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
     cudaError_t e = bl::launch_prep_onebit(x, g, M, K, planes, step, ts, cs(stream));
     if (e != cudaSuccess) return BL_ERR_CUDA;
     if (M >= bl::kOnebitPrefillMinM) {
-        unsigned int* flags = device_flags();
-        if (!flags) return BL_ERR_CUDA;
         e = bl::launch_onebit_prefill(s1, planes, step, ts, h, M, K, N, y, flags, cs(stream));
     } else {
         e = bl::launch_onebit_skinny(s1, planes, step, ts, h, M, K, N, y, cs(stream));

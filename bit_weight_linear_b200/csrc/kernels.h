@@ -46,6 +46,19 @@ cudaError_t launch_onebit_prefill(const uint32_t* s1, const int8_t* planes, cons
                                   const int32_t* tsum, const uint16_t* h, int M, int K, int N,
                                   uint16_t* y, unsigned int* flags, cudaStream_t s);
 
+// Fused decode (decode.cu): activation preparation + contraction in one kernel,
+// 8-CTA clusters, weights bulk-copied to shared memory before the
+// programmatic-dependent-launch wait.  Used when M <= 32 columns of MMA fit and
+// the CTA's shared memory (16 weight rows + the prepared activations) fits.
+constexpr int kDecodeMaxSmem = 227 * 1024;
+bool decode_fused_fits(int form, int M, int K);
+cudaError_t launch_ternary_decode(const uint16_t* x, const uint32_t* w2, int M, int K, int N,
+                                  float w_scale, uint16_t* y, int32_t* acc_out,
+                                  unsigned int* flags, cudaStream_t s);
+cudaError_t launch_onebit_decode(const uint16_t* x, const uint16_t* g, const uint16_t* h,
+                                 const uint32_t* s1, int M, int K, int N, uint16_t* y,
+                                 unsigned int* flags, cudaStream_t s);
+
 // Token counts at or above which the tensor-core prefill kernel is used.
 constexpr int kTernaryPrefillMinM = 33;
 constexpr int kOnebitPrefillMinM = 17;

@@ -277,3 +277,83 @@ def test_decode_full_size_layers(blw, oref):
         torch.cuda.synchronize()
         y_ref, acc_ref = oref.ternary_linear(x.numpy(), w2, 0.02)
         assert np.array_equal(acc.cpu().numpy(), acc_ref)
+
+
+# ----------------------------------- fused decode chains and fallbacks -----
+
+def test_fallback_two_kernel_path(blw, oref):
+    """Shapes whose fused-decode shared memory would not fit take the
+    activation-kernel + skinny-kernel path; both forms stay exact."""
+    M, K, N = 8, 28672, 64
+    x = synth.activations(M, K, seed=101)
+    w2 = oref.pack_ternary(synth.ternary_weights(N, K, seed=102).numpy())
+    y, acc = blw.bl_ternary_linear(x.cuda(), torch.from_numpy(w2.view(np.int32)).cuda(), 0.02,
+                                   return_acc=True)
+    torch.cuda.synchronize()
+    y_ref, acc_ref = oref.ternary_linear(x.numpy(), w2, 0.02)
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    M, K, N = 16, 13824, 64
+    x, ws, g, h = _onebit_inputs(M, K, N, seed=103)
+    s1 = oref.pack_sign(ws.numpy())
+    y = blw.ob_linear(x.cuda(), torch.from_numpy(s1.view(np.int32)).cuda(), g.cuda(), h.cuda())
+    torch.cuda.synchronize()
+    _, z_ref = oref.ob_linear(x.numpy(), s1, g.numpy(), h.numpy())
+    assert _rel_err(y.cpu().numpy(), z_ref) <= OB_TOL
+
+
+@pytest.mark.parametrize("use_graph", [False, True])
+def test_dependent_decode_chain(blw, oref, use_graph):
+    """Eight M=1 layers where each layer's output is the next layer's input.
+    The decode kernel streams weights before its programmatic-launch wait and
+    reads x after it; the chained outputs must equal the oracle's chain
+    bit for bit."""
+    K = N = 1024
+    layers = 8
+    ws = [synth.ternary_weights(N, K, seed=200 + i) for i in range(layers)]
+    w2s = [oref.pack_ternary(w.numpy()) for w in ws]
+    w2d = [torch.from_numpy(w.view(np.int32)).cuda() for w in w2s]
+    x0 = synth.activations(1, K, seed=199)
+    xd = x0.cuda()
+    bufs = [torch.empty((1, N), dtype=torch.float16, device="cuda") for _ in range(layers)]
+    wsp = torch.empty((blw.bl_ternary_workspace_bytes(1, K, N),), dtype=torch.uint8, device="cuda")
+
+    def run():
+        cur = xd
+        for i in range(layers):
+            blw.bl_ternary_linear(cur, w2d[i], 0.5, workspace=wsp, out=bufs[i])
+            cur = bufs[i]
+
+    if use_graph:
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            run()
+        torch.cuda.current_stream().wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run()
+        for b in bufs:
+            b.zero_()
+        g.replay()
+    else:
+        run()
+    torch.cuda.synchronize()
+    cur = x0.numpy()
+    for i in range(layers):
+        y_ref, _ = oref.ternary_linear(cur, w2s[i], 0.5)
+        assert np.array_equal(bufs[i].cpu().numpy().view(np.uint16), y_ref.view(np.uint16)), i
+        cur = y_ref
+
+
+def test_decode_all_token_counts_fused(blw, oref):
+    """Every M the fused decode kernel serves (ternary 1..32), one shape each."""
+    K, N = 640, 48
+    w = synth.ternary_weights(N, K, seed=300)
+    w2 = oref.pack_ternary(w.numpy())
+    w2d = torch.from_numpy(w2.view(np.int32)).cuda()
+    for M in range(1, 33):
+        x = synth.activations(M, K, seed=300 + M)
+        y, acc = blw.bl_ternary_linear(x.cuda(), w2d, 0.02, return_acc=True)
+        torch.cuda.synchronize()
+        _, acc_ref = oref.ternary_linear(x.numpy(), w2, 0.02)
+        assert np.array_equal(acc.cpu().numpy(), acc_ref), M
