@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
 BL_OK = 0
 STATUS_NAMES = {0: "BL_OK", 1: "BL_ERR_NULL", 2: "BL_ERR_SHAPE", 3: "BL_ERR_ALIGN",
                 4: "BL_ERR_INVALID_VALUE", 5: "BL_ERR_CUDA", 6: "BL_ERR_TIMEOUT",
-                7: "BL_ERR_WORKSPACE"}
+                7: "BL_ERR_WORKSPACE", 8: "BL_ERR_SCRATCH_LIMIT"}
 
 # Entry points declared in include/bitlinear.h: name -> (argtypes, restype)
 _P = ctypes.c_void_p
@@ -45,6 +45,7 @@ ABI = {
     "ob_workspace_bytes": ([_I, _I, _I], _SZ),
     "ob_linear": ([_P, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P], _I),
     "bl_device_status": ([_P], _I),
+    "bl_ternary_linear_noalloc": ([_P, _I, _I, _I, _P, ctypes.c_float, _P, _P, _P], _I),
 }
 
 
@@ -175,10 +176,29 @@ def ob_linear(x: torch.Tensor, s1: torch.Tensor, g: torch.Tensor, h: torch.Tenso
     return y
 
 
+def bl_ternary_linear_noalloc(x: torch.Tensor, w2: torch.Tensor, w_scale: float, *,
+                              return_acc: bool = False, out: torch.Tensor | None = None):
+    """BitLinear forward without a workspace, for callers that cannot allocate device
+    memory where they run the layer: the library's fixed scratch array stands in
+    for it (M*K up to about 16.7 million; calls that overlap on the GPU race on
+    the shared array).  Same result as ``bl_ternary_linear``."""
+    _need_cuda(x, w2)
+    M, K = x.shape
+    N = w2.shape[0]
+    if w2.shape[1] * 16 != K:
+        raise ValueError("w2 must be [N, K/16]")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
+    acc = torch.empty((M, N), dtype=torch.int32, device=x.device) if return_acc else None
+    st = lib().bl_ternary_linear_noalloc(_ptr(x), M, K, N, _ptr(w2), float(w_scale), _ptr(y),
+                                         _ptr(acc), _stream())
+    _check("bl_ternary_linear_noalloc", st)
+    return (y, acc) if return_acc else y
+
+
 def bl_device_status() -> int:
     return int(lib().bl_device_status(_stream()))
 
 
 __all__ = ["bl_pack_ternary", "ob_pack_sign", "bl_quant_act", "bl_ternary_linear",
            "ob_linear", "bl_ternary_workspace_bytes", "ob_workspace_bytes",
-           "bl_device_status", "BitLinearError", "lib", "ABI"]
+           "bl_device_status", "bl_ternary_linear_noalloc", "BitLinearError", "lib", "ABI"]

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libbitlinear.so")
-SOURCES = ["api.cu", "pack.cu", "quant.cu", "skinny.cu", "prefill.cu", "decode.cu"]
+SOURCES = ["api.cu", "pack.cu", "quant.cu", "skinny.cu", "prefill.cu", "decode.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h", "tc_prims.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -86,6 +86,8 @@ bl_status pack_begin(unsigned int** flag, cudaStream_t s) {
 
 }  // namespace
 
+unsigned int* bl::device_flags_address() { return device_flags(); }
+
 extern "C" {
 
 const char* bl_status_string(int status) {
@@ -98,6 +100,8 @@ const char* bl_status_string(int status) {
         case BL_ERR_CUDA: return "BL_ERR_CUDA: a CUDA call or kernel launch failed";
         case BL_ERR_TIMEOUT: return "BL_ERR_TIMEOUT: a bounded device-side wait expired";
         case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE: workspace missing or too small";
+        case BL_ERR_SCRATCH_LIMIT:
+            return "BL_ERR_SCRATCH_LIMIT: shape exceeds the fixed scratch of the no-allocation entry point";
         default: return "unknown bl_status";
     }
 }

@@ -59,6 +59,9 @@ cudaError_t launch_onebit_decode(const uint16_t* x, const uint16_t* g, const uin
                                  const uint32_t* s1, int M, int K, int N, uint16_t* y,
                                  unsigned int* flags, cudaStream_t s);
 
+// Device address of the condition word bounded waits mark (nullptr on error).
+unsigned int* device_flags_address();
+
 // Token counts at or above which the tensor-core prefill kernel is used.
 constexpr int kTernaryPrefillMinM = 33;
 constexpr int kOnebitPrefillMinM = 17;

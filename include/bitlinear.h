@@ -58,7 +58,8 @@ typedef enum {
     BL_ERR_INVALID_VALUE = 4, /* an input value outside the format (packers) */
     BL_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
     BL_ERR_TIMEOUT = 6,       /* a bounded device-side wait expired */
-    BL_ERR_WORKSPACE = 7      /* workspace missing or smaller than required */
+    BL_ERR_WORKSPACE = 7,     /* workspace missing or smaller than required */
+    BL_ERR_SCRATCH_LIMIT = 8  /* shape needs more than bl_ternary_linear_noalloc's fixed scratch */
 } bl_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -150,6 +151,38 @@ size_t ob_workspace_bytes(int M, int K, int N);
 bl_status ob_linear(const uint16_t *x, int M, int K, int N, const uint32_t *s1,
                     const uint16_t *g, const uint16_t *h, uint16_t *y,
                     void *workspace, size_t workspace_bytes, bl_stream_t stream);
+
+/*
+ * bl_ternary_linear_noalloc -- bl_ternary_linear for callers that cannot
+ * allocate device memory.  (No counterpart on the pages: this is a calling
+ * convention, not part of the method.)
+ *
+ * Some callers cannot call cudaMalloc or any other allocator where they run the
+ * layer -- for example a plugin inside a host program that owns all device
+ * memory and gives the plugin no allocator, or a latency-critical loop that
+ * forbids allocation because cudaMalloc can block the whole device.  This entry
+ * point takes no workspace: its scratch is a fixed array of
+ * BL_NOALLOC_SCRATCH_BYTES compiled into the library, held by every GPU that
+ * loads the library until the process exits.  It computes exactly what
+ * bl_ternary_linear computes (same arguments minus the workspace).
+ *   - Shapes needing more than the array, i.e. when
+ *       round256(M*K) + round256(4*M) + round256(4*M) > BL_NOALLOC_SCRATCH_BYTES
+ *     (M*K up to about 16.7 million int8 activations), return
+ *     BL_ERR_SCRATCH_LIMIT before anything is launched.
+ *   - It allocates nothing and frees nothing.
+ *   - The first call on each device looks up that device's copy of the array
+ *     (with the caller's device current); make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the one array, and it keeps the previous
+ *     call's contents (each call overwrites what it reads, so no clearing is
+ *     needed).  Calls that may overlap on the GPU (different streams without
+ *     ordering between them) race on it: order them, or use bl_ternary_linear
+ *     with separate workspaces.
+ */
+#define BL_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+bl_status bl_ternary_linear_noalloc(const uint16_t *x, int M, int K, int N, const uint32_t *w2,
+                                    float w_scale, uint16_t *y, int32_t *acc_out,
+                                    bl_stream_t stream);
 
 /*
  * bl_device_status -- synchronise `stream` and report (then clear) any
