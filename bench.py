@@ -35,6 +35,9 @@ sys.path.insert(0, ROOT)
 LLAMA7B_BLOCK = [("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
                  ("gate", 4096, 11008), ("up", 4096, 11008), ("down", 11008, 4096)]  # (name, K, N)
 LLAMA7B_LAYERS = 32
+# the same block with the projections that share an input fused into one call each
+LLAMA7B_BLOCK_FUSED = [("qkv", 4096, 3 * 4096), ("o", 4096, 4096), ("gate+up", 4096, 2 * 11008),
+                       ("down", 11008, 4096)]
 LLAMA70B_PREFILL = [("qkvo-like", 8192, 8192), ("gate/up", 8192, 28672), ("down", 28672, 8192)]
 PREFILL_M = 512
 W_SCALE = 0.02
@@ -127,11 +130,13 @@ class ClockSampler:
 
 # ----------------------------------------------------------- workloads ----
 
-def decode_stack(blw, synth, dev, form: str, M: int = 1, layers: int = LLAMA7B_LAYERS):
+def decode_stack(blw, synth, dev, form: str, M: int = 1, layers: int = LLAMA7B_LAYERS,
+                 block=None):
     """Allocate and pack the 7B-shaped stack.  Every call's input and output are
     views into one contiguous device buffer each (so an end-to-end step is one
     host->device copy, the graph, and one device->host copy)."""
-    shapes = [(layer, j, K, N) for layer in range(layers) for j, (_, K, N) in enumerate(LLAMA7B_BLOCK)]
+    block = block or LLAMA7B_BLOCK
+    shapes = [(layer, j, K, N) for layer in range(layers) for j, (_, K, N) in enumerate(block)]
     x_all = torch.empty((sum(M * K for _, _, K, _ in shapes),), dtype=torch.float16, device=dev)
     y_all = torch.empty((sum(M * N for _, _, _, N in shapes),), dtype=torch.float16, device=dev)
     calls = []
@@ -256,6 +261,35 @@ def oracle_decode_sample(synth, form: str, budget_s: float = 12.0):
     return total_bytes / t_total / 1e9, f"{layer} of 32 blocks (x7 linears, M=1), CPU-generated seeds", t_total
 
 
+def run_prefill(blw, synth, dev, args, dist_on, world, peaks):
+    """M=512 on the LLaMA-70B-shaped ternary layers (tcgen05 prefill path)."""
+    pcalls = []
+    flops = 0
+    for j, (name, K, N) in enumerate(LLAMA70B_PREFILL):
+        seed = 3_000_000 + j
+        x = synth.activations(PREFILL_M, K, seed=seed, device=dev, outlier_frac=0.01)
+        w = synth.ternary_weights(N, K, seed=seed + 7, device=dev)
+        w2 = blw.bl_pack_ternary(w)
+        del w
+        ws = torch.empty((blw.bl_ternary_workspace_bytes(PREFILL_M, K, N),), dtype=torch.uint8,
+                         device=dev)
+        pcalls.append(dict(x=x, w=w2, y=torch.empty((PREFILL_M, N), dtype=torch.float16,
+                                                   device=dev), ws=ws, K=K, N=N))
+        flops += 2 * PREFILL_M * K * N
+    pg = capture(lambda: run_calls(blw, pcalls, "ternary"))
+    pms = time_replays(pg, max(5, args.steps // 20), args.warmup, dist_on, dev)
+    tops = flops * world / (pms * 1e-3) / 1e12
+    i8_peak = 2.0 * peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    del pg, pcalls
+    torch.cuda.synchronize()
+    return {
+        "workload": "llama70b-prefill-M512-ternary (8192x8192, 8192x28672, 28672x8192; 1% outlier channels x20)",
+        "value": round(tops, 2), "unit": "TOPS", "ms_per_step": round(pms, 4),
+        "roofline": {"bound": "tensor", "achieved": round(tops / world, 2), "peak": round(i8_peak, 1),
+                     "unit": "TOPS", "frac": round(tops / world / i8_peak, 4),
+                     "peak_source": "2 x measured sustained bf16 (nominal int8/bf16 ratio)"}}
+
+
 # --------------------------------------------------------------- main -----
 
 def main():
@@ -268,6 +302,8 @@ def main():
     ap.add_argument("--layers", type=int, default=LLAMA7B_LAYERS,
                     help="blocks in the decode stack (fewer = a small profiling case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="run only the M=512 prefill layers (a profiling case)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -311,6 +347,14 @@ def main():
     from bit_weight_linear_b200 import build
     build.build()
     peaks = load_peaks()
+
+    if args.prefill_only:
+        res = run_prefill(blw, synth, dev, args, dist_on, world, peaks)
+        if rank == 0:
+            print(json.dumps({"prefill": res}), flush=True)
+        if dist_on:
+            torch.distributed.destroy_process_group()
+        return 0
 
     # ---- headline: ternary decode stack, M=1
     calls, wbytes, x_all, y_all = decode_stack(blw, synth, dev, "ternary", layers=args.layers)
@@ -367,6 +411,22 @@ def main():
 
     extras = {}
     if not args.no_extras:
+        # ---- same stack with fused QKV and gate+up projections (4 calls per block)
+        fcalls, fwbytes, _fx, _fy = decode_stack(blw, synth, dev, "ternary", layers=args.layers,
+                                                 block=LLAMA7B_BLOCK_FUSED)
+        fg = capture(lambda: run_calls(blw, fcalls, "ternary"))
+        fms = time_replays(fg, args.steps, args.warmup, dist_on, dev)
+        fval = fwbytes * world / (fms * 1e-3) / 1e9
+        extras["decode_fused_projections"] = {
+            "workload": "llama7b-decode-M1-ternary, qkv (4096->12288) and gate+up (4096->22016) fused",
+            "calls_per_step": len(fcalls), "value": round(fval, 2), "unit": "GB/s",
+            "ms_per_step": round(fms, 4), "weight_bytes_per_step": fwbytes,
+            "roofline": {"bound": "hbm", "achieved": round(fval / world, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(fval / world / peaks["hbm_gbs"], 4)}}
+        del fg, fcalls, _fx, _fy
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
         # ---- OneBit decode stack, M=1
         ocalls, owbytes, _ox, _oy = decode_stack(blw, synth, dev, "onebit", layers=args.layers)
         og = capture(lambda: run_calls(blw, ocalls, "onebit"))
@@ -381,32 +441,7 @@ def main():
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
 
-        # ---- prefill M=512, 70B-shaped ternary layers
-        pcalls = []
-        flops = 0
-        for j, (name, K, N) in enumerate(LLAMA70B_PREFILL):
-            seed = 3_000_000 + j
-            x = synth.activations(PREFILL_M, K, seed=seed, device=dev, outlier_frac=0.01)
-            w = synth.ternary_weights(N, K, seed=seed + 7, device=dev)
-            w2 = blw.bl_pack_ternary(w)
-            del w
-            ws = torch.empty((blw.bl_ternary_workspace_bytes(PREFILL_M, K, N),), dtype=torch.uint8,
-                             device=dev)
-            pcalls.append(dict(x=x, w=w2, y=torch.empty((PREFILL_M, N), dtype=torch.float16,
-                                                       device=dev), ws=ws, K=K, N=N))
-            flops += 2 * PREFILL_M * K * N
-        pg = capture(lambda: run_calls(blw, pcalls, "ternary"))
-        pms = time_replays(pg, max(5, args.steps // 20), args.warmup, dist_on, dev)
-        tops = flops * world / (pms * 1e-3) / 1e12
-        i8_peak = 2.0 * peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-        extras["prefill"] = {
-            "workload": "llama70b-prefill-M512-ternary (8192x8192, 8192x28672, 28672x8192; 1% outlier channels x20)",
-            "value": round(tops, 2), "unit": "TOPS", "ms_per_step": round(pms, 4),
-            "roofline": {"bound": "tensor", "achieved": round(tops / world, 2), "peak": round(i8_peak, 1),
-                         "unit": "TOPS", "frac": round(tops / world / i8_peak, 4),
-                         "peak_source": "2 x measured sustained bf16 (nominal int8/bf16 ratio)"}}
-        del pg, pcalls
-        torch.cuda.synchronize()
+        extras["prefill"] = run_prefill(blw, synth, dev, args, dist_on, world, peaks)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,

@@ -14,17 +14,16 @@
 //      call's weights start streaming while this call computes.
 //   2. griddepcontrol.wait -- only now is x (the previous call's output, in a
 //      model) read.
-//   3. Activation preparation is split over an 8-CTA thread-block cluster:
-//      CTA r handles every 8th group of 16 (ternary) / 32 (sign) inputs.  The
-//      per-token absmax and the per-token row sums are exchanged through
-//      distributed shared memory, and each quantised, permuted group is stored
-//      into all eight CTAs' activation tiles (st.shared::cluster), so x is read
-//      once per cluster instead of once per CTA.
+//   3. Activation preparation in the CTA: per-token absmax (warp shuffles +
+//      one CTA barrier), then every thread quantises its 16- (ternary) or
+//      32-element (sign) groups straight into the permuted shared-memory tile.
+//      x is small at decode sizes and L2-resident, so each CTA reading it is
+//      cheaper than any cross-CTA exchange.
 //   4. The contraction runs from shared memory on the warp-level u8 x s8 MMA
 //      (byte-SIMD unpack as in skinny.cu), warps split K, and reduce through
 //      shared memory for the epilogue.
-// Shared-memory rows are padded by 16 bytes so that the 8 row groups a warp
-// reads land on different banks.
+// Weight rows in shared memory are padded to a stride of 64 (mod 128) bytes so
+// that every quarter-warp's 16-byte loads hit 8 distinct bank groups.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_prims.cuh"
@@ -35,7 +34,6 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kCluster = 8;
 constexpr int kMaxTok = 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -55,6 +53,7 @@ struct DF<1> {
 };
 
 struct DecodeParams {
+    int stage_x;            // 1: x (and g) are staged in shared memory between the two passes
     const uint16_t* x;
     const uint16_t* g;      // OneBit input value vector
     const uint16_t* h;      // OneBit output value vector
@@ -67,22 +66,40 @@ struct DecodeParams {
 };
 
 struct DecodeLayout {
-    int wstride, astride, off_a, off_red, off_tok, off_bar, total;
+    int wstride, astride, off_a, off_x, off_red, off_tok, off_bar, total;
 };
 
+// Shared memory: weight slab [16][wstride] | prepared activations [cols][astride] |
+// staged x [M][K] (+ g [K]) fp16 when stage_x | partial sums | token scratch | mbarrier
 template <int FORM, int NT>
-__host__ __device__ inline DecodeLayout decode_layout(int M, int K) {
+__host__ __device__ inline DecodeLayout decode_layout(int M, int K, int stage_x) {
     DecodeLayout l;
-    l.wstride = K / DF<FORM>::kPerWord * 4 + 16;
+    // row stride = 64 (mod 128) bytes: the 8 lanes of a quarter-warp (rows 2q,
+    // 2q+1; chunks t = 0..3) then read 8 disjoint 16-byte bank groups
+    const int rowbytes = K / DF<FORM>::kPerWord * 4;
+    l.wstride = rowbytes + ((64 - rowbytes % 128) + 128) % 128;
     l.astride = K + 16;
     l.off_a = 16 * l.wstride;
-    l.off_red = l.off_a + M * DF<FORM>::kCPT * l.astride;
+    l.off_x = l.off_a + M * DF<FORM>::kCPT * l.astride;
+    l.off_red = l.off_x + (stage_x ? 2 * K * (M + (FORM == 1 ? 1 : 0)) : 0);
     l.off_tok = l.off_red + kWarps * NT * 16 * 8 * 4;       // contraction partials
-    // token scratch: warp partials (2 x kWarps x kMaxTok) + cluster partials
-    // (2 x kCluster x kMaxTok), 4 bytes each
-    l.off_bar = l.off_tok + 4 * (2 * kWarps * kMaxTok + 2 * kCluster * kMaxTok);
+    // token scratch: warp partials of the max and of the row sums (2 x kWarps x kMaxTok)
+    l.off_bar = l.off_tok + 4 * (2 * kWarps * kMaxTok);
     l.total = l.off_bar + 16;
     return l;
+}
+
+// 16-byte read of x or g in pass B: from the shared-memory copy when staged,
+// else (coherently) from global memory.
+__device__ __forceinline__ uint4 ld_act(const uint16_t* p, int staged) {
+    return staged ? *reinterpret_cast<const uint4*>(p) : tc::ld_v4(p);
+}
+
+// low bytes of a, b, c, d -> one word (a in the lowest byte)
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+    const uint32_t lo = __byte_perm((uint32_t)a, (uint32_t)b, 0x0040);
+    const uint32_t hi = __byte_perm((uint32_t)c, (uint32_t)d, 0x0040);
+    return __byte_perm(lo, hi, 0x5410);
 }
 
 __device__ __forceinline__ float hbits(uint32_t v) {
@@ -93,52 +110,55 @@ template <int FORM, int NT>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
     using F = DF<FORM>;
     extern __shared__ __align__(16) uint8_t smem[];
-    const DecodeLayout L = decode_layout<FORM, NT>(p.M, p.K);
+    const DecodeLayout L = decode_layout<FORM, NT>(p.M, p.K, p.stage_x);
     const int K = p.K, M = p.M;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t sb = tc::smem_u32(smem);
     const uint32_t bar = sb + L.off_bar;
-    float* red_max = reinterpret_cast<float*>(smem + L.off_tok);             // [kWarps][kMaxTok]
-    int* red_sum = reinterpret_cast<int*>(red_max + kWarps * kMaxTok);       // [kWarps][kMaxTok]
-    float* cl_max = reinterpret_cast<float*>(red_sum + kWarps * kMaxTok);    // [kCluster][kMaxTok]
-    int* cl_sum = reinterpret_cast<int*>(cl_max + kCluster * kMaxTok);       // [kCluster][kMaxTok]
+    float* red_max = reinterpret_cast<float*>(smem + L.off_tok);        // [kWarps][kMaxTok]
+    int* red_sum = reinterpret_cast<int*>(red_max + kWarps * kMaxTok);  // [kWarps][kMaxTok]
     const int rg = blockIdx.x;                 // 16-row group
-    const bool has_rows = rg * 16 < p.N;       // trailing CTAs of the last cluster may be idle
     const int wbytes = K / F::kPerWord * 4;    // packed bytes per weight row
 
     // 1. stream this CTA's weight slab into shared memory (independent of x)
     if (threadIdx.x == 0) {
         tc::mbar_init(bar, 1);
         tc::mbar_fence_init();
-        if (has_rows) {
-            tc::mbar_arrive_expect_tx(bar, (uint32_t)(16 * wbytes));
-            const uint8_t* src = reinterpret_cast<const uint8_t*>(p.w) + (size_t)rg * 16 * wbytes;
-            for (int r = 0; r < 16; ++r)
-                tc::bulk_g2s(sb + r * L.wstride, src + (size_t)r * wbytes, (uint32_t)wbytes, bar);
-        }
+        tc::mbar_arrive_expect_tx(bar, (uint32_t)(16 * wbytes));
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.w) + (size_t)rg * 16 * wbytes;
+        for (int r = 0; r < 16; ++r)
+            tc::bulk_g2s(sb + r * L.wstride, src + (size_t)r * wbytes, (uint32_t)wbytes, bar);
     }
-    // every CTA of the cluster must be running before any distributed
-    // shared-memory store; the matching wait comes just before the first one
-    tc::cluster_arrive_relaxed();
+    __syncthreads();  // the mbarrier is initialised before any thread waits on it
     tc::pdl_trigger();
     tc::pdl_wait();
 
-    // 2-3. cluster-split activation preparation
-    const uint32_t rank = tc::cluster_ctarank();
-    const int ngroups = K / F::kGroup;
+    // 2-3. activation preparation
     constexpr int G = F::kGroup;
-    // pass A: per-token max |x| (ternary) or |x*g| (OneBit) over this CTA's groups
+    const int ngroups = K / G;
+    // pass A: per-token max |x| (ternary) or |x*g| (OneBit); x (and g) are copied
+    // into shared memory on the way, so pass B does not go back to L2
+    uint16_t* xs_s = reinterpret_cast<uint16_t*>(smem + L.off_x);
+    uint16_t* gs_s = xs_s + (size_t)M * K;
+    if (FORM == 1 && p.stage_x) {
+        for (int c = threadIdx.x; c < K / 8; c += kThreads)
+            reinterpret_cast<uint4*>(gs_s)[c] = tc::ld_v4(p.g + 8 * c);
+    }
     for (int m = 0; m < M; ++m) {
         float mx = 0.f;
-        for (int i = (int)rank + kCluster * threadIdx.x; i < ngroups; i += kCluster * kThreads) {
+        for (int i = threadIdx.x; i < ngroups; i += kThreads) {
             const uint16_t* xs = p.x + (size_t)m * K + (size_t)i * G;
 #pragma unroll
             for (int v = 0; v < G / 8; ++v) {
                 uint4 a = tc::ld_v4(xs + 8 * v);
+                if (p.stage_x)
+                    *reinterpret_cast<uint4*>(xs_s + (size_t)m * K + (size_t)i * G + 8 * v) = a;
                 const uint32_t av[4] = {a.x, a.y, a.z, a.w};
                 if (FORM == 0) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(hbits(av[e >> 1] >> (16 * (e & 1)))));
+                    // max of |fp16| bit patterns, two lanes per word (monotone for finite values)
+                    uint32_t mb = __vmaxu2(__vmaxu2(av[0] & 0x7fff7fffu, av[1] & 0x7fff7fffu),
+                                           __vmaxu2(av[2] & 0x7fff7fffu, av[3] & 0x7fff7fffu));
+                    mx = fmaxf(mx, hbits(max(mb & 0xffffu, mb >> 16)));
                 } else {
                     uint4 gg = tc::ld_v4(p.g + (size_t)i * G + 8 * v);
                     const uint32_t gv[4] = {gg.x, gg.y, gg.z, gg.w};
@@ -153,104 +173,87 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         if (lane == 0) red_max[warp * kMaxTok + m] = mx;
     }
     __syncthreads();
-    tc::cluster_wait();
-    if (threadIdx.x < M) {
-        float mx = 0.f;
-        for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, red_max[w * kMaxTok + threadIdx.x]);
-        const uint32_t off = tc::smem_u32(cl_max + rank * kMaxTok + threadIdx.x);
-        for (int d = 0; d < kCluster; ++d) tc::st_cluster_u32(tc::mapa(off, d), __float_as_uint(mx));
-    }
-    tc::cluster_sync();
+    const uint16_t* xsrc = p.stage_x ? xs_s : p.x;
+    const uint16_t* gsrc = p.stage_x ? gs_s : p.g;
 
-    // pass B: quantise this CTA's groups into every CTA's activation tile
+    // pass B: quantise into the permuted shared-memory activation tile
     for (int m = 0; m < M; ++m) {
         float amax = 0.f;
-        for (int r = 0; r < kCluster; ++r) amax = fmaxf(amax, cl_max[r * kMaxTok + m]);
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) amax = fmaxf(amax, red_max[w * kMaxTok + m]);
         int sum = 0;
-        for (int i = (int)rank + kCluster * threadIdx.x; i < ngroups; i += kCluster * kThreads) {
-            const uint16_t* xs = p.x + (size_t)m * K + (size_t)i * G;
+        for (int i = threadIdx.x; i < ngroups; i += kThreads) {
+            const uint16_t* xs = xsrc + (size_t)m * K + (size_t)i * G;
             if (FORM == 0) {
+                // |x * inv| <= 127 (1 + 2^-24) for inv = rn(127/amax): the rounded
+                // value never leaves [-127, 127], so no clamp is needed
                 const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
                 int qv[16];
 #pragma unroll
                 for (int v = 0; v < 2; ++v) {
-                    uint4 a = tc::ld_v4(xs + 8 * v);
+                    uint4 a = ld_act(xs + 8 * v, p.stage_x);
                     const uint32_t av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        int r = __float2int_rn(__fmul_rn(hbits(av[e >> 1] >> (16 * (e & 1))), inv));
-                        r = min(127, max(-127, r));
-                        qv[8 * v + e] = r;
-                        sum += r;
-                    }
+                    for (int e = 0; e < 8; ++e)
+                        qv[8 * v + e] = __float2int_rn(__fmul_rn(hbits(av[e >> 1] >> (16 * (e & 1))), inv));
                 }
-                uint32_t o[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t wv = 0;
-#pragma unroll
-                    for (int bb = 0; bb < 4; ++bb) wv |= ((uint32_t)qv[4 * bb + j] & 0xffu) << (8 * bb);
-                    o[j] = wv;
-                }
-                const uint32_t off = sb + L.off_a + m * L.astride + i * G;
-                const uint4 val = make_uint4(o[0], o[1], o[2], o[3]);
-                for (int d = 0; d < kCluster; ++d) tc::st_cluster_v4(tc::mapa(off, d), val);
+                // byte 4j+b of the group holds element 4b+j
+                uint4 o;
+                o.x = pack4(qv[0], qv[4], qv[8], qv[12]);
+                o.y = pack4(qv[1], qv[5], qv[9], qv[13]);
+                o.z = pack4(qv[2], qv[6], qv[10], qv[14]);
+                o.w = pack4(qv[3], qv[7], qv[11], qv[15]);
+                *reinterpret_cast<uint4*>(smem + L.off_a + m * L.astride + i * G) = o;
+                sum = __dp4a((int)o.x, 0x01010101, sum);
+                sum = __dp4a((int)o.y, 0x01010101, sum);
+                sum = __dp4a((int)o.z, 0x01010101, sum);
+                sum = __dp4a((int)o.w, 0x01010101, sum);
             } else {
                 constexpr int kFix = 32639;
                 const float inv = amax > 0.f ? __fdiv_rn((float)kFix, amax) : 0.f;
                 int hv[32], lv[32];
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
-                    uint4 a = tc::ld_v4(xs + 8 * v);
-                    uint4 gg = tc::ld_v4(p.g + (size_t)i * G + 8 * v);
+                    uint4 a = ld_act(xs + 8 * v, p.stage_x);
+                    uint4 gg = ld_act(gsrc + (size_t)i * G + 8 * v, p.stage_x);
                     const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {gg.x, gg.y, gg.z, gg.w};
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const float pr = __fmul_rn(hbits(av[e >> 1] >> (16 * (e & 1))),
                                                    hbits(gv[e >> 1] >> (16 * (e & 1))));
-                        int X = __float2int_rn(__fmul_rn(pr, inv));
-                        X = min(kFix, max(-kFix, X));
+                        // |pr * inv| <= 32639 (1 + 2^-24): no clamp needed
+                        const int X = __float2int_rn(__fmul_rn(pr, inv));
                         const int hi = (X + 128) >> 8;
                         hv[8 * v + e] = hi;
                         lv[8 * v + e] = X - 256 * hi;
-                        sum += X;
                     }
                 }
+                // byte 4j+b of the 32-byte group holds element 8b+j
                 uint32_t ho[8], lo[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    uint32_t a = 0, b = 0;
+                    ho[j] = pack4(hv[j], hv[8 + j], hv[16 + j], hv[24 + j]);
+                    lo[j] = pack4(lv[j], lv[8 + j], lv[16 + j], lv[24 + j]);
+                }
+                int shi = 0, slo = 0;
 #pragma unroll
-                    for (int bb = 0; bb < 4; ++bb) {
-                        a |= ((uint32_t)hv[8 * bb + j] & 0xffu) << (8 * bb);
-                        b |= ((uint32_t)lv[8 * bb + j] & 0xffu) << (8 * bb);
-                    }
-                    ho[j] = a;
-                    lo[j] = b;
+                for (int j = 0; j < 8; ++j) {
+                    shi = __dp4a((int)ho[j], 0x01010101, shi);
+                    slo = __dp4a((int)lo[j], 0x01010101, slo);
                 }
-                const uint32_t offh = sb + L.off_a + (2 * m) * L.astride + i * G;
-                const uint32_t offl = offh + L.astride;
-                for (int d = 0; d < kCluster; ++d) {
-                    tc::st_cluster_v4(tc::mapa(offh, d), make_uint4(ho[0], ho[1], ho[2], ho[3]));
-                    tc::st_cluster_v4(tc::mapa(offh + 16, d), make_uint4(ho[4], ho[5], ho[6], ho[7]));
-                    tc::st_cluster_v4(tc::mapa(offl, d), make_uint4(lo[0], lo[1], lo[2], lo[3]));
-                    tc::st_cluster_v4(tc::mapa(offl + 16, d), make_uint4(lo[4], lo[5], lo[6], lo[7]));
-                }
+                sum += 256 * shi + slo;  // sum of X over the group
+                uint4* dh = reinterpret_cast<uint4*>(smem + L.off_a + (2 * m) * L.astride + i * G);
+                uint4* dl = reinterpret_cast<uint4*>(smem + L.off_a + (2 * m + 1) * L.astride + i * G);
+                dh[0] = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+                dh[1] = make_uint4(ho[4], ho[5], ho[6], ho[7]);
+                dl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                dl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
             }
         }
         sum = warp_sum(sum);
         if (lane == 0) red_sum[warp * kMaxTok + m] = sum;
     }
     __syncthreads();
-    if (threadIdx.x < M) {
-        int s = 0;
-        for (int w = 0; w < kWarps; ++w) s += red_sum[w * kMaxTok + threadIdx.x];
-        const uint32_t off = tc::smem_u32(cl_sum + rank * kMaxTok + threadIdx.x);
-        for (int d = 0; d < kCluster; ++d) tc::st_cluster_u32(tc::mapa(off, d), (uint32_t)s);
-    }
-    tc::cluster_sync();
-    // From here on no CTA touches another CTA's shared memory.
-    if (!has_rows) return;
 
     const bool w_ok = __syncthreads_and(tc::mbar_wait(bar, 0, p.flags, kWaitLimitNs));
     if (!w_ok) return;
@@ -268,9 +271,13 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         bvalid[nt] = col < ncols;
         bsrc[nt] = smem + L.off_a + (bvalid[nt] ? col : 0) * L.astride + t * F::kChunkK;
     }
-    int acc[NT][4];
+    // four independent accumulator chains (one per word of the lane's 4-word
+    // chunk) cut the dependent MMA latency per step
+    int acc[NT][4][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[nt][c][0] = acc[nt][c][1] = acc[nt][c][2] = acc[nt][c][3] = 0;
     const int nsteps = (K + F::kStepK - 1) / F::kStepK;
     for (int s = warp; s < nsteps; s += kWarps) {
         const bool lane_ok = s * F::kStepK + t * F::kChunkK < K;
@@ -308,7 +315,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                 }
 #pragma unroll
                 for (int j = 0; j < F::kRegs; j += 2)
-                    mma_u8s8_16832(acc[nt], u0[j], u1[j], u0[j + 1], u1[j + 1], b[j], b[j + 1]);
+                    mma_u8s8_16832(acc[nt][om], u0[j], u1[j], u0[j + 1], u1[j + 1], b[j], b[j + 1]);
             }
         }
     }
@@ -317,10 +324,13 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         int* rb = red + ((warp * NT + nt) * 16) * 8;
-        rb[g * 8 + 2 * t] = acc[nt][0];
-        rb[g * 8 + 2 * t + 1] = acc[nt][1];
-        rb[(g + 8) * 8 + 2 * t] = acc[nt][2];
-        rb[(g + 8) * 8 + 2 * t + 1] = acc[nt][3];
+        int v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = acc[nt][0][e] + acc[nt][1][e] + acc[nt][2][e] + acc[nt][3][e];
+        rb[g * 8 + 2 * t] = v[0];
+        rb[g * 8 + 2 * t + 1] = v[1];
+        rb[(g + 8) * 8 + 2 * t] = v[2];
+        rb[(g + 8) * 8 + 2 * t + 1] = v[3];
     }
     __syncthreads();
     auto part = [&](int col, int r) {
@@ -334,9 +344,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
             const int m = o >> 4, r = o & 15;
             float amax = 0.f;
             int qs = 0;
-            for (int c = 0; c < kCluster; ++c) {
-                amax = fmaxf(amax, cl_max[c * kMaxTok + m]);
-                qs += cl_sum[c * kMaxTok + m];
+            for (int w = 0; w < kWarps; ++w) {
+                amax = fmaxf(amax, red_max[w * kMaxTok + m]);
+                qs += red_sum[w * kMaxTok + m];
             }
             const float sc = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
             const int accv = part(m, r) - qs;
@@ -350,9 +360,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
             const int m = o >> 4, r = o & 15;
             float amax = 0.f;
             long long ts = 0;
-            for (int c = 0; c < kCluster; ++c) {
-                amax = fmaxf(amax, cl_max[c * kMaxTok + m]);
-                ts += cl_sum[c * kMaxTok + m];
+            for (int w = 0; w < kWarps; ++w) {
+                amax = fmaxf(amax, red_max[w * kMaxTok + m]);
+                ts += red_sum[w * kMaxTok + m];
             }
             const float st = amax > 0.f ? __fdiv_rn(amax, 32639.0f) : 0.f;
             const long long P = 256ll * part(2 * m, r) + part(2 * m + 1, r);
@@ -366,6 +376,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
 
 template <int FORM, int NT>
 cudaError_t launch_decode(const DecodeParams& p, int smem, cudaStream_t s) {
+    static_assert(NT >= 1, "");
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(decode_kernel<FORM, NT>,
@@ -374,21 +385,16 @@ cudaError_t launch_decode(const DecodeParams& p, int smem, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    const int groups = p.N / 16;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((groups + kCluster - 1) / kCluster * kCluster);
+    cfg.gridDim = dim3(p.N / 16);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = s;
-    cudaLaunchAttribute attrs[2];
-    attrs[0].id = cudaLaunchAttributeClusterDimension;
-    attrs[0].val.clusterDim.x = kCluster;
-    attrs[0].val.clusterDim.y = 1;
-    attrs[0].val.clusterDim.z = 1;
-    attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attrs[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attrs[1];
+    attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, decode_kernel<FORM, NT>, p);
 }
 
@@ -399,17 +405,25 @@ int pick_nt(int M) {
 }
 
 template <int FORM>
-int decode_smem(int M, int K) {
+int decode_smem(int M, int K, int stage_x) {
     const int nt = pick_nt<FORM>(M);
     if (nt == 0) return -1;
-    if (nt == 1) return decode_layout<FORM, 1>(M, K).total;
-    if (nt == 2) return decode_layout<FORM, 2>(M, K).total;
-    return decode_layout<FORM, 4>(M, K).total;
+    if (nt == 1) return decode_layout<FORM, 1>(M, K, stage_x).total;
+    if (nt == 2) return decode_layout<FORM, 2>(M, K, stage_x).total;
+    return decode_layout<FORM, 4>(M, K, stage_x).total;
+}
+
+// Stage x in shared memory whenever that still fits next to the weight slab.
+template <int FORM>
+int decode_stage_x(int M, int K) {
+    const int s = decode_smem<FORM>(M, K, 1);
+    return (s > 0 && s <= kDecodeMaxSmem) ? 1 : 0;
 }
 
 template <int FORM>
-cudaError_t launch_decode_form(const DecodeParams& p, cudaStream_t s) {
-    const int smem = decode_smem<FORM>(p.M, p.K);
+cudaError_t launch_decode_form(DecodeParams p, cudaStream_t s) {
+    p.stage_x = decode_stage_x<FORM>(p.M, p.K);
+    const int smem = decode_smem<FORM>(p.M, p.K, p.stage_x);
     switch (pick_nt<FORM>(p.M)) {
         case 1: return launch_decode<FORM, 1>(p, smem, s);
         case 2: return launch_decode<FORM, 2>(p, smem, s);
@@ -421,21 +435,21 @@ cudaError_t launch_decode_form(const DecodeParams& p, cudaStream_t s) {
 
 bool decode_fused_fits(int form, int M, int K) {
     if (M < 1 || M > kMaxTok) return false;
-    const int smem = form == 0 ? decode_smem<0>(M, K) : decode_smem<1>(M, K);
+    const int smem = form == 0 ? decode_smem<0>(M, K, 0) : decode_smem<1>(M, K, 0);
     return smem > 0 && smem <= kDecodeMaxSmem;
 }
 
 cudaError_t launch_ternary_decode(const uint16_t* x, const uint32_t* w2, int M, int K, int N,
                                   float w_scale, uint16_t* y, int32_t* acc_out,
                                   unsigned int* flags, cudaStream_t s) {
-    DecodeParams p{x, nullptr, nullptr, w2, w_scale, M, K, N, y, acc_out, flags};
+    DecodeParams p{0, x, nullptr, nullptr, w2, w_scale, M, K, N, y, acc_out, flags};
     return launch_decode_form<0>(p, s);
 }
 
 cudaError_t launch_onebit_decode(const uint16_t* x, const uint16_t* g, const uint16_t* h,
                                  const uint32_t* s1, int M, int K, int N, uint16_t* y,
                                  unsigned int* flags, cudaStream_t s) {
-    DecodeParams p{x, g, h, s1, 0.f, M, K, N, y, nullptr, flags};
+    DecodeParams p{0, x, g, h, s1, 0.f, M, K, N, y, nullptr, flags};
     return launch_decode_form<1>(p, s);
 }
 

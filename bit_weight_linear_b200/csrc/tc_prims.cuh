@@ -224,6 +224,15 @@ __device__ __forceinline__ uint4 ld_v4(const void* p) {
     return v;
 }
 
+// Per-thread 16-byte asynchronous copy global -> shared (L2 only), the
+// load/store-unit path, independent of the bulk-copy engine's queue.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Untiled bulk copy global -> this CTA's shared memory (16-byte aligned
 // addresses, size a multiple of 16), completion counted on `bar`.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
