@@ -38,6 +38,8 @@ LLAMA7B_LAYERS = 32
 # the same block with the projections that share an input fused into one call each
 LLAMA7B_BLOCK_FUSED = [("qkv", 4096, 3 * 4096), ("o", 4096, 4096), ("gate+up", 4096, 2 * 11008),
                        ("down", 11008, 4096)]
+LLAMA13B_SWEEP = [("up", 5120, 13824), ("down", 13824, 5120)]   # (name, K, N)
+SWEEP_M = [1, 4, 16, 64, 256, 1024]
 LLAMA70B_PREFILL = [("qkvo-like", 8192, 8192), ("gate/up", 8192, 28672), ("down", 28672, 8192)]
 PREFILL_M = 512
 W_SCALE = 0.02
@@ -290,6 +292,58 @@ def run_prefill(blw, synth, dev, args, dist_on, world, peaks):
                      "peak_source": "2 x measured sustained bf16 (nominal int8/bf16 ratio)"}}
 
 
+def run_sweep(blw, synth, dev, peaks, reps=10):
+    """Batch sweep on the LLaMA-13B-shaped layers, both forms: per (form, shape, M)
+    the effective weight GB/s and int8 TOPS of one call, over rotating weight
+    copies that total more than twice the L2 (each call streams its weights)."""
+    l2_bytes = 126 * 2 ** 20
+    i8_peak = 2.0 * peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    out = []
+    for form in ("ternary", "onebit"):
+        for (name, K, N) in LLAMA13B_SWEEP:
+            wb = N * K // (4 if form == "ternary" else 8)
+            copies = max(2, -(-2 * l2_bytes // wb) + 1)
+            ws, gs, hs = [], None, None
+            for c in range(copies):
+                seed = 4_000_000 + 100 * c + (0 if name == "up" else 50)
+                if form == "ternary":
+                    w = synth.ternary_weights(N, K, seed=seed, device=dev)
+                    ws.append(blw.bl_pack_ternary(w))
+                else:
+                    w = synth.sign_weights(N, K, seed=seed, device=dev)
+                    ws.append(blw.ob_pack_sign(w))
+                del w
+            if form == "onebit":
+                gs = synth.value_vector(K, seed=4_000_900, device=dev)
+                hs = synth.value_vector(N, seed=4_000_901, device=dev)
+            for M in SWEEP_M:
+                x = synth.activations(M, K, seed=4_001_000 + M, device=dev)
+                y = torch.empty((M, N), dtype=torch.float16, device=dev)
+                nws = (blw.bl_ternary_workspace_bytes if form == "ternary" else blw.ob_workspace_bytes)(M, K, N)
+                wsp = torch.empty((nws,), dtype=torch.uint8, device=dev)
+
+                def step():
+                    for w2 in ws:
+                        if form == "ternary":
+                            blw.bl_ternary_linear(x, w2, W_SCALE, workspace=wsp, out=y)
+                        else:
+                            blw.ob_linear(x, w2, gs, hs, workspace=wsp, out=y)
+
+                g = capture(step)
+                ms = time_replays(g, reps, 3, False, dev) / copies
+                gbs = (wb + (2 * (K + N) if form == "onebit" else 0)) / (ms * 1e-3) / 1e9
+                tops = 2 * M * K * N / (ms * 1e-3) / 1e12
+                out.append({"form": form, "layer": f"{name} {K}->{N}", "M": M, "us_per_call": round(ms * 1e3, 2),
+                            "weight_GBs": round(gbs, 1), "TOPS": round(tops, 2),
+                            "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+                            "int8_frac": round(tops / i8_peak, 4)})
+                del g, x, y, wsp
+            del ws
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+    return out
+
+
 # --------------------------------------------------------------- main -----
 
 def main():
@@ -302,6 +356,7 @@ def main():
     ap.add_argument("--layers", type=int, default=LLAMA7B_LAYERS,
                     help="blocks in the decode stack (fewer = a small profiling case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the 13B batch sweep")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the M=512 prefill layers (a profiling case)")
     args = ap.parse_args()
@@ -442,6 +497,8 @@ def main():
         torch.cuda.empty_cache()
 
         extras["prefill"] = run_prefill(blw, synth, dev, args, dist_on, world, peaks)
+        if not args.no_sweep:
+            extras["batch_sweep_13b"] = run_sweep(blw, synth, dev, peaks)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,

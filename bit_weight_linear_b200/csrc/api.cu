@@ -4,7 +4,7 @@
 #include <cstdlib>
 #include <cstring>
 
-#include "../../include/bitlinear.h"
+#include "bitlinear.h"
 #include "common.cuh"
 #include "kernels.h"
 

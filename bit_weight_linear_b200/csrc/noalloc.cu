@@ -18,7 +18,7 @@
 // caches it; make that first call before any stream capture.
 #include <mutex>
 
-#include "../../include/bitlinear.h"
+#include "bitlinear.h"
 #include "common.cuh"
 #include "kernels.h"
 

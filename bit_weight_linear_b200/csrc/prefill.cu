@@ -5,22 +5,32 @@
 // "BitNet b1.58 介绍": 8-bit activations against ternary weights; OneBit page,
 // "1. 新的 1bit 结构": the +-1 matrix between x*g and h), so the weights are
 // expanded on chip to int8 and run through the int8 tensor cores:
-//   ternary: B = code in {0,1,2} (= t + 1), D = q . code^T, acc = D - sum_k q
-//   OneBit : B = bit in {0,1}, A rows = the two int8 limbs (hi, lo) of each
+//   ternary: code in {0,1,2} (= t + 1), D = code . q^T, acc = D - sum_k q
+//   OneBit : bit in {0,1}, activation rows = the two int8 limbs (hi, lo) of each
 //            token's 16-bit fixed-point image X of x*g, so
 //            sum X*S = 2 (256 D_hi + D_lo) - sum X
 // Both are exact in int32.
 //
-// CTA tile: 128 A rows (tokens, or token limbs) x 256 weight rows, K in
-// 128-byte stages.  Warp roles (192 threads):
-//   warp 0     TMA producer: A tile (128x128 B, 128-byte swizzle) and the packed
-//              weight tile (256 rows x 32 B or 16 B) into a 3-stage ring;
+// The expanded weights never touch shared memory: they are the MMA's A
+// operand and live in TENSOR memory.  Each unpack thread owns one weight row
+// (one TMEM lane), expands that row's 128 k of a stage to 128 bytes and writes
+// them with one tcgen05.st; the MMA reads A from TMEM and only the activations
+// (B operand, TMA-loaded, 128-byte swizzle) come from shared memory.  That
+// keeps shared-memory traffic per MMA at the activation tile alone.
+//
+// CTA tile: 128 weight rows (MMA M, TMEM lanes) x 256 activation rows (MMA N:
+// tokens, or token limb rows), K in 128-byte stages; tiles ordered
+// activation-tile-fastest so CTAs sharing a weight tile run together.
+// Warp roles (192 threads):
+//   warp 0     TMA producer: activation tile (256 x 128 B) and packed weight tile
+//              (128 rows x 32 B or 16 B) into a 5-stage shared-memory ring;
 //   warp 1     TMEM allocator + single-thread MMA issuer (4 x K=32 per stage);
-//   warps 2-5  unpack the packed tile into the UMMA K-major 128-byte-swizzled
-//              int8 layout, then run the epilogue (tcgen05.ld -> scale -> fp16).
-// The unpacked byte order inside each 16-byte (ternary) / 32-byte (sign) group
+//   warps 2-5  one thread per weight row: unpack into a 4-slot TMEM ring, then
+//              the epilogue (tcgen05.ld -> correction and scale -> fp16), in
+//              which a warp's lanes are 32 consecutive output columns.
+// The expanded byte order inside each 16-byte (ternary) / 32-byte (sign) group
 // is the order the byte-SIMD unpack produces; the activation preparation
-// kernels store A in the same order, so no shuffle is needed anywhere.
+// kernels store the activations in the same order.
 // Every mbarrier wait is bounded (a timeout sets the device condition word).
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -33,20 +43,22 @@ namespace bl {
 
 namespace {
 
-constexpr int BM = 128;          // A rows per tile (MMA M)
-constexpr int BN = 256;          // weight rows per tile (MMA N)
-constexpr int BK = 128;          // k per stage (bytes of int8 A per row)
-constexpr int STAGES = 3;
+constexpr int BW = 128;          // weight rows per tile (MMA M)
+constexpr int BT = 256;          // activation rows per tile (MMA N)
+constexpr int BK = 128;          // k per stage (bytes of int8 per activation row)
+constexpr int SS = 5;            // shared-memory ring stages
+constexpr int SU = 4;            // TMEM slots for expanded weights
 constexpr int kThreads = 192;
-constexpr int A_STAGE = BM * BK;        // 16 KB
-constexpr int BU_STAGE = BN * BK;       // 32 KB
-constexpr int BP_STAGE_MAX = BN * BK / 4;  // 8 KB (ternary); sign uses half
-constexpr int OFF_A = 0;
-constexpr int OFF_BU = OFF_A + STAGES * A_STAGE;
-constexpr int OFF_BP = OFF_BU + STAGES * BU_STAGE;
-constexpr int OFF_BAR = OFF_BP + STAGES * BP_STAGE_MAX;
-constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
-constexpr uint32_t TMEM_COLS = 256;
+constexpr int ACT_STAGE = BT * BK;        // 32 KB
+constexpr int BP_STAGE = BW * BK / 4;     // 4 KB (ternary); sign uses half
+constexpr int OFF_ACT = 0;
+constexpr int OFF_BP = OFF_ACT + SS * ACT_STAGE;
+constexpr int OFF_TOK = OFF_BP + SS * BP_STAGE;          // per-token scale / row sum [BT]
+constexpr int OFF_BAR = OFF_TOK + 2 * BT * 4;
+constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;         // barriers + alignment slack
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t kAccCol = 0;          // accumulator: columns [0, 256)
+constexpr uint32_t kWCol = 256;          // expanded-weight slots: 32 columns each
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 template <int FORM>
@@ -61,7 +73,7 @@ struct PF<1> {  // sign
 };
 
 struct PrefillParams {
-    int rows_a;        // M (ternary) or 2M (OneBit limb rows)
+    int rows_a;        // activation rows: M (ternary) or 2M (OneBit limb rows)
     int M, K, N;
     const float* scale;   // per token: ternary scale / OneBit fixed-point step
     const int32_t* rsum;  // per token: sum q / sum X
@@ -74,35 +86,39 @@ struct PrefillParams {
 
 template <int FORM>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                   const __grid_constant__ CUtensorMap tmap_b, const PrefillParams p) {
+    prefill_kernel(const __grid_constant__ CUtensorMap tmap_act,
+                   const __grid_constant__ CUtensorMap tmap_w, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = tc::smem_u32(smem);
-    const uint32_t bar_full = sbase + OFF_BAR;             // TMA landed   [STAGES]
-    const uint32_t bar_unp = bar_full + 8 * STAGES;        // unpacked     [STAGES]
-    const uint32_t bar_empty = bar_unp + 8 * STAGES;       // MMA consumed [STAGES]
-    const uint32_t bar_acc = bar_empty + 8 * STAGES;       // accumulator complete
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * (3 * STAGES + 1));
+    const uint32_t bar_full = sbase + OFF_BAR;        // activation + packed tile landed [SS]
+    const uint32_t bar_empty = bar_full + 8 * SS;     // MMA done with the stage        [SS]
+    const uint32_t bar_ufull = bar_empty + 8 * SS;    // expanded weights in TMEM      [SU]
+    const uint32_t bar_uempty = bar_ufull + 8 * SU;   // MMA done with a TMEM slot     [SU]
+    const uint32_t bar_acc = bar_uempty + 8 * SU;     // accumulator complete
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * (2 * SS + 2 * SU + 1));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN;
-    const int m0 = blockIdx.y * BM;
+    const int ttiles = (p.rows_a + BT - 1) / BT;
+    const int t0 = (blockIdx.x % ttiles) * BT;   // first activation row of the tile
+    const int n0 = (blockIdx.x / ttiles) * BW;   // first weight row of the tile
     const int nk = p.K / BK;
-    constexpr int kBp = PF<FORM>::kPackedRowBytes * BN;
-    constexpr uint32_t kTx = A_STAGE + kBp;
+    constexpr uint32_t kTx = ACT_STAGE + PF<FORM>::kPackedRowBytes * BW;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < SS; ++s) {
             tc::mbar_init(bar_full + 8 * s, 1);
-            tc::mbar_init(bar_unp + 8 * s, 128);
             tc::mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int u = 0; u < SU; ++u) {
+            tc::mbar_init(bar_ufull + 8 * u, 128);
+            tc::mbar_init(bar_uempty + 8 * u, 1);
         }
         tc::mbar_init(bar_acc, 1);
         tc::mbar_fence_init();
-        tc::prefetch_tmap(&tmap_a);
-        tc::prefetch_tmap(&tmap_b);
+        tc::prefetch_tmap(&tmap_act);
+        tc::prefetch_tmap(&tmap_w);
     }
     if (warp == 1) {
         tc::tmem_alloc(tc::smem_u32(tmem_slot), TMEM_COLS);
@@ -111,181 +127,134 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    const uint32_t tmem_d = *tmem_slot;
+    const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
         if (lane == 0) {
             int issued = 0;
             bool ok = true;
             for (int kb = 0; kb < nk && ok; ++kb) {
-                const int s = kb % STAGES;
-                if (kb >= STAGES)
-                    ok = tc::mbar_wait(bar_empty + 8 * s, ((kb / STAGES) - 1) & 1, p.flags,
-                                       kWaitLimitNs);
+                const int s = kb % SS;
+                if (kb >= SS)
+                    ok = tc::mbar_wait(bar_empty + 8 * s, ((kb / SS) - 1) & 1, p.flags, kWaitLimitNs);
                 if (!ok) break;
                 tc::mbar_arrive_expect_tx(bar_full + 8 * s, kTx);
-                tc::tma_load_2d(sbase + OFF_A + s * A_STAGE, &tmap_a, kb * BK, m0, bar_full + 8 * s);
-                tc::tma_load_2d(sbase + OFF_BP + s * BP_STAGE_MAX, &tmap_b,
+                tc::tma_load_2d(sbase + OFF_ACT + s * ACT_STAGE, &tmap_act, kb * BK, t0,
+                                bar_full + 8 * s);
+                tc::tma_load_2d(sbase + OFF_BP + s * BP_STAGE, &tmap_w,
                                 kb * PF<FORM>::kPackedRowBytes, n0, bar_full + 8 * s);
                 ++issued;
             }
             if (!ok) {
                 // drain copies still in flight before the CTA's shared memory goes away
-                for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
-                    tc::mbar_wait(bar_full + 8 * (kb % STAGES), (kb / STAGES) & 1, p.flags,
-                                  kWaitLimitNs);
+                for (int kb = (issued > SS ? issued - SS : 0); kb < issued; ++kb)
+                    tc::mbar_wait(bar_full + 8 * (kb % SS), (kb / SS) & 1, p.flags, kWaitLimitNs);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = tc::idesc_i8(BM, BN);
+            constexpr uint32_t idesc = tc::idesc_i8(BW, BT);
             bool ok = true;
             for (int kb = 0; kb < nk && ok; ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t par = (kb / STAGES) & 1;
-                ok = tc::mbar_wait(bar_full + 8 * s, par, p.flags, kWaitLimitNs) &&
-                     tc::mbar_wait(bar_unp + 8 * s, par, p.flags, kWaitLimitNs);
+                const int s = kb % SS, u = kb % SU;
+                ok = tc::mbar_wait(bar_full + 8 * s, (kb / SS) & 1, p.flags, kWaitLimitNs) &&
+                     tc::mbar_wait(bar_ufull + 8 * u, (kb / SU) & 1, p.flags, kWaitLimitNs);
                 if (!ok) break;
                 tc::tc_fence_after();
-                const uint32_t a_s = sbase + OFF_A + s * A_STAGE;
-                const uint32_t b_s = sbase + OFF_BU + s * BU_STAGE;
+                const uint32_t act_s = sbase + OFF_ACT + s * ACT_STAGE;
 #pragma unroll
                 for (int j = 0; j < BK / 32; ++j)
-                    tc::mma_i8(tmem_d, tc::desc_kmajor_sw128(a_s + 32 * j),
-                               tc::desc_kmajor_sw128(b_s + 32 * j), idesc, kb > 0 || j > 0);
+                    tc::mma_i8_ts(tmem + kAccCol, tmem + kWCol + 32 * u + 8 * j,
+                                  tc::desc_kmajor_sw128(act_s + 32 * j), idesc, kb > 0 || j > 0);
                 tc::mma_commit(bar_empty + 8 * s);
+                tc::mma_commit(bar_uempty + 8 * u);
             }
             // completion of everything issued (also on the abort path)
             tc::mma_commit(bar_acc);
             tc::mbar_wait(bar_acc, 0, p.flags, kWaitLimitNs);
         }
     } else {
-        // ---------------- unpack (warps 2-5, 128 threads) -------------------
-        const int ut = threadIdx.x - 64;  // 0..127
+        // ------- expand (warps 2-5): thread = weight row = TMEM lane -------
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int r = 32 * q + lane;            // weight row within the tile
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         bool ok = true;
         for (int kb = 0; kb < nk && ok; ++kb) {
-            const int s = kb % STAGES;
-            ok = tc::mbar_wait(bar_full + 8 * s, (kb / STAGES) & 1, p.flags, kWaitLimitNs);
+            const int s = kb % SS, u = kb % SU;
+            ok = tc::mbar_wait(bar_full + 8 * s, (kb / SS) & 1, p.flags, kWaitLimitNs);
+            if (ok && kb >= SU)
+                ok = tc::mbar_wait(bar_uempty + 8 * u, ((kb / SU) - 1) & 1, p.flags, kWaitLimitNs);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
-            const uint8_t* bp = smem + OFF_BP + s * BP_STAGE_MAX;
-            uint8_t* bu = smem + OFF_BU + s * BU_STAGE;
+            const uint8_t* bp = smem + OFF_BP + s * BP_STAGE;
+            uint32_t e[32];
+            if (FORM == 0) {
+                const uint4 w0 = *reinterpret_cast<const uint4*>(bp + r * 32);
+                const uint4 w1 = *reinterpret_cast<const uint4*>(bp + r * 32 + 16);
+                const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int r = ut + 128 * half;   // weight row within the tile
-                uint8_t* rowp = bu + r * BK;
-                const int sw = r & 7;
-                if (FORM == 0) {
-                    const uint4* src = reinterpret_cast<const uint4*>(bp + r * 32);
+                for (int o = 0; o < 8; ++o)
 #pragma unroll
-                    for (int v = 0; v < 2; ++v) {
-                        const uint4 w = src[v];
-                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                    for (int j = 0; j < 4; ++j) e[4 * o + j] = (ws[o] >> (2 * j)) & 0x03030303u;
+            } else {
+                const uint4 w0 = *reinterpret_cast<const uint4*>(bp + r * 16);
+                const uint32_t ws[4] = {w0.x, w0.y, w0.z, w0.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const uint32_t x = ws[e];
-                            const int c = 4 * v + e;  // 16-byte chunk = packed word
-                            *reinterpret_cast<uint4*>(rowp + ((c ^ sw) << 4)) =
-                                make_uint4(x & 0x03030303u, (x >> 2) & 0x03030303u,
-                                           (x >> 4) & 0x03030303u, (x >> 6) & 0x03030303u);
-                        }
-                    }
-                } else {
-                    const uint4 w = *reinterpret_cast<const uint4*>(bp + r * 16);
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                for (int o = 0; o < 4; ++o)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t x = ws[e];
-                        const int c0 = 2 * e, c1 = 2 * e + 1;
-                        *reinterpret_cast<uint4*>(rowp + ((c0 ^ sw) << 4)) =
-                            make_uint4(x & 0x01010101u, (x >> 1) & 0x01010101u,
-                                       (x >> 2) & 0x01010101u, (x >> 3) & 0x01010101u);
-                        *reinterpret_cast<uint4*>(rowp + ((c1 ^ sw) << 4)) =
-                            make_uint4((x >> 4) & 0x01010101u, (x >> 5) & 0x01010101u,
-                                       (x >> 6) & 0x01010101u, (x >> 7) & 0x01010101u);
-                    }
-                }
+                    for (int j = 0; j < 8; ++j) e[8 * o + j] = (ws[o] >> j) & 0x01010101u;
             }
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(bar_unp + 8 * s);
+            tc::tmem_st_32x32b_x32(lane_base + kWCol + 32 * u, e);
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            tc::mbar_arrive(bar_ufull + 8 * u);
         }
 
         // ---------------- epilogue ----------------------------------------
+        // per-token scale and row sum of this activation tile, staged once
+        float* tok_scale = reinterpret_cast<float*>(smem + OFF_TOK);
+        int* tok_rsum = reinterpret_cast<int*>(tok_scale + BT);
+        const int et = threadIdx.x - 64;        // 0..127
+        for (int i = et; i < BT; i += 128) {
+            const int row = t0 + i;
+            const int tok = FORM == 0 ? row : row >> 1;
+            const bool in = FORM == 0 ? row < p.M : tok < p.M;
+            tok_scale[i] = in ? p.scale[tok] : 0.f;
+            tok_rsum[i] = in ? p.rsum[tok] : 0;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");   // the four epilogue warps only
         const bool acc_ok =
             __all_sync(0xffffffffu, tc::mbar_wait(bar_acc, 0, p.flags, kWaitLimitNs));
         tc::tc_fence_after();
+        const int n = n0 + r;                    // output column held by this thread
         if (ok && acc_ok) {
-            const int q = warp & 3;             // TMEM lane quarter this warp may read
-            const int arow = m0 + 32 * q + lane;  // A row held by this thread
+            const float hn = (FORM == 1 && n < p.N) ? __half2float(__ushort_as_half(p.h[n])) : 0.f;
 #pragma unroll 1
-            for (int cc = 0; cc < BN / 32; ++cc) {
-                uint32_t r[32];
-                tc::tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(32 * q) << 16) + 32 * cc, r);
+            for (int cc = 0; cc < BT / 32; ++cc) {
+                uint32_t d[32];
+                tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * cc, d);
                 tc::tmem_ld_wait();
-                const int nb = n0 + 32 * cc;
+                if (n >= p.N) continue;
                 if (FORM == 0) {
-                    if (arow < p.M && nb < p.N) {
-                        const float sc = p.scale[arow];
-                        const int rs = p.rsum[arow];
-                        uint32_t packed[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int a0 = (int)r[2 * i] - rs, a1 = (int)r[2 * i + 1] - rs;
-                            const float v0 = __fmul_rn(__fmul_rn((float)a0, sc), p.w_scale);
-                            const float v1 = __fmul_rn(__fmul_rn((float)a1, sc), p.w_scale);
-                            packed[i] = (uint32_t)__half_as_ushort(__float2half_rn(v0)) |
-                                        ((uint32_t)__half_as_ushort(__float2half_rn(v1)) << 16);
-                            r[2 * i] = (uint32_t)a0;
-                            r[2 * i + 1] = (uint32_t)a1;
-                        }
-                        uint16_t* yrow = p.y + (size_t)arow * p.N + nb;
-#pragma unroll
-                        for (int g8 = 0; g8 < 4; ++g8)
-                            if (nb + 8 * g8 < p.N)
-                                reinterpret_cast<uint4*>(yrow)[g8] =
-                                    make_uint4(packed[4 * g8], packed[4 * g8 + 1],
-                                               packed[4 * g8 + 2], packed[4 * g8 + 3]);
-                        if (p.acc_out) {
-                            int32_t* arw = p.acc_out + (size_t)arow * p.N + nb;
-#pragma unroll
-                            for (int g4 = 0; g4 < 8; ++g4)
-                                if (nb + 4 * g4 < p.N)
-                                    reinterpret_cast<uint4*>(arw)[g4] =
-                                        make_uint4(r[4 * g4], r[4 * g4 + 1], r[4 * g4 + 2],
-                                                   r[4 * g4 + 3]);
+                    for (int i = 0; i < 32; ++i) {
+                        const int ti = 32 * cc + i, m = t0 + ti;
+                        if (m < p.M) {
+                            const int a = (int)d[i] - tok_rsum[ti];
+                            const float v = __fmul_rn(__fmul_rn((float)a, tok_scale[ti]), p.w_scale);
+                            p.y[(size_t)m * p.N + n] = __half_as_ushort(__float2half_rn(v));
+                            if (p.acc_out) p.acc_out[(size_t)m * p.N + n] = a;
                         }
                     }
                 } else {
-                    // lanes (2i, 2i+1) hold the hi and lo limb rows of one token
-                    uint32_t lo[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) lo[i] = __shfl_down_sync(0xffffffffu, r[i], 1);
-                    const int tok = arow >> 1;
-                    if ((lane & 1) == 0 && tok < p.M && nb < p.N) {
-                        const float st = p.scale[tok];
-                        const long long ts = p.rsum[tok];
-                        uint32_t packed[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            float v[2];
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int c = 2 * i + e;
-                                const long long P = 256ll * (int)r[c] + (int)lo[c];
-                                const float z = __fmul_rn(st, (float)(2 * P - ts));
-                                const int n = min(nb + c, p.N - 1);
-                                v[e] = __fmul_rn(z, __half2float(__ushort_as_half(p.h[n])));
-                            }
-                            packed[i] = (uint32_t)__half_as_ushort(__float2half_rn(v[0])) |
-                                        ((uint32_t)__half_as_ushort(__float2half_rn(v[1])) << 16);
+                    for (int i = 0; i < 32; i += 2) {
+                        const int ti = 32 * cc + i, tok = (t0 + ti) >> 1;
+                        if (tok < p.M) {
+                            const long long P = 256ll * (int)d[i] + (int)d[i + 1];
+                            const float z = __fmul_rn(tok_scale[ti], (float)(2 * P - (long long)tok_rsum[ti]));
+                            p.y[(size_t)tok * p.N + n] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hn)));
                         }
-                        uint16_t* yrow = p.y + (size_t)tok * p.N + nb;
-#pragma unroll
-                        for (int g8 = 0; g8 < 4; ++g8)
-                            if (nb + 8 * g8 < p.N)
-                                reinterpret_cast<uint4*>(yrow)[g8] =
-                                    make_uint4(packed[4 * g8], packed[4 * g8 + 1],
-                                               packed[4 * g8 + 2], packed[4 * g8 + 3]);
                     }
                 }
             }
@@ -297,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         __syncwarp();
         tc::tc_fence_after();
-        tc::tmem_dealloc(tmem_d, TMEM_COLS);
+        tc::tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
@@ -340,16 +309,16 @@ cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, const PrefillPa
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    CUtensorMap ta, tb;
-    if (!make_tmap(&ta, act, (uint64_t)p.rows_a, (uint64_t)p.K, BK, BM,
+    CUtensorMap ta, tw;
+    if (!make_tmap(&ta, act, (uint64_t)p.rows_a, (uint64_t)p.K, BK, BT,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     const uint64_t prow = (uint64_t)p.K / (FORM == 0 ? 4 : 8);
-    if (!make_tmap(&tb, w, (uint64_t)p.N, prow, PF<FORM>::kPackedRowBytes, BN,
+    if (!make_tmap(&tw, w, (uint64_t)p.N, prow, PF<FORM>::kPackedRowBytes, BW,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    dim3 grid((p.N + BN - 1) / BN, (p.rows_a + BM - 1) / BM);
-    prefill_kernel<FORM><<<grid, kThreads, SMEM_BYTES, s>>>(ta, tb, p);
+    const int tiles = ((p.N + BW - 1) / BW) * ((p.rows_a + BT - 1) / BT);
+    prefill_kernel<FORM><<<tiles, kThreads, SMEM_BYTES, s>>>(ta, tw, p);
     return cudaGetLastError();
 }
 
