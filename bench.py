@@ -200,11 +200,17 @@ def barrier(dist_on):
 
 
 def max_over_ranks(v: float, dist_on: bool, dev) -> float:
+    """Slowest rank's time: every rank takes part, in the same order on all ranks."""
     if not dist_on:
         return v
     t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: units all ranks processed / slowest rank's time (ms)."""
+    return units_per_rank * world / (ms_max * 1e-3)
 
 
 def time_replays(g, steps, warmup, dist_on, dev, clocks=None):
