@@ -54,6 +54,9 @@ struct DF<1> {
 
 struct DecodeParams {
     int stage_x;            // 1: x (and g) are staged in shared memory between the two passes
+    const int8_t* prep;     // prepared activations [cols][K] (PREP kernels only)
+    const float* pscale;    // per token: scale (ternary) / fixed-point step (OneBit)
+    const int32_t* prsum;   // per token: row sum of the prepared activations
     const uint16_t* x;
     const uint16_t* g;      // OneBit input value vector
     const uint16_t* h;      // OneBit output value vector
@@ -106,7 +109,10 @@ __device__ __forceinline__ float hbits(uint32_t v) {
     return __half2float(__ushort_as_half((unsigned short)(v & 0xffffu)));
 }
 
-template <int FORM, int NT>
+// PREP = 0: the kernel prepares the activations from x itself (decode sizes).
+// PREP = 1: they were prepared by the activation kernel launched just before
+// (quant.cu); the kernel only copies them into shared memory.
+template <int FORM, int NT, int PREP>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
     using F = DF<FORM>;
     extern __shared__ __align__(16) uint8_t smem[];
@@ -133,6 +139,17 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     tc::pdl_trigger();
     tc::pdl_wait();
 
+    if (PREP) {
+        // prepared activations -> shared memory as 16-byte asynchronous copies
+        const int cols = M * F::kCPT, per_row = K / 16;
+        for (int c = threadIdx.x; c < cols * per_row; c += kThreads) {
+            const int row = c / per_row, off = c - row * per_row;
+            tc::cp_async16(sb + L.off_a + row * L.astride + 16 * off,
+                           p.prep + (size_t)row * K + 16 * off);
+        }
+        tc::cp_async_wait_all();
+        __syncthreads();
+    } else {
     // 2-3. activation preparation
     constexpr int G = F::kGroup;
     const int ngroups = K / G;
@@ -255,6 +272,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     }
     __syncthreads();
 
+    }
+
     const bool w_ok = __syncthreads_and(tc::mbar_wait(bar, 0, p.flags, kWaitLimitNs));
     if (!w_ok) return;
 
@@ -342,13 +361,19 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     if (FORM == 0) {
         for (int o = threadIdx.x; o < M * 16; o += kThreads) {
             const int m = o >> 4, r = o & 15;
-            float amax = 0.f;
+            float sc;
             int qs = 0;
-            for (int w = 0; w < kWarps; ++w) {
-                amax = fmaxf(amax, red_max[w * kMaxTok + m]);
-                qs += red_sum[w * kMaxTok + m];
+            if (PREP) {
+                sc = p.pscale[m];
+                qs = p.prsum[m];
+            } else {
+                float amax = 0.f;
+                for (int w = 0; w < kWarps; ++w) {
+                    amax = fmaxf(amax, red_max[w * kMaxTok + m]);
+                    qs += red_sum[w * kMaxTok + m];
+                }
+                sc = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
             }
-            const float sc = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
             const int accv = part(m, r) - qs;
             const int n = rg * 16 + r;
             const float v = __fmul_rn(__fmul_rn((float)accv, sc), p.w_scale);
@@ -358,13 +383,19 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     } else {
         for (int o = threadIdx.x; o < M * 16; o += kThreads) {
             const int m = o >> 4, r = o & 15;
-            float amax = 0.f;
+            float st;
             long long ts = 0;
-            for (int w = 0; w < kWarps; ++w) {
-                amax = fmaxf(amax, red_max[w * kMaxTok + m]);
-                ts += red_sum[w * kMaxTok + m];
+            if (PREP) {
+                st = p.pscale[m];
+                ts = p.prsum[m];
+            } else {
+                float amax = 0.f;
+                for (int w = 0; w < kWarps; ++w) {
+                    amax = fmaxf(amax, red_max[w * kMaxTok + m]);
+                    ts += red_sum[w * kMaxTok + m];
+                }
+                st = amax > 0.f ? __fdiv_rn(amax, 32639.0f) : 0.f;
             }
-            const float st = amax > 0.f ? __fdiv_rn(amax, 32639.0f) : 0.f;
             const long long P = 256ll * part(2 * m, r) + part(2 * m + 1, r);
             const int n = rg * 16 + r;
             const float z = __fmul_rn(st, (float)(2 * P - ts));
@@ -374,12 +405,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     }
 }
 
-template <int FORM, int NT>
+template <int FORM, int NT, int PREP>
 cudaError_t launch_decode(const DecodeParams& p, int smem, cudaStream_t s) {
     static_assert(NT >= 1, "");
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<FORM, NT>,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<FORM, NT, PREP>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kDecodeMaxSmem);
         if (e != cudaSuccess) return e;
@@ -395,7 +426,7 @@ cudaError_t launch_decode(const DecodeParams& p, int smem, cudaStream_t s) {
     attrs[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<FORM, NT>, p);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<FORM, NT, PREP>, p);
 }
 
 template <int FORM>
@@ -420,14 +451,14 @@ int decode_stage_x(int M, int K) {
     return (s > 0 && s <= kDecodeMaxSmem) ? 1 : 0;
 }
 
-template <int FORM>
+template <int FORM, int PREP>
 cudaError_t launch_decode_form(DecodeParams p, cudaStream_t s) {
-    p.stage_x = decode_stage_x<FORM>(p.M, p.K);
+    p.stage_x = PREP ? 0 : decode_stage_x<FORM>(p.M, p.K);
     const int smem = decode_smem<FORM>(p.M, p.K, p.stage_x);
     switch (pick_nt<FORM>(p.M)) {
-        case 1: return launch_decode<FORM, 1>(p, smem, s);
-        case 2: return launch_decode<FORM, 2>(p, smem, s);
-        default: return launch_decode<FORM, 4>(p, smem, s);
+        case 1: return launch_decode<FORM, 1, PREP>(p, smem, s);
+        case 2: return launch_decode<FORM, 2, PREP>(p, smem, s);
+        default: return launch_decode<FORM, 4, PREP>(p, smem, s);
     }
 }
 
@@ -442,15 +473,39 @@ bool decode_fused_fits(int form, int M, int K) {
 cudaError_t launch_ternary_decode(const uint16_t* x, const uint32_t* w2, int M, int K, int N,
                                   float w_scale, uint16_t* y, int32_t* acc_out,
                                   unsigned int* flags, cudaStream_t s) {
-    DecodeParams p{0, x, nullptr, nullptr, w2, w_scale, M, K, N, y, acc_out, flags};
-    return launch_decode_form<0>(p, s);
+    DecodeParams p{0, nullptr, nullptr, nullptr, x, nullptr, nullptr, w2, w_scale, M, K, N, y,
+                   acc_out, flags};
+    return launch_decode_form<0, 0>(p, s);
 }
 
 cudaError_t launch_onebit_decode(const uint16_t* x, const uint16_t* g, const uint16_t* h,
                                  const uint32_t* s1, int M, int K, int N, uint16_t* y,
                                  unsigned int* flags, cudaStream_t s) {
-    DecodeParams p{0, x, g, h, s1, 0.f, M, K, N, y, nullptr, flags};
-    return launch_decode_form<1>(p, s);
+    DecodeParams p{0, nullptr, nullptr, nullptr, x, g, h, s1, 0.f, M, K, N, y, nullptr, flags};
+    return launch_decode_form<1, 0>(p, s);
+}
+
+cudaError_t launch_ternary_decode_prepared(const int8_t* qp, const float* scale, const int32_t* qsum,
+                                           const uint32_t* w2, int M, int K, int N, float w_scale,
+                                           uint16_t* y, int32_t* acc_out, unsigned int* flags,
+                                           cudaStream_t s) {
+    DecodeParams p{0, qp, scale, qsum, nullptr, nullptr, nullptr, w2, w_scale, M, K, N, y,
+                   acc_out, flags};
+    return launch_decode_form<0, 1>(p, s);
+}
+
+cudaError_t launch_onebit_decode_prepared(const int8_t* planes, const float* step,
+                                          const int32_t* tsum, const uint16_t* h,
+                                          const uint32_t* s1, int M, int K, int N, uint16_t* y,
+                                          unsigned int* flags, cudaStream_t s) {
+    DecodeParams p{0, planes, step, tsum, nullptr, nullptr, h, s1, 0.f, M, K, N, y, nullptr, flags};
+    return launch_decode_form<1, 1>(p, s);
+}
+
+bool decode_prepared_fits(int form, int M, int K) {
+    if (M < 1 || M > kMaxTok) return false;
+    const int smem = form == 0 ? decode_smem<0>(M, K, 0) : decode_smem<1>(M, K, 0);
+    return smem > 0 && smem <= kDecodeMaxSmem;
 }
 
 }  // namespace bl

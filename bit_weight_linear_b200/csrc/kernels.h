@@ -47,10 +47,13 @@ cudaError_t launch_onebit_prefill(const uint32_t* s1, const int8_t* planes, cons
                                   uint16_t* y, unsigned int* flags, cudaStream_t s);
 
 // Fused decode (decode.cu): activation preparation + contraction in one kernel,
-// 8-CTA clusters, weights bulk-copied to shared memory before the
-// programmatic-dependent-launch wait.  Used when M <= 32 columns of MMA fit and
-// the CTA's shared memory (16 weight rows + the prepared activations) fits.
+// weights bulk-copied to shared memory before the programmatic-dependent-launch
+// wait.  Used for M <= 8 (ternary) / 4 (OneBit) when a CTA's shared memory
+// (weight rows + the prepared activations) stays within kDecodeSmemTarget.
 constexpr int kDecodeMaxSmem = 227 * 1024;
+// Shared-memory budget per decode CTA: small enough that two CTAs of a layer
+// (and the next layer's, launched early) share an SM.
+constexpr int kDecodeSmemTarget = 100 * 1024;
 bool decode_fused_fits(int form, int M, int K);
 cudaError_t launch_ternary_decode(const uint16_t* x, const uint32_t* w2, int M, int K, int N,
                                   float w_scale, uint16_t* y, int32_t* acc_out,
@@ -61,6 +64,22 @@ cudaError_t launch_onebit_decode(const uint16_t* x, const uint16_t* g, const uin
 
 // Device address of the condition word bounded waits mark (nullptr on error).
 unsigned int* device_flags_address();
+
+// The same decode kernel on activations prepared by launch_quant_ternary_perm /
+// launch_prep_onebit (launched just before; both kernels use programmatic
+// dependent launch).  Used for small M > kFusedMaxM, where preparing the
+// activations once beats preparing them in every CTA.
+cudaError_t launch_ternary_decode_prepared(const int8_t* qp, const float* scale, const int32_t* qsum,
+                                           const uint32_t* w2, int M, int K, int N, float w_scale,
+                                           uint16_t* y, int32_t* acc_out, unsigned int* flags,
+                                           cudaStream_t s);
+cudaError_t launch_onebit_decode_prepared(const int8_t* planes, const float* step,
+                                          const int32_t* tsum, const uint16_t* h,
+                                          const uint32_t* s1, int M, int K, int N, uint16_t* y,
+                                          unsigned int* flags, cudaStream_t s);
+bool decode_prepared_fits(int form, int M, int K);
+// Largest M for which the decode kernel prepares the activations itself.
+constexpr int kFusedMaxM = 2;
 
 // Token counts at or above which the tensor-core prefill kernel is used.
 constexpr int kTernaryPrefillMinM = 33;

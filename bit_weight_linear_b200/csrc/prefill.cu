@@ -18,8 +18,9 @@
 // (B operand, TMA-loaded, 128-byte swizzle) come from shared memory.  That
 // keeps shared-memory traffic per MMA at the activation tile alone.
 //
-// CTA tile: 128 weight rows (MMA M, TMEM lanes) x 256 activation rows (MMA N:
-// tokens, or token limb rows), K in 128-byte stages; tiles ordered
+// CTA tile: 128 weight rows (MMA M, TMEM lanes) x bt activation rows (MMA N:
+// tokens, or token limb rows; bt = the smallest multiple of 32 covering them,
+// at most 256), K in 128-byte stages; tiles ordered
 // activation-tile-fastest so CTAs sharing a weight tile run together.
 // Warp roles (192 threads):
 //   warp 0     TMA producer: activation tile (256 x 128 B) and packed weight tile
@@ -44,7 +45,7 @@ namespace bl {
 namespace {
 
 constexpr int BW = 128;          // weight rows per tile (MMA M)
-constexpr int BT = 256;          // activation rows per tile (MMA N)
+constexpr int BT = 256;          // max activation rows per tile (MMA N); per call bt <= BT
 constexpr int BK = 128;          // k per stage (bytes of int8 per activation row)
 constexpr int SS = 5;            // shared-memory ring stages
 constexpr int SU = 4;            // TMEM slots for expanded weights
@@ -74,6 +75,7 @@ struct PF<1> {  // sign
 
 struct PrefillParams {
     int rows_a;        // activation rows: M (ternary) or 2M (OneBit limb rows)
+    int bt;            // activation rows per tile: multiple of 32, <= BT
     int M, K, N;
     const float* scale;   // per token: ternary scale / OneBit fixed-point step
     const int32_t* rsum;  // per token: sum q / sum X
@@ -100,11 +102,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * (2 * SS + 2 * SU + 1));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ttiles = (p.rows_a + BT - 1) / BT;
-    const int t0 = (blockIdx.x % ttiles) * BT;   // first activation row of the tile
+    const int bt = p.bt;
+    const int ttiles = (p.rows_a + bt - 1) / bt;
+    const int t0 = (blockIdx.x % ttiles) * bt;   // first activation row of the tile
     const int n0 = (blockIdx.x / ttiles) * BW;   // first weight row of the tile
     const int nk = p.K / BK;
-    constexpr uint32_t kTx = ACT_STAGE + PF<FORM>::kPackedRowBytes * BW;
+    const uint32_t kTx = (uint32_t)(bt * BK + PF<FORM>::kPackedRowBytes * BW);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SS; ++s) {
@@ -153,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = tc::idesc_i8(BW, BT);
+            const uint32_t idesc = tc::idesc_i8(BW, bt);
             bool ok = true;
             for (int kb = 0; kb < nk && ok; ++kb) {
                 const int s = kb % SS, u = kb % SU;
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* tok_scale = reinterpret_cast<float*>(smem + OFF_TOK);
         int* tok_rsum = reinterpret_cast<int*>(tok_scale + BT);
         const int et = threadIdx.x - 64;        // 0..127
-        for (int i = et; i < BT; i += 128) {
+        for (int i = et; i < bt; i += 128) {
             const int row = t0 + i;
             const int tok = FORM == 0 ? row : row >> 1;
             const bool in = FORM == 0 ? row < p.M : tok < p.M;
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && acc_ok) {
             const float hn = (FORM == 1 && n < p.N) ? __half2float(__ushort_as_half(p.h[n])) : 0.f;
 #pragma unroll 1
-            for (int cc = 0; cc < BT / 32; ++cc) {
+            for (int cc = 0; cc < bt / 32; ++cc) {
                 uint32_t d[32];
                 tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * cc, d);
                 tc::tmem_ld_wait();
@@ -298,9 +301,17 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
     return r == CUDA_SUCCESS;
 }
 
+// Activation rows per tile: the smallest multiple of 32 that covers them, at most
+// BT (a tile never computes more than 31 padding columns when rows_a <= BT).
+inline int choose_bt(int rows_a) {
+    const int r = (rows_a + 31) / 32 * 32;
+    return r < BT ? r : BT;
+}
+
 template <int FORM>
-cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, const PrefillParams& p,
+cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, PrefillParams p,
                            cudaStream_t s) {
+    p.bt = choose_bt(p.rows_a);
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(prefill_kernel<FORM>,
@@ -310,14 +321,14 @@ cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, const PrefillPa
         attr_set = true;
     }
     CUtensorMap ta, tw;
-    if (!make_tmap(&ta, act, (uint64_t)p.rows_a, (uint64_t)p.K, BK, BT,
+    if (!make_tmap(&ta, act, (uint64_t)p.rows_a, (uint64_t)p.K, BK, (uint32_t)p.bt,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     const uint64_t prow = (uint64_t)p.K / (FORM == 0 ? 4 : 8);
     if (!make_tmap(&tw, w, (uint64_t)p.N, prow, PF<FORM>::kPackedRowBytes, BW,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    const int tiles = ((p.N + BW - 1) / BW) * ((p.rows_a + BT - 1) / BT);
+    const int tiles = ((p.N + BW - 1) / BW) * ((p.rows_a + p.bt - 1) / p.bt);
     prefill_kernel<FORM><<<tiles, kThreads, SMEM_BYTES, s>>>(ta, tw, p);
     return cudaGetLastError();
 }
@@ -329,7 +340,7 @@ cudaError_t launch_ternary_prefill(const uint32_t* w2, const int8_t* qp, const f
                                    uint16_t* y, int32_t* acc_out, unsigned int* flags,
                                    cudaStream_t s) {
     if (M == 0 || N == 0) return cudaSuccess;
-    PrefillParams p{M, M, K, N, scale, qsum, nullptr, w_scale, y, acc_out, flags};
+    PrefillParams p{M, 0, M, K, N, scale, qsum, nullptr, w_scale, y, acc_out, flags};
     return launch_prefill<0>(qp, w2, p, s);
 }
 
@@ -337,7 +348,7 @@ cudaError_t launch_onebit_prefill(const uint32_t* s1, const int8_t* planes, cons
                                   const int32_t* tsum, const uint16_t* h, int M, int K, int N,
                                   uint16_t* y, unsigned int* flags, cudaStream_t s) {
     if (M == 0 || N == 0) return cudaSuccess;
-    PrefillParams p{2 * M, M, K, N, step, tsum, h, 0.f, y, nullptr, flags};
+    PrefillParams p{2 * M, 0, M, K, N, step, tsum, h, 0.f, y, nullptr, flags};
     return launch_prefill<1>(planes, s1, p, s);
 }
 

@@ -17,6 +17,7 @@
 // HBM-bound: the plain/ternary kernels read 2 B and write 1 B per element.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_prims.cuh"
 
 namespace bl {
 
@@ -71,11 +72,15 @@ __global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t* __r
     __shared__ int redi[kWarps];
     const int m = blockIdx.x;
     const uint16_t* row = x + (size_t)m * K;
+    // programmatic dependent launch: let the consumer start streaming its
+    // weights, and read x / write the outputs only after the producer of x is done
+    tc::pdl_trigger();
+    tc::pdl_wait();
 
     // pass 1: amax as the max of |x| bit patterns (monotone for finite halves)
     uint32_t mx = 0;
     for (int c = threadIdx.x; c < K / 8; c += kThreads) {
-        uint4 v = ld_ro_v4(row + 8 * c);
+        uint4 v = tc::ld_v4(row + 8 * c);
         mx = __vmaxu2(mx, v.x & 0x7fff7fffu);
         mx = __vmaxu2(mx, v.y & 0x7fff7fffu);
         mx = __vmaxu2(mx, v.z & 0x7fff7fffu);
@@ -89,8 +94,8 @@ __global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t* __r
     int sum = 0;
     int8_t* qrow = q + (size_t)m * K;
     for (int c = threadIdx.x; c < K / 16; c += kThreads) {
-        uint4 a = ld_ro_v4(row + 16 * c);
-        uint4 b = ld_ro_v4(row + 16 * c + 8);
+        uint4 a = tc::ld_v4(row + 16 * c);
+        uint4 b = tc::ld_v4(row + 16 * c + 8);
         uint32_t hv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
         int qv[16];
 #pragma unroll
@@ -129,10 +134,12 @@ __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* _
     __shared__ int redi[kWarps];
     const int m = blockIdx.x;
     const uint16_t* row = x + (size_t)m * K;
+    tc::pdl_trigger();
+    tc::pdl_wait();
 
     float mx = 0.f;
     for (int c = threadIdx.x; c < K / 8; c += kThreads) {
-        uint4 v = ld_ro_v4(row + 8 * c);
+        uint4 v = tc::ld_v4(row + 8 * c);
         uint4 gv = ld_ro_v4(g + 8 * c);
         uint32_t xs[4] = {v.x, v.y, v.z, v.w}, gs[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
@@ -152,7 +159,7 @@ __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* _
         int hv[32], lv[32];
 #pragma unroll
         for (int part = 0; part < 4; ++part) {
-            uint4 v = ld_ro_v4(row + 32 * c + 8 * part);
+            uint4 v = tc::ld_v4(row + 32 * c + 8 * part);
             uint4 gv = ld_ro_v4(g + 32 * c + 8 * part);
             uint32_t xs[4] = {v.x, v.y, v.z, v.w}, gs[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
@@ -195,27 +202,38 @@ __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* _
     }
 }
 
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kern, int blocks, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attrs[1];
+    attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 }  // namespace
 
 cudaError_t launch_quant_plain(const uint16_t* x, int M, int K, int8_t* q, float* scale,
                                cudaStream_t s) {
     if (M == 0) return cudaSuccess;
-    quant_act_kernel<0><<<M, kThreads, 0, s>>>(x, K, q, scale, nullptr);
-    return cudaGetLastError();
+    return launch_pdl(quant_act_kernel<0>, M, s, x, K, q, scale, (int32_t*)nullptr);
 }
 
 cudaError_t launch_quant_ternary_perm(const uint16_t* x, int M, int K, int8_t* qp,
                                       float* scale, int32_t* qsum, cudaStream_t s) {
     if (M == 0) return cudaSuccess;
-    quant_act_kernel<1><<<M, kThreads, 0, s>>>(x, K, qp, scale, qsum);
-    return cudaGetLastError();
+    return launch_pdl(quant_act_kernel<1>, M, s, x, K, qp, scale, qsum);
 }
 
 cudaError_t launch_prep_onebit(const uint16_t* x, const uint16_t* g, int M, int K,
                                int8_t* planes, float* step, int32_t* tsum, cudaStream_t s) {
     if (M == 0) return cudaSuccess;
-    prep_onebit_kernel<<<M, kThreads, 0, s>>>(x, g, K, planes, step, tsum);
-    return cudaGetLastError();
+    return launch_pdl(prep_onebit_kernel, M, s, x, g, K, planes, step, tsum);
 }
 
 }  // namespace bl

@@ -214,7 +214,9 @@ __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 }
 
-// Coherent 16-byte global load (data written by the preceding grid).
+// Coherent (weak, default-cached) 16-byte global load, for data written by the
+// preceding grid and read after griddepcontrol.wait, which makes that grid's
+// writes visible.  Several CTAs on an SM reading the same x share L1 lines.
 __device__ __forceinline__ uint4 ld_v4(const void* p) {
     uint4 v;
     asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
