@@ -298,15 +298,18 @@ def run_prefill(blw, synth, dev, args, dist_on, world, peaks):
                      "peak_source": "2 x measured sustained bf16 (nominal int8/bf16 ratio)"}}
 
 
-def run_sweep(blw, synth, dev, peaks, reps=10):
-    """Batch sweep on the LLaMA-13B-shaped layers, both forms: per (form, shape, M)
-    the effective weight GB/s and int8 TOPS of one call, over rotating weight
-    copies that total more than twice the L2 (each call streams its weights)."""
+def run_sweep(blw, synth, dev, peaks, reps=10, forms=("ternary", "onebit"), layers=None,
+              ms_list=None):
+    """Per (form, layer, M): the effective weight GB/s and int8 TOPS of one call,
+    over rotating weight copies that total more than twice the L2 (each call
+    streams its weights from HBM).  Defaults: the LLaMA-13B-shaped batch sweep."""
     l2_bytes = 126 * 2 ** 20
     i8_peak = 2.0 * peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    layers = layers or LLAMA13B_SWEEP
+    ms_list = ms_list or SWEEP_M
     out = []
-    for form in ("ternary", "onebit"):
-        for (name, K, N) in LLAMA13B_SWEEP:
+    for form in forms:
+        for (name, K, N) in layers:
             wb = N * K // (4 if form == "ternary" else 8)
             copies = max(2, -(-2 * l2_bytes // wb) + 1)
             ws, gs, hs = [], None, None
@@ -322,7 +325,7 @@ def run_sweep(blw, synth, dev, peaks, reps=10):
             if form == "onebit":
                 gs = synth.value_vector(K, seed=4_000_900, device=dev)
                 hs = synth.value_vector(N, seed=4_000_901, device=dev)
-            for M in SWEEP_M:
+            for M in ms_list:
                 x = synth.activations(M, K, seed=4_001_000 + M, device=dev)
                 y = torch.empty((M, N), dtype=torch.float16, device=dev)
                 nws = (blw.bl_ternary_workspace_bytes if form == "ternary" else blw.ob_workspace_bytes)(M, K, N)
@@ -503,6 +506,11 @@ def main():
         torch.cuda.empty_cache()
 
         extras["prefill"] = run_prefill(blw, synth, dev, args, dist_on, world, peaks)
+        # the two small configurations: BitLinear M=8 and OneBit M=1 / M=16 on 4096x4096
+        extras["bitlinear_m8_4096"] = run_sweep(blw, synth, dev, peaks, forms=("ternary",),
+                                                layers=[("q", 4096, 4096)], ms_list=[8])
+        extras["onebit_4096"] = run_sweep(blw, synth, dev, peaks, forms=("onebit",),
+                                          layers=[("q", 4096, 4096)], ms_list=[1, 16])
         if not args.no_sweep:
             extras["batch_sweep_13b"] = run_sweep(blw, synth, dev, peaks)
 
