@@ -157,6 +157,9 @@ bl_status bl_ternary_linear(const uint16_t* x, int M, int K, int N, const uint32
     if (misaligned(workspace)) return BL_ERR_ALIGN;
     unsigned int* flags = device_flags();
     if (!flags) return BL_ERR_CUDA;
+    if (M <= bl::kFusedMaxM && bl::stream_fits(0, M, K, N, 0))
+        return from_cuda(
+            bl::launch_ternary_stream(x, w2, M, K, N, w_scale, y, acc_out, flags, cs(stream)));
     if (M <= bl::kFusedMaxM && bl::decode_fused_fits(0, M, K))
         return from_cuda(
             bl::launch_ternary_decode(x, w2, M, K, N, w_scale, y, acc_out, flags, cs(stream)));
@@ -170,7 +173,10 @@ bl_status bl_ternary_linear(const uint16_t* x, int M, int K, int N, const uint32
         e = bl::launch_ternary_prefill(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, flags,
                                        cs(stream));
     } else {
-        e = bl::decode_prepared_fits(0, M, K)
+        e = bl::stream_fits(0, M, K, N, 1)
+                ? bl::launch_ternary_stream_prepared(qp, sc, qs, w2, M, K, N, w_scale, y, acc_out,
+                                                     flags, cs(stream))
+            : bl::decode_prepared_fits(0, M, K)
                 ? bl::launch_ternary_decode_prepared(qp, sc, qs, w2, M, K, N, w_scale, y, acc_out,
                                                      flags, cs(stream))
                 : bl::launch_ternary_skinny(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, cs(stream));
@@ -199,6 +205,8 @@ bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
     if (misaligned(workspace)) return BL_ERR_ALIGN;
     unsigned int* flags = device_flags();
     if (!flags) return BL_ERR_CUDA;
+    if (M <= bl::kFusedMaxM && bl::stream_fits(1, M, K, N, 0))
+        return from_cuda(bl::launch_onebit_stream(x, g, h, s1, M, K, N, y, flags, cs(stream)));
     if (M <= bl::kFusedMaxM && bl::decode_fused_fits(1, M, K))
         return from_cuda(bl::launch_onebit_decode(x, g, h, s1, M, K, N, y, flags, cs(stream)));
     char* ws = static_cast<char*>(workspace);
@@ -210,7 +218,10 @@ bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
     if (M >= bl::kOnebitPrefillMinM) {
         e = bl::launch_onebit_prefill(s1, planes, step, ts, h, M, K, N, y, flags, cs(stream));
     } else {
-        e = bl::decode_prepared_fits(1, M, K)
+        e = bl::stream_fits(1, M, K, N, 1)
+                ? bl::launch_onebit_stream_prepared(planes, step, ts, h, s1, M, K, N, y, flags,
+                                                    cs(stream))
+            : bl::decode_prepared_fits(1, M, K)
                 ? bl::launch_onebit_decode_prepared(planes, step, ts, h, s1, M, K, N, y, flags,
                                                     cs(stream))
                 : bl::launch_onebit_skinny(s1, planes, step, ts, h, M, K, N, y, cs(stream));

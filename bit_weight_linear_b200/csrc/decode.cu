@@ -25,6 +25,7 @@
 // Weight rows in shared memory are padded to a stride of 64 (mod 128) bytes so
 // that every quarter-warp's 16-byte loads hit 8 distinct bank groups.
 #include "common.cuh"
+#include "decode_forms.cuh"
 #include "kernels.h"
 #include "tc_prims.cuh"
 
@@ -36,21 +37,6 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxTok = 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-
-template <int FORM>
-struct DF;
-template <>
-struct DF<0> {
-    static constexpr int kPerWord = 16, kRegs = 4, kShift = 2, kStepK = 256, kChunkK = 64;
-    static constexpr int kCPT = 1, kGroup = 16;
-    static constexpr uint32_t kMask = 0x03030303u;
-};
-template <>
-struct DF<1> {
-    static constexpr int kPerWord = 32, kRegs = 8, kShift = 1, kStepK = 512, kChunkK = 128;
-    static constexpr int kCPT = 2, kGroup = 32;
-    static constexpr uint32_t kMask = 0x01010101u;
-};
 
 struct DecodeParams {
     int stage_x;            // 1: x (and g) are staged in shared memory between the two passes
@@ -96,17 +82,6 @@ __host__ __device__ inline DecodeLayout decode_layout(int M, int K, int stage_x)
 // else (coherently) from global memory.
 __device__ __forceinline__ uint4 ld_act(const uint16_t* p, int staged) {
     return staged ? *reinterpret_cast<const uint4*>(p) : tc::ld_v4(p);
-}
-
-// low bytes of a, b, c, d -> one word (a in the lowest byte)
-__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-    const uint32_t lo = __byte_perm((uint32_t)a, (uint32_t)b, 0x0040);
-    const uint32_t hi = __byte_perm((uint32_t)c, (uint32_t)d, 0x0040);
-    return __byte_perm(lo, hi, 0x5410);
-}
-
-__device__ __forceinline__ float hbits(uint32_t v) {
-    return __half2float(__ushort_as_half((unsigned short)(v & 0xffffu)));
 }
 
 // PREP = 0: the kernel prepares the activations from x itself (decode sizes).
@@ -413,6 +388,8 @@ cudaError_t launch_decode(const DecodeParams& p, int smem, cudaStream_t s) {
         cudaError_t e = cudaFuncSetAttribute(decode_kernel<FORM, NT, PREP>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kDecodeMaxSmem);
+        if (e != cudaSuccess) return e;
+        e = use_max_shared_carveout(decode_kernel<FORM, NT, PREP>);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }

@@ -46,14 +46,11 @@ cudaError_t launch_onebit_prefill(const uint32_t* s1, const int8_t* planes, cons
                                   const int32_t* tsum, const uint16_t* h, int M, int K, int N,
                                   uint16_t* y, unsigned int* flags, cudaStream_t s);
 
-// Fused decode (decode.cu): activation preparation + contraction in one kernel,
-// weights bulk-copied to shared memory before the programmatic-dependent-launch
-// wait.  Used for M <= 8 (ternary) / 4 (OneBit) when a CTA's shared memory
-// (weight rows + the prepared activations) stays within kDecodeSmemTarget.
+// Per-16-row decode (decode.cu): activation preparation + contraction in one
+// kernel, one CTA per 16 weight rows, weights bulk-copied to shared memory
+// before the programmatic-dependent-launch wait.  The fallback for shapes the
+// streamed decode kernel (stream.cu) has no plan for.
 constexpr int kDecodeMaxSmem = 227 * 1024;
-// Shared-memory budget per decode CTA: small enough that two CTAs of a layer
-// (and the next layer's, launched early) share an SM.
-constexpr int kDecodeSmemTarget = 100 * 1024;
 bool decode_fused_fits(int form, int M, int K);
 cudaError_t launch_ternary_decode(const uint16_t* x, const uint32_t* w2, int M, int K, int N,
                                   float w_scale, uint16_t* y, int32_t* acc_out,
@@ -78,6 +75,38 @@ cudaError_t launch_onebit_decode_prepared(const int8_t* planes, const float* ste
                                           const uint32_t* s1, int M, int K, int N, uint16_t* y,
                                           unsigned int* flags, cudaStream_t s);
 bool decode_prepared_fits(int form, int M, int K);
+// Streamed decode (stream.cu): at most one 512-thread CTA per SM, each owning a
+// contiguous range of 16-row tiles streamed through a shared-memory ring that
+// is filled before the programmatic-dependent-launch wait.  prep = 0: the CTA
+// prepares the activations from x; prep = 1: they come from the activation
+// kernel.  stream_fits tells whether the shape has a plan.
+bool stream_fits(int form, int M, int K, int N, int prep);
+cudaError_t launch_ternary_stream(const uint16_t* x, const uint32_t* w2, int M, int K, int N,
+                                  float w_scale, uint16_t* y, int32_t* acc_out, unsigned int* flags,
+                                  cudaStream_t s);
+cudaError_t launch_onebit_stream(const uint16_t* x, const uint16_t* g, const uint16_t* h,
+                                 const uint32_t* s1, int M, int K, int N, uint16_t* y,
+                                 unsigned int* flags, cudaStream_t s);
+cudaError_t launch_ternary_stream_prepared(const int8_t* qp, const float* scale, const int32_t* qsum,
+                                           const uint32_t* w2, int M, int K, int N, float w_scale,
+                                           uint16_t* y, int32_t* acc_out, unsigned int* flags,
+                                           cudaStream_t s);
+cudaError_t launch_onebit_stream_prepared(const int8_t* planes, const float* step,
+                                          const int32_t* tsum, const uint16_t* h,
+                                          const uint32_t* s1, int M, int K, int N, uint16_t* y,
+                                          unsigned int* flags, cudaStream_t s);
+
+// Every kernel of the library runs with the whole L1/shared-memory carveout
+// given to shared memory.  An SM changes its carveout only when it is idle, so
+// kernels with differing carveouts could not share an SM: the next call's CTAs
+// (launched early, programmatic dependent launch) would then wait for SMs to
+// drain and pile up two to an SM.
+template <typename Kern>
+inline cudaError_t use_max_shared_carveout(Kern kern) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                (int)cudaSharedmemCarveoutMaxShared);
+}
+
 // Largest M for which the decode kernel prepares the activations itself.
 constexpr int kFusedMaxM = 2;
 

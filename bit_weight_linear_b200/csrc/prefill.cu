@@ -33,12 +33,10 @@
 // is the order the byte-SIMD unpack produces; the activation preparation
 // kernels store the activations in the same order.
 // Every mbarrier wait is bounded (a timeout sets the device condition word).
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_prims.cuh"
+#include "tmap.cuh"
 
 namespace bl {
 
@@ -273,32 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
 // 2-D uint8 tensor map: rows x cols bytes (row stride = cols), box box_cols x box_rows.
 bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                uint32_t box_rows, CUtensorMapSwizzle swz) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    return encode_u8_map(m, base, 2, dims, strides, box, swz);
 }
 
 // Activation rows per tile: the smallest multiple of 32 that covers them, at most
@@ -317,6 +296,8 @@ cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, PrefillParams p
         cudaError_t e = cudaFuncSetAttribute(prefill_kernel<FORM>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        e = use_max_shared_carveout(prefill_kernel<FORM>);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }

@@ -202,8 +202,14 @@ __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* _
     }
 }
 
-template <typename Kern, typename... Args>
-cudaError_t launch_pdl(Kern kern, int blocks, cudaStream_t s, Args... args) {
+template <auto KERN, typename... Args>
+cudaError_t launch_pdl(int blocks, cudaStream_t s, Args... args) {
+    static bool attr_set = false;  // one flag per kernel
+    if (!attr_set) {
+        cudaError_t e = use_max_shared_carveout(KERN);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(blocks);
     cfg.blockDim = dim3(kThreads);
@@ -213,7 +219,7 @@ cudaError_t launch_pdl(Kern kern, int blocks, cudaStream_t s, Args... args) {
     attrs[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, args...);
+    return cudaLaunchKernelEx(&cfg, KERN, args...);
 }
 
 }  // namespace
@@ -221,19 +227,19 @@ cudaError_t launch_pdl(Kern kern, int blocks, cudaStream_t s, Args... args) {
 cudaError_t launch_quant_plain(const uint16_t* x, int M, int K, int8_t* q, float* scale,
                                cudaStream_t s) {
     if (M == 0) return cudaSuccess;
-    return launch_pdl(quant_act_kernel<0>, M, s, x, K, q, scale, (int32_t*)nullptr);
+    return launch_pdl<quant_act_kernel<0>>(M, s, x, K, q, scale, (int32_t*)nullptr);
 }
 
 cudaError_t launch_quant_ternary_perm(const uint16_t* x, int M, int K, int8_t* qp,
                                       float* scale, int32_t* qsum, cudaStream_t s) {
     if (M == 0) return cudaSuccess;
-    return launch_pdl(quant_act_kernel<1>, M, s, x, K, qp, scale, qsum);
+    return launch_pdl<quant_act_kernel<1>>(M, s, x, K, qp, scale, qsum);
 }
 
 cudaError_t launch_prep_onebit(const uint16_t* x, const uint16_t* g, int M, int K,
                                int8_t* planes, float* step, int32_t* tsum, cudaStream_t s) {
     if (M == 0) return cudaSuccess;
-    return launch_pdl(prep_onebit_kernel, M, s, x, g, K, planes, step, tsum);
+    return launch_pdl<prep_onebit_kernel>(M, s, x, g, K, planes, step, tsum);
 }
 
 }  // namespace bl

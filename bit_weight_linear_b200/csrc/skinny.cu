@@ -194,6 +194,12 @@ template <int FORM, int NT>
 cudaError_t launch(const SkinnyParams& p, cudaStream_t s) {
     constexpr int kTokPerCta = NT * 8 / Form<FORM>::kColsPerToken;
     dim3 grid(p.N / 16, (p.M + kTokPerCta - 1) / kTokPerCta);
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = use_max_shared_carveout(skinny_kernel<FORM, NT>);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
     skinny_kernel<FORM, NT><<<grid, kThreads, 0, s>>>(p);
     return cudaGetLastError();
 }

@@ -1,0 +1,788 @@
+// stream.cu -- streamed decode-shaped (small M) forward of both layer forms:
+// one 512-thread CTA per SM owns a contiguous range of 16-row weight tiles and
+// streams them through a shared-memory ring.
+//
+// Arithmetic is that of the other decode kernels:
+//   BitLinear (BitNet b1.58 page, "BitNet b1.58 介绍"): per-token absmax int8
+//     q = rne(x * rn(127/amax)), acc = sum q*code - sum q, y = fp16((acc*s)*w_scale);
+//   OneBit (OneBit page, "1. 新的 1bit 结构"): 16-bit fixed-point image X of
+//     x*g in two int8 limbs, sum X*S = 2 sum X*b - sum X, y = fp16(step*Z*h).
+//
+// Why this shape on B200.  At M = 1 a call is a chain: wait for the previous
+// grid, read x, reduce its absmax, quantise, contract, write y.  The weights
+// do not depend on that chain, so they are read before it:
+//   * The grid has at most one CTA per SM, and a CTA fits twice per SM
+//     (512 threads x 64 registers, <= 112 KB shared memory), so the CTA of the
+//     NEXT call becomes resident beside the running one and streams its tiles
+//     while this call finishes (programmatic dependent launch).
+//   * At launch, one thread fills the ring: ONE 3-D TMA load per stage
+//     (16 rows x up to 32 k-steps, laid out [step][row][64 B], so the MMA
+//     fragment loads are bank-conflict free).  Large copies matter: per-row
+//     1 KB bulk copies stream at under half of HBM bandwidth per SM, 8 KB and
+//     larger ones at full rate.  x is prefetched into L2.  Only then does the
+//     CTA wait for the preceding grid.
+//   * x is quantised once per SM (not once per 16 rows), by all 16 warps.
+//   * Warps split each ring stage's 256-k (ternary) / 512-k (sign) steps and
+//     run the u8 x s8 warp MMA; the last warp to finish a stage refills its
+//     slot.  Per-tile partial sums meet in shared memory through integer
+//     atomics (exact in any order).
+#include "common.cuh"
+#include "decode_forms.cuh"
+#include "kernels.h"
+#include "tc_prims.cuh"
+#include "tmap.cuh"
+
+#include <mutex>
+
+namespace bl {
+
+namespace {
+
+constexpr int kSWarps = 16;
+constexpr int kSThreads = kSWarps * 32;
+constexpr int kMaxSlots = 16;
+constexpr int kMaxTokS = 32;
+constexpr uint64_t kSWaitLimitNs = 2000000000ull;
+constexpr uint64_t kSDrainLimitNs = 100000000ull;
+// two CTAs per SM: (228 KB - 2 x 1 KB reserved) / 2, rounded down
+constexpr int kStreamSmemPair = 112 * 1024;
+
+struct StreamParams {
+    const int8_t* prep;     // prepared activations [cols][K] (PREP kernels only)
+    const float* pscale;    // per token: scale (ternary) / fixed-point step (OneBit)
+    const int32_t* prsum;   // per token: row sum of the prepared activations
+    const uint16_t* x;
+    const uint16_t* g;      // OneBit input value vector
+    const uint16_t* h;      // OneBit output value vector
+    const uint32_t* w;      // packed weights
+    float w_scale;
+    int M, K, N;
+    uint16_t* y;
+    int32_t* acc_out;
+    unsigned int* flags;
+    // plan (host-computed)
+    int t_lo, t_rem, t_max;  // tiles per CTA: t_lo + (cta < t_rem)
+    int steps, nch, S;       // k-steps per row, ring stages per tile, ring slots
+    int nfull, bsteps;       // whole 64-byte steps per row; steps per stage (box depth)
+    int ragged;              // 1: the last step is partial: `tail` bytes per row (tail map)
+    int tail;                // 16, 32 or 48 bytes (sign); 32 (ternary)
+    int slot_bytes;
+    int off_act, astride, off_red, off_tok, off_h, off_bar, off_cnt;
+};
+
+// Quantise one 16-element ternary group (fp16 in a, b) into the permuted
+// activation tile; returns the group's sum of q.
+// |x * inv| <= 127 (1 + 2^-24) for inv = rn(127/amax), so the rounded value
+// never leaves [-127, 127] and no clamp is needed.
+__device__ __forceinline__ int quant_group_t(uint4 a, uint4 b, float inv, uint8_t* dst) {
+    const uint32_t hv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    int qv[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+        qv[e] = __float2int_rn(__fmul_rn(hbits(hv[e >> 1] >> (16 * (e & 1))), inv));
+    uint4 o;
+    o.x = pack4(qv[0], qv[4], qv[8], qv[12]);
+    o.y = pack4(qv[1], qv[5], qv[9], qv[13]);
+    o.z = pack4(qv[2], qv[6], qv[10], qv[14]);
+    o.w = pack4(qv[3], qv[7], qv[11], qv[15]);
+    *reinterpret_cast<uint4*>(dst) = o;
+    int sum = __dp4a((int)o.x, 0x01010101, 0);
+    sum = __dp4a((int)o.y, 0x01010101, sum);
+    sum = __dp4a((int)o.z, 0x01010101, sum);
+    return __dp4a((int)o.w, 0x01010101, sum);
+}
+
+__device__ __forceinline__ uint32_t absmax_bits_t(uint4 a) {
+    const uint32_t mb = __vmaxu2(__vmaxu2(a.x & 0x7fff7fffu, a.y & 0x7fff7fffu),
+                                 __vmaxu2(a.z & 0x7fff7fffu, a.w & 0x7fff7fffu));
+    return max(mb & 0xffffu, mb >> 16);
+}
+
+// max |x*g| over 8 elements (fp32 products, exact for fp16 inputs)
+__device__ __forceinline__ float absmax_prod(uint4 a, uint4 gg) {
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {gg.x, gg.y, gg.z, gg.w};
+    float mx = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+        mx = fmaxf(mx, fabsf(__fmul_rn(hbits(av[e >> 1] >> (16 * (e & 1))),
+                                       hbits(gv[e >> 1] >> (16 * (e & 1))))));
+    return mx;
+}
+
+// OneBit: one 32-element group of x*g -> X = rne(x*g*inv) in two int8 limbs,
+// hi = floor((X+128)/256), lo = X - 256 hi, written permuted into the two
+// limb rows; returns the group's sum of X.  |x*g*inv| <= 32639 (1 + 2^-24),
+// so no clamp is needed.
+__device__ __forceinline__ int quant_group_s(const uint4 (&xa)[4], const uint4 (&ga)[4], float inv,
+                                             uint8_t* dh, uint8_t* dl) {
+    uint32_t ho[8], lo[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ho[j] = lo[j] = 0;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        const uint32_t av[4] = {xa[v].x, xa[v].y, xa[v].z, xa[v].w};
+        const uint32_t gv[4] = {ga[v].x, ga[v].y, ga[v].z, ga[v].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float pr = __fmul_rn(hbits(av[e >> 1] >> (16 * (e & 1))),
+                                       hbits(gv[e >> 1] >> (16 * (e & 1))));
+            const int X = __float2int_rn(__fmul_rn(pr, inv));
+            const int hi = (X + 128) >> 8;
+            // element 8v+e goes to byte v of word e
+            ho[e] |= ((uint32_t)hi & 0xffu) << (8 * v);
+            lo[e] |= ((uint32_t)(X - 256 * hi) & 0xffu) << (8 * v);
+        }
+    }
+    int shi = 0, slo = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        shi = __dp4a((int)ho[j], 0x01010101, shi);
+        slo = __dp4a((int)lo[j], 0x01010101, slo);
+    }
+    uint4* h4 = reinterpret_cast<uint4*>(dh);
+    uint4* l4 = reinterpret_cast<uint4*>(dl);
+    h4[0] = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+    h4[1] = make_uint4(ho[4], ho[5], ho[6], ho[7]);
+    l4[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    l4[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+    return 256 * shi + slo;
+}
+
+// Steps [s0, s1) of chunk c of a tile: chunks of bsteps steps, the last one
+// shorter (its box runs past the row end and is zero-filled without reading).
+struct Chunk {
+    int s0, s1;
+};
+__host__ __device__ __forceinline__ Chunk chunk_of(int c, int steps, int bsteps) {
+    Chunk ch;
+    ch.s0 = c * bsteps;
+    ch.s1 = min(ch.s0 + bsteps, steps);
+    return ch;
+}
+
+// sum of one partial over the 16 warps' copies (warp stride `stride` ints)
+__device__ __forceinline__ int warp_rows_sum(const int* red, int idx, int stride) {
+    int v = 0;
+#pragma unroll
+    for (int w = 0; w < kSWarps; ++w) v += red[w * stride + idx];
+    return v;
+}
+
+// Ring stage u = (tile u / nch, chunk u % nch): one box of bsteps whole steps
+// ([step][row][64 B]) and, for the chunk holding a partial last step, the tail
+// box ([row][tail B]) behind it.  The caller arms the barrier with stage_bytes.
+__device__ __forceinline__ uint32_t stage_bytes(const StreamParams& p, int u) {
+    const Chunk ch = chunk_of(u % p.nch, p.steps, p.bsteps);
+    uint32_t b = ch.s0 < p.nfull ? (uint32_t)p.bsteps * 1024u : 0u;
+    if (p.ragged && ch.s1 == p.steps) b += 16u * (uint32_t)p.tail;
+    return b;
+}
+
+__device__ __forceinline__ void issue_stage(const StreamParams& p, const CUtensorMap* tm_main,
+                                            const CUtensorMap* tm_tail, uint32_t sb, int tile0,
+                                            int u) {
+    const int lt = u / p.nch;
+    const Chunk ch = chunk_of(u - lt * p.nch, p.steps, p.bsteps);
+    const int slot = u % p.S;
+    const uint32_t dst = sb + slot * p.slot_bytes;
+    const uint32_t bar = sb + p.off_bar + 8 * slot;
+    const int row0 = (tile0 + lt) * 16;
+    if (ch.s0 < p.nfull) tc::tma_load_3d(dst, tm_main, 0, row0, ch.s0, bar);
+    if (p.ragged && ch.s1 == p.steps) tc::tma_load_2d(dst + p.bsteps * 1024, tm_tail, 0, row0, bar);
+}
+
+// PREP = 0: the CTA prepares the activations from x (M <= a few tokens).
+//   XREG = 1 (M == 1 and few groups per thread): x stays in registers between
+//   the absmax and the quantisation pass.
+// PREP = 1: the activation kernel prepared them; they are copied in.
+template <int FORM, int NT, int PREP, int XREG>
+__global__ void __launch_bounds__(kSThreads, 2)
+    stream_kernel(const __grid_constant__ CUtensorMap tm_main,
+                  const __grid_constant__ CUtensorMap tm_tail, const StreamParams p) {
+    using F = DF<FORM>;
+    constexpr int CH = 4 / NT;  // independent accumulator chains per column tile
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int K = p.K, M = p.M;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t sb = tc::smem_u32(smem);
+    const int cta = blockIdx.x;
+    const int T = p.t_lo + (cta < p.t_rem ? 1 : 0);
+    const int tile0 = cta * p.t_lo + min(cta, p.t_rem);
+    const int nstages = T * p.nch;
+    const int S = p.S;
+    const int ncols = M * F::kCPT;
+    uint8_t* act = smem + p.off_act;
+    int* racc = reinterpret_cast<int*>(smem + p.off_red);             // [16 warps][t_max*16][ncols]
+    float* red_max = reinterpret_cast<float*>(smem + p.off_tok);      // [16][M]
+    int* red_sum = reinterpret_cast<int*>(red_max + kSWarps * M);     // [16][M]
+    uint16_t* hs = reinterpret_cast<uint16_t*>(smem + p.off_h);       // [t_max*16]
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + p.off_cnt);    // [S] releases, [S] rounds issued
+    const uint32_t cnt_sb = sb + p.off_cnt;
+
+    // 1. weights and parameters: independent of the preceding grid
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) tc::mbar_init(sb + p.off_bar + 8 * i, 1);
+        tc::mbar_fence_init();
+        if (p.nfull > 0) tc::prefetch_tmap(&tm_main);
+        if (p.ragged) tc::prefetch_tmap(&tm_tail);
+    }
+    for (int i = tid; i < 2 * S; i += kSThreads) cnt[i] = 0;
+    for (int i = tid; i < kSWarps * p.t_max * 16 * ncols; i += kSThreads) racc[i] = 0;
+    if (FORM == 1)
+        for (int i = tid; i < T * 16; i += kSThreads) hs[i] = p.h[tile0 * 16 + i];
+    // Warp-local activation preparation (XREG): warp w owns the k-steps
+    // s = w, w + 16, ... (the steps it contracts); lane l takes group l % 16 of
+    // its owned steps 2i + l / 16.  OneBit's g is a parameter, read before the wait.
+    constexpr int G = F::kGroup;
+    const int gi = lane & 15;
+    uint4 ga[4];
+    if (FORM == 1 && XREG) {
+        const int s_own = warp + 16 * (lane >> 4), k0 = s_own * F::kStepK + gi * G;
+        if (s_own < p.steps && k0 < K) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) ga[v] = ld_ro_v4(p.g + k0 + 8 * v);
+        }
+    }
+    __syncthreads();  // barriers initialised, counters and partial sums zeroed
+    tc::pdl_trigger();
+    if (tid == 0) {
+        const int nfill = min(S, nstages);
+        for (int u = 0; u < nfill; ++u) {
+            tc::mbar_arrive_expect_tx(sb + p.off_bar + 8 * u, stage_bytes(p, u));
+            issue_stage(p, &tm_main, &tm_tail, sb, tile0, u);
+        }
+    } else if (!PREP && cta == 0 && tid == 32) {
+        tc::bulk_prefetch_l2(p.x, (uint32_t)(2 * (size_t)M * K));
+    }
+    tc::pdl_wait();
+
+    // 2. activations
+    if (PREP) {
+        const int per_row = K / 16;
+        for (int c = tid; c < ncols * per_row; c += kSThreads) {
+            const int row = c / per_row, off = c - row * per_row;
+            tc::cp_async16(sb + p.off_act + row * p.astride + 16 * off,
+                           p.prep + (size_t)row * K + 16 * off);
+        }
+        tc::cp_async_wait_all();
+        __syncthreads();
+    } else if (XREG) {
+        // M == 1: x stays in registers; one CTA barrier (the absmax); each warp
+        // then quantises exactly the steps it contracts, so the contraction
+        // needs only the warp's own writes (__syncwarp, no CTA barrier)
+        constexpr int R = FORM == 0 ? 4 : 1;  // owned step pairs per lane
+        uint4 xa[R][G / 8];
+        bool has[R];
+        float mx = 0.f;
+        uint32_t mb = 0;
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int s_own = warp + 16 * (2 * i + (lane >> 4)), k0 = s_own * F::kStepK + gi * G;
+            has[i] = s_own < p.steps && k0 < K;
+            if (has[i]) {
+#pragma unroll
+                for (int v = 0; v < G / 8; ++v) xa[i][v] = tc::ld_v4(p.x + k0 + 8 * v);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            if (!has[i]) continue;
+            if constexpr (FORM == 0) {
+                mb = max(mb, max(absmax_bits_t(xa[i][0]), absmax_bits_t(xa[i][1])));
+            } else {
+#pragma unroll
+                for (int v = 0; v < G / 8; ++v) mx = fmaxf(mx, absmax_prod(xa[i][v], ga[v]));
+            }
+        }
+        if (FORM == 0) mx = hbits(mb);
+        mx = warp_max(mx);
+        if (lane == 0) red_max[warp] = mx;
+        __syncthreads();
+        float amax = 0.f;
+#pragma unroll
+        for (int w = 0; w < kSWarps; ++w) amax = fmaxf(amax, red_max[w]);
+        int sum = 0;
+        if constexpr (FORM == 0) {
+            const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                if (!has[i]) continue;
+                const int k0 = (warp + 16 * (2 * i + (lane >> 4))) * F::kStepK + gi * G;
+                sum += quant_group_t(xa[i][0], xa[i][1], inv, act + k0);
+            }
+        } else {
+            const float inv = amax > 0.f ? __fdiv_rn(32639.0f, amax) : 0.f;
+            if (has[0]) {
+                const int k0 = (warp + 16 * (lane >> 4)) * F::kStepK + gi * G;
+                sum = quant_group_s(xa[0], ga, inv, act + k0, act + p.astride + k0);
+            }
+        }
+        sum = warp_sum(sum);
+        if (lane == 0) red_sum[warp] = sum;
+        __syncwarp();
+    } else {
+        // general M: x is read twice (the second pass hits L1/L2)
+        constexpr int G = F::kGroup;
+        const int ngroups = K / G;
+        for (int m = 0; m < M; ++m) {
+            const uint16_t* xr = p.x + (size_t)m * K;
+            float mx = 0.f;
+            for (int i = tid; i < ngroups; i += kSThreads) {
+                if (FORM == 0) {
+                    const uint32_t mb = max(absmax_bits_t(tc::ld_v4(xr + 16 * i)),
+                                            absmax_bits_t(tc::ld_v4(xr + 16 * i + 8)));
+                    mx = fmaxf(mx, hbits(mb));
+                } else {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        mx = fmaxf(mx, absmax_prod(tc::ld_v4(xr + 32 * i + 8 * v),
+                                                   ld_ro_v4(p.g + 32 * i + 8 * v)));
+                }
+            }
+            mx = warp_max(mx);
+            if (lane == 0) red_max[warp * M + m] = mx;
+        }
+        __syncthreads();
+        for (int m = 0; m < M; ++m) {
+            const uint16_t* xr = p.x + (size_t)m * K;
+            float amax = 0.f;
+#pragma unroll
+            for (int w = 0; w < kSWarps; ++w) amax = fmaxf(amax, red_max[w * M + m]);
+            int sum = 0;
+            if (FORM == 0) {
+                const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+                for (int i = tid; i < ngroups; i += kSThreads)
+                    sum += quant_group_t(tc::ld_v4(xr + 16 * i), tc::ld_v4(xr + 16 * i + 8), inv,
+                                         act + m * p.astride + 16 * i);
+            } else {
+                const float inv = amax > 0.f ? __fdiv_rn(32639.0f, amax) : 0.f;
+                for (int i = tid; i < ngroups; i += kSThreads) {
+                    uint4 xa[4], gg[4];
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        xa[v] = tc::ld_v4(xr + 32 * i + 8 * v);
+                        gg[v] = ld_ro_v4(p.g + 32 * i + 8 * v);
+                    }
+                    sum += quant_group_s(xa, gg, inv, act + (2 * m) * p.astride + 32 * i,
+                                         act + (2 * m + 1) * p.astride + 32 * i);
+                }
+            }
+            sum = warp_sum(sum);
+            if (lane == 0) red_sum[warp * M + m] = sum;
+        }
+        __syncthreads();
+    }
+
+    // 3. contraction, one ring stage at a time (tile-major).  The warps split a
+    // stage's steps; a warp accumulates a tile in registers (CH independent
+    // chains) and adds it into its own rows of wred, which the epilogue sums
+    // over the 16 warps (no atomics).
+    const int g8 = lane >> 2, t = lane & 3;
+    const uint8_t* bsrc[NT];
+    bool bvalid[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int col = nt * 8 + g8;
+        bvalid[nt] = col < ncols;
+        bsrc[nt] = act + (bvalid[nt] ? col : 0) * p.astride + t * F::kChunkK;
+    }
+    int* wred_w = racc + warp * p.t_max * 16 * ncols;  // this warp's [t_max*16][ncols]
+    int acc[NT][CH][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int c = 0; c < CH; ++c) acc[nt][c][0] = acc[nt][c][1] = acc[nt][c][2] = acc[nt][c][3] = 0;
+    bool ok = true;
+    int slot = 0, phase = 0, chunk = 0, lt = 0;  // stage u = lt * nch + chunk, in slot u % S
+    for (int u = 0; u < nstages; ++u) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(sb + p.off_bar + 8 * slot, (uint32_t)phase,
+                                                   p.flags, kSWaitLimitNs));
+        if (!ok) break;
+        const int s0 = chunk * p.bsteps, s1 = min(s0 + p.bsteps, p.steps);
+        const uint8_t* slot_p = smem + slot * p.slot_bytes;
+        for (int s = s0 + warp; s < s1; s += kSWarps) {
+            // whole step: [step][row][64 B]; partial last step: tail box [row][tail B]
+            const bool part = s >= p.nfull;
+            const uint8_t* w0 = part ? slot_p + p.bsteps * 1024 + p.tail * g8 + 16 * t
+                                     : slot_p + (s - s0) * 1024 + 64 * g8 + 16 * t;
+            const int rs8 = part ? 8 * p.tail : 512;  // 8 rows further down
+            const bool lane_ok = s * F::kStepK + t * F::kChunkK < K;
+            uint4 a0 = make_uint4(0, 0, 0, 0), a1 = make_uint4(0, 0, 0, 0);
+            if (lane_ok) {
+                a0 = *reinterpret_cast<const uint4*>(w0);
+                a1 = *reinterpret_cast<const uint4*>(w0 + rs8);
+            }
+            const uint32_t r0[4] = {a0.x, a0.y, a0.z, a0.w};
+            const uint32_t r1[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+            for (int om = 0; om < 4; ++om) {
+                uint32_t u0r[F::kRegs], u1r[F::kRegs];
+#pragma unroll
+                for (int j = 0; j < F::kRegs; ++j) {
+                    u0r[j] = (r0[om] >> (F::kShift * j)) & F::kMask;
+                    u1r[j] = (r1[om] >> (F::kShift * j)) & F::kMask;
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    uint32_t b[F::kRegs];
+                    if (lane_ok && bvalid[nt]) {
+                        const uint8_t* src = bsrc[nt] + s * F::kStepK + om * (4 * F::kRegs);
+#pragma unroll
+                        for (int q = 0; q < F::kRegs / 4; ++q) {
+                            const uint4 bv = *reinterpret_cast<const uint4*>(src + 16 * q);
+                            b[4 * q + 0] = bv.x;
+                            b[4 * q + 1] = bv.y;
+                            b[4 * q + 2] = bv.z;
+                            b[4 * q + 3] = bv.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < F::kRegs; ++j) b[j] = 0;
+                    }
+#pragma unroll
+                    for (int j = 0; j < F::kRegs; j += 2)
+                        mma_u8s8_16832(acc[nt][om % CH], u0r[j], u1r[j], u0r[j + 1], u1r[j + 1],
+                                       b[j], b[j + 1]);
+                }
+            }
+        }
+        // release the slot (only when it is to be refilled); the warp that
+        // releases it last refills it
+        if (u + S < nstages) {
+            __syncwarp();
+            if (lane == 0) {
+                const uint32_t old = tc::atom_add_acq_rel_smem(cnt_sb + 4 * slot, 1u);
+                if ((old + 1) % kSWarps == 0) {
+                    tc::fence_proxy_async_smem();
+                    const int un = u + S;
+                    tc::mbar_arrive_expect_tx(sb + p.off_bar + 8 * slot, stage_bytes(p, un));
+                    issue_stage(p, &tm_main, &tm_tail, sb, tile0, un);
+                    cnt[S + slot] = (uint32_t)(un / S);  // newest round issued into the slot
+                }
+            }
+            __syncwarp();
+        }
+        if (chunk == p.nch - 1) {
+            // tile finished: fold the chains into the warp's partial sums
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    int v = 0;
+#pragma unroll
+                    for (int cc = 0; cc < CH; ++cc) {
+                        v += acc[nt][cc][e];
+                        acc[nt][cc][e] = 0;
+                    }
+                    const int row = g8 + 8 * (e >> 1), col = nt * 8 + 2 * t + (e & 1);
+                    if (col < ncols) wred_w[(lt * 16 + row) * ncols + col] = v;
+                }
+            }
+        }
+        if (++slot == S) {
+            slot = 0;
+            phase ^= 1;
+        }
+        if (++chunk == p.nch) {
+            chunk = 0;
+            ++lt;
+        }
+    }
+    if (!__syncthreads_and(ok)) {
+        // a stage never arrived: let the copies still in flight land before the
+        // CTA's shared memory is released, then leave (the flag is set)
+        if (tid == 0) {
+            for (int sl = 0; sl < min(S, nstages); ++sl)
+                tc::mbar_wait(sb + p.off_bar + 8 * sl, cnt[S + sl] & 1u, p.flags, kSDrainLimitNs);
+        }
+        __syncthreads();
+        return;
+    }
+
+    // 4. epilogue: one output per thread and step, consecutive threads on consecutive n
+    const int rows = T * 16;
+    if (FORM == 0) {
+        for (int o = tid; o < M * rows; o += kSThreads) {
+            const int m = o / rows, r = o - m * rows;
+            float sc;
+            int qs = 0;
+            if (PREP) {
+                sc = p.pscale[m];
+                qs = p.prsum[m];
+            } else {
+                float amax = 0.f;
+#pragma unroll
+                for (int w = 0; w < kSWarps; ++w) {
+                    amax = fmaxf(amax, red_max[w * M + m]);
+                    qs += red_sum[w * M + m];
+                }
+                sc = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
+            }
+            const int accv = warp_rows_sum(racc, r * ncols + m, p.t_max * 16 * ncols) - qs;
+            const int n = tile0 * 16 + r;
+            const float v = __fmul_rn(__fmul_rn((float)accv, sc), p.w_scale);
+            p.y[(size_t)m * p.N + n] = __half_as_ushort(__float2half_rn(v));
+            if (p.acc_out) p.acc_out[(size_t)m * p.N + n] = accv;
+        }
+    } else {
+        for (int o = tid; o < M * rows; o += kSThreads) {
+            const int m = o / rows, r = o - m * rows;
+            float st;
+            long long ts = 0;
+            if (PREP) {
+                st = p.pscale[m];
+                ts = p.prsum[m];
+            } else {
+                float amax = 0.f;
+#pragma unroll
+                for (int w = 0; w < kSWarps; ++w) {
+                    amax = fmaxf(amax, red_max[w * M + m]);
+                    ts += red_sum[w * M + m];
+                }
+                st = amax > 0.f ? __fdiv_rn(amax, 32639.0f) : 0.f;
+            }
+            const long long P = 256ll * warp_rows_sum(racc, r * ncols + 2 * m, p.t_max * 16 * ncols) +
+                                warp_rows_sum(racc, r * ncols + 2 * m + 1, p.t_max * 16 * ncols);
+            const int n = tile0 * 16 + r;
+            const float z = __fmul_rn(st, (float)(2 * P - ts));
+            const float hv = __half2float(__ushort_as_half(hs[r]));
+            p.y[(size_t)m * p.N + n] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hv)));
+        }
+    }
+}
+
+// ------------------------------------------------------------------ host --
+
+int sm_count() {
+    static std::mutex mu;
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+struct StreamPlan {
+    int grid, nt, xreg, smem;
+};
+
+// Fill the plan fields of p and choose the launch.  Shared memory is laid out
+// as: ring slots [S][bsteps][16][64 B] (+ [16][32 B] ragged tail) | activation tile [cols][K+16] | per-tile
+// partial sums [t_max*16][cols] int32 | token scratch [2][16][M] | h [t_max*16]
+// fp16 | full barriers [S] | release counters [S] + rounds issued [S].
+template <int FORM>
+bool stream_plan(StreamParams& p, int prep, StreamPlan& pl) {
+    using F = DF<FORM>;
+    const int M = p.M, K = p.K, N = p.N;
+    const int cols = M * F::kCPT;
+    if (M < 1 || M > kMaxTokS || cols > 32 || N % 16 != 0 || K % 128 != 0 || K <= 0) return false;
+    pl.nt = cols <= 8 ? 1 : cols <= 16 ? 2 : 4;
+    const int sms = sm_count();
+    if (sms <= 0) return false;
+    const int tiles = N / 16;
+    pl.grid = tiles < sms ? tiles : sms;
+    p.t_lo = tiles / pl.grid;
+    p.t_rem = tiles % pl.grid;
+    p.t_max = p.t_lo + (p.t_rem > 0 ? 1 : 0);
+    const int wbytes = K / (F::kPerWord / 4);  // packed bytes per row, a multiple of 16
+    p.nfull = wbytes / 64;
+    p.tail = wbytes % 64;                      // a partial last step of 16/32/48 bytes
+    p.ragged = p.tail != 0 ? 1 : 0;
+    p.steps = p.nfull + p.ragged;
+    // stage depth: a row's steps in one box when they fit (<= 48 steps), else
+    // boxes of a multiple of 16 steps, so every chunk starts at a step that is
+    // 0 mod 16 (a warp owns the same steps in every chunk)
+    auto set_depth = [&](int max_steps) {
+        p.nch = (p.steps + max_steps - 1) / max_steps;
+        p.bsteps = (p.steps + p.nch - 1) / p.nch;
+        if (p.nch > 1) p.bsteps = (p.bsteps + 15) / 16 * 16;
+        p.slot_bytes = (p.bsteps * 1024 + 16 * p.tail + 127) / 128 * 128;
+    };
+    p.astride = K + 16;
+    const int act = cols * p.astride;
+    const int red = kSWarps * p.t_max * 16 * cols * 4;
+    const int tok = prep ? 0 : 2 * kSWarps * M * 4;
+    const int hbytes = FORM == 1 ? p.t_max * 16 * 2 : 0;
+    auto up16 = [](int v) { return (v + 15) & ~15; };
+    const int fixed = up16(act) + up16(red) + up16(tok) + up16(hbytes) + 16 * kMaxSlots + 8 * kMaxSlots;
+    for (int cand = 0; cand < 4; ++cand) {
+        // (depth, budget): two CTAs per SM with 48-, 32- then 16-step boxes, else one
+        const int depth = cand == 0 ? 48 : cand == 1 ? 32 : 16;
+        const int budget = cand < 3 ? kStreamSmemPair : kDecodeMaxSmem;
+        set_depth(depth);
+        const int nst = p.t_max * p.nch;
+        int S = (budget - fixed) / p.slot_bytes;
+        if (S > kMaxSlots) S = kMaxSlots;
+        if (S > nst) S = nst;
+        if (S < 1 || (S < 2 && nst > 1)) continue;
+        p.S = S;
+        int off = S * p.slot_bytes;
+        p.off_act = off;
+        off += up16(act);
+        p.off_red = off;
+        off += up16(red);
+        p.off_tok = off;
+        off += up16(tok);
+        p.off_h = off;
+        off += up16(hbytes);
+        p.off_bar = off;
+        off += 8 * S;
+        p.off_cnt = off;
+        off += 8 * S;
+        pl.smem = off;
+        // warp-local M = 1 path: every lane holds at most 4 (ternary) / 1 (sign)
+        // owned step pairs, i.e. at most 128 / 32 steps per row
+        pl.xreg = (!prep && M == 1 && p.steps <= (FORM == 0 ? 128 : 32)) ? 1 : 0;
+        return true;
+    }
+    return false;
+}
+
+template <int FORM, int NT, int PREP, int XREG>
+cudaError_t launch_stream(const CUtensorMap& tm_main, const CUtensorMap& tm_tail,
+                          const StreamParams& p, const StreamPlan& pl, cudaStream_t s) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(stream_kernel<FORM, NT, PREP, XREG>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kDecodeMaxSmem);
+        if (e != cudaSuccess) return e;
+        e = use_max_shared_carveout(stream_kernel<FORM, NT, PREP, XREG>);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.grid);
+    cfg.blockDim = dim3(kSThreads);
+    cfg.dynamicSmemBytes = (size_t)pl.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attrs[1];
+    attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, stream_kernel<FORM, NT, PREP, XREG>, tm_main, tm_tail, p);
+}
+
+template <int FORM, int PREP>
+cudaError_t launch_stream_form(StreamParams p, cudaStream_t s) {
+    StreamPlan pl;
+    if (!stream_plan<FORM>(p, PREP, pl)) return cudaErrorInvalidConfiguration;
+    // weights as [step][row][64 B] boxes: dim 0 = the 64 bytes of a step,
+    // dim 1 = rows (stride = packed row bytes), dim 2 = steps (stride 64)
+    const uint64_t wbytes = (uint64_t)p.K / (DF<FORM>::kPerWord / 4);
+    CUtensorMap tm_main = {}, tm_tail = {};
+    if (p.nfull > 0) {
+        const cuuint64_t dims[3] = {64, (cuuint64_t)p.N, (cuuint64_t)p.nfull};
+        const cuuint64_t strides[2] = {wbytes, 64};
+        const cuuint32_t box[3] = {64, 16, (cuuint32_t)p.bsteps};
+        if (!encode_u8_map(&tm_main, p.w, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidConfiguration;
+    }
+    if (p.ragged) {
+        const cuuint64_t dims[2] = {(cuuint64_t)p.tail, (cuuint64_t)p.N};
+        const cuuint64_t strides[1] = {wbytes};
+        const cuuint32_t box[2] = {(cuuint32_t)p.tail, 16};
+        const uint8_t* tail = reinterpret_cast<const uint8_t*>(p.w) + 64 * (size_t)p.nfull;
+        if (!encode_u8_map(&tm_tail, tail, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidConfiguration;
+    }
+    if constexpr (!PREP) {
+        if (pl.xreg) {
+            if (pl.nt == 1) return launch_stream<FORM, 1, 0, 1>(tm_main, tm_tail, p, pl, s);
+            return cudaErrorInvalidConfiguration;  // M == 1 always has one column tile
+        }
+    }
+    switch (pl.nt) {
+        case 1: return launch_stream<FORM, 1, PREP, 0>(tm_main, tm_tail, p, pl, s);
+        case 2: return launch_stream<FORM, 2, PREP, 0>(tm_main, tm_tail, p, pl, s);
+        default: return launch_stream<FORM, 4, PREP, 0>(tm_main, tm_tail, p, pl, s);
+    }
+}
+
+}  // namespace
+
+bool stream_fits(int form, int M, int K, int N, int prep) {
+    StreamParams p = {};
+    p.M = M;
+    p.K = K;
+    p.N = N;
+    StreamPlan pl;
+    return form == 0 ? stream_plan<0>(p, prep, pl) : stream_plan<1>(p, prep, pl);
+}
+
+cudaError_t launch_ternary_stream(const uint16_t* x, const uint32_t* w2, int M, int K, int N,
+                                  float w_scale, uint16_t* y, int32_t* acc_out, unsigned int* flags,
+                                  cudaStream_t s) {
+    StreamParams p = {};
+    p.x = x;
+    p.w = w2;
+    p.w_scale = w_scale;
+    p.M = M;
+    p.K = K;
+    p.N = N;
+    p.y = y;
+    p.acc_out = acc_out;
+    p.flags = flags;
+    return launch_stream_form<0, 0>(p, s);
+}
+
+cudaError_t launch_onebit_stream(const uint16_t* x, const uint16_t* g, const uint16_t* h,
+                                 const uint32_t* s1, int M, int K, int N, uint16_t* y,
+                                 unsigned int* flags, cudaStream_t s) {
+    StreamParams p = {};
+    p.x = x;
+    p.g = g;
+    p.h = h;
+    p.w = s1;
+    p.M = M;
+    p.K = K;
+    p.N = N;
+    p.y = y;
+    p.flags = flags;
+    return launch_stream_form<1, 0>(p, s);
+}
+
+cudaError_t launch_ternary_stream_prepared(const int8_t* qp, const float* scale, const int32_t* qsum,
+                                           const uint32_t* w2, int M, int K, int N, float w_scale,
+                                           uint16_t* y, int32_t* acc_out, unsigned int* flags,
+                                           cudaStream_t s) {
+    StreamParams p = {};
+    p.prep = qp;
+    p.pscale = scale;
+    p.prsum = qsum;
+    p.w = w2;
+    p.w_scale = w_scale;
+    p.M = M;
+    p.K = K;
+    p.N = N;
+    p.y = y;
+    p.acc_out = acc_out;
+    p.flags = flags;
+    return launch_stream_form<0, 1>(p, s);
+}
+
+cudaError_t launch_onebit_stream_prepared(const int8_t* planes, const float* step,
+                                          const int32_t* tsum, const uint16_t* h,
+                                          const uint32_t* s1, int M, int K, int N, uint16_t* y,
+                                          unsigned int* flags, cudaStream_t s) {
+    StreamParams p = {};
+    p.prep = planes;
+    p.pscale = step;
+    p.prsum = tsum;
+    p.h = h;
+    p.w = s1;
+    p.M = M;
+    p.K = K;
+    p.N = N;
+    p.y = y;
+    p.flags = flags;
+    return launch_stream_form<1, 1>(p, s);
+}
+
+}  // namespace bl

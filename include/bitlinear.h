@@ -24,6 +24,13 @@
  *   - Calls are asynchronous on `stream` (NULL = the legacy default stream)
  *     except the two packers, which synchronise `stream` to report invalid
  *     input values.
+ *   - Overlap with the preceding kernel (programmatic dependent launch): the
+ *     linear layers start streaming their PARAMETERS (w2 / s1, g, h) into
+ *     on-chip memory while the kernel queued just before them on `stream` is
+ *     still running, and read x (and the workspace) only after it completes.
+ *     So parameters must not be written by the kernel immediately preceding a
+ *     call on the same stream; activations may be.  (The packers synchronise,
+ *     so packing and then calling is always safe.)
  *   - Shapes: M >= 0 and N >= 0 (0 is a no-op returning BL_OK); N % 16 == 0;
  *     K > 0 and K % 128 == 0.  Anything else returns BL_ERR_SHAPE without
  *     touching memory.
