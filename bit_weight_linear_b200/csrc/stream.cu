@@ -192,7 +192,9 @@ __device__ __forceinline__ void issue_stage(const StreamParams& p, const CUtenso
 }
 
 // PREP = 0: the CTA prepares the activations from x (M <= a few tokens).
-//   XREG = 1 (M == 1 and few groups per thread): x stays in registers between
+//   XREG = 1 or 2 (M == 1, at most 64 / 32 steps): warp-local preparation, x
+//   in registers; XREG = 2 when K is a whole number of steps (no partial step
+//   to guard in the contraction).  XREG = 0: general M; x stays in registers between
 //   the absmax and the quantisation pass.
 // PREP = 1: the activation kernel prepared them; they are copied in.
 template <int FORM, int NT, int PREP, int XREG>
@@ -227,7 +229,6 @@ __global__ void __launch_bounds__(kSThreads, 2)
         if (p.ragged) tc::prefetch_tmap(&tm_tail);
     }
     for (int i = tid; i < 2 * S; i += kSThreads) cnt[i] = 0;
-    for (int i = tid; i < kSWarps * p.t_max * 16 * ncols; i += kSThreads) racc[i] = 0;
     if (FORM == 1)
         for (int i = tid; i < T * 16; i += kSThreads) hs[i] = p.h[tile0 * 16 + i];
     // Warp-local activation preparation (XREG): warp w owns the k-steps
@@ -243,7 +244,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
             for (int v = 0; v < 4; ++v) ga[v] = ld_ro_v4(p.g + k0 + 8 * v);
         }
     }
-    __syncthreads();  // barriers initialised, counters and partial sums zeroed
+    __syncthreads();  // barriers initialised, counters zeroed
     tc::pdl_trigger();
     if (tid == 0) {
         const int nfill = min(S, nstages);
@@ -257,6 +258,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     tc::pdl_wait();
 
     // 2. activations
+    float tok_amax = 0.f;  // XREG: the token's absmax, kept for the epilogue
     if (PREP) {
         const int per_row = K / 16;
         for (int c = tid; c < ncols * per_row; c += kSThreads) {
@@ -270,7 +272,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         // M == 1: x stays in registers; one CTA barrier (the absmax); each warp
         // then quantises exactly the steps it contracts, so the contraction
         // needs only the warp's own writes (__syncwarp, no CTA barrier)
-        constexpr int R = FORM == 0 ? 4 : 1;  // owned step pairs per lane
+        constexpr int R = FORM == 0 ? 2 : 1;  // owned step pairs per lane
         uint4 xa[R][G / 8];
         bool has[R];
         float mx = 0.f;
@@ -294,13 +296,18 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 for (int v = 0; v < G / 8; ++v) mx = fmaxf(mx, absmax_prod(xa[i][v], ga[v]));
             }
         }
+        // non-negative floats order like their bit patterns: one redux.sync max
         if (FORM == 0) mx = hbits(mb);
-        mx = warp_max(mx);
+        mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
         if (lane == 0) red_max[warp] = mx;
         __syncthreads();
         float amax = 0.f;
 #pragma unroll
-        for (int w = 0; w < kSWarps; ++w) amax = fmaxf(amax, red_max[w]);
+        for (int w = 0; w < kSWarps; w += 4) {
+            const float4 r4 = *reinterpret_cast<const float4*>(red_max + w);
+            amax = fmaxf(fmaxf(amax, r4.x), fmaxf(r4.y, fmaxf(r4.z, r4.w)));
+        }
+        tok_amax = amax;
         int sum = 0;
         if constexpr (FORM == 0) {
             const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
@@ -317,7 +324,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 sum = quant_group_s(xa[0], ga, inv, act + k0, act + p.astride + k0);
             }
         }
-        sum = warp_sum(sum);
+        sum = __reduce_add_sync(0xffffffffu, sum);
         if (lane == 0) red_sum[warp] = sum;
         __syncwarp();
     } else {
@@ -402,11 +409,11 @@ __global__ void __launch_bounds__(kSThreads, 2)
         const uint8_t* slot_p = smem + slot * p.slot_bytes;
         for (int s = s0 + warp; s < s1; s += kSWarps) {
             // whole step: [step][row][64 B]; partial last step: tail box [row][tail B]
-            const bool part = s >= p.nfull;
+            const bool part = XREG == 2 ? false : s >= p.nfull;
             const uint8_t* w0 = part ? slot_p + p.bsteps * 1024 + p.tail * g8 + 16 * t
                                      : slot_p + (s - s0) * 1024 + 64 * g8 + 16 * t;
             const int rs8 = part ? 8 * p.tail : 512;  // 8 rows further down
-            const bool lane_ok = s * F::kStepK + t * F::kChunkK < K;
+            const bool lane_ok = XREG == 2 || s * F::kStepK + t * F::kChunkK < K;
             uint4 a0 = make_uint4(0, 0, 0, 0), a1 = make_uint4(0, 0, 0, 0);
             if (lane_ok) {
                 a0 = *reinterpret_cast<const uint4*>(w0);
@@ -510,11 +517,19 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 sc = p.pscale[m];
                 qs = p.prsum[m];
             } else {
-                float amax = 0.f;
+                float amax = tok_amax;
+                if (XREG) {  // M == 1: the 16 warp sums are contiguous
 #pragma unroll
-                for (int w = 0; w < kSWarps; ++w) {
-                    amax = fmaxf(amax, red_max[w * M + m]);
-                    qs += red_sum[w * M + m];
+                    for (int w = 0; w < kSWarps; w += 4) {
+                        const int4 r4 = *reinterpret_cast<const int4*>(red_sum + w);
+                        qs += (r4.x + r4.y) + (r4.z + r4.w);
+                    }
+                } else {
+#pragma unroll
+                    for (int w = 0; w < kSWarps; ++w) {
+                        amax = fmaxf(amax, red_max[w * M + m]);
+                        qs += red_sum[w * M + m];
+                    }
                 }
                 sc = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
             }
@@ -533,11 +548,19 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 st = p.pscale[m];
                 ts = p.prsum[m];
             } else {
-                float amax = 0.f;
+                float amax = tok_amax;
+                if (XREG) {  // M == 1: the 16 warp sums are contiguous
 #pragma unroll
-                for (int w = 0; w < kSWarps; ++w) {
-                    amax = fmaxf(amax, red_max[w * M + m]);
-                    ts += red_sum[w * M + m];
+                    for (int w = 0; w < kSWarps; w += 4) {
+                        const int4 r4 = *reinterpret_cast<const int4*>(red_sum + w);
+                        ts += (r4.x + r4.y) + (r4.z + r4.w);
+                    }
+                } else {
+#pragma unroll
+                    for (int w = 0; w < kSWarps; ++w) {
+                        amax = fmaxf(amax, red_max[w * M + m]);
+                        ts += red_sum[w * M + m];
+                    }
                 }
                 st = amax > 0.f ? __fdiv_rn(amax, 32639.0f) : 0.f;
             }
@@ -635,9 +658,9 @@ bool stream_plan(StreamParams& p, int prep, StreamPlan& pl) {
         p.off_cnt = off;
         off += 8 * S;
         pl.smem = off;
-        // warp-local M = 1 path: every lane holds at most 4 (ternary) / 1 (sign)
-        // owned step pairs, i.e. at most 128 / 32 steps per row
-        pl.xreg = (!prep && M == 1 && p.steps <= (FORM == 0 ? 128 : 32)) ? 1 : 0;
+        // warp-local M = 1 path: every lane holds at most 2 (ternary) / 1 (sign)
+        // owned step pairs, i.e. at most 64 / 32 steps per row
+        pl.xreg = (!prep && M == 1 && p.steps <= (FORM == 0 ? 64 : 32)) ? (p.ragged ? 1 : 2) : 0;
         return true;
     }
     return false;
@@ -694,7 +717,9 @@ cudaError_t launch_stream_form(StreamParams p, cudaStream_t s) {
     }
     if constexpr (!PREP) {
         if (pl.xreg) {
-            if (pl.nt == 1) return launch_stream<FORM, 1, 0, 1>(tm_main, tm_tail, p, pl, s);
+            if (pl.nt == 1)
+                return pl.xreg == 2 ? launch_stream<FORM, 1, 0, 2>(tm_main, tm_tail, p, pl, s)
+                                    : launch_stream<FORM, 1, 0, 1>(tm_main, tm_tail, p, pl, s);
             return cudaErrorInvalidConfiguration;  // M == 1 always has one column tile
         }
     }
