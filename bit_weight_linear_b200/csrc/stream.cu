@@ -203,6 +203,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
                   const __grid_constant__ CUtensorMap tm_tail, const StreamParams p) {
     using F = DF<FORM>;
     constexpr int CH = 4 / NT;  // independent accumulator chains per column tile
+    // ternary with one column tile: in-place masked unpack (one AND per register)
+    constexpr bool kMasked = FORM == 0 && NT == 1;
     extern __shared__ __align__(128) uint8_t smem[];
     const int K = p.K, M = p.M;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -421,6 +423,33 @@ __global__ void __launch_bounds__(kSThreads, 2)
             }
             const uint32_t r0[4] = {a0.x, a0.y, a0.z, a0.w};
             const uint32_t r1[4] = {a1.x, a1.y, a1.z, a1.w};
+            if constexpr (kMasked) {
+                // ternary, one column tile: field j of every byte is masked in
+                // place (value code * 4^j) and multiplies activation word j; the
+                // two words of a pair share j, so each MMA has one scale 4^j and
+                // accumulates into chain j
+                uint32_t b[4][4];
+#pragma unroll
+                for (int om = 0; om < 4; ++om) {
+                    if (lane_ok && bvalid[0]) {
+                        const uint4 bv = *reinterpret_cast<const uint4*>(bsrc[0] + s * F::kStepK + 16 * om);
+                        b[om][0] = bv.x;
+                        b[om][1] = bv.y;
+                        b[om][2] = bv.z;
+                        b[om][3] = bv.w;
+                    } else {
+                        b[om][0] = b[om][1] = b[om][2] = b[om][3] = 0;
+                    }
+                }
+#pragma unroll
+                for (int op = 0; op < 4; op += 2)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t m = 0x03030303u << (2 * j);
+                        mma_u8s8_16832(acc[0][j], r0[op] & m, r1[op] & m, r0[op + 1] & m,
+                                       r1[op + 1] & m, b[op][j], b[op + 1][j]);
+                    }
+            } else {
 #pragma unroll
             for (int om = 0; om < 4; ++om) {
                 uint32_t u0r[F::kRegs], u1r[F::kRegs];
@@ -452,6 +481,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
                                        b[j], b[j + 1]);
                 }
             }
+            }
         }
         // release the slot (only when it is to be refilled); the warp that
         // releases it last refills it
@@ -478,7 +508,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
                     int v = 0;
 #pragma unroll
                     for (int cc = 0; cc < CH; ++cc) {
-                        v += acc[nt][cc][e];
+                        // masked chains hold 4^cc times their sums (exact shifts)
+                        v += kMasked ? (acc[nt][cc][e] >> (2 * cc)) : acc[nt][cc][e];
                         acc[nt][cc][e] = 0;
                     }
                     const int row = g8 + 8 * (e >> 1), col = nt * 8 + 2 * t + (e & 1);
@@ -604,6 +635,8 @@ bool stream_plan(StreamParams& p, int prep, StreamPlan& pl) {
     const int M = p.M, K = p.K, N = p.N;
     const int cols = M * F::kCPT;
     if (M < 1 || M > kMaxTokS || cols > 32 || N % 16 != 0 || K % 128 != 0 || K <= 0) return false;
+    // int32 partial sums: the masked ternary chain 3 reaches K/4 * 128 * 127
+    if (K > 262144) return false;
     pl.nt = cols <= 8 ? 1 : cols <= 16 ? 2 : 4;
     const int sms = sm_count();
     if (sms <= 0) return false;
