@@ -67,6 +67,7 @@ struct StreamParams {
     int ragged;              // 1: the last step is partial: `tail` bytes per row (tail map)
     int tail;                // 16, 32 or 48 bytes (sign); 32 (ternary)
     int slot_bytes;
+    int compact;             // 1: per-tile reduction through one [16 warps][16][cols] scratch
     int off_act, astride, off_red, off_tok, off_h, off_bar, off_cnt;
 };
 
@@ -166,6 +167,12 @@ __device__ __forceinline__ int warp_rows_sum(const int* red, int idx, int stride
 #pragma unroll
     for (int w = 0; w < kSWarps; ++w) v += red[w * stride + idx];
     return v;
+}
+
+// partial sum idx ([row][col] over the CTA's tiles): the 16 warps' copies, or
+// the compact mode's reduced result rows
+__device__ __forceinline__ int tile_sum(const int* red, const StreamParams& p, int idx, int ncols) {
+    return p.compact ? red[kSWarps * 16 * ncols + idx] : warp_rows_sum(red, idx, p.t_max * 16 * ncols);
 }
 
 // Ring stage u = (tile u / nch, chunk u % nch): one box of bsteps whole steps
@@ -395,7 +402,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
         bvalid[nt] = col < ncols;
         bsrc[nt] = act + (bvalid[nt] ? col : 0) * p.astride + t * F::kChunkK;
     }
-    int* wred_w = racc + warp * p.t_max * 16 * ncols;  // this warp's [t_max*16][ncols]
+    // this warp's partial sums: [t_max*16][ncols], or (compact) [16][ncols] for the current tile
+    // (M = 1 kernels never use the compact layout: its code is compiled out there)
+    const bool compact = XREG == 0 && p.compact;
+    int* wred_w = racc + warp * (compact ? 16 : p.t_max * 16) * ncols;
     int acc[NT][CH][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -404,10 +414,18 @@ __global__ void __launch_bounds__(kSThreads, 2)
     bool ok = true;
     int slot = 0, phase = 0, chunk = 0, lt = 0;  // stage u = lt * nch + chunk, in slot u % S
     for (int u = 0; u < nstages; ++u) {
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(sb + p.off_bar + 8 * slot, (uint32_t)phase,
-                                                   p.flags, kSWaitLimitNs));
-        if (!ok) break;
-        const int s0 = chunk * p.bsteps, s1 = min(s0 + p.bsteps, p.steps);
+        // compact mode has CTA barriers inside the loop: a failed wait skips
+        // the work but keeps the warp in step until the tile's barrier, where
+        // the CTA agrees to stop
+        if (!compact) {
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(sb + p.off_bar + 8 * slot, (uint32_t)phase,
+                                                       p.flags, kSWaitLimitNs));
+            if (!ok) break;
+        } else if (ok) {
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(sb + p.off_bar + 8 * slot, (uint32_t)phase,
+                                                       p.flags, kSWaitLimitNs));
+        }
+        const int s0 = chunk * p.bsteps, s1 = ok ? min(s0 + p.bsteps, p.steps) : s0;
         const uint8_t* slot_p = smem + slot * p.slot_bytes;
         for (int s = s0 + warp; s < s1; s += kSWarps) {
             // whole step: [step][row][64 B]; partial last step: tail box [row][tail B]
@@ -485,7 +503,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         }
         // release the slot (only when it is to be refilled); the warp that
         // releases it last refills it
-        if (u + S < nstages) {
+        if (ok && u + S < nstages) {
             __syncwarp();
             if (lane == 0) {
                 const uint32_t old = tc::atom_add_acq_rel_smem(cnt_sb + 4 * slot, 1u);
@@ -513,8 +531,20 @@ __global__ void __launch_bounds__(kSThreads, 2)
                         acc[nt][cc][e] = 0;
                     }
                     const int row = g8 + 8 * (e >> 1), col = nt * 8 + 2 * t + (e & 1);
-                    if (col < ncols) wred_w[(lt * 16 + row) * ncols + col] = v;
+                    // compact: wred_w is this warp's [16][ncols] scratch for the tile
+                    if (col < ncols) wred_w[((compact ? 0 : lt) * 16 + row) * ncols + col] = v;
                 }
+            }
+            if (compact) {
+                // add the 16 warps' partials of this tile into its result rows
+                if (!__syncthreads_and(ok)) {
+                    ok = false;
+                    break;
+                }
+                int* res = racc + kSWarps * 16 * ncols;  // [t_max*16][ncols]
+                for (int i = tid; i < 16 * ncols; i += kSThreads)
+                    res[lt * 16 * ncols + i] = warp_rows_sum(racc, i, 16 * ncols);
+                __syncthreads();
             }
         }
         if (++slot == S) {
@@ -564,7 +594,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 }
                 sc = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
             }
-            const int accv = warp_rows_sum(racc, r * ncols + m, p.t_max * 16 * ncols) - qs;
+            const int accv = tile_sum(racc, p, r * ncols + m, ncols) - qs;
             const int n = tile0 * 16 + r;
             const float v = __fmul_rn(__fmul_rn((float)accv, sc), p.w_scale);
             p.y[(size_t)m * p.N + n] = __half_as_ushort(__float2half_rn(v));
@@ -595,8 +625,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 }
                 st = amax > 0.f ? __fdiv_rn(amax, 32639.0f) : 0.f;
             }
-            const long long P = 256ll * warp_rows_sum(racc, r * ncols + 2 * m, p.t_max * 16 * ncols) +
-                                warp_rows_sum(racc, r * ncols + 2 * m + 1, p.t_max * 16 * ncols);
+            const long long P = 256ll * tile_sum(racc, p, r * ncols + 2 * m, ncols) +
+                                tile_sum(racc, p, r * ncols + 2 * m + 1, ncols);
             const int n = tile0 * 16 + r;
             const float z = __fmul_rn(st, (float)(2 * P - ts));
             const float hv = __half2float(__ushort_as_half(hs[r]));
@@ -661,7 +691,12 @@ bool stream_plan(StreamParams& p, int prep, StreamPlan& pl) {
     };
     p.astride = K + 16;
     const int act = cols * p.astride;
-    const int red = kSWarps * p.t_max * 16 * cols * 4;
+    // per-warp partial sums for every tile, or (compact) one tile's worth plus
+    // the reduced rows, when the first does not fit beside the activations
+    const int red_full = kSWarps * p.t_max * 16 * cols * 4;
+    const int red_compact = (kSWarps * 16 + p.t_max * 16) * cols * 4;
+    p.compact = cols * p.astride + red_full > kStreamSmemPair / 2 ? 1 : 0;
+    const int red = p.compact ? red_compact : red_full;
     const int tok = prep ? 0 : 2 * kSWarps * M * 4;
     const int hbytes = FORM == 1 ? p.t_max * 16 * 2 : 0;
     auto up16 = [](int v) { return (v + 15) & ~15; };
