@@ -157,7 +157,7 @@ bl_status bl_ternary_linear(const uint16_t* x, int M, int K, int N, const uint32
     if (misaligned(workspace)) return BL_ERR_ALIGN;
     unsigned int* flags = device_flags();
     if (!flags) return BL_ERR_CUDA;
-    if (M <= bl::kFusedMaxM && bl::stream_fits(0, M, K, N, 0))
+    if (M <= bl::kStreamFusedMaxM && bl::stream_fits(0, M, K, N, 0))
         return from_cuda(
             bl::launch_ternary_stream(x, w2, M, K, N, w_scale, y, acc_out, flags, cs(stream)));
     if (M <= bl::kFusedMaxM && bl::decode_fused_fits(0, M, K))
@@ -205,7 +205,7 @@ bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
     if (misaligned(workspace)) return BL_ERR_ALIGN;
     unsigned int* flags = device_flags();
     if (!flags) return BL_ERR_CUDA;
-    if (M <= bl::kFusedMaxM && bl::stream_fits(1, M, K, N, 0))
+    if (M <= bl::kStreamFusedMaxM / 2 && bl::stream_fits(1, M, K, N, 0))
         return from_cuda(bl::launch_onebit_stream(x, g, h, s1, M, K, N, y, flags, cs(stream)));
     if (M <= bl::kFusedMaxM && bl::decode_fused_fits(1, M, K))
         return from_cuda(bl::launch_onebit_decode(x, g, h, s1, M, K, N, y, flags, cs(stream)));

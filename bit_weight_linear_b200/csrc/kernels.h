@@ -109,6 +109,9 @@ inline cudaError_t use_max_shared_carveout(Kern kern) {
 
 // Largest M for which the decode kernel prepares the activations itself.
 constexpr int kFusedMaxM = 2;
+// Largest M (ternary; half of it for OneBit, two columns per token) for which
+// the streamed decode CTA prepares the activations itself.
+constexpr int kStreamFusedMaxM = 8;
 
 // Token counts at or above which the tensor-core prefill kernel is used.
 constexpr int kTernaryPrefillMinM = 33;

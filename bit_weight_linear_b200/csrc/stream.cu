@@ -198,11 +198,12 @@ __device__ __forceinline__ void issue_stage(const StreamParams& p, const CUtenso
     if (p.ragged && ch.s1 == p.steps) tc::tma_load_2d(dst + p.bsteps * 1024, tm_tail, 0, row0, bar);
 }
 
-// PREP = 0: the CTA prepares the activations from x (M <= a few tokens).
-//   XREG = 1 or 2 (M == 1, at most 64 / 32 steps): warp-local preparation, x
-//   in registers; XREG = 2 when K is a whole number of steps (no partial step
-//   to guard in the contraction).  XREG = 0: general M; x stays in registers between
-//   the absmax and the quantisation pass.
+// PREP = 0: the CTA prepares the activations from x.
+//   XREG != 0: warp-local preparation with x in registers; 1, 2: M == 1
+//   (2 when K is a whole number of steps, so the contraction has no partial
+//   step to guard); 3: M > 1 (up to 2 units per lane, 1 for sign); 4: M > 1,
+//   4 units per lane, whole steps (ternary).
+//   XREG = 0: general M, x read twice (second pass from L1/L2).
 // PREP = 1: the activation kernel prepared them; they are copied in.
 template <int FORM, int NT, int PREP, int XREG>
 __global__ void __launch_bounds__(kSThreads, 2)
@@ -241,16 +242,39 @@ __global__ void __launch_bounds__(kSThreads, 2)
     if (FORM == 1)
         for (int i = tid; i < T * 16; i += kSThreads) hs[i] = p.h[tile0 * 16 + i];
     // Warp-local activation preparation (XREG): warp w owns the k-steps
-    // s = w, w + 16, ... (the steps it contracts); lane l takes group l % 16 of
-    // its owned steps 2i + l / 16.  OneBit's g is a parameter, read before the wait.
+    // s = w, w + 16, ... (the steps it contracts).  Its work is the units
+    // (token m, group q of its owned steps), token-major; lane l takes units
+    // l, l + 32, ... (at most U).  OneBit's g is a parameter, read before the wait.
     constexpr int G = F::kGroup;
-    const int gi = lane & 15;
-    uint4 ga[4];
-    if (FORM == 1 && XREG) {
-        const int s_own = warp + 16 * (lane >> 4), k0 = s_own * F::kStepK + gi * G;
-        if (s_own < p.steps && k0 < K) {
+    constexpr bool kOne = XREG == 1 || XREG == 2;            // M == 1 variants
+    constexpr int U = XREG == 4 ? 4 : (FORM == 0 ? 2 : 1);  // units per lane
+    const int Mx = kOne ? 1 : M;                             // compile-time 1 for M == 1
+    int um[U], uk[U];
+    bool has[U];
+    if constexpr (XREG != 0) {
+        const int own = warp < p.steps ? (p.steps - 1 - warp) / 16 + 1 : 0;
+        const int gw = own * 16;  // groups per token owned by this warp
 #pragma unroll
-            for (int v = 0; v < 4; ++v) ga[v] = ld_ro_v4(p.g + k0 + 8 * v);
+        for (int i = 0; i < U; ++i) {
+            const int v = lane + 32 * i;
+            int m, q;
+            if constexpr (kOne) {
+                m = v < gw ? 0 : 1;
+                q = v;
+            } else {
+                m = gw > 0 ? v / gw : M;
+                q = gw > 0 ? v - m * gw : 0;
+            }
+            um[i] = m;
+            uk[i] = (warp + 16 * (q >> 4)) * F::kStepK + (q & 15) * G;
+            has[i] = m < Mx && uk[i] < K;
+        }
+    }
+    uint4 ga[4];
+    if constexpr (FORM == 1 && XREG != 0) {
+        if (has[0]) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) ga[v] = ld_ro_v4(p.g + uk[0] + 8 * v);
         }
     }
     __syncthreads();  // barriers initialised, counters zeroed
@@ -278,63 +302,75 @@ __global__ void __launch_bounds__(kSThreads, 2)
         tc::cp_async_wait_all();
         __syncthreads();
     } else if (XREG) {
-        // M == 1: x stays in registers; one CTA barrier (the absmax); each warp
-        // then quantises exactly the steps it contracts, so the contraction
-        // needs only the warp's own writes (__syncwarp, no CTA barrier)
-        constexpr int R = FORM == 0 ? 2 : 1;  // owned step pairs per lane
-        uint4 xa[R][G / 8];
-        bool has[R];
-        float mx = 0.f;
-        uint32_t mb = 0;
+        // M <= 8 (ternary) / 2 (sign): x stays in registers; one CTA barrier
+        // (the per-token absmax); each warp then quantises exactly the steps it
+        // contracts, so the contraction needs only the warp's own writes
+        uint4 xa[U][G / 8];
+        float umx[U];
 #pragma unroll
-        for (int i = 0; i < R; ++i) {
-            const int s_own = warp + 16 * (2 * i + (lane >> 4)), k0 = s_own * F::kStepK + gi * G;
-            has[i] = s_own < p.steps && k0 < K;
+        for (int i = 0; i < U; ++i) {
             if (has[i]) {
 #pragma unroll
-                for (int v = 0; v < G / 8; ++v) xa[i][v] = tc::ld_v4(p.x + k0 + 8 * v);
+                for (int v = 0; v < G / 8; ++v) xa[i][v] = tc::ld_v4(p.x + (size_t)um[i] * K + uk[i] + 8 * v);
             }
         }
 #pragma unroll
-        for (int i = 0; i < R; ++i) {
+        for (int i = 0; i < U; ++i) {
+            umx[i] = 0.f;
             if (!has[i]) continue;
             if constexpr (FORM == 0) {
-                mb = max(mb, max(absmax_bits_t(xa[i][0]), absmax_bits_t(xa[i][1])));
+                umx[i] = hbits(max(absmax_bits_t(xa[i][0]), absmax_bits_t(xa[i][1])));
             } else {
 #pragma unroll
-                for (int v = 0; v < G / 8; ++v) mx = fmaxf(mx, absmax_prod(xa[i][v], ga[v]));
+                for (int v = 0; v < G / 8; ++v) umx[i] = fmaxf(umx[i], absmax_prod(xa[i][v], ga[v]));
             }
         }
-        // non-negative floats order like their bit patterns: one redux.sync max
-        if (FORM == 0) mx = hbits(mb);
-        mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
-        if (lane == 0) red_max[warp] = mx;
+        // non-negative floats order like their bit patterns: one redux.sync max per token
+        for (int m = 0; m < Mx; ++m) {
+            float v = 0.f;
+#pragma unroll
+            for (int i = 0; i < U; ++i)
+                if (has[i] && um[i] == m) v = fmaxf(v, umx[i]);
+            v = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(v)));
+            if (lane == 0) red_max[warp * Mx + m] = v;
+        }
         __syncthreads();
-        float amax = 0.f;
+        // lane m < M reduces token m's absmax and inverse step; units fetch theirs by shuffle
+        float amax_l = 0.f;
+        if (Mx == 1) {
 #pragma unroll
-        for (int w = 0; w < kSWarps; w += 4) {
-            const float4 r4 = *reinterpret_cast<const float4*>(red_max + w);
-            amax = fmaxf(fmaxf(amax, r4.x), fmaxf(r4.y, fmaxf(r4.z, r4.w)));
-        }
-        tok_amax = amax;
-        int sum = 0;
-        if constexpr (FORM == 0) {
-            const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+            for (int w = 0; w < kSWarps; w += 4) {
+                const float4 r4 = *reinterpret_cast<const float4*>(red_max + w);
+                amax_l = fmaxf(fmaxf(amax_l, r4.x), fmaxf(r4.y, fmaxf(r4.z, r4.w)));
+            }
+        } else if (lane < Mx) {
 #pragma unroll
-            for (int i = 0; i < R; ++i) {
-                if (!has[i]) continue;
-                const int k0 = (warp + 16 * (2 * i + (lane >> 4))) * F::kStepK + gi * G;
-                sum += quant_group_t(xa[i][0], xa[i][1], inv, act + k0);
-            }
-        } else {
-            const float inv = amax > 0.f ? __fdiv_rn(32639.0f, amax) : 0.f;
-            if (has[0]) {
-                const int k0 = (warp + 16 * (lane >> 4)) * F::kStepK + gi * G;
-                sum = quant_group_s(xa[0], ga, inv, act + k0, act + p.astride + k0);
+            for (int w = 0; w < kSWarps; ++w) amax_l = fmaxf(amax_l, red_max[w * Mx + lane]);
+        }
+        tok_amax = amax_l;
+        const float qmax = FORM == 0 ? 127.0f : 32639.0f;
+        const float inv_l = amax_l > 0.f ? __fdiv_rn(qmax, amax_l) : 0.f;
+        int usum[U];
+#pragma unroll
+        for (int i = 0; i < U; ++i) {
+            const float inv = Mx == 1 ? inv_l : __shfl_sync(0xffffffffu, inv_l, um[i] < Mx ? um[i] : 0);
+            usum[i] = 0;
+            if (!has[i]) continue;
+            uint8_t* dst = act + (kOne ? 0 : um[i]) * F::kCPT * p.astride + uk[i];
+            if constexpr (FORM == 0) {
+                usum[i] = quant_group_t(xa[i][0], xa[i][1], inv, dst);
+            } else {
+                usum[i] = quant_group_s(xa[i], ga, inv, dst, dst + p.astride);
             }
         }
-        sum = __reduce_add_sync(0xffffffffu, sum);
-        if (lane == 0) red_sum[warp] = sum;
+        for (int m = 0; m < Mx; ++m) {
+            int v = 0;
+#pragma unroll
+            for (int i = 0; i < U; ++i)
+                if (has[i] && um[i] == m) v += usum[i];
+            v = __reduce_add_sync(0xffffffffu, v);
+            if (lane == 0) red_sum[warp * Mx + m] = v;
+        }
         __syncwarp();
     } else {
         // general M: x is read twice (the second pass hits L1/L2)
@@ -429,11 +465,11 @@ __global__ void __launch_bounds__(kSThreads, 2)
         const uint8_t* slot_p = smem + slot * p.slot_bytes;
         for (int s = s0 + warp; s < s1; s += kSWarps) {
             // whole step: [step][row][64 B]; partial last step: tail box [row][tail B]
-            const bool part = XREG == 2 ? false : s >= p.nfull;
+            const bool part = (XREG == 2 || XREG == 4) ? false : s >= p.nfull;
             const uint8_t* w0 = part ? slot_p + p.bsteps * 1024 + p.tail * g8 + 16 * t
                                      : slot_p + (s - s0) * 1024 + 64 * g8 + 16 * t;
             const int rs8 = part ? 8 * p.tail : 512;  // 8 rows further down
-            const bool lane_ok = XREG == 2 || s * F::kStepK + t * F::kChunkK < K;
+            const bool lane_ok = XREG == 2 || XREG == 4 || s * F::kStepK + t * F::kChunkK < K;
             uint4 a0 = make_uint4(0, 0, 0, 0), a1 = make_uint4(0, 0, 0, 0);
             if (lane_ok) {
                 a0 = *reinterpret_cast<const uint4*>(w0);
@@ -579,13 +615,14 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 qs = p.prsum[m];
             } else {
                 float amax = tok_amax;
-                if (XREG) {  // M == 1: the 16 warp sums are contiguous
+                if (kOne) {  // M == 1: the 16 warp sums are contiguous
 #pragma unroll
                     for (int w = 0; w < kSWarps; w += 4) {
                         const int4 r4 = *reinterpret_cast<const int4*>(red_sum + w);
                         qs += (r4.x + r4.y) + (r4.z + r4.w);
                     }
                 } else {
+                    amax = 0.f;
 #pragma unroll
                     for (int w = 0; w < kSWarps; ++w) {
                         amax = fmaxf(amax, red_max[w * M + m]);
@@ -610,13 +647,14 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 ts = p.prsum[m];
             } else {
                 float amax = tok_amax;
-                if (XREG) {  // M == 1: the 16 warp sums are contiguous
+                if (kOne) {  // M == 1: the 16 warp sums are contiguous
 #pragma unroll
                     for (int w = 0; w < kSWarps; w += 4) {
                         const int4 r4 = *reinterpret_cast<const int4*>(red_sum + w);
                         ts += (r4.x + r4.y) + (r4.z + r4.w);
                     }
                 } else {
+                    amax = 0.f;
 #pragma unroll
                     for (int w = 0; w < kSWarps; ++w) {
                         amax = fmaxf(amax, red_max[w * M + m]);
@@ -726,9 +764,17 @@ bool stream_plan(StreamParams& p, int prep, StreamPlan& pl) {
         p.off_cnt = off;
         off += 8 * S;
         pl.smem = off;
-        // warp-local M = 1 path: every lane holds at most 2 (ternary) / 1 (sign)
-        // owned step pairs, i.e. at most 64 / 32 steps per row
-        pl.xreg = (!prep && M == 1 && p.steps <= (FORM == 0 ? 64 : 32)) ? (p.ragged ? 1 : 2) : 0;
+        // warp-local preparation: a warp's units (tokens x owned groups) spread
+        // over its 32 lanes, at most 2 (4 when K has whole steps) per lane for
+        // ternary, 1 for sign; M > 1 without it is prepared by the activation kernel
+        // (xreg 1, 2: M == 1; 3: M > 1; 4: M > 1 with 4 units per lane, whole steps)
+        const int units = (p.steps + 15) / 16 * 16 * M;
+        pl.xreg = 0;
+        if (!prep && cols <= 8) {
+            if (units <= 32 * (FORM == 0 ? 2 : 1)) pl.xreg = M == 1 ? (p.ragged ? 1 : 2) : 3;
+            else if (FORM == 0 && !p.ragged && units <= 128) pl.xreg = 4;
+        }
+        if (!prep && M > 1 && pl.xreg == 0) return false;
         return true;
     }
     return false;
@@ -785,9 +831,13 @@ cudaError_t launch_stream_form(StreamParams p, cudaStream_t s) {
     }
     if constexpr (!PREP) {
         if (pl.xreg) {
-            if (pl.nt == 1)
+            if (pl.nt == 1) {
+                if constexpr (FORM == 0)
+                    if (pl.xreg == 4) return launch_stream<FORM, 1, 0, 4>(tm_main, tm_tail, p, pl, s);
+                if (pl.xreg == 3) return launch_stream<FORM, 1, 0, 3>(tm_main, tm_tail, p, pl, s);
                 return pl.xreg == 2 ? launch_stream<FORM, 1, 0, 2>(tm_main, tm_tail, p, pl, s)
                                     : launch_stream<FORM, 1, 0, 1>(tm_main, tm_tail, p, pl, s);
+            }
             return cudaErrorInvalidConfiguration;  // M == 1 always has one column tile
         }
     }

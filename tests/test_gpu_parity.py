@@ -361,3 +361,31 @@ def test_decode_all_token_counts_fused(blw, oref):
         torch.cuda.synchronize()
         _, acc_ref = oref.ternary_linear(x.numpy(), w2, 0.02)
         assert np.array_equal(acc.cpu().numpy(), acc_ref), M
+
+
+@pytest.mark.parametrize("M,K,N", [(2, 4096, 272), (3, 4096, 272), (5, 4096, 48), (8, 4096, 4096),
+                                   (4, 2048, 64), (8, 1024, 96), (2, 11008, 64)])
+def test_decode_warp_local_multi_token(blw, oref, M, K, N):
+    """Small-M calls whose activations each warp prepares for exactly the
+    k-steps it contracts (up to four token/group units per lane; K = 2048 and
+    1024 leave warps that own no step)."""
+    x = synth.activations(M, K, seed=400 + M + K, outlier_frac=0.01)
+    w2 = oref.pack_ternary(synth.ternary_weights(N, K, seed=401 + M).numpy())
+    y, acc = blw.bl_ternary_linear(x.cuda(), torch.from_numpy(w2.view(np.int32)).cuda(), 0.02,
+                                   return_acc=True)
+    torch.cuda.synchronize()
+    y_ref, acc_ref = oref.ternary_linear(x.numpy(), w2, 0.02)
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert np.array_equal(y.cpu().numpy().view(np.uint16), y_ref.view(np.uint16))
+
+
+@pytest.mark.parametrize("M,K,N", [(2, 4096, 48), (2, 384, 32), (1, 8192, 64), (2, 11008, 32)])
+def test_onebit_decode_warp_local_two_tokens(blw, oref, M, K, N):
+    """OneBit at M <= 2 with warp-local preparation (partial last step for
+    K = 384 and 11008)."""
+    x, ws, g, h = _onebit_inputs(M, K, N, seed=420 + M + K)
+    s1 = oref.pack_sign(ws.numpy())
+    y = blw.ob_linear(x.cuda(), torch.from_numpy(s1.view(np.int32)).cuda(), g.cuda(), h.cuda())
+    torch.cuda.synchronize()
+    _, z_ref = oref.ob_linear(x.numpy(), s1, g.numpy(), h.numpy())
+    assert _rel_err(y.cpu().numpy(), z_ref) <= OB_TOL
