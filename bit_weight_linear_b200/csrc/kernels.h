@@ -114,7 +114,7 @@ constexpr int kFusedMaxM = 2;
 constexpr int kStreamFusedMaxM = 8;
 
 // Token counts at or above which the tensor-core prefill kernel is used.
-constexpr int kTernaryPrefillMinM = 33;
-constexpr int kOnebitPrefillMinM = 17;
+constexpr int kTernaryPrefillMinM = 17;
+constexpr int kOnebitPrefillMinM = 9;
 
 }  // namespace bl

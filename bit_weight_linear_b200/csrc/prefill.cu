@@ -44,21 +44,29 @@ namespace {
 
 constexpr int BW = 128;          // weight rows per tile (MMA M)
 constexpr int BT = 256;          // max activation rows per tile (MMA N); per call bt <= BT
-constexpr int BK = 128;          // k per stage (bytes of int8 per activation row)
-constexpr int SS = 5;            // shared-memory ring stages
-constexpr int SU = 4;            // TMEM slots for expanded weights
+constexpr int BK = 128;          // k per block (bytes of int8 per activation row)
 constexpr int kThreads = 192;
-constexpr int ACT_STAGE = BT * BK;        // 32 KB
-constexpr int BP_STAGE = BW * BK / 4;     // 4 KB (ternary); sign uses half
-constexpr int OFF_ACT = 0;
-constexpr int OFF_BP = OFF_ACT + SS * ACT_STAGE;
-constexpr int OFF_TOK = OFF_BP + SS * BP_STAGE;          // per-token scale / row sum [BT]
-constexpr int OFF_BAR = OFF_TOK + 2 * BT * 4;
-constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;         // barriers + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t kAccCol = 0;          // accumulator: columns [0, 256)
-constexpr uint32_t kWCol = 256;          // expanded-weight slots: 32 columns each
+constexpr uint32_t kWCol = 256;          // expanded-weight slots: columns [256, 512)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
+
+// A ring stage carries KB consecutive 128-k blocks: KB = 1 for 256-row activation
+// tiles, 2 for <= 128 rows, 4 for <= 64 rows.  The activation part of a stage
+// stays 32 KB, so small token counts still move enough bytes per stage to keep
+// the SM's copy pipeline full.
+template <int KB>
+struct PS {
+    static constexpr int SS = KB == 1 ? 5 : 4;             // shared-memory ring stages
+    static constexpr int SU = KB == 1 ? 4 : 8 / KB;        // TMEM weight slots (32*KB columns each)
+    static constexpr int ACT_STAGE = BT * BK;              // 32 KB: KB blocks of bt <= BT/KB rows
+    static constexpr int BP_STAGE = BW * BK / 4 * KB;      // packed weights (ternary; sign uses half)
+    static constexpr int OFF_ACT = 0;
+    static constexpr int OFF_BP = OFF_ACT + SS * ACT_STAGE;
+    static constexpr int OFF_TOK = OFF_BP + SS * BP_STAGE;  // per-token scale / row sum [BT]
+    static constexpr int OFF_BAR = OFF_TOK + 2 * BT * 4;
+    static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
+};
 
 template <int FORM>
 struct PF;
@@ -84,10 +92,14 @@ struct PrefillParams {
     unsigned int* flags;
 };
 
-template <int FORM>
+template <int FORM, int KB>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_act,
                    const __grid_constant__ CUtensorMap tmap_w, const PrefillParams p) {
+    using L = PS<KB>;
+    constexpr int SS = L::SS, SU = L::SU, ACT_STAGE = L::ACT_STAGE, BP_STAGE = L::BP_STAGE;
+    constexpr int OFF_ACT = L::OFF_ACT, OFF_BP = L::OFF_BP, OFF_TOK = L::OFF_TOK, OFF_BAR = L::OFF_BAR;
+    constexpr int kRowBytes = PF<FORM>::kPackedRowBytes * KB;  // packed bytes of a row per stage
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -104,8 +116,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ttiles = (p.rows_a + bt - 1) / bt;
     const int t0 = (blockIdx.x % ttiles) * bt;   // first activation row of the tile
     const int n0 = (blockIdx.x / ttiles) * BW;   // first weight row of the tile
-    const int nk = p.K / BK;
-    const uint32_t kTx = (uint32_t)(bt * BK + PF<FORM>::kPackedRowBytes * BW);
+    const int nblk = p.K / BK;                 // 128-k blocks
+    const int nk = (nblk + KB - 1) / KB;       // stages; the last may hold fewer blocks
+    // blocks in stage kb; the weight box of a short last stage runs past the row
+    // end and is zero-filled (codes 0 expand to 0, so those products vanish)
+    auto blocks = [&](int kb) { return KB == 1 ? 1 : min(KB, nblk - kb * KB); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SS; ++s) {
@@ -139,11 +154,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (kb >= SS)
                     ok = tc::mbar_wait(bar_empty + 8 * s, ((kb / SS) - 1) & 1, p.flags, kWaitLimitNs);
                 if (!ok) break;
-                tc::mbar_arrive_expect_tx(bar_full + 8 * s, kTx);
-                tc::tma_load_2d(sbase + OFF_ACT + s * ACT_STAGE, &tmap_act, kb * BK, t0,
+                const int nb = blocks(kb);
+                tc::mbar_arrive_expect_tx(bar_full + 8 * s,
+                                          (uint32_t)(nb * bt * BK + kRowBytes * BW));
+                for (int b = 0; b < nb; ++b)
+                    tc::tma_load_2d(sbase + OFF_ACT + s * ACT_STAGE + b * bt * BK, &tmap_act,
+                                    (kb * KB + b) * BK, t0, bar_full + 8 * s);
+                tc::tma_load_2d(sbase + OFF_BP + s * BP_STAGE, &tmap_w, kb * kRowBytes, n0,
                                 bar_full + 8 * s);
-                tc::tma_load_2d(sbase + OFF_BP + s * BP_STAGE, &tmap_w,
-                                kb * PF<FORM>::kPackedRowBytes, n0, bar_full + 8 * s);
                 ++issued;
             }
             if (!ok) {
@@ -163,10 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 tc::tc_fence_after();
                 const uint32_t act_s = sbase + OFF_ACT + s * ACT_STAGE;
+                const int nj = 4 * blocks(kb);
 #pragma unroll
-                for (int j = 0; j < BK / 32; ++j)
-                    tc::mma_i8_ts(tmem + kAccCol, tmem + kWCol + 32 * u + 8 * j,
-                                  tc::desc_kmajor_sw128(act_s + 32 * j), idesc, kb > 0 || j > 0);
+                for (int j = 0; j < KB * BK / 32; ++j)
+                    if (j < nj)
+                    tc::mma_i8_ts(tmem + kAccCol, tmem + kWCol + 32 * KB * u + 8 * j,
+                                  tc::desc_kmajor_sw128(act_s + (j >> 2) * bt * BK + 32 * (j & 3)),
+                                  idesc, kb > 0 || j > 0);
                 tc::mma_commit(bar_empty + 8 * s);
                 tc::mma_commit(bar_uempty + 8 * u);
             }
@@ -187,25 +208,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = tc::mbar_wait(bar_uempty + 8 * u, ((kb / SU) - 1) & 1, p.flags, kWaitLimitNs);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
-            const uint8_t* bp = smem + OFF_BP + s * BP_STAGE;
-            uint32_t e[32];
-            if (FORM == 0) {
-                const uint4 w0 = *reinterpret_cast<const uint4*>(bp + r * 32);
-                const uint4 w1 = *reinterpret_cast<const uint4*>(bp + r * 32 + 16);
-                const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-                for (int o = 0; o < 8; ++o)
+            for (int b = 0; b < KB; ++b) {
+                const uint8_t* bp = smem + OFF_BP + s * BP_STAGE + r * kRowBytes +
+                                    b * PF<FORM>::kPackedRowBytes;
+                uint32_t e[32];
+                if (FORM == 0) {
+                    const uint4 w0 = *reinterpret_cast<const uint4*>(bp);
+                    const uint4 w1 = *reinterpret_cast<const uint4*>(bp + 16);
+                    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) e[4 * o + j] = (ws[o] >> (2 * j)) & 0x03030303u;
-            } else {
-                const uint4 w0 = *reinterpret_cast<const uint4*>(bp + r * 16);
-                const uint32_t ws[4] = {w0.x, w0.y, w0.z, w0.w};
+                    for (int o = 0; o < 8; ++o)
 #pragma unroll
-                for (int o = 0; o < 4; ++o)
+                        for (int j = 0; j < 4; ++j) e[4 * o + j] = (ws[o] >> (2 * j)) & 0x03030303u;
+                } else {
+                    const uint4 w0 = *reinterpret_cast<const uint4*>(bp);
+                    const uint32_t ws[4] = {w0.x, w0.y, w0.z, w0.w};
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) e[8 * o + j] = (ws[o] >> j) & 0x01010101u;
+                    for (int o = 0; o < 4; ++o)
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) e[8 * o + j] = (ws[o] >> j) & 0x01010101u;
+                }
+                tc::tmem_st_32x32b_x32(lane_base + kWCol + 32 * KB * u + 32 * b, e);
             }
-            tc::tmem_st_32x32b_x32(lane_base + kWCol + 32 * u, e);
             tc::tmem_st_wait();
             tc::tc_fence_before();
             tc::mbar_arrive(bar_ufull + 8 * u);
@@ -287,17 +312,16 @@ inline int choose_bt(int rows_a) {
     return r < BT ? r : BT;
 }
 
-template <int FORM>
-cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, PrefillParams p,
-                           cudaStream_t s) {
-    p.bt = choose_bt(p.rows_a);
+template <int FORM, int KB>
+cudaError_t launch_prefill_kb(const int8_t* act, const uint32_t* w, PrefillParams p,
+                              cudaStream_t s) {
+    constexpr int smem = PS<KB>::SMEM_BYTES;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_kernel<FORM>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(prefill_kernel<FORM, KB>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        e = use_max_shared_carveout(prefill_kernel<FORM>);
+        e = use_max_shared_carveout(prefill_kernel<FORM, KB>);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -306,12 +330,21 @@ cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, PrefillParams p
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     const uint64_t prow = (uint64_t)p.K / (FORM == 0 ? 4 : 8);
-    if (!make_tmap(&tw, w, (uint64_t)p.N, prow, PF<FORM>::kPackedRowBytes, BW,
+    if (!make_tmap(&tw, w, (uint64_t)p.N, prow, PF<FORM>::kPackedRowBytes * KB, BW,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     const int tiles = ((p.N + BW - 1) / BW) * ((p.rows_a + p.bt - 1) / p.bt);
-    prefill_kernel<FORM><<<tiles, kThreads, SMEM_BYTES, s>>>(ta, tw, p);
+    prefill_kernel<FORM, KB><<<tiles, kThreads, smem, s>>>(ta, tw, p);
     return cudaGetLastError();
+}
+
+template <int FORM>
+cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, PrefillParams p,
+                           cudaStream_t s) {
+    p.bt = choose_bt(p.rows_a);
+    if (p.bt <= BT / 4) return launch_prefill_kb<FORM, 4>(act, w, p, s);
+    if (p.bt <= BT / 2) return launch_prefill_kb<FORM, 2>(act, w, p, s);
+    return launch_prefill_kb<FORM, 1>(act, w, p, s);
 }
 
 }  // namespace

@@ -203,7 +203,9 @@ def test_ob_linear_zero_token(blw):
 # ------------------------------------------------- tensor-core prefill ------
 
 PREFILL_TERNARY = [(33, 128, 16), (128, 4096, 512), (200, 384, 272), (512, 1024, 1024),
-                   (77, 11008, 256), (300, 640, 48)]
+                   (77, 11008, 256), (300, 640, 48),
+                   # 4 and 2 k-blocks per stage with a short last stage (9 and 15 blocks)
+                   (40, 1152, 96), (100, 1920, 128)]
 
 
 @pytest.mark.parametrize("M,K,N", PREFILL_TERNARY)
@@ -222,7 +224,8 @@ def test_ternary_prefill_parity(blw, oref, M, K, N):
     assert np.array_equal(yg.view(np.uint16), y_ref.view(np.uint16))
 
 
-PREFILL_ONEBIT = [(17, 128, 16), (64, 4096, 512), (150, 640, 272), (256, 1024, 1024)]
+PREFILL_ONEBIT = [(17, 128, 16), (64, 4096, 512), (150, 640, 272), (256, 1024, 1024),
+                  (40, 640, 64)]
 
 
 @pytest.mark.parametrize("M,K,N", PREFILL_ONEBIT)
