@@ -392,3 +392,29 @@ def test_onebit_decode_warp_local_two_tokens(blw, oref, M, K, N):
     torch.cuda.synchronize()
     _, z_ref = oref.ob_linear(x.numpy(), s1, g.numpy(), h.numpy())
     assert _rel_err(y.cpu().numpy(), z_ref) <= OB_TOL
+
+
+@pytest.mark.parametrize("M", [1, 4, 12, 20])
+def test_quant_two_step_rounding_on_every_path(blw, oref, M):
+    """x = amax/2 whose fp32 product with rn(127/amax) is exactly 63.5 (the exact
+    product is just below it): every activation path must round the fp32 product,
+    giving 64, like the oracle (M = 1 and 4: in-kernel warp-local preparation;
+    12: the activation kernel; 20: the activation kernel before the tensor-core GEMM)."""
+    K, N = 4096, 64
+    x = synth.activations(M, K, seed=500 + M)
+    amax = np.float16(4.6328125)
+    x[:, :] = torch.clamp(x, -4.5, 4.5)
+    x[:, 7] = float(amax)
+    x[:, 100] = float(np.float16(amax / 2))
+    x[:, 2049] = -float(np.float16(amax / 2))
+    w2 = oref.pack_ternary(synth.ternary_weights(N, K, seed=501).numpy())
+    y, acc = blw.bl_ternary_linear(x.cuda(), torch.from_numpy(w2.view(np.int32)).cuda(), 0.02,
+                                   return_acc=True)
+    torch.cuda.synchronize()
+    q_ref, _ = oref.quant_act(x.numpy())
+    assert q_ref[0, 100] == 64 and q_ref[0, 2049] == -64
+    _, acc_ref = oref.ternary_linear(x.numpy(), w2, 0.02)
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    q, s = blw.bl_quant_act(x.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), q_ref)

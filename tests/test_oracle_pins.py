@@ -169,6 +169,25 @@ def test_act_quant_invariants(oref):
     assert q[6, 17] == -127
 
 
+def test_act_quant_rounds_fp32_product_then_to_integer(oref):
+    """q = rne(fp32(x * fp32(127/amax))): the product is rounded to fp32 first
+    (the reading of the BitNet b1.58 page's quantiser: scale by the fp32 inverse,
+    then round half to even).  For amax = 4.6328125 and x = amax/2 the exact
+    product 127/2 * (1 + delta) lies just below 63.5, rounds to 63.5 in fp32 and
+    then to 64; a single rounding of the exact product would give 63."""
+    amax = np.float16(4.6328125)
+    x = np.zeros((1, 16), dtype=np.float16)
+    x[0, 0] = amax
+    x[0, 3] = np.float16(amax / 2)
+    x[0, 9] = np.float16(-amax / 2)
+    inv = np.float32(127.0) / np.float32(amax)
+    exact = float(np.float64(x[0, 3]) * np.float64(inv))
+    assert 63.49 < exact < 63.5                        # below the tie in exact arithmetic
+    assert np.float32(np.float32(x[0, 3]) * inv) == np.float32(63.5)
+    q, s = oref.quant_act(x)
+    assert q[0, 0] == 127 and q[0, 3] == 64 and q[0, 9] == -64
+
+
 # ------------------------------------------------- ternary contraction -----
 
 def _bitlinear_case(oref, M, K, N, seed, w=None):
