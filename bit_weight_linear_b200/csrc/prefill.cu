@@ -104,12 +104,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = tc::smem_u32(smem);
-    const uint32_t bar_full = sbase + OFF_BAR;        // activation + packed tile landed [SS]
-    const uint32_t bar_empty = bar_full + 8 * SS;     // MMA done with the stage        [SS]
+    const uint32_t bar_full = sbase + OFF_BAR;        // activation tile landed         [SS]
+    const uint32_t bar_wfull = bar_full + 8 * SS;     // packed weight tile landed      [SS]
+    const uint32_t bar_empty = bar_wfull + 8 * SS;    // MMA done with the stage        [SS]
     const uint32_t bar_ufull = bar_empty + 8 * SS;    // expanded weights in TMEM      [SU]
     const uint32_t bar_uempty = bar_ufull + 8 * SU;   // MMA done with a TMEM slot     [SU]
     const uint32_t bar_acc = bar_uempty + 8 * SU;     // accumulator complete
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * (2 * SS + 2 * SU + 1));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * (3 * SS + 2 * SU + 1));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bt = p.bt;
@@ -125,6 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < SS; ++s) {
             tc::mbar_init(bar_full + 8 * s, 1);
+            tc::mbar_init(bar_wfull + 8 * s, 1);
             tc::mbar_init(bar_empty + 8 * s, 1);
         }
         for (int u = 0; u < SU; ++u) {
@@ -147,27 +149,42 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            int issued = 0;
+            // The packed weights are call parameters, not written by the kernel
+            // this launch may overlap (programmatic dependent launch): the first
+            // ring of weight tiles is requested before waiting for the producer
+            // of the activations, so the expansion warps can start early.
+            const int pre = nk < SS ? nk : SS;
+            int wissued = 0, issued = 0;
+            for (; wissued < pre; ++wissued) {
+                tc::mbar_arrive_expect_tx(bar_wfull + 8 * wissued, (uint32_t)(kRowBytes * BW));
+                tc::tma_load_2d(sbase + OFF_BP + wissued * BP_STAGE, &tmap_w,
+                                wissued * kRowBytes, n0, bar_wfull + 8 * wissued);
+            }
+            tc::pdl_wait();
             bool ok = true;
             for (int kb = 0; kb < nk && ok; ++kb) {
                 const int s = kb % SS;
-                if (kb >= SS)
+                if (kb >= SS) {
                     ok = tc::mbar_wait(bar_empty + 8 * s, ((kb / SS) - 1) & 1, p.flags, kWaitLimitNs);
-                if (!ok) break;
+                    if (!ok) break;
+                    tc::mbar_arrive_expect_tx(bar_wfull + 8 * s, (uint32_t)(kRowBytes * BW));
+                    tc::tma_load_2d(sbase + OFF_BP + s * BP_STAGE, &tmap_w, kb * kRowBytes, n0,
+                                    bar_wfull + 8 * s);
+                    ++wissued;
+                }
                 const int nb = blocks(kb);
-                tc::mbar_arrive_expect_tx(bar_full + 8 * s,
-                                          (uint32_t)(nb * bt * BK + kRowBytes * BW));
+                tc::mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)(nb * bt * BK));
                 for (int b = 0; b < nb; ++b)
                     tc::tma_load_2d(sbase + OFF_ACT + s * ACT_STAGE + b * bt * BK, &tmap_act,
                                     (kb * KB + b) * BK, t0, bar_full + 8 * s);
-                tc::tma_load_2d(sbase + OFF_BP + s * BP_STAGE, &tmap_w, kb * kRowBytes, n0,
-                                bar_full + 8 * s);
                 ++issued;
             }
             if (!ok) {
                 // drain copies still in flight before the CTA's shared memory goes away
                 for (int kb = (issued > SS ? issued - SS : 0); kb < issued; ++kb)
                     tc::mbar_wait(bar_full + 8 * (kb % SS), (kb / SS) & 1, p.flags, kWaitLimitNs);
+                for (int kb = (wissued > SS ? wissued - SS : 0); kb < wissued; ++kb)
+                    tc::mbar_wait(bar_wfull + 8 * (kb % SS), (kb / SS) & 1, p.flags, kWaitLimitNs);
             }
         }
     } else if (warp == 1) {
@@ -191,6 +208,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::mma_commit(bar_empty + 8 * s);
                 tc::mma_commit(bar_uempty + 8 * u);
             }
+            // the next kernel on the stream may start launching now; it waits for
+            // this grid's completion before touching anything this grid writes
+            tc::pdl_trigger();
             // completion of everything issued (also on the abort path)
             tc::mma_commit(bar_acc);
             tc::mbar_wait(bar_acc, 0, p.flags, kWaitLimitNs);
@@ -203,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int kb = 0; kb < nk && ok; ++kb) {
             const int s = kb % SS, u = kb % SU;
-            ok = tc::mbar_wait(bar_full + 8 * s, (kb / SS) & 1, p.flags, kWaitLimitNs);
+            ok = tc::mbar_wait(bar_wfull + 8 * s, (kb / SS) & 1, p.flags, kWaitLimitNs);
             if (ok && kb >= SU)
                 ok = tc::mbar_wait(bar_uempty + 8 * u, ((kb / SU) - 1) & 1, p.flags, kWaitLimitNs);
             ok = __all_sync(0xffffffffu, ok);
@@ -241,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* tok_scale = reinterpret_cast<float*>(smem + OFF_TOK);
         int* tok_rsum = reinterpret_cast<int*>(tok_scale + BT);
         const int et = threadIdx.x - 64;        // 0..127
+        tc::pdl_wait();                          // scale / row sums come from the previous kernel
         for (int i = et; i < bt; i += 128) {
             const int row = t0 + i;
             const int tok = FORM == 0 ? row : row >> 1;
@@ -334,8 +355,17 @@ cudaError_t launch_prefill_kb(const int8_t* act, const uint32_t* w, PrefillParam
                    CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     const int tiles = ((p.N + BW - 1) / BW) * ((p.rows_a + p.bt - 1) / p.bt);
-    prefill_kernel<FORM, KB><<<tiles, kThreads, smem, s>>>(ta, tw, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(tiles);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attrs[1];
+    attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<FORM, KB>, ta, tw, p);
 }
 
 template <int FORM>

@@ -123,6 +123,110 @@ __global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t* __r
     if (threadIdx.x == 0) scale[m] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
 }
 
+// Register-resident variant: a 512-thread CTA per token loads the whole token
+// into registers (NCH 16-element chunks per thread, all loads in flight at
+// once), takes amax, then quantises from registers.  One read of x instead of
+// two, and no loop-carried load latency; used while K <= 16 * 512 * 8.
+constexpr int kRegThreads = 512;
+constexpr int kRegMaxChunks = 8;
+
+template <int NW>
+__device__ __forceinline__ uint32_t block_max_u32_n(uint32_t v, uint32_t* red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    uint32_t r = red[lane < NW ? lane : 0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) r = max(r, __shfl_xor_sync(0xffffffffu, r, o));
+    return r;
+}
+
+template <int NW>
+__device__ __forceinline__ int block_sum_i32_n(int v, int* red) {
+    v = warp_sum(v);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    return warp_sum(lane < NW ? red[lane] : 0);
+}
+
+template <int LAYOUT, int NCH>
+__global__ void __launch_bounds__(kRegThreads, NCH <= 4 ? 2 : 1)
+    quant_act_reg_kernel(const uint16_t* __restrict__ x, int K, int8_t* __restrict__ q,
+                         float* __restrict__ scale, int32_t* __restrict__ qsum) {
+    constexpr int NW = kRegThreads / 32;
+    __shared__ uint32_t redu[NW];
+    __shared__ int redi[NW];
+    const int m = blockIdx.x;
+    const int nc = K / 16;
+    const uint16_t* row = x + (size_t)m * K;
+    tc::pdl_trigger();
+    tc::pdl_wait();
+
+    uint4 va[NCH], vb[NCH];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+        const int c = threadIdx.x + i * kRegThreads;
+        if (c < nc) {
+            va[i] = tc::ld_v4(row + 16 * c);
+            vb[i] = tc::ld_v4(row + 16 * c + 8);
+        } else {
+            va[i] = make_uint4(0, 0, 0, 0);
+            vb[i] = va[i];
+        }
+    }
+    uint32_t mx = 0;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+        mx = __vmaxu2(mx, va[i].x & 0x7fff7fffu);
+        mx = __vmaxu2(mx, va[i].y & 0x7fff7fffu);
+        mx = __vmaxu2(mx, va[i].z & 0x7fff7fffu);
+        mx = __vmaxu2(mx, va[i].w & 0x7fff7fffu);
+        mx = __vmaxu2(mx, vb[i].x & 0x7fff7fffu);
+        mx = __vmaxu2(mx, vb[i].y & 0x7fff7fffu);
+        mx = __vmaxu2(mx, vb[i].z & 0x7fff7fffu);
+        mx = __vmaxu2(mx, vb[i].w & 0x7fff7fffu);
+    }
+    mx = max(mx & 0xffffu, mx >> 16);
+    const float amax = half_bits_to_float(block_max_u32_n<NW>(mx, redu));
+    const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+
+    int sum = 0;
+    int8_t* qrow = q + (size_t)m * K;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+        const int c = threadIdx.x + i * kRegThreads;
+        if (c >= nc) break;
+        const uint32_t hv[8] = {va[i].x, va[i].y, va[i].z, va[i].w,
+                                vb[i].x, vb[i].y, vb[i].z, vb[i].w};
+        int qv[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            qv[e] = quant127(half_bits_to_float(hv[e >> 1] >> (16 * (e & 1))), inv);
+            sum += qv[e];
+        }
+        uint32_t out[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t wv = 0;
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                const int src = LAYOUT == 0 ? 4 * j + bb : 4 * bb + j;
+                wv |= ((uint32_t)qv[src] & 0xffu) << (8 * bb);
+            }
+            out[j] = wv;
+        }
+        *reinterpret_cast<uint4*>(qrow + 16 * c) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+    if (LAYOUT == 1) {
+        const int tot = block_sum_i32_n<NW>(sum, redi);
+        if (threadIdx.x == 0) qsum[m] = tot;
+    }
+    if (threadIdx.x == 0) scale[m] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
+}
+
 constexpr int kFixMax = 32639;  // |X| <= 32639 keeps hi = floor((X+128)/256) in int8
 
 __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* __restrict__ x,
@@ -202,7 +306,7 @@ __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* _
     }
 }
 
-template <auto KERN, typename... Args>
+template <auto KERN, int THREADS = kThreads, typename... Args>
 cudaError_t launch_pdl(int blocks, cudaStream_t s, Args... args) {
     static bool attr_set = false;  // one flag per kernel
     if (!attr_set) {
@@ -212,7 +316,7 @@ cudaError_t launch_pdl(int blocks, cudaStream_t s, Args... args) {
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(blocks);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(THREADS);
     cfg.stream = s;
     cudaLaunchAttribute attrs[1];
     attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -222,18 +326,38 @@ cudaError_t launch_pdl(int blocks, cudaStream_t s, Args... args) {
     return cudaLaunchKernelEx(&cfg, KERN, args...);
 }
 
+// chunks of 16 elements per thread for the register-resident kernel, 0 = too long
+inline int reg_chunks(int K) {
+    const int need = (K / 16 + kRegThreads - 1) / kRegThreads;
+    for (int c = 1; c <= kRegMaxChunks; c *= 2)
+        if (need <= c) return c;
+    return 0;
+}
+
+template <int LAYOUT>
+cudaError_t launch_quant(const uint16_t* x, int M, int K, int8_t* q, float* scale,
+                         int32_t* qsum, cudaStream_t s) {
+    switch (reg_chunks(K)) {
+        case 1: return launch_pdl<quant_act_reg_kernel<LAYOUT, 1>, kRegThreads>(M, s, x, K, q, scale, qsum);
+        case 2: return launch_pdl<quant_act_reg_kernel<LAYOUT, 2>, kRegThreads>(M, s, x, K, q, scale, qsum);
+        case 4: return launch_pdl<quant_act_reg_kernel<LAYOUT, 4>, kRegThreads>(M, s, x, K, q, scale, qsum);
+        case 8: return launch_pdl<quant_act_reg_kernel<LAYOUT, 8>, kRegThreads>(M, s, x, K, q, scale, qsum);
+        default: return launch_pdl<quant_act_kernel<LAYOUT>>(M, s, x, K, q, scale, qsum);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_quant_plain(const uint16_t* x, int M, int K, int8_t* q, float* scale,
                                cudaStream_t s) {
     if (M == 0) return cudaSuccess;
-    return launch_pdl<quant_act_kernel<0>>(M, s, x, K, q, scale, (int32_t*)nullptr);
+    return launch_quant<0>(x, M, K, q, scale, (int32_t*)nullptr, s);
 }
 
 cudaError_t launch_quant_ternary_perm(const uint16_t* x, int M, int K, int8_t* qp,
                                       float* scale, int32_t* qsum, cudaStream_t s) {
     if (M == 0) return cudaSuccess;
-    return launch_pdl<quant_act_kernel<1>>(M, s, x, K, qp, scale, qsum);
+    return launch_quant<1>(x, M, K, qp, scale, qsum, s);
 }
 
 cudaError_t launch_prep_onebit(const uint16_t* x, const uint16_t* g, int M, int K,
