@@ -95,7 +95,8 @@ struct PrefillParams {
 template <int FORM, int KB>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_act,
-                   const __grid_constant__ CUtensorMap tmap_w, const PrefillParams p) {
+                   const __grid_constant__ CUtensorMap tmap_w,
+                   const __grid_constant__ CUtensorMap tmap_y, const PrefillParams p) {
     using L = PS<KB>;
     constexpr int SS = L::SS, SU = L::SU, ACT_STAGE = L::ACT_STAGE, BP_STAGE = L::BP_STAGE;
     constexpr int OFF_ACT = L::OFF_ACT, OFF_BP = L::OFF_BP, OFF_TOK = L::OFF_TOK, OFF_BAR = L::OFF_BAR;
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_fence_init();
         tc::prefetch_tmap(&tmap_act);
         tc::prefetch_tmap(&tmap_w);
+        tc::prefetch_tmap(&tmap_y);
     }
     if (warp == 1) {
         tc::tmem_alloc(tc::smem_u32(tmem_slot), TMEM_COLS);
@@ -269,41 +271,55 @@ __global__ void __launch_bounds__(kThreads, 1)
             tok_scale[i] = in ? p.scale[tok] : 0.f;
             tok_rsum[i] = in ? p.rsum[tok] : 0;
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");   // the four epilogue warps only
-        const bool acc_ok =
-            __all_sync(0xffffffffu, tc::mbar_wait(bar_acc, 0, p.flags, kWaitLimitNs));
+        const bool acc_ok = tc::mbar_wait(bar_acc, 0, p.flags, kWaitLimitNs);
+        // one decision for the four epilogue warps; also publishes the token table
+        const bool good = tc::bar_and(1, 128, ok && acc_ok);
         tc::tc_fence_after();
-        const int n = n0 + r;                    // output column held by this thread
-        if (ok && acc_ok) {
+        if (good) {
+            // The fp16 tile is staged in the (now idle) activation ring as
+            // [token][128 columns] and leaves with one tensor store, which also
+            // drops the rows past M and the columns past N.
+            uint16_t* stage = reinterpret_cast<uint16_t*>(smem + OFF_ACT);
+            const int n = n0 + r;                // output column held by this thread
             const float hn = (FORM == 1 && n < p.N) ? __half2float(__ushort_as_half(p.h[n])) : 0.f;
 #pragma unroll 1
             for (int cc = 0; cc < bt / 32; ++cc) {
                 uint32_t d[32];
                 tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * cc, d);
                 tc::tmem_ld_wait();
-                if (n >= p.N) continue;
                 if (FORM == 0) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int ti = 32 * cc + i, m = t0 + ti;
-                        if (m < p.M) {
-                            const int a = (int)d[i] - tok_rsum[ti];
-                            const float v = __fmul_rn(__fmul_rn((float)a, tok_scale[ti]), p.w_scale);
-                            p.y[(size_t)m * p.N + n] = __half_as_ushort(__float2half_rn(v));
-                            if (p.acc_out) p.acc_out[(size_t)m * p.N + n] = a;
+                    for (int i4 = 0; i4 < 32; i4 += 4) {
+                        const int tb = 32 * cc + i4;
+                        const float4 sc = *reinterpret_cast<const float4*>(tok_scale + tb);
+                        const int4 rs = *reinterpret_cast<const int4*>(tok_rsum + tb);
+                        const float scs[4] = {sc.x, sc.y, sc.z, sc.w};
+                        const int rss[4] = {rs.x, rs.y, rs.z, rs.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int a = (int)d[i4 + j] - rss[j];
+                            const float v = __fmul_rn(__fmul_rn((float)a, scs[j]), p.w_scale);
+                            stage[(tb + j) * BW + r] = __half_as_ushort(__float2half_rn(v));
+                            const int m = t0 + tb + j;
+                            if (p.acc_out && m < p.M && n < p.N) p.acc_out[(size_t)m * p.N + n] = a;
                         }
                     }
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
-                        const int ti = 32 * cc + i, tok = (t0 + ti) >> 1;
-                        if (tok < p.M) {
-                            const long long P = 256ll * (int)d[i] + (int)d[i + 1];
-                            const float z = __fmul_rn(tok_scale[ti], (float)(2 * P - (long long)tok_rsum[ti]));
-                            p.y[(size_t)tok * p.N + n] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hn)));
-                        }
+                        const int ti = 32 * cc + i;
+                        const long long P = 256ll * (int)d[i] + (int)d[i + 1];
+                        const float z = __fmul_rn(tok_scale[ti], (float)(2 * P - (long long)tok_rsum[ti]));
+                        stage[(ti >> 1) * BW + r] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hn)));
                     }
                 }
+            }
+            tc::fence_proxy_async_smem();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (et == 0) {
+                tc::tma_store_2d(&tmap_y, sbase + OFF_ACT, n0 * 2, FORM == 0 ? t0 : t0 >> 1);
+                tc::bulk_commit_group();
+                tc::bulk_wait_group_read0();
             }
         }
     }
@@ -354,6 +370,11 @@ cudaError_t launch_prefill_kb(const int8_t* act, const uint32_t* w, PrefillParam
     if (!make_tmap(&tw, w, (uint64_t)p.N, prow, PF<FORM>::kPackedRowBytes * KB, BW,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
+    // y as bytes: N * 2 per row; one box = 128 columns x the tile's tokens
+    CUtensorMap ty;
+    if (!make_tmap(&ty, p.y, (uint64_t)p.M, (uint64_t)p.N * 2, BW * 2,
+                   (uint32_t)(FORM == 0 ? p.bt : p.bt / 2), CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
     const int tiles = ((p.N + BW - 1) / BW) * ((p.rows_a + p.bt - 1) / p.bt);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles);
@@ -365,7 +386,7 @@ cudaError_t launch_prefill_kb(const int8_t* act, const uint32_t* w, PrefillParam
     attrs[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_kernel<FORM, KB>, ta, tw, p);
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<FORM, KB>, ta, tw, ty, p);
 }
 
 template <int FORM>
