@@ -22,13 +22,19 @@
 // tokens, or token limb rows; bt = the smallest multiple of 32 covering them,
 // at most 256), K in 128-byte stages; tiles ordered
 // activation-tile-fastest so CTAs sharing a weight tile run together.
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0     TMA producer: activation tile (256 x 128 B) and packed weight tile
-//              (128 rows x 32 B or 16 B) into a 5-stage shared-memory ring;
+//              (128 rows x 32 B or 16 B) into a 5-stage shared-memory ring; the
+//              weight tiles have their own full barriers and the first ring of
+//              them is requested before the wait on the previous kernel
+//              (programmatic dependent launch), the activations after it;
 //   warp 1     TMEM allocator + single-thread MMA issuer (4 x K=32 per stage);
-//   warps 2-5  one thread per weight row: unpack into a 4-slot TMEM ring, then
-//              the epilogue (tcgen05.ld -> correction and scale -> fp16), in
-//              which a warp's lanes are 32 consecutive output columns.
+//   warps 2-5  one thread per weight row: unpack into a 4-slot TMEM ring;
+//   warps 2-9  the epilogue (tcgen05.ld -> correction and scale -> fp16), two
+//              warps per TMEM lane quarter taking alternate 32-column chunks; a
+//              warp's lanes are 32 consecutive output columns.  The fp16 tile
+//              is staged in the idle activation ring and leaves by one TMA
+//              tensor store.
 // The expanded byte order inside each 16-byte (ternary) / 32-byte (sign) group
 // is the order the byte-SIMD unpack produces; the activation preparation
 // kernels store the activations in the same order.
@@ -45,7 +51,8 @@ namespace {
 constexpr int BW = 128;          // weight rows per tile (MMA M)
 constexpr int BT = 256;          // max activation rows per tile (MMA N); per call bt <= BT
 constexpr int BK = 128;          // k per block (bytes of int8 per activation row)
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kEpiThreads = kThreads - 64;   // warps 2-9: the epilogue (2-5 also expand)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t kAccCol = 0;          // accumulator: columns [0, 256)
 constexpr uint32_t kWCol = 256;          // expanded-weight slots: columns [256, 512)
@@ -220,10 +227,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------- expand (warps 2-5): thread = weight row = TMEM lane -------
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int hsel = (warp - 2) >> 2;       // 0: warps 2-5, 1: warps 6-9 (epilogue only)
         const int r = 32 * q + lane;            // weight row within the tile
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         bool ok = true;
-        for (int kb = 0; kb < nk && ok; ++kb) {
+        for (int kb = 0; hsel == 0 && kb < nk && ok; ++kb) {
             const int s = kb % SS, u = kb % SU;
             ok = tc::mbar_wait(bar_wfull + 8 * s, (kb / SS) & 1, p.flags, kWaitLimitNs);
             if (ok && kb >= SU)
@@ -262,9 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // per-token scale and row sum of this activation tile, staged once
         float* tok_scale = reinterpret_cast<float*>(smem + OFF_TOK);
         int* tok_rsum = reinterpret_cast<int*>(tok_scale + BT);
-        const int et = threadIdx.x - 64;        // 0..127
+        const int et = threadIdx.x - 64;        // 0..kEpiThreads-1
         tc::pdl_wait();                          // scale / row sums come from the previous kernel
-        for (int i = et; i < bt; i += 128) {
+        for (int i = et; i < bt; i += kEpiThreads) {
             const int row = t0 + i;
             const int tok = FORM == 0 ? row : row >> 1;
             const bool in = FORM == 0 ? row < p.M : tok < p.M;
@@ -272,8 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tok_rsum[i] = in ? p.rsum[tok] : 0;
         }
         const bool acc_ok = tc::mbar_wait(bar_acc, 0, p.flags, kWaitLimitNs);
-        // one decision for the four epilogue warps; also publishes the token table
-        const bool good = tc::bar_and(1, 128, ok && acc_ok);
+        // one decision for the eight epilogue warps; also publishes the token table
+        const bool good = tc::bar_and(1, kEpiThreads, ok && acc_ok);
         tc::tc_fence_after();
         if (good) {
             // The fp16 tile is staged in the (now idle) activation ring as
@@ -283,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n = n0 + r;                // output column held by this thread
             const float hn = (FORM == 1 && n < p.N) ? __half2float(__ushort_as_half(p.h[n])) : 0.f;
 #pragma unroll 1
-            for (int cc = 0; cc < bt / 32; ++cc) {
+            for (int cc = hsel; cc < bt / 32; cc += 2) {
                 uint32_t d[32];
                 tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * cc, d);
                 tc::tmem_ld_wait();
@@ -315,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             tc::fence_proxy_async_smem();
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
             if (et == 0) {
                 tc::tma_store_2d(&tmap_y, sbase + OFF_ACT, n0 * 2, FORM == 0 ? t0 : t0 >> 1);
                 tc::bulk_commit_group();
