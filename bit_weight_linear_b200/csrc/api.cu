@@ -3,6 +3,7 @@
 // caller's.
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "bitlinear.h"
 #include "common.cuh"
@@ -42,18 +43,27 @@ bl_status check_nk(int N, int K) {
 }
 
 // Workspace layouts (offsets in bytes, each region 256-byte aligned):
-//   ternary: [0] permuted q  M*K int8 | scale M fp32 | row sums M int32
-//   onebit : [0] limb planes 2*M*K int8 | step M fp32 | row sums M int32
+//   ternary: [0] permuted q  M*K int8 | scale M fp32 | row sums M int32 | split
+//   onebit : [0] limb planes 2*M*K int8 | step M fp32 | row sums M int32 | split
+// `split` is the prefill kernel's scratch for sharing out its last round
+// (arrival counters + partial accumulators); empty unless the call takes the
+// prefill path and its tiles leave SMs idle in the last round.
 struct WsLayout {
-    size_t act, scale, rsum, total;
+    size_t act, scale, rsum, split, split_bytes, total;
+    int n_ctr;
 };
 
-WsLayout ws_layout(int M, int K, int planes) {
+WsLayout ws_layout(int form, int M, int K, int N) {
     WsLayout l;
     l.act = 0;
-    l.scale = align_up((size_t)M * (size_t)K * (size_t)planes);
+    l.scale = align_up((size_t)M * (size_t)K * (size_t)(form == 0 ? 1 : 2));
     l.rsum = l.scale + align_up((size_t)M * sizeof(float));
-    l.total = l.rsum + align_up((size_t)M * sizeof(int32_t));
+    l.split = l.rsum + align_up((size_t)M * sizeof(int32_t));
+    l.split_bytes = 0;
+    l.n_ctr = 0;
+    const int min_m = form == 0 ? bl::kTernaryPrefillMinM : bl::kOnebitPrefillMinM;
+    if (M >= min_m) l.split_bytes = bl::prefill_split_bytes(form, M, K, N, &l.n_ctr);
+    l.total = l.split + align_up(l.split_bytes);
     return l;
 }
 
@@ -87,6 +97,20 @@ bl_status pack_begin(unsigned int** flag, cudaStream_t s) {
 }  // namespace
 
 unsigned int* bl::device_flags_address() { return device_flags(); }
+
+int bl::device_sm_count() {
+    static std::mutex mu;
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
 
 extern "C" {
 
@@ -138,9 +162,8 @@ bl_status bl_quant_act(const uint16_t* x, int M, int K, int8_t* q, float* scale,
 }
 
 size_t bl_ternary_workspace_bytes(int M, int K, int N) {
-    (void)N;
-    if (check_mk(M, K) != BL_OK) return 0;
-    return ws_layout(M, K, 1).total;
+    if (check_mk(M, K) != BL_OK || check_nk(N, K) != BL_OK) return 0;
+    return ws_layout(0, M, K, N).total;
 }
 
 bl_status bl_ternary_linear(const uint16_t* x, int M, int K, int N, const uint32_t* w2,
@@ -152,7 +175,7 @@ bl_status bl_ternary_linear(const uint16_t* x, int M, int K, int N, const uint32
     if (!x || !w2 || !y) return BL_ERR_NULL;
     if (misaligned(x) || misaligned(w2) || misaligned(y) || misaligned(acc_out))
         return BL_ERR_ALIGN;
-    const WsLayout l = ws_layout(M, K, 1);
+    const WsLayout l = ws_layout(0, M, K, N);
     if (!workspace || workspace_bytes < l.total) return BL_ERR_WORKSPACE;
     if (misaligned(workspace)) return BL_ERR_ALIGN;
     unsigned int* flags = device_flags();
@@ -167,11 +190,12 @@ bl_status bl_ternary_linear(const uint16_t* x, int M, int K, int N, const uint32
     int8_t* qp = reinterpret_cast<int8_t*>(ws + l.act);
     float* sc = reinterpret_cast<float*>(ws + l.scale);
     int32_t* qs = reinterpret_cast<int32_t*>(ws + l.rsum);
-    cudaError_t e = bl::launch_quant_ternary_perm(x, M, K, qp, sc, qs, cs(stream));
+    unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + l.split);
+    cudaError_t e = bl::launch_quant_ternary_perm(x, M, K, qp, sc, qs, cs(stream), ctr, l.n_ctr);
     if (e != cudaSuccess) return BL_ERR_CUDA;
     if (M >= bl::kTernaryPrefillMinM) {
         e = bl::launch_ternary_prefill(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, flags,
-                                       cs(stream));
+                                       cs(stream), ws + l.split, l.split_bytes);
     } else {
         e = bl::stream_fits(0, M, K, N, 1)
                 ? bl::launch_ternary_stream_prepared(qp, sc, qs, w2, M, K, N, w_scale, y, acc_out,
@@ -185,9 +209,8 @@ bl_status bl_ternary_linear(const uint16_t* x, int M, int K, int N, const uint32
 }
 
 size_t ob_workspace_bytes(int M, int K, int N) {
-    (void)N;
-    if (check_mk(M, K) != BL_OK || K > 65536) return 0;
-    return ws_layout(M, K, 2).total;
+    if (check_mk(M, K) != BL_OK || check_nk(N, K) != BL_OK || K > 65536) return 0;
+    return ws_layout(1, M, K, N).total;
 }
 
 bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
@@ -200,7 +223,7 @@ bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
     if (!x || !s1 || !g || !h || !y) return BL_ERR_NULL;
     if (misaligned(x) || misaligned(s1) || misaligned(g) || misaligned(h) || misaligned(y))
         return BL_ERR_ALIGN;
-    const WsLayout l = ws_layout(M, K, 2);
+    const WsLayout l = ws_layout(1, M, K, N);
     if (!workspace || workspace_bytes < l.total) return BL_ERR_WORKSPACE;
     if (misaligned(workspace)) return BL_ERR_ALIGN;
     unsigned int* flags = device_flags();
@@ -213,10 +236,12 @@ bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
     int8_t* planes = reinterpret_cast<int8_t*>(ws + l.act);
     float* step = reinterpret_cast<float*>(ws + l.scale);
     int32_t* ts = reinterpret_cast<int32_t*>(ws + l.rsum);
-    cudaError_t e = bl::launch_prep_onebit(x, g, M, K, planes, step, ts, cs(stream));
+    unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + l.split);
+    cudaError_t e = bl::launch_prep_onebit(x, g, M, K, planes, step, ts, cs(stream), ctr, l.n_ctr);
     if (e != cudaSuccess) return BL_ERR_CUDA;
     if (M >= bl::kOnebitPrefillMinM) {
-        e = bl::launch_onebit_prefill(s1, planes, step, ts, h, M, K, N, y, flags, cs(stream));
+        e = bl::launch_onebit_prefill(s1, planes, step, ts, h, M, K, N, y, flags, cs(stream),
+                                      ws + l.split, l.split_bytes);
     } else {
         e = bl::stream_fits(1, M, K, N, 1)
                 ? bl::launch_onebit_stream_prepared(planes, step, ts, h, s1, M, K, N, y, flags,

@@ -22,10 +22,14 @@ cudaError_t launch_pack_sign(const uint16_t* w, int N, int K, uint32_t* s1,
 //             [M][2][K] (permuted), fixed-point step [M], row sum of the image
 cudaError_t launch_quant_plain(const uint16_t* x, int M, int K, int8_t* q, float* scale,
                                cudaStream_t s);
+// The ternary and onebit preparations also zero `n_zero` words at `zero` (the
+// prefill kernel's arrival counters) once the previous kernel has finished.
 cudaError_t launch_quant_ternary_perm(const uint16_t* x, int M, int K, int8_t* qp,
-                                      float* scale, int32_t* qsum, cudaStream_t s);
+                                      float* scale, int32_t* qsum, cudaStream_t s,
+                                      unsigned int* zero = nullptr, int n_zero = 0);
 cudaError_t launch_prep_onebit(const uint16_t* x, const uint16_t* g, int M, int K,
-                               int8_t* planes, float* step, int32_t* tsum, cudaStream_t s);
+                               int8_t* planes, float* step, int32_t* tsum, cudaStream_t s,
+                               unsigned int* zero = nullptr, int n_zero = 0);
 
 // Decode-shaped (small M) packed-weight kernels on warp-level int8 MMA (skinny.cu).
 cudaError_t launch_ternary_skinny(const uint32_t* w2, const int8_t* qp, const float* scale,
@@ -38,13 +42,24 @@ cudaError_t launch_onebit_skinny(const uint32_t* s1, const int8_t* planes, const
 // Prefill-shaped (large M) GEMM on tcgen05 int8 tensor cores with TMEM
 // accumulators (prefill.cu).  `flags` is the device condition word that bounded
 // waits mark on timeout.
+// When the tiles would leave SMs idle in the last round, the kernel shares
+// that round's work out evenly in k-stages; that needs `split_ws` of
+// prefill_split_bytes() bytes whose first n_counters uint32 are zero at launch
+// (the activation preparation kernel zeroes them).  Without it (NULL or too
+// small) every tile runs whole.
+size_t prefill_split_bytes(int form, int M, int K, int N, int* n_counters);
 cudaError_t launch_ternary_prefill(const uint32_t* w2, const int8_t* qp, const float* scale,
                                    const int32_t* qsum, int M, int K, int N, float w_scale,
                                    uint16_t* y, int32_t* acc_out, unsigned int* flags,
-                                   cudaStream_t s);
+                                   cudaStream_t s, void* split_ws = nullptr,
+                                   size_t split_ws_bytes = 0);
 cudaError_t launch_onebit_prefill(const uint32_t* s1, const int8_t* planes, const float* step,
                                   const int32_t* tsum, const uint16_t* h, int M, int K, int N,
-                                  uint16_t* y, unsigned int* flags, cudaStream_t s);
+                                  uint16_t* y, unsigned int* flags, cudaStream_t s,
+                                  void* split_ws = nullptr, size_t split_ws_bytes = 0);
+
+// Number of SMs of the current device (cached per device; 0 on error).
+int device_sm_count();
 
 // Per-16-row decode (decode.cu): activation preparation + contraction in one
 // kernel, one CTA per 16 weight rows, weights bulk-copied to shared memory

@@ -97,8 +97,17 @@ struct PrefillParams {
     uint16_t* y;
     int32_t* acc_out;
     unsigned int* flags;
+    // Work split.  CTAs [0, dp_tiles) each compute one whole tile.  The
+    // remaining sk_tiles tiles form one balanced round: CTA dp_tiles + c
+    // (c < sk_ctas) takes the (tile, k-stage) units [c U / G, (c+1) U / G) of
+    // them (U = sk_tiles * stages, G = sk_ctas), tile by tile.  A tile split
+    // between CTAs is finished by whichever of them arrives last.
+    int dp_tiles, sk_tiles, sk_ctas;
+    unsigned int* sk_ctr;  // [sk_tiles] arrival counts, zero when the kernel starts
+    int32_t* sk_slots;     // [2 * sk_ctas][bt * BW] partial accumulators
 };
 
+// One whole tile per CTA (launches without a balanced round).
 template <int FORM, int KB>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_act,
@@ -341,6 +350,369 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// The same tile pipeline over a CTA's run of (tile, k-stage) units, used for
+// launches with a balanced round: pieces of tiles, int32 partial slots and
+// per-tile arrival counts (see PrefillParams).  Ring and TMEM-slot phases run
+// on across the pieces of a CTA; the accumulator and the staging area are
+// handed back by two more barriers before the next piece starts.
+template <int FORM, int KB>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_split_kernel(const __grid_constant__ CUtensorMap tmap_act,
+                   const __grid_constant__ CUtensorMap tmap_w,
+                   const __grid_constant__ CUtensorMap tmap_y, const PrefillParams p) {
+    using L = PS<KB>;
+    constexpr int SS = L::SS, SU = L::SU, ACT_STAGE = L::ACT_STAGE, BP_STAGE = L::BP_STAGE;
+    constexpr int OFF_ACT = L::OFF_ACT, OFF_BP = L::OFF_BP, OFF_TOK = L::OFF_TOK, OFF_BAR = L::OFF_BAR;
+    constexpr int kRowBytes = PF<FORM>::kPackedRowBytes * KB;  // packed bytes of a row per stage
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = tc::smem_u32(smem);
+    const uint32_t bar_full = sbase + OFF_BAR;        // activation tile landed         [SS]
+    const uint32_t bar_wfull = bar_full + 8 * SS;     // packed weight tile landed      [SS]
+    const uint32_t bar_empty = bar_wfull + 8 * SS;    // MMA done with the stage        [SS]
+    const uint32_t bar_ufull = bar_empty + 8 * SS;    // expanded weights in TMEM      [SU]
+    const uint32_t bar_uempty = bar_ufull + 8 * SU;   // MMA done with a TMEM slot     [SU]
+    const uint32_t bar_acc = bar_uempty + 8 * SU;     // accumulator of a piece complete
+    const uint32_t bar_accfree = bar_acc + 8;         // epilogue done reading it
+    const uint32_t bar_stfree = bar_accfree + 8;      // epilogue done with the staging area
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * (3 * SS + 2 * SU + 3));
+    unsigned int* arrivals = reinterpret_cast<unsigned int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bt = p.bt;
+    const int ttiles = (p.rows_a + bt - 1) / bt;
+    const int nblk = p.K / BK;                 // 128-k blocks
+    const int nk = (nblk + KB - 1) / KB;       // stages; the last may hold fewer blocks
+    // blocks in stage kb; the weight box of a short last stage runs past the row
+    // end and is zero-filled (codes 0 expand to 0, so those products vanish)
+    auto blocks = [&](int kb) { return KB == 1 ? 1 : min(KB, nblk - kb * KB); };
+
+    // This CTA's (tile, stage) units [ua, ub), walked in pieces of one tile each.
+    const long long U = (long long)p.sk_tiles * nk;
+    const int G = p.sk_ctas > 0 ? p.sk_ctas : 1;
+    const int cme = (int)blockIdx.x - p.dp_tiles;       // >= 0: a CTA of the balanced round
+    auto sk_start = [&](int c) { return (long long)c * U / G; };   // relative to the round
+    long long ua, ub;
+    if (cme < 0) {
+        ua = (long long)blockIdx.x * nk;
+        ub = ua + nk;
+    } else {
+        const long long base = (long long)p.dp_tiles * nk;
+        ua = base + sk_start(cme);
+        ub = base + sk_start(cme + 1);
+    }
+    auto piece = [&](long long u, int& tile, int& kb0, int& kb1) {
+        tile = (int)(u / nk);
+        kb0 = (int)(u - (long long)tile * nk);
+        kb1 = (int)min((long long)nk, kb0 + (ub - u));
+    };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < SS; ++s) {
+            tc::mbar_init(bar_full + 8 * s, 1);
+            tc::mbar_init(bar_wfull + 8 * s, 1);
+            tc::mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int u = 0; u < SU; ++u) {
+            tc::mbar_init(bar_ufull + 8 * u, 128);
+            tc::mbar_init(bar_uempty + 8 * u, 1);
+        }
+        tc::mbar_init(bar_acc, 1);
+        tc::mbar_init(bar_accfree, kEpiThreads);
+        tc::mbar_init(bar_stfree, 1);
+        tc::mbar_fence_init();
+        tc::prefetch_tmap(&tmap_act);
+        tc::prefetch_tmap(&tmap_w);
+        tc::prefetch_tmap(&tmap_y);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tc::smem_u32(tmem_slot), TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // Ring and TMEM-slot positions run on across pieces: g counts this CTA's stages.
+    if (warp == 0) {
+        if (lane == 0) {
+            int tile, kb0, kb1;
+            piece(ua, tile, kb0, kb1);
+            // The packed weights are call parameters, not written by the kernel
+            // this launch may overlap (programmatic dependent launch): the first
+            // ring of weight tiles is requested before waiting for the producer
+            // of the activations, so the expansion warps can start early.
+            const int pre = min(SS, kb1 - kb0);
+            int ag = 0, wg = 0;                  // activation / weight stages issued
+            for (; wg < pre; ++wg) {
+                tc::mbar_arrive_expect_tx(bar_wfull + 8 * wg, (uint32_t)(kRowBytes * BW));
+                tc::tma_load_2d(sbase + OFF_BP + wg * BP_STAGE, &tmap_w, (kb0 + wg) * kRowBytes,
+                                (tile / ttiles) * BW, bar_wfull + 8 * wg);
+            }
+            tc::pdl_wait();
+            bool ok = true;
+            int item = 0;
+            for (long long u = ua; u < ub && ok; ++item) {
+                piece(u, tile, kb0, kb1);
+                u += kb1 - kb0;
+                const int t0 = (tile % ttiles) * bt, n0 = (tile / ttiles) * BW;
+                // the previous piece's epilogue stages its output in the ring
+                if (item > 0) ok = tc::mbar_wait(bar_stfree, (item - 1) & 1, p.flags, kWaitLimitNs);
+                for (int kb = kb0; kb < kb1 && ok; ++kb) {
+                    const int g = ag, s = g % SS;
+                    if (g >= SS) {
+                        ok = tc::mbar_wait(bar_empty + 8 * s, ((g / SS) - 1) & 1, p.flags, kWaitLimitNs);
+                        if (!ok) break;
+                    }
+                    if (g >= wg) {
+                        tc::mbar_arrive_expect_tx(bar_wfull + 8 * s, (uint32_t)(kRowBytes * BW));
+                        tc::tma_load_2d(sbase + OFF_BP + s * BP_STAGE, &tmap_w, kb * kRowBytes, n0,
+                                        bar_wfull + 8 * s);
+                        ++wg;
+                    }
+                    const int nb = blocks(kb);
+                    tc::mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)(nb * bt * BK));
+                    for (int b = 0; b < nb; ++b)
+                        tc::tma_load_2d(sbase + OFF_ACT + s * ACT_STAGE + b * bt * BK, &tmap_act,
+                                        (kb * KB + b) * BK, t0, bar_full + 8 * s);
+                    ++ag;
+                }
+            }
+            if (!ok) {
+                // drain copies still in flight before the CTA's shared memory goes away
+                for (int g = (ag > SS ? ag - SS : 0); g < ag; ++g)
+                    tc::mbar_wait(bar_full + 8 * (g % SS), (g / SS) & 1, p.flags, kWaitLimitNs);
+                for (int g = (wg > SS ? wg - SS : 0); g < wg; ++g)
+                    tc::mbar_wait(bar_wfull + 8 * (g % SS), (g / SS) & 1, p.flags, kWaitLimitNs);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = tc::idesc_i8(BW, bt);
+            bool ok = true;
+            int g = 0, item = 0;
+            for (long long u = ua; u < ub && ok; ++item) {
+                int tile, kb0, kb1;
+                piece(u, tile, kb0, kb1);
+                u += kb1 - kb0;
+                if (item > 0) {
+                    // the accumulator is reused: the previous piece's epilogue must have read it
+                    ok = tc::mbar_wait(bar_accfree, (item - 1) & 1, p.flags, kWaitLimitNs);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                }
+                for (int kb = kb0; kb < kb1; ++kb, ++g) {
+                    const int s = g % SS, uu = g % SU;
+                    ok = tc::mbar_wait(bar_full + 8 * s, (g / SS) & 1, p.flags, kWaitLimitNs) &&
+                         tc::mbar_wait(bar_ufull + 8 * uu, (g / SU) & 1, p.flags, kWaitLimitNs);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                    const uint32_t act_s = sbase + OFF_ACT + s * ACT_STAGE;
+                    const int nj = 4 * blocks(kb);
+#pragma unroll
+                    for (int j = 0; j < KB * BK / 32; ++j)
+                        if (j < nj)
+                        tc::mma_i8_ts(tmem + kAccCol, tmem + kWCol + 32 * KB * uu + 8 * j,
+                                      tc::desc_kmajor_sw128(act_s + (j >> 2) * bt * BK + 32 * (j & 3)),
+                                      idesc, kb > kb0 || j > 0);
+                    tc::mma_commit(bar_empty + 8 * s);
+                    tc::mma_commit(bar_uempty + 8 * uu);
+                }
+                // completion of this piece's MMAs (also on the abort path)
+                tc::mma_commit(bar_acc);
+            }
+            // the next kernel on the stream may start launching now; it waits for
+            // this grid's completion before touching anything this grid writes
+            tc::pdl_trigger();
+            // everything issued has completed before the accumulator is freed
+            if (item > 0) tc::mbar_wait(bar_acc, (item - 1) & 1, p.flags, kWaitLimitNs);
+        }
+    } else {
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int hsel = (warp - 2) >> 2;       // 0: warps 2-5 (expand + epilogue), 1: warps 6-9
+        const int r = 32 * q + lane;            // weight row within the tile = TMEM lane
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        float* tok_scale = reinterpret_cast<float*>(smem + OFF_TOK);
+        int* tok_rsum = reinterpret_cast<int*>(tok_scale + BT);
+        const int et = threadIdx.x - 64;        // 0..kEpiThreads-1
+        const size_t slot_elems = (size_t)bt * BW;
+        bool ok = true;
+        int g = 0, item = 0;
+        for (long long u = ua; u < ub; ++item) {
+            const long long upiece = u;
+            int tile, kb0, kb1;
+            piece(u, tile, kb0, kb1);
+            u += kb1 - kb0;
+            const int t0 = (tile % ttiles) * bt, n0 = (tile / ttiles) * BW;
+
+            // ------- expand (warps 2-5): one thread per weight row -------
+            for (int kb = kb0; hsel == 0 && kb < kb1 && ok; ++kb, ++g) {
+                const int s = g % SS, uu = g % SU;
+                ok = tc::mbar_wait(bar_wfull + 8 * s, (g / SS) & 1, p.flags, kWaitLimitNs);
+                if (ok && g >= SU)
+                    ok = tc::mbar_wait(bar_uempty + 8 * uu, ((g / SU) - 1) & 1, p.flags, kWaitLimitNs);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+#pragma unroll
+                for (int b = 0; b < KB; ++b) {
+                    const uint8_t* bp = smem + OFF_BP + s * BP_STAGE + r * kRowBytes +
+                                        b * PF<FORM>::kPackedRowBytes;
+                    uint32_t e[32];
+                    if (FORM == 0) {
+                        const uint4 w0 = *reinterpret_cast<const uint4*>(bp);
+                        const uint4 w1 = *reinterpret_cast<const uint4*>(bp + 16);
+                        const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                        for (int o = 0; o < 8; ++o)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) e[4 * o + j] = (ws[o] >> (2 * j)) & 0x03030303u;
+                    } else {
+                        const uint4 w0 = *reinterpret_cast<const uint4*>(bp);
+                        const uint32_t ws[4] = {w0.x, w0.y, w0.z, w0.w};
+#pragma unroll
+                        for (int o = 0; o < 4; ++o)
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) e[8 * o + j] = (ws[o] >> j) & 0x01010101u;
+                    }
+                    tc::tmem_st_32x32b_x32(lane_base + kWCol + 32 * KB * uu + 32 * b, e);
+                }
+                tc::tmem_st_wait();
+                tc::tc_fence_before();
+                tc::mbar_arrive(bar_ufull + 8 * uu);
+            }
+
+            // ---------------- epilogue (warps 2-9) ----------------------------
+            if (item == 0) tc::pdl_wait();       // scale / row sums come from the previous kernel
+            // per-token scale and row sum of this activation tile
+            for (int i = et; i < bt; i += kEpiThreads) {
+                const int row = t0 + i;
+                const int tok = FORM == 0 ? row : row >> 1;
+                const bool in = FORM == 0 ? row < p.M : tok < p.M;
+                tok_scale[i] = in ? p.scale[tok] : 0.f;
+                tok_rsum[i] = in ? p.rsum[tok] : 0;
+            }
+            const bool acc_ok = tc::mbar_wait(bar_acc, item & 1, p.flags, kWaitLimitNs);
+            // one decision for the eight epilogue warps; also publishes the token table
+            const bool good = tc::bar_and(1, kEpiThreads, ok && acc_ok);
+            if (!good) break;
+            tc::tc_fence_after();
+
+            // A piece that is not a whole tile: store its int32 accumulator in
+            // this CTA's slot (0: its first piece, 1: its last), then count the
+            // arrival; the last of the tile's pieces to arrive finishes the tile.
+            const bool whole = kb0 == 0 && kb1 == nk;
+            int ts = 0, c_first = 0, c_last = 0;
+            if (!whole) {
+                ts = tile - p.dp_tiles;
+                const long long t_lo = (long long)ts * nk, t_hi = t_lo + nk - 1;
+                c_first = (int)(((t_lo + 1) * G - 1) / U);   // CTA holding the tile's first unit
+                c_last = (int)(((t_hi + 1) * G - 1) / U);    // ... and its last unit
+                int32_t* slot = p.sk_slots + (size_t)(2 * cme + (upiece == ua ? 0 : 1)) * slot_elems;
+#pragma unroll 1
+                for (int cc = hsel; cc < bt / 32; cc += 2) {
+                    uint32_t d[32];
+                    tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * cc, d);
+                    tc::tmem_ld_wait();
+                    int4* dst = reinterpret_cast<int4*>(slot) + (size_t)cc * 8 * BW + r;
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4)
+                        dst[i4 * BW] = make_int4((int)d[4 * i4], (int)d[4 * i4 + 1],
+                                                 (int)d[4 * i4 + 2], (int)d[4 * i4 + 3]);
+                }
+                __threadfence();
+                asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+                if (et == 0) *arrivals = atomicAdd(p.sk_ctr + ts, 1u);
+                asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+                if (*arrivals != (unsigned int)(c_last - c_first)) {
+                    // another piece of this tile is still running; it finishes the tile
+                    tc::tc_fence_before();
+                    tc::mbar_arrive(bar_accfree);
+                    if (et == 0) tc::mbar_arrive(bar_stfree);
+                    continue;
+                }
+                __threadfence();
+            }
+
+            // The fp16 tile is staged in the activation ring as [token][128
+            // columns] and leaves with one tensor store, which also drops the
+            // rows past M and the columns past N.
+            uint16_t* stage = reinterpret_cast<uint16_t*>(smem + OFF_ACT);
+            const int n = n0 + r;                // output column held by this thread
+            const float hn = (FORM == 1 && n < p.N) ? __half2float(__ushort_as_half(p.h[n])) : 0.f;
+#pragma unroll 1
+            for (int cc = hsel; cc < bt / 32; cc += 2) {
+                uint32_t d[32];
+                tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * cc, d);
+                tc::tmem_ld_wait();
+                if (!whole) {
+                    // add the other pieces' partial accumulators (exact in int32)
+                    for (int c = c_first; c <= c_last; ++c) {
+                        if (c == cme) continue;
+                        const int which = (c == c_first && sk_start(c) < (long long)ts * nk) ? 1 : 0;
+                        const int4* src = reinterpret_cast<const int4*>(
+                                              p.sk_slots + (size_t)(2 * c + which) * slot_elems) +
+                                          (size_t)cc * 8 * BW + r;
+#pragma unroll
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const int4 v = __ldcg(src + i4 * BW);   // written by another CTA
+                            d[4 * i4] += (uint32_t)v.x;
+                            d[4 * i4 + 1] += (uint32_t)v.y;
+                            d[4 * i4 + 2] += (uint32_t)v.z;
+                            d[4 * i4 + 3] += (uint32_t)v.w;
+                        }
+                    }
+                }
+                if (FORM == 0) {
+#pragma unroll
+                    for (int i4 = 0; i4 < 32; i4 += 4) {
+                        const int tb = 32 * cc + i4;
+                        const float4 sc = *reinterpret_cast<const float4*>(tok_scale + tb);
+                        const int4 rs = *reinterpret_cast<const int4*>(tok_rsum + tb);
+                        const float scs[4] = {sc.x, sc.y, sc.z, sc.w};
+                        const int rss[4] = {rs.x, rs.y, rs.z, rs.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int a = (int)d[i4 + j] - rss[j];
+                            const float v = __fmul_rn(__fmul_rn((float)a, scs[j]), p.w_scale);
+                            stage[(tb + j) * BW + r] = __half_as_ushort(__float2half_rn(v));
+                            const int m = t0 + tb + j;
+                            if (p.acc_out && m < p.M && n < p.N) p.acc_out[(size_t)m * p.N + n] = a;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const int ti = 32 * cc + i;
+                        const long long P = 256ll * (int)d[i] + (int)d[i + 1];
+                        const float z = __fmul_rn(tok_scale[ti], (float)(2 * P - (long long)tok_rsum[ti]));
+                        stage[(ti >> 1) * BW + r] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hn)));
+                    }
+                }
+            }
+            tc::tc_fence_before();
+            tc::mbar_arrive(bar_accfree);
+            tc::fence_proxy_async_smem();
+            asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+            if (et == 0) {
+                tc::tma_store_2d(&tmap_y, sbase + OFF_ACT, n0 * 2, FORM == 0 ? t0 : t0 >> 1);
+                tc::bulk_commit_group();
+                tc::bulk_wait_group_read0();
+                tc::mbar_arrive(bar_stfree);
+            }
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
 // 2-D uint8 tensor map: rows x cols bytes (row stride = cols), box box_cols x box_rows.
 bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                uint32_t box_rows, CUtensorMapSwizzle swz) {
@@ -357,16 +729,70 @@ inline int choose_bt(int rows_a) {
     return r < BT ? r : BT;
 }
 
-template <int FORM, int KB>
+// Tile geometry of a call: activation rows per tile, k-blocks per stage,
+// stages per tile and the number of (weight-row, activation-row) tiles.
+struct Geometry {
+    int bt, kb, nk, tiles;
+};
+
+Geometry geometry(int rows_a, int K, int N) {
+    Geometry g;
+    g.bt = choose_bt(rows_a);
+    g.kb = g.bt <= BT / 4 ? 4 : g.bt <= BT / 2 ? 2 : 1;
+    g.nk = (K / BK + g.kb - 1) / g.kb;
+    g.tiles = ((N + BW - 1) / BW) * ((rows_a + g.bt - 1) / g.bt);
+    return g;
+}
+
+// One CTA per SM at a time (the ring takes most of shared memory), so the
+// tiles run in rounds of G.  When the last round would leave SMs idle, the
+// last one or two rounds' tiles are instead shared out evenly in k-stages over
+// G CTAs.  The cost model, in stage-times (measured on the 70B-shaped layers):
+// a whole tile's epilogue is worth about 10 stages; a CTA of the balanced
+// round pays about 36 more (writing a partial slot, the refill before its
+// next piece, and finishing a split tile from another CTA's slot).  The
+// balanced round must win by 5 % to be used.
+struct SplitPlan {
+    int dp_tiles, sk_tiles, sk_ctas;
+};
+
+SplitPlan plan_split(const Geometry& g, int G) {
+    SplitPlan pl{g.tiles, 0, 0};
+    if (G <= 0 || g.tiles % G == 0) return pl;
+    const int rounds = g.tiles / G;
+    const int dp = rounds >= 1 ? (rounds - 1) * G : 0;
+    const int skt = g.tiles - dp;
+    if ((long long)skt * g.nk < 4ll * G) return pl;   // too little work to share out
+    constexpr double kEpi = 10.0, kSplit = 36.0;
+    const double dp_cost = (double)((g.tiles + G - 1) / G) * (g.nk + kEpi);
+    const double sk_cost = (double)(dp / G) * (g.nk + kEpi) + (double)skt * g.nk / G + kSplit;
+    if (sk_cost >= 0.95 * dp_cost) return pl;
+    pl.dp_tiles = dp;
+    pl.sk_tiles = skt;
+    pl.sk_ctas = G;
+    return pl;
+}
+
+inline size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Scratch of a balanced round: arrival counters, then two partial-accumulator
+// slots per CTA.
+size_t split_bytes(const Geometry& g, const SplitPlan& pl) {
+    if (pl.sk_ctas == 0) return 0;
+    return round256((size_t)pl.sk_tiles * 4) + (size_t)2 * pl.sk_ctas * g.bt * BW * 4;
+}
+
+template <int FORM, int KB, bool SPLIT>
 cudaError_t launch_prefill_kb(const int8_t* act, const uint32_t* w, PrefillParams p,
                               cudaStream_t s) {
     constexpr int smem = PS<KB>::SMEM_BYTES;
+    constexpr auto kern = SPLIT ? prefill_split_kernel<FORM, KB> : prefill_kernel<FORM, KB>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_kernel<FORM, KB>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        e = use_max_shared_carveout(prefill_kernel<FORM, KB>);
+        e = use_max_shared_carveout(kern);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -383,9 +809,8 @@ cudaError_t launch_prefill_kb(const int8_t* act, const uint32_t* w, PrefillParam
     if (!make_tmap(&ty, p.y, (uint64_t)p.M, (uint64_t)p.N * 2, BW * 2,
                    (uint32_t)(FORM == 0 ? p.bt : p.bt / 2), CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    const int tiles = ((p.N + BW - 1) / BW) * ((p.rows_a + p.bt - 1) / p.bt);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(tiles);
+    cfg.gridDim = dim3(p.dp_tiles + p.sk_ctas);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
@@ -394,35 +819,63 @@ cudaError_t launch_prefill_kb(const int8_t* act, const uint32_t* w, PrefillParam
     attrs[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_kernel<FORM, KB>, ta, tw, ty, p);
+    return cudaLaunchKernelEx(&cfg, kern, ta, tw, ty, p);
 }
 
 template <int FORM>
-cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, PrefillParams p,
-                           cudaStream_t s) {
-    p.bt = choose_bt(p.rows_a);
-    if (p.bt <= BT / 4) return launch_prefill_kb<FORM, 4>(act, w, p, s);
-    if (p.bt <= BT / 2) return launch_prefill_kb<FORM, 2>(act, w, p, s);
-    return launch_prefill_kb<FORM, 1>(act, w, p, s);
+cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, PrefillParams p, void* split_ws,
+                           size_t split_ws_bytes, cudaStream_t s) {
+    const Geometry g = geometry(p.rows_a, p.K, p.N);
+    p.bt = g.bt;
+    SplitPlan pl = plan_split(g, device_sm_count());
+    const size_t need = split_bytes(g, pl);
+    if (need == 0 || split_ws == nullptr || split_ws_bytes < need) pl = SplitPlan{g.tiles, 0, 0};
+    p.dp_tiles = pl.dp_tiles;
+    p.sk_tiles = pl.sk_tiles;
+    p.sk_ctas = pl.sk_ctas;
+    p.sk_ctr = pl.sk_ctas ? static_cast<unsigned int*>(split_ws) : nullptr;
+    p.sk_slots = pl.sk_ctas ? reinterpret_cast<int32_t*>(static_cast<char*>(split_ws) +
+                                                         round256((size_t)pl.sk_tiles * 4))
+                            : nullptr;
+    if (pl.sk_ctas > 0) {
+        if (g.kb == 4) return launch_prefill_kb<FORM, 4, true>(act, w, p, s);
+        if (g.kb == 2) return launch_prefill_kb<FORM, 2, true>(act, w, p, s);
+        return launch_prefill_kb<FORM, 1, true>(act, w, p, s);
+    }
+    if (g.kb == 4) return launch_prefill_kb<FORM, 4, false>(act, w, p, s);
+    if (g.kb == 2) return launch_prefill_kb<FORM, 2, false>(act, w, p, s);
+    return launch_prefill_kb<FORM, 1, false>(act, w, p, s);
 }
 
 }  // namespace
 
+size_t prefill_split_bytes(int form, int M, int K, int N, int* n_counters) {
+    *n_counters = 0;
+    if (M <= 0 || N <= 0) return 0;
+    const Geometry g = geometry(form == 0 ? M : 2 * M, K, N);
+    const SplitPlan pl = plan_split(g, device_sm_count());
+    *n_counters = pl.sk_tiles;
+    return split_bytes(g, pl);
+}
+
 cudaError_t launch_ternary_prefill(const uint32_t* w2, const int8_t* qp, const float* scale,
                                    const int32_t* qsum, int M, int K, int N, float w_scale,
                                    uint16_t* y, int32_t* acc_out, unsigned int* flags,
-                                   cudaStream_t s) {
+                                   cudaStream_t s, void* split_ws, size_t split_ws_bytes) {
     if (M == 0 || N == 0) return cudaSuccess;
-    PrefillParams p{M, 0, M, K, N, scale, qsum, nullptr, w_scale, y, acc_out, flags};
-    return launch_prefill<0>(qp, w2, p, s);
+    PrefillParams p{M, 0, M, K, N, scale, qsum, nullptr, w_scale, y, acc_out, flags,
+                    0, 0, 0, nullptr, nullptr};
+    return launch_prefill<0>(qp, w2, p, split_ws, split_ws_bytes, s);
 }
 
 cudaError_t launch_onebit_prefill(const uint32_t* s1, const int8_t* planes, const float* step,
                                   const int32_t* tsum, const uint16_t* h, int M, int K, int N,
-                                  uint16_t* y, unsigned int* flags, cudaStream_t s) {
+                                  uint16_t* y, unsigned int* flags, cudaStream_t s,
+                                  void* split_ws, size_t split_ws_bytes) {
     if (M == 0 || N == 0) return cudaSuccess;
-    PrefillParams p{2 * M, 0, M, K, N, step, tsum, h, 0.f, y, nullptr, flags};
-    return launch_prefill<1>(planes, s1, p, s);
+    PrefillParams p{2 * M, 0, M, K, N, step, tsum, h, 0.f, y, nullptr, flags,
+                    0, 0, 0, nullptr, nullptr};
+    return launch_prefill<1>(planes, s1, p, split_ws, split_ws_bytes, s);
 }
 
 }  // namespace bl

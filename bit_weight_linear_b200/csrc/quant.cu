@@ -51,6 +51,13 @@ __device__ __forceinline__ int block_sum_i32(int v, int* red) {
     return r;
 }
 
+// Zero the consumer's arrival counters (CTA 0 only; called after the PDL wait,
+// so the previous user of the counters has finished).
+__device__ __forceinline__ void zero_words(unsigned int* zero, int n_zero) {
+    if (zero != nullptr && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0u;
+}
+
 __device__ __forceinline__ float half_bits_to_float(uint32_t bits) {
     return __half2float(__ushort_as_half((unsigned short)(bits & 0xffffu)));
 }
@@ -67,7 +74,8 @@ template <int LAYOUT>
 __global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t* __restrict__ x,
                                                              int K, int8_t* __restrict__ q,
                                                              float* __restrict__ scale,
-                                                             int32_t* __restrict__ qsum) {
+                                                             int32_t* __restrict__ qsum,
+                                                             unsigned int* zero, int n_zero) {
     __shared__ uint32_t redu[kWarps];
     __shared__ int redi[kWarps];
     const int m = blockIdx.x;
@@ -76,6 +84,7 @@ __global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t* __r
     // weights, and read x / write the outputs only after the producer of x is done
     tc::pdl_trigger();
     tc::pdl_wait();
+    zero_words(zero, n_zero);
 
     // pass 1: amax as the max of |x| bit patterns (monotone for finite halves)
     uint32_t mx = 0;
@@ -155,7 +164,8 @@ __device__ __forceinline__ int block_sum_i32_n(int v, int* red) {
 template <int LAYOUT, int NCH>
 __global__ void __launch_bounds__(kRegThreads, NCH <= 4 ? 2 : 1)
     quant_act_reg_kernel(const uint16_t* __restrict__ x, int K, int8_t* __restrict__ q,
-                         float* __restrict__ scale, int32_t* __restrict__ qsum) {
+                         float* __restrict__ scale, int32_t* __restrict__ qsum,
+                         unsigned int* zero, int n_zero) {
     constexpr int NW = kRegThreads / 32;
     __shared__ uint32_t redu[NW];
     __shared__ int redi[NW];
@@ -164,6 +174,7 @@ __global__ void __launch_bounds__(kRegThreads, NCH <= 4 ? 2 : 1)
     const uint16_t* row = x + (size_t)m * K;
     tc::pdl_trigger();
     tc::pdl_wait();
+    zero_words(zero, n_zero);
 
     uint4 va[NCH], vb[NCH];
 #pragma unroll
@@ -233,13 +244,15 @@ __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* _
                                                                const uint16_t* __restrict__ g,
                                                                int K, int8_t* __restrict__ planes,
                                                                float* __restrict__ step,
-                                                               int32_t* __restrict__ tsum) {
+                                                               int32_t* __restrict__ tsum,
+                                                               unsigned int* zero, int n_zero) {
     __shared__ uint32_t redu[kWarps];
     __shared__ int redi[kWarps];
     const int m = blockIdx.x;
     const uint16_t* row = x + (size_t)m * K;
     tc::pdl_trigger();
     tc::pdl_wait();
+    zero_words(zero, n_zero);
 
     float mx = 0.f;
     for (int c = threadIdx.x; c < K / 8; c += kThreads) {
@@ -336,13 +349,13 @@ inline int reg_chunks(int K) {
 
 template <int LAYOUT>
 cudaError_t launch_quant(const uint16_t* x, int M, int K, int8_t* q, float* scale,
-                         int32_t* qsum, cudaStream_t s) {
+                         int32_t* qsum, unsigned int* zero, int n_zero, cudaStream_t s) {
     switch (reg_chunks(K)) {
-        case 1: return launch_pdl<quant_act_reg_kernel<LAYOUT, 1>, kRegThreads>(M, s, x, K, q, scale, qsum);
-        case 2: return launch_pdl<quant_act_reg_kernel<LAYOUT, 2>, kRegThreads>(M, s, x, K, q, scale, qsum);
-        case 4: return launch_pdl<quant_act_reg_kernel<LAYOUT, 4>, kRegThreads>(M, s, x, K, q, scale, qsum);
-        case 8: return launch_pdl<quant_act_reg_kernel<LAYOUT, 8>, kRegThreads>(M, s, x, K, q, scale, qsum);
-        default: return launch_pdl<quant_act_kernel<LAYOUT>>(M, s, x, K, q, scale, qsum);
+        case 1: return launch_pdl<quant_act_reg_kernel<LAYOUT, 1>, kRegThreads>(M, s, x, K, q, scale, qsum, zero, n_zero);
+        case 2: return launch_pdl<quant_act_reg_kernel<LAYOUT, 2>, kRegThreads>(M, s, x, K, q, scale, qsum, zero, n_zero);
+        case 4: return launch_pdl<quant_act_reg_kernel<LAYOUT, 4>, kRegThreads>(M, s, x, K, q, scale, qsum, zero, n_zero);
+        case 8: return launch_pdl<quant_act_reg_kernel<LAYOUT, 8>, kRegThreads>(M, s, x, K, q, scale, qsum, zero, n_zero);
+        default: return launch_pdl<quant_act_kernel<LAYOUT>>(M, s, x, K, q, scale, qsum, zero, n_zero);
     }
 }
 
@@ -351,19 +364,21 @@ cudaError_t launch_quant(const uint16_t* x, int M, int K, int8_t* q, float* scal
 cudaError_t launch_quant_plain(const uint16_t* x, int M, int K, int8_t* q, float* scale,
                                cudaStream_t s) {
     if (M == 0) return cudaSuccess;
-    return launch_quant<0>(x, M, K, q, scale, (int32_t*)nullptr, s);
+    return launch_quant<0>(x, M, K, q, scale, (int32_t*)nullptr, (unsigned int*)nullptr, 0, s);
 }
 
 cudaError_t launch_quant_ternary_perm(const uint16_t* x, int M, int K, int8_t* qp,
-                                      float* scale, int32_t* qsum, cudaStream_t s) {
+                                      float* scale, int32_t* qsum, cudaStream_t s,
+                                      unsigned int* zero, int n_zero) {
     if (M == 0) return cudaSuccess;
-    return launch_quant<1>(x, M, K, qp, scale, qsum, s);
+    return launch_quant<1>(x, M, K, qp, scale, qsum, zero, n_zero, s);
 }
 
 cudaError_t launch_prep_onebit(const uint16_t* x, const uint16_t* g, int M, int K,
-                               int8_t* planes, float* step, int32_t* tsum, cudaStream_t s) {
+                               int8_t* planes, float* step, int32_t* tsum, cudaStream_t s,
+                               unsigned int* zero, int n_zero) {
     if (M == 0) return cudaSuccess;
-    return launch_pdl<prep_onebit_kernel>(M, s, x, g, K, planes, step, tsum);
+    return launch_pdl<prep_onebit_kernel>(M, s, x, g, K, planes, step, tsum, zero, n_zero);
 }
 
 }  // namespace bl

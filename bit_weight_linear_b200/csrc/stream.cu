@@ -675,19 +675,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
 
 // ------------------------------------------------------------------ host --
 
-int sm_count() {
-    static std::mutex mu;
-    static int cached[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    std::lock_guard<std::mutex> lk(mu);
-    if (cached[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-        cached[dev] = n;
-    }
-    return cached[dev];
-}
+int sm_count() { return device_sm_count(); }
 
 struct StreamPlan {
     int grid, nt, xreg, smem;

@@ -113,7 +113,12 @@ bl_status ob_pack_sign(const uint16_t *w, int N, int K, uint32_t *s1, bl_stream_
 bl_status bl_quant_act(const uint16_t *x, int M, int K, int8_t *q, float *scale,
                        bl_stream_t stream);
 
-/* Workspace bytes bl_ternary_linear needs for this shape (a multiple of 256). */
+/* Workspace bytes bl_ternary_linear needs for this shape (a multiple of 256),
+ * 0 for an invalid shape.  The size depends on the current device's SM count:
+ * for prefill-sized M, when the (128-row x token) tiles would leave SMs idle
+ * in the last round, it includes scratch (per-tile arrival counters and two
+ * int32 partial tiles per SM) that lets the kernel share that round out in
+ * k-stages.  Query it with the device that will run the call current. */
 size_t bl_ternary_workspace_bytes(int M, int K, int N);
 
 /*
@@ -138,7 +143,8 @@ bl_status bl_ternary_linear(const uint16_t *x, int M, int K, int N, const uint32
                             float w_scale, uint16_t *y, int32_t *acc_out,
                             void *workspace, size_t workspace_bytes, bl_stream_t stream);
 
-/* Workspace bytes ob_linear needs for this shape (a multiple of 256). */
+/* Workspace bytes ob_linear needs for this shape (a multiple of 256), 0 for an
+ * invalid shape; device-dependent like bl_ternary_workspace_bytes. */
 size_t ob_workspace_bytes(int M, int K, int N);
 
 /*

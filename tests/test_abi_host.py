@@ -50,6 +50,8 @@ def test_workspace_sizes(L):
     assert L.bl_ternary_workspace_bytes(8, 4096, 4096) == 8 * 4096 + 256 + 256
     assert L.ob_workspace_bytes(16, 4096, 4096) == 2 * 16 * 4096 + 256 + 256
     assert L.bl_ternary_workspace_bytes(1, 100, 16) == 0       # bad K
+    assert L.bl_ternary_workspace_bytes(1, 128, 24) == 0       # bad N (not a multiple of 16)
+    assert L.ob_workspace_bytes(1, 128, -16) == 0
     assert L.ob_workspace_bytes(1, 65536 + 128, 16) == 0        # OneBit K limit
     for v in (L.bl_ternary_workspace_bytes(3, 384, 16), L.ob_workspace_bytes(5, 640, 32)):
         assert v % 256 == 0

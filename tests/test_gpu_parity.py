@@ -244,6 +244,8 @@ def test_ternary_prefill_70b_full_size_sampled_rows(blw, oref):
     channels, run whole on the GPU; the oracle recomputes 96 sampled weight rows
     for all 512 tokens (rows are independent)."""
     M, K, N = 512, 8192, 28672
+    # 448 tiles: two whole-tile rounds, then a balanced round of the last 152
+    assert blw.bl_ternary_workspace_bytes(M, K, N) > M * K + 1_000_000
     x = synth.activations(M, K, seed=3_000_001, outlier_frac=0.01)
     w = synth.ternary_weights(N, K, seed=3_000_008)
     y, acc = blw.bl_ternary_linear(x.cuda(), blw.bl_pack_ternary(w.cuda()), 0.02, return_acc=True)
@@ -256,9 +258,37 @@ def test_ternary_prefill_70b_full_size_sampled_rows(blw, oref):
     assert np.array_equal(y.cpu().numpy()[:, rows].view(np.uint16), y_ref.view(np.uint16))
 
 
+# Shapes whose tiles leave most SMs idle in the last round on a 148-SM part, so
+# the kernel shares the work out in k-stages and finishes split tiles from int32
+# partials: 150 tiles of 100 tokens with two 128-k blocks per ring stage, and
+# 150 ragged tiles (a 44-row token tile, an 80-column weight tile).
+BALANCED_ROUND = [(100, 16384, 19200), (300, 8192, 9552)]
+
+
+@pytest.mark.parametrize("M,K,N", BALANCED_ROUND)
+def test_ternary_prefill_balanced_round(blw, oref, M, K, N):
+    """The integer accumulators of split tiles must still be exact.  Sampled
+    weight rows (first and last included), all tokens."""
+    # the workspace carries the split scratch only when the plan uses it
+    assert blw.bl_ternary_workspace_bytes(M, K, N) > M * K + 1_000_000
+    x = synth.activations(M, K, seed=3_100_001 + M, outlier_frac=0.01)
+    w = synth.ternary_weights(N, K, seed=3_100_002 + M)
+    y, acc = blw.bl_ternary_linear(x.cuda(), blw.bl_pack_ternary(w.cuda()), 0.02, return_acc=True)
+    torch.cuda.synchronize()
+    assert blw.bl_device_status() == 0
+    rows = np.sort(np.random.default_rng(7).choice(N, size=128, replace=False))
+    rows[0], rows[-1] = 0, N - 1
+    w2s = oref.pack_ternary(w.numpy()[rows])
+    y_ref, acc_ref = oref.ternary_linear(x.numpy(), w2s, 0.02)
+    assert np.array_equal(acc.cpu().numpy()[:, rows], acc_ref)
+    assert np.array_equal(y.cpu().numpy()[:, rows].view(np.uint16), y_ref.view(np.uint16))
+
+
 def test_onebit_prefill_13b_full_size_sampled_rows(blw, oref):
     """The 13B-shaped down layer (K=13824, N=5120) at M=256, sampled rows."""
     M, K, N = 256, 13824, 5120
+    # 80 tiles of 256 limb rows: shared out over all SMs in k-stages
+    assert blw.ob_workspace_bytes(M, K, N) > 2 * M * K + 1_000_000
     x, ws, g, h = _onebit_inputs(M, K, N, seed=4_000_000)
     y = blw.ob_linear(x.cuda(), blw.ob_pack_sign(ws.cuda()), g.cuda(), h.cuda())
     torch.cuda.synchronize()
