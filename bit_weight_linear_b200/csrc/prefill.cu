@@ -107,6 +107,42 @@ struct PrefillParams {
     int32_t* sk_slots;     // [2 * sk_ctas][bt * BW] partial accumulators
 };
 
+// Epilogue of one 32-token chunk of accumulators d (TMEM lane = weight row r,
+// output column n): bias by the token row sums, scale, round to fp16 and stage
+// as [token][128 columns]; optionally also store the int32 accumulators.
+template <int FORM>
+__device__ __forceinline__ void convert_chunk(const uint32_t (&d)[32], int cc, uint16_t* stage,
+                                              const float* tok_scale, const int* tok_rsum,
+                                              const PrefillParams& p, int r, int n, int t0,
+                                              float hn) {
+    if (FORM == 0) {
+#pragma unroll
+        for (int i4 = 0; i4 < 32; i4 += 4) {
+            const int tb = 32 * cc + i4;
+            const float4 sc = *reinterpret_cast<const float4*>(tok_scale + tb);
+            const int4 rs = *reinterpret_cast<const int4*>(tok_rsum + tb);
+            const float scs[4] = {sc.x, sc.y, sc.z, sc.w};
+            const int rss[4] = {rs.x, rs.y, rs.z, rs.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int a = (int)d[i4 + j] - rss[j];
+                const float v = __fmul_rn(__fmul_rn((float)a, scs[j]), p.w_scale);
+                stage[(tb + j) * BW + r] = __half_as_ushort(__float2half_rn(v));
+                const int m = t0 + tb + j;
+                if (p.acc_out && m < p.M && n < p.N) p.acc_out[(size_t)m * p.N + n] = a;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+            const int ti = 32 * cc + i;
+            const long long P = 256ll * (int)d[i] + (int)d[i + 1];
+            const float z = __fmul_rn(tok_scale[ti], (float)(2 * P - (long long)tok_rsum[ti]));
+            stage[(ti >> 1) * BW + r] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hn)));
+        }
+    }
+}
+
 // One whole tile per CTA (launches without a balanced round).
 template <int FORM, int KB>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -299,37 +335,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint16_t* stage = reinterpret_cast<uint16_t*>(smem + OFF_ACT);
             const int n = n0 + r;                // output column held by this thread
             const float hn = (FORM == 1 && n < p.N) ? __half2float(__ushort_as_half(p.h[n])) : 0.f;
+            // chunks cc = hsel, hsel+2, ...; the TMEM load of the next chunk is
+            // in flight while this one is converted
+            const int nch = bt / 32;
+            uint32_t da[32], db[32];
+            if (hsel < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * hsel, da);
+            tc::tmem_ld_wait();
 #pragma unroll 1
-            for (int cc = hsel; cc < bt / 32; cc += 2) {
-                uint32_t d[32];
-                tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * cc, d);
+            for (int cc = hsel; cc < nch; cc += 4) {
+                if (cc + 2 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 2), db);
+                convert_chunk<FORM>(da, cc, stage, tok_scale, tok_rsum, p, r, n, t0, hn);
                 tc::tmem_ld_wait();
-                if (FORM == 0) {
-#pragma unroll
-                    for (int i4 = 0; i4 < 32; i4 += 4) {
-                        const int tb = 32 * cc + i4;
-                        const float4 sc = *reinterpret_cast<const float4*>(tok_scale + tb);
-                        const int4 rs = *reinterpret_cast<const int4*>(tok_rsum + tb);
-                        const float scs[4] = {sc.x, sc.y, sc.z, sc.w};
-                        const int rss[4] = {rs.x, rs.y, rs.z, rs.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int a = (int)d[i4 + j] - rss[j];
-                            const float v = __fmul_rn(__fmul_rn((float)a, scs[j]), p.w_scale);
-                            stage[(tb + j) * BW + r] = __half_as_ushort(__float2half_rn(v));
-                            const int m = t0 + tb + j;
-                            if (p.acc_out && m < p.M && n < p.N) p.acc_out[(size_t)m * p.N + n] = a;
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const int ti = 32 * cc + i;
-                        const long long P = 256ll * (int)d[i] + (int)d[i + 1];
-                        const float z = __fmul_rn(tok_scale[ti], (float)(2 * P - (long long)tok_rsum[ti]));
-                        stage[(ti >> 1) * BW + r] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hn)));
-                    }
-                }
+                if (cc + 2 >= nch) break;
+                if (cc + 4 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 4), da);
+                convert_chunk<FORM>(db, cc + 2, stage, tok_scale, tok_rsum, p, r, n, t0, hn);
+                tc::tmem_ld_wait();
             }
             tc::fence_proxy_async_smem();
             asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
@@ -641,55 +661,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint16_t* stage = reinterpret_cast<uint16_t*>(smem + OFF_ACT);
             const int n = n0 + r;                // output column held by this thread
             const float hn = (FORM == 1 && n < p.N) ? __half2float(__ushort_as_half(p.h[n])) : 0.f;
+            // add the other pieces' partial accumulators of chunk cc (exact in int32)
+            auto add_parts = [&](uint32_t (&d)[32], int cc) {
+                if (whole) return;
+                for (int c = c_first; c <= c_last; ++c) {
+                    if (c == cme) continue;
+                    const int which = (c == c_first && sk_start(c) < (long long)ts * nk) ? 1 : 0;
+                    const int4* src = reinterpret_cast<const int4*>(
+                                          p.sk_slots + (size_t)(2 * c + which) * slot_elems) +
+                                      (size_t)cc * 8 * BW + r;
+                    int4 v[8];
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) v[i4] = __ldcg(src + i4 * BW);   // another CTA's
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        d[4 * i4] += (uint32_t)v[i4].x;
+                        d[4 * i4 + 1] += (uint32_t)v[i4].y;
+                        d[4 * i4 + 2] += (uint32_t)v[i4].z;
+                        d[4 * i4 + 3] += (uint32_t)v[i4].w;
+                    }
+                }
+            };
+            // chunks cc = hsel, hsel+2, ...; the TMEM load of the next chunk is
+            // in flight while this one is finished
+            const int nch = bt / 32;
+            uint32_t da[32], db[32];
+            if (hsel < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * hsel, da);
+            tc::tmem_ld_wait();
 #pragma unroll 1
-            for (int cc = hsel; cc < bt / 32; cc += 2) {
-                uint32_t d[32];
-                tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * cc, d);
+            for (int cc = hsel; cc < nch; cc += 4) {
+                if (cc + 2 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 2), db);
+                add_parts(da, cc);
+                convert_chunk<FORM>(da, cc, stage, tok_scale, tok_rsum, p, r, n, t0, hn);
                 tc::tmem_ld_wait();
-                if (!whole) {
-                    // add the other pieces' partial accumulators (exact in int32)
-                    for (int c = c_first; c <= c_last; ++c) {
-                        if (c == cme) continue;
-                        const int which = (c == c_first && sk_start(c) < (long long)ts * nk) ? 1 : 0;
-                        const int4* src = reinterpret_cast<const int4*>(
-                                              p.sk_slots + (size_t)(2 * c + which) * slot_elems) +
-                                          (size_t)cc * 8 * BW + r;
-#pragma unroll
-                        for (int i4 = 0; i4 < 8; ++i4) {
-                            const int4 v = __ldcg(src + i4 * BW);   // written by another CTA
-                            d[4 * i4] += (uint32_t)v.x;
-                            d[4 * i4 + 1] += (uint32_t)v.y;
-                            d[4 * i4 + 2] += (uint32_t)v.z;
-                            d[4 * i4 + 3] += (uint32_t)v.w;
-                        }
-                    }
-                }
-                if (FORM == 0) {
-#pragma unroll
-                    for (int i4 = 0; i4 < 32; i4 += 4) {
-                        const int tb = 32 * cc + i4;
-                        const float4 sc = *reinterpret_cast<const float4*>(tok_scale + tb);
-                        const int4 rs = *reinterpret_cast<const int4*>(tok_rsum + tb);
-                        const float scs[4] = {sc.x, sc.y, sc.z, sc.w};
-                        const int rss[4] = {rs.x, rs.y, rs.z, rs.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int a = (int)d[i4 + j] - rss[j];
-                            const float v = __fmul_rn(__fmul_rn((float)a, scs[j]), p.w_scale);
-                            stage[(tb + j) * BW + r] = __half_as_ushort(__float2half_rn(v));
-                            const int m = t0 + tb + j;
-                            if (p.acc_out && m < p.M && n < p.N) p.acc_out[(size_t)m * p.N + n] = a;
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const int ti = 32 * cc + i;
-                        const long long P = 256ll * (int)d[i] + (int)d[i + 1];
-                        const float z = __fmul_rn(tok_scale[ti], (float)(2 * P - (long long)tok_rsum[ti]));
-                        stage[(ti >> 1) * BW + r] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hn)));
-                    }
-                }
+                if (cc + 2 >= nch) break;
+                if (cc + 4 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 4), da);
+                add_parts(db, cc + 2);
+                convert_chunk<FORM>(db, cc + 2, stage, tok_scale, tok_rsum, p, r, n, t0, hn);
+                tc::tmem_ld_wait();
             }
             tc::tc_fence_before();
             tc::mbar_arrive(bar_accfree);
