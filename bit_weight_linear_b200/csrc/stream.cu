@@ -161,18 +161,20 @@ __host__ __device__ __forceinline__ Chunk chunk_of(int c, int steps, int bsteps)
     return ch;
 }
 
-// sum of one partial over the 16 warps' copies (warp stride `stride` ints)
+// sum of one partial over the NW warps' copies (warp stride `stride` ints)
+template <int NW>
 __device__ __forceinline__ int warp_rows_sum(const int* red, int idx, int stride) {
     int v = 0;
 #pragma unroll
-    for (int w = 0; w < kSWarps; ++w) v += red[w * stride + idx];
+    for (int w = 0; w < NW; ++w) v += red[w * stride + idx];
     return v;
 }
 
-// partial sum idx ([row][col] over the CTA's tiles): the 16 warps' copies, or
+// partial sum idx ([row][col] over the CTA's tiles): the NW warps' copies, or
 // the compact mode's reduced result rows
+template <int NW>
 __device__ __forceinline__ int tile_sum(const int* red, const StreamParams& p, int idx, int ncols) {
-    return p.compact ? red[kSWarps * 16 * ncols + idx] : warp_rows_sum(red, idx, p.t_max * 16 * ncols);
+    return p.compact ? red[NW * 16 * ncols + idx] : warp_rows_sum<NW>(red, idx, p.t_max * 16 * ncols);
 }
 
 // Ring stage u = (tile u / nch, chunk u % nch): one box of bsteps whole steps
@@ -205,8 +207,11 @@ __device__ __forceinline__ void issue_stage(const StreamParams& p, const CUtenso
 //   4 units per lane, whole steps (ternary).
 //   XREG = 0: general M, x read twice (second pass from L1/L2).
 // PREP = 1: the activation kernel prepared them; they are copied in.
-template <int FORM, int NT, int PREP, int XREG>
-__global__ void __launch_bounds__(kSThreads, 2)
+// NW: warps per CTA (16; 8 for single-token launches with a register
+// preparation, where each warp takes more steps of a stage and the per-stage
+// warp overhead -- waits, releases, folds -- is paid half as often).
+template <int FORM, int NT, int PREP, int XREG, int NW = kSWarps>
+__global__ void __launch_bounds__(NW * 32, 2)
     stream_kernel(const __grid_constant__ CUtensorMap tm_main,
                   const __grid_constant__ CUtensorMap tm_tail, const StreamParams p) {
     using F = DF<FORM>;
@@ -214,6 +219,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     // ternary with one column tile: in-place masked unpack (one AND per register)
     constexpr bool kMasked = FORM == 0 && NT == 1;
     extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int kW = NW, kT = NW * 32;
     const int K = p.K, M = p.M;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sb = tc::smem_u32(smem);
@@ -224,9 +230,9 @@ __global__ void __launch_bounds__(kSThreads, 2)
     const int S = p.S;
     const int ncols = M * F::kCPT;
     uint8_t* act = smem + p.off_act;
-    int* racc = reinterpret_cast<int*>(smem + p.off_red);             // [16 warps][t_max*16][ncols]
-    float* red_max = reinterpret_cast<float*>(smem + p.off_tok);      // [16][M]
-    int* red_sum = reinterpret_cast<int*>(red_max + kSWarps * M);     // [16][M]
+    int* racc = reinterpret_cast<int*>(smem + p.off_red);             // [NW warps][t_max*16][ncols]
+    float* red_max = reinterpret_cast<float*>(smem + p.off_tok);      // [NW][M]
+    int* red_sum = reinterpret_cast<int*>(red_max + kW * M);          // [NW][M]
     uint16_t* hs = reinterpret_cast<uint16_t*>(smem + p.off_h);       // [t_max*16]
     uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + p.off_cnt);    // [S] releases, [S] rounds issued
     const uint32_t cnt_sb = sb + p.off_cnt;
@@ -238,9 +244,9 @@ __global__ void __launch_bounds__(kSThreads, 2)
         if (p.nfull > 0) tc::prefetch_tmap(&tm_main);
         if (p.ragged) tc::prefetch_tmap(&tm_tail);
     }
-    for (int i = tid; i < 2 * S; i += kSThreads) cnt[i] = 0;
+    for (int i = tid; i < 2 * S; i += kT) cnt[i] = 0;
     if (FORM == 1)
-        for (int i = tid; i < T * 16; i += kSThreads) hs[i] = p.h[tile0 * 16 + i];
+        for (int i = tid; i < T * 16; i += kT) hs[i] = p.h[tile0 * 16 + i];
     // Warp-local activation preparation (XREG): warp w owns the k-steps
     // s = w, w + 16, ... (the steps it contracts).  Its work is the units
     // (token m, group q of its owned steps), token-major; lane l takes units
@@ -252,7 +258,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     int um[U], uk[U];
     bool has[U];
     if constexpr (XREG != 0) {
-        const int own = warp < p.steps ? (p.steps - 1 - warp) / 16 + 1 : 0;
+        const int own = warp < p.steps ? (p.steps - 1 - warp) / kW + 1 : 0;
         const int gw = own * 16;  // groups per token owned by this warp
 #pragma unroll
         for (int i = 0; i < U; ++i) {
@@ -266,7 +272,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 q = gw > 0 ? v - m * gw : 0;
             }
             um[i] = m;
-            uk[i] = (warp + 16 * (q >> 4)) * F::kStepK + (q & 15) * G;
+            uk[i] = (warp + kW * (q >> 4)) * F::kStepK + (q & 15) * G;
             has[i] = m < Mx && uk[i] < K;
         }
     }
@@ -294,7 +300,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     float tok_amax = 0.f;  // XREG: the token's absmax, kept for the epilogue
     if (PREP) {
         const int per_row = K / 16;
-        for (int c = tid; c < ncols * per_row; c += kSThreads) {
+        for (int c = tid; c < ncols * per_row; c += kT) {
             const int row = c / per_row, off = c - row * per_row;
             tc::cp_async16(sb + p.off_act + row * p.astride + 16 * off,
                            p.prep + (size_t)row * K + 16 * off);
@@ -339,13 +345,13 @@ __global__ void __launch_bounds__(kSThreads, 2)
         float amax_l = 0.f;
         if (Mx == 1) {
 #pragma unroll
-            for (int w = 0; w < kSWarps; w += 4) {
+            for (int w = 0; w < kW; w += 4) {
                 const float4 r4 = *reinterpret_cast<const float4*>(red_max + w);
                 amax_l = fmaxf(fmaxf(amax_l, r4.x), fmaxf(r4.y, fmaxf(r4.z, r4.w)));
             }
         } else if (lane < Mx) {
 #pragma unroll
-            for (int w = 0; w < kSWarps; ++w) amax_l = fmaxf(amax_l, red_max[w * Mx + lane]);
+            for (int w = 0; w < kW; ++w) amax_l = fmaxf(amax_l, red_max[w * Mx + lane]);
         }
         tok_amax = amax_l;
         const float qmax = FORM == 0 ? 127.0f : 32639.0f;
@@ -379,7 +385,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         for (int m = 0; m < M; ++m) {
             const uint16_t* xr = p.x + (size_t)m * K;
             float mx = 0.f;
-            for (int i = tid; i < ngroups; i += kSThreads) {
+            for (int i = tid; i < ngroups; i += kT) {
                 if (FORM == 0) {
                     const uint32_t mb = max(absmax_bits_t(tc::ld_v4(xr + 16 * i)),
                                             absmax_bits_t(tc::ld_v4(xr + 16 * i + 8)));
@@ -399,16 +405,16 @@ __global__ void __launch_bounds__(kSThreads, 2)
             const uint16_t* xr = p.x + (size_t)m * K;
             float amax = 0.f;
 #pragma unroll
-            for (int w = 0; w < kSWarps; ++w) amax = fmaxf(amax, red_max[w * M + m]);
+            for (int w = 0; w < kW; ++w) amax = fmaxf(amax, red_max[w * M + m]);
             int sum = 0;
             if (FORM == 0) {
                 const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
-                for (int i = tid; i < ngroups; i += kSThreads)
+                for (int i = tid; i < ngroups; i += kT)
                     sum += quant_group_t(tc::ld_v4(xr + 16 * i), tc::ld_v4(xr + 16 * i + 8), inv,
                                          act + m * p.astride + 16 * i);
             } else {
                 const float inv = amax > 0.f ? __fdiv_rn(32639.0f, amax) : 0.f;
-                for (int i = tid; i < ngroups; i += kSThreads) {
+                for (int i = tid; i < ngroups; i += kT) {
                     uint4 xa[4], gg[4];
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
@@ -463,7 +469,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         }
         const int s0 = chunk * p.bsteps, s1 = ok ? min(s0 + p.bsteps, p.steps) : s0;
         const uint8_t* slot_p = smem + slot * p.slot_bytes;
-        for (int s = s0 + warp; s < s1; s += kSWarps) {
+        for (int s = s0 + warp; s < s1; s += kW) {
             // whole step: [step][row][64 B]; partial last step: tail box [row][tail B]
             const bool part = (XREG == 2 || XREG == 4) ? false : s >= p.nfull;
             const uint8_t* w0 = part ? slot_p + p.bsteps * 1024 + p.tail * g8 + 16 * t
@@ -543,7 +549,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
             __syncwarp();
             if (lane == 0) {
                 const uint32_t old = tc::atom_add_acq_rel_smem(cnt_sb + 4 * slot, 1u);
-                if ((old + 1) % kSWarps == 0) {
+                if ((old + 1) % kW == 0) {
                     tc::fence_proxy_async_smem();
                     const int un = u + S;
                     tc::mbar_arrive_expect_tx(sb + p.off_bar + 8 * slot, stage_bytes(p, un));
@@ -577,9 +583,9 @@ __global__ void __launch_bounds__(kSThreads, 2)
                     ok = false;
                     break;
                 }
-                int* res = racc + kSWarps * 16 * ncols;  // [t_max*16][ncols]
-                for (int i = tid; i < 16 * ncols; i += kSThreads)
-                    res[lt * 16 * ncols + i] = warp_rows_sum(racc, i, 16 * ncols);
+                int* res = racc + kW * 16 * ncols;  // [t_max*16][ncols]
+                for (int i = tid; i < 16 * ncols; i += kT)
+                    res[lt * 16 * ncols + i] = warp_rows_sum<kW>(racc, i, 16 * ncols);
                 __syncthreads();
             }
         }
@@ -606,7 +612,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     // 4. epilogue: one output per thread and step, consecutive threads on consecutive n
     const int rows = T * 16;
     if (FORM == 0) {
-        for (int o = tid; o < M * rows; o += kSThreads) {
+        for (int o = tid; o < M * rows; o += kT) {
             const int m = o / rows, r = o - m * rows;
             float sc;
             int qs = 0;
@@ -617,28 +623,28 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 float amax = tok_amax;
                 if (kOne) {  // M == 1: the 16 warp sums are contiguous
 #pragma unroll
-                    for (int w = 0; w < kSWarps; w += 4) {
+                    for (int w = 0; w < kW; w += 4) {
                         const int4 r4 = *reinterpret_cast<const int4*>(red_sum + w);
                         qs += (r4.x + r4.y) + (r4.z + r4.w);
                     }
                 } else {
                     amax = 0.f;
 #pragma unroll
-                    for (int w = 0; w < kSWarps; ++w) {
+                    for (int w = 0; w < kW; ++w) {
                         amax = fmaxf(amax, red_max[w * M + m]);
                         qs += red_sum[w * M + m];
                     }
                 }
                 sc = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
             }
-            const int accv = tile_sum(racc, p, r * ncols + m, ncols) - qs;
+            const int accv = tile_sum<kW>(racc, p, r * ncols + m, ncols) - qs;
             const int n = tile0 * 16 + r;
             const float v = __fmul_rn(__fmul_rn((float)accv, sc), p.w_scale);
             p.y[(size_t)m * p.N + n] = __half_as_ushort(__float2half_rn(v));
             if (p.acc_out) p.acc_out[(size_t)m * p.N + n] = accv;
         }
     } else {
-        for (int o = tid; o < M * rows; o += kSThreads) {
+        for (int o = tid; o < M * rows; o += kT) {
             const int m = o / rows, r = o - m * rows;
             float st;
             long long ts = 0;
@@ -649,22 +655,22 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 float amax = tok_amax;
                 if (kOne) {  // M == 1: the 16 warp sums are contiguous
 #pragma unroll
-                    for (int w = 0; w < kSWarps; w += 4) {
+                    for (int w = 0; w < kW; w += 4) {
                         const int4 r4 = *reinterpret_cast<const int4*>(red_sum + w);
                         ts += (r4.x + r4.y) + (r4.z + r4.w);
                     }
                 } else {
                     amax = 0.f;
 #pragma unroll
-                    for (int w = 0; w < kSWarps; ++w) {
+                    for (int w = 0; w < kW; ++w) {
                         amax = fmaxf(amax, red_max[w * M + m]);
                         ts += red_sum[w * M + m];
                     }
                 }
                 st = amax > 0.f ? __fdiv_rn(amax, 32639.0f) : 0.f;
             }
-            const long long P = 256ll * tile_sum(racc, p, r * ncols + 2 * m, ncols) +
-                                tile_sum(racc, p, r * ncols + 2 * m + 1, ncols);
+            const long long P = 256ll * tile_sum<kW>(racc, p, r * ncols + 2 * m, ncols) +
+                                tile_sum<kW>(racc, p, r * ncols + 2 * m + 1, ncols);
             const int n = tile0 * 16 + r;
             const float z = __fmul_rn(st, (float)(2 * P - ts));
             const float hv = __half2float(__ushort_as_half(hs[r]));
@@ -678,7 +684,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
 int sm_count() { return device_sm_count(); }
 
 struct StreamPlan {
-    int grid, nt, xreg, smem;
+    int grid, nt, xreg, smem, nw;
 };
 
 // Fill the plan fields of p and choose the launch.  Shared memory is laid out
@@ -686,7 +692,7 @@ struct StreamPlan {
 // partial sums [t_max*16][cols] int32 | token scratch [2][16][M] | h [t_max*16]
 // fp16 | full barriers [S] | release counters [S] + rounds issued [S].
 template <int FORM>
-bool stream_plan(StreamParams& p, int prep, StreamPlan& pl) {
+bool stream_plan(StreamParams& p, int prep, StreamPlan& pl, int nw = kSWarps) {
     using F = DF<FORM>;
     const int M = p.M, K = p.K, N = p.N;
     const int cols = M * F::kCPT;
@@ -719,11 +725,11 @@ bool stream_plan(StreamParams& p, int prep, StreamPlan& pl) {
     const int act = cols * p.astride;
     // per-warp partial sums for every tile, or (compact) one tile's worth plus
     // the reduced rows, when the first does not fit beside the activations
-    const int red_full = kSWarps * p.t_max * 16 * cols * 4;
-    const int red_compact = (kSWarps * 16 + p.t_max * 16) * cols * 4;
+    const int red_full = nw * p.t_max * 16 * cols * 4;
+    const int red_compact = (nw * 16 + p.t_max * 16) * cols * 4;
     p.compact = cols * p.astride + red_full > kStreamSmemPair / 2 ? 1 : 0;
     const int red = p.compact ? red_compact : red_full;
-    const int tok = prep ? 0 : 2 * kSWarps * M * 4;
+    const int tok = prep ? 0 : 2 * nw * M * 4;
     const int hbytes = FORM == 1 ? p.t_max * 16 * 2 : 0;
     auto up16 = [](int v) { return (v + 15) & ~15; };
     const int fixed = up16(act) + up16(red) + up16(tok) + up16(hbytes) + 16 * kMaxSlots + 8 * kMaxSlots;
@@ -756,34 +762,35 @@ bool stream_plan(StreamParams& p, int prep, StreamPlan& pl) {
         // over its 32 lanes, at most 2 (4 when K has whole steps) per lane for
         // ternary, 1 for sign; M > 1 without it is prepared by the activation kernel
         // (xreg 1, 2: M == 1; 3: M > 1; 4: M > 1 with 4 units per lane, whole steps)
-        const int units = (p.steps + 15) / 16 * 16 * M;
+        const int units = (p.steps + nw - 1) / nw * 16 * M;
         pl.xreg = 0;
         if (!prep && cols <= 8) {
             if (units <= 32 * (FORM == 0 ? 2 : 1)) pl.xreg = M == 1 ? (p.ragged ? 1 : 2) : 3;
             else if (FORM == 0 && !p.ragged && units <= 128) pl.xreg = 4;
         }
         if (!prep && M > 1 && pl.xreg == 0) return false;
+        pl.nw = nw;
         return true;
     }
     return false;
 }
 
-template <int FORM, int NT, int PREP, int XREG>
+template <int FORM, int NT, int PREP, int XREG, int NW = kSWarps>
 cudaError_t launch_stream(const CUtensorMap& tm_main, const CUtensorMap& tm_tail,
                           const StreamParams& p, const StreamPlan& pl, cudaStream_t s) {
+    constexpr auto kern = stream_kernel<FORM, NT, PREP, XREG, NW>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(stream_kernel<FORM, NT, PREP, XREG>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kDecodeMaxSmem);
         if (e != cudaSuccess) return e;
-        e = use_max_shared_carveout(stream_kernel<FORM, NT, PREP, XREG>);
+        e = use_max_shared_carveout(kern);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.grid);
-    cfg.blockDim = dim3(kSThreads);
+    cfg.blockDim = dim3(NW * 32);
     cfg.dynamicSmemBytes = (size_t)pl.smem;
     cfg.stream = s;
     cudaLaunchAttribute attrs[1];
@@ -791,13 +798,22 @@ cudaError_t launch_stream(const CUtensorMap& tm_main, const CUtensorMap& tm_tail
     attrs[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, stream_kernel<FORM, NT, PREP, XREG>, tm_main, tm_tail, p);
+    return cudaLaunchKernelEx(&cfg, kern, tm_main, tm_tail, p);
 }
 
 template <int FORM, int PREP>
 cudaError_t launch_stream_form(StreamParams p, cudaStream_t s) {
     StreamPlan pl;
-    if (!stream_plan<FORM>(p, PREP, pl)) return cudaErrorInvalidConfiguration;
+    // One token: 8 warps whenever the activations still take a register
+    // preparation.  A chain of dependent calls runs much slower when its
+    // kernels alternate between 8- and 16-warp CTAs (measured: a 7B-shaped
+    // stack of single-token calls lost 20 %), so every single-token call of a
+    // given form makes the same choice unless K is too long for it.
+    // (OneBit keeps 16: with 8 warps its 11008-long rows no longer fit a
+    // register preparation, which would mix the two in a 7B-shaped stack.)
+    bool planned = false;
+    if (FORM == 0 && !PREP && p.M == 1) planned = stream_plan<FORM>(p, PREP, pl, 8) && pl.xreg != 0;
+    if (!planned && !stream_plan<FORM>(p, PREP, pl)) return cudaErrorInvalidConfiguration;
     // weights as [step][row][64 B] boxes: dim 0 = the 64 bytes of a step,
     // dim 1 = rows (stride = packed row bytes), dim 2 = steps (stride 64)
     const uint64_t wbytes = (uint64_t)p.K / (DF<FORM>::kPerWord / 4);
@@ -821,8 +837,14 @@ cudaError_t launch_stream_form(StreamParams p, cudaStream_t s) {
         if (pl.xreg) {
             if (pl.nt == 1) {
                 if constexpr (FORM == 0)
-                    if (pl.xreg == 4) return launch_stream<FORM, 1, 0, 4>(tm_main, tm_tail, p, pl, s);
+                    if (pl.xreg == 4)
+                        return pl.nw == 8 ? launch_stream<FORM, 1, 0, 4, 8>(tm_main, tm_tail, p, pl, s)
+                                          : launch_stream<FORM, 1, 0, 4>(tm_main, tm_tail, p, pl, s);
                 if (pl.xreg == 3) return launch_stream<FORM, 1, 0, 3>(tm_main, tm_tail, p, pl, s);
+                if constexpr (FORM == 0)
+                    if (pl.nw == 8)
+                        return pl.xreg == 2 ? launch_stream<FORM, 1, 0, 2, 8>(tm_main, tm_tail, p, pl, s)
+                                            : launch_stream<FORM, 1, 0, 1, 8>(tm_main, tm_tail, p, pl, s);
                 return pl.xreg == 2 ? launch_stream<FORM, 1, 0, 2>(tm_main, tm_tail, p, pl, s)
                                     : launch_stream<FORM, 1, 0, 1>(tm_main, tm_tail, p, pl, s);
             }
