@@ -49,8 +49,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per launch of the M = 1 decode kernel over one 7-call LLaMA-7B block
 # (4 x 4096->4096, 2 x 4096->11008, 11008->4096), from one ncu capture of the
-# current kernel: 50.90 MB / 7 launches, i.e. 1.006 x the packed-weight bytes.
-DECODE_TRAFFIC_PER_LAUNCH = 7.271e6
+# current (8-warp) kernel: 50.93 MB / 7 launches, i.e. 1.006 x the packed-weight bytes.
+DECODE_TRAFFIC_PER_LAUNCH = 7.275e6
 
 
 def load_peaks():
@@ -443,7 +443,8 @@ def main():
     alg_bytes_per_launch = (wbytes + in_b + out_b) / n_calls
     launch_ms = ms / n_calls          # upper bound: includes the per-call activation quant
     achieved = alg_bytes_per_launch / (launch_ms * 1e-3) / 1e9
-    roofline = {"kernel": "streamed ternary decode (stream_kernel<0,1,0,2>)", "bound": "hbm",
+    roofline = {"kernel": "streamed ternary decode (stream_kernel<0,1,0,2,8>; the 11008-long "
+                          "down rows use stream_kernel<0,1,0,4,8>)", "bound": "hbm",
                 "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": DECODE_TRAFFIC_PER_LAUNCH, "traffic_unit": "bytes",
