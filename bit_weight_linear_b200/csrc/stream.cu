@@ -253,7 +253,9 @@ __global__ void __launch_bounds__(NW * 32, 2)
     // l, l + 32, ... (at most U).  OneBit's g is a parameter, read before the wait.
     constexpr int G = F::kGroup;
     constexpr bool kOne = XREG == 1 || XREG == 2;            // M == 1 variants
-    constexpr int U = XREG == 4 ? 4 : (FORM == 0 ? 2 : 1);  // units per lane
+    // units per lane: OneBit's 32-element units also hold their g, so two of
+    // them only for one token on 8 warps (16 would spill at 64 registers)
+    constexpr int U = XREG == 4 ? 4 : (FORM == 0 || (kOne && NW == 8) ? 2 : 1);
     const int Mx = kOne ? 1 : M;                             // compile-time 1 for M == 1
     int um[U], uk[U];
     bool has[U];
@@ -276,11 +278,16 @@ __global__ void __launch_bounds__(NW * 32, 2)
             has[i] = m < Mx && uk[i] < K;
         }
     }
-    uint4 ga[4];
+    // OneBit: each unit's g (with several tokens, a lane's units share one group)
+    constexpr int UG = FORM == 1 && kOne ? U : 1;
+    uint4 ga[UG][4];
     if constexpr (FORM == 1 && XREG != 0) {
-        if (has[0]) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) ga[v] = ld_ro_v4(p.g + uk[0] + 8 * v);
+        for (int i = 0; i < UG; ++i) {
+            if (has[i]) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) ga[i][v] = ld_ro_v4(p.g + uk[i] + 8 * v);
+            }
         }
     }
     __syncthreads();  // barriers initialised, counters zeroed
@@ -328,7 +335,8 @@ __global__ void __launch_bounds__(NW * 32, 2)
                 umx[i] = hbits(max(absmax_bits_t(xa[i][0]), absmax_bits_t(xa[i][1])));
             } else {
 #pragma unroll
-                for (int v = 0; v < G / 8; ++v) umx[i] = fmaxf(umx[i], absmax_prod(xa[i][v], ga[v]));
+                for (int v = 0; v < G / 8; ++v)
+                    umx[i] = fmaxf(umx[i], absmax_prod(xa[i][v], ga[UG > 1 ? i : 0][v]));
             }
         }
         // non-negative floats order like their bit patterns: one redux.sync max per token
@@ -366,7 +374,7 @@ __global__ void __launch_bounds__(NW * 32, 2)
             if constexpr (FORM == 0) {
                 usum[i] = quant_group_t(xa[i][0], xa[i][1], inv, dst);
             } else {
-                usum[i] = quant_group_s(xa[i], ga, inv, dst, dst + p.astride);
+                usum[i] = quant_group_s(xa[i], ga[UG > 1 ? i : 0], inv, dst, dst + p.astride);
             }
         }
         for (int m = 0; m < Mx; ++m) {
@@ -760,12 +768,14 @@ bool stream_plan(StreamParams& p, int prep, StreamPlan& pl, int nw = kSWarps) {
         pl.smem = off;
         // warp-local preparation: a warp's units (tokens x owned groups) spread
         // over its 32 lanes, at most 2 (4 when K has whole steps) per lane for
-        // ternary, 1 for sign; M > 1 without it is prepared by the activation kernel
+        // ternary, for sign 2 at M == 1 on 8 warps and 1 otherwise; M > 1
+        // without it is prepared by the activation kernel
         // (xreg 1, 2: M == 1; 3: M > 1; 4: M > 1 with 4 units per lane, whole steps)
         const int units = (p.steps + nw - 1) / nw * 16 * M;
         pl.xreg = 0;
         if (!prep && cols <= 8) {
-            if (units <= 32 * (FORM == 0 ? 2 : 1)) pl.xreg = M == 1 ? (p.ragged ? 1 : 2) : 3;
+            if (units <= 32 * (FORM == 0 || (M == 1 && nw == 8) ? 2 : 1))
+                pl.xreg = M == 1 ? (p.ragged ? 1 : 2) : 3;
             else if (FORM == 0 && !p.ragged && units <= 128) pl.xreg = 4;
         }
         if (!prep && M > 1 && pl.xreg == 0) return false;
@@ -809,10 +819,8 @@ cudaError_t launch_stream_form(StreamParams p, cudaStream_t s) {
     // kernels alternate between 8- and 16-warp CTAs (measured: a 7B-shaped
     // stack of single-token calls lost 20 %), so every single-token call of a
     // given form makes the same choice unless K is too long for it.
-    // (OneBit keeps 16: with 8 warps its 11008-long rows no longer fit a
-    // register preparation, which would mix the two in a 7B-shaped stack.)
     bool planned = false;
-    if (FORM == 0 && !PREP && p.M == 1) planned = stream_plan<FORM>(p, PREP, pl, 8) && pl.xreg != 0;
+    if (!PREP && p.M == 1) planned = stream_plan<FORM>(p, PREP, pl, 8) && pl.xreg != 0;
     if (!planned && !stream_plan<FORM>(p, PREP, pl)) return cudaErrorInvalidConfiguration;
     // weights as [step][row][64 B] boxes: dim 0 = the 64 bytes of a step,
     // dim 1 = rows (stride = packed row bytes), dim 2 = steps (stride 64)
@@ -841,10 +849,9 @@ cudaError_t launch_stream_form(StreamParams p, cudaStream_t s) {
                         return pl.nw == 8 ? launch_stream<FORM, 1, 0, 4, 8>(tm_main, tm_tail, p, pl, s)
                                           : launch_stream<FORM, 1, 0, 4>(tm_main, tm_tail, p, pl, s);
                 if (pl.xreg == 3) return launch_stream<FORM, 1, 0, 3>(tm_main, tm_tail, p, pl, s);
-                if constexpr (FORM == 0)
-                    if (pl.nw == 8)
-                        return pl.xreg == 2 ? launch_stream<FORM, 1, 0, 2, 8>(tm_main, tm_tail, p, pl, s)
-                                            : launch_stream<FORM, 1, 0, 1, 8>(tm_main, tm_tail, p, pl, s);
+                if (pl.nw == 8)
+                    return pl.xreg == 2 ? launch_stream<FORM, 1, 0, 2, 8>(tm_main, tm_tail, p, pl, s)
+                                        : launch_stream<FORM, 1, 0, 1, 8>(tm_main, tm_tail, p, pl, s);
                 return pl.xreg == 2 ? launch_stream<FORM, 1, 0, 2>(tm_main, tm_tail, p, pl, s)
                                     : launch_stream<FORM, 1, 0, 1>(tm_main, tm_tail, p, pl, s);
             }
