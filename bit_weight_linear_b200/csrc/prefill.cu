@@ -772,7 +772,10 @@ SplitPlan plan_split(const Geometry& g, int G) {
     const int dp = rounds >= 1 ? (rounds - 1) * G : 0;
     const int skt = g.tiles - dp;
     if ((long long)skt * g.nk < 4ll * G) return pl;   // too little work to share out
-    constexpr double kEpi = 10.0, kSplit = 36.0;
+    // both overheads scale with the activation rows of a tile (bt) on top of a
+    // fixed part: at bt = 256 they are the measured 10 and 36 stages
+    const double r = g.bt / 256.0;
+    const double kEpi = 2.0 + 8.0 * r, kSplit = 8.0 + 28.0 * r;
     const double dp_cost = (double)((g.tiles + G - 1) / G) * (g.nk + kEpi);
     const double sk_cost = (double)(dp / G) * (g.nk + kEpi) + (double)skt * g.nk / G + kSplit;
     if (sk_cost >= 0.95 * dp_cost) return pl;
