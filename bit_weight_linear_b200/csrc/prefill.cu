@@ -396,7 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_acc = bar_uempty + 8 * SU;     // accumulator of a piece complete
     const uint32_t bar_accfree = bar_acc + 8;         // epilogue done reading it
     const uint32_t bar_stfree = bar_accfree + 8;      // epilogue done with the staging area
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * (3 * SS + 2 * SU + 3));
+    const uint32_t bar_part = bar_stfree + 8;         // another piece's partial slot landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * (3 * SS + 2 * SU + 4));
     unsigned int* arrivals = reinterpret_cast<unsigned int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -441,6 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_init(bar_acc, 1);
         tc::mbar_init(bar_accfree, kEpiThreads);
         tc::mbar_init(bar_stfree, 1);
+        tc::mbar_init(bar_part, 1);
         tc::mbar_fence_init();
         tc::prefetch_tmap(&tmap_act);
         tc::prefetch_tmap(&tmap_w);
@@ -558,8 +560,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         int* tok_rsum = reinterpret_cast<int*>(tok_scale + BT);
         const int et = threadIdx.x - 64;        // 0..kEpiThreads-1
         const size_t slot_elems = (size_t)bt * BW;
+        // a finisher brings the other piece's slot into the idle activation
+        // ring, behind the fp16 staging area (at most 64 KB)
+        constexpr int kPartOff = 32 * 1024;
         bool ok = true;
-        int g = 0, item = 0;
+        int g = 0, item = 0, nfin = 0;
         for (long long u = ua; u < ub; ++item) {
             const long long upiece = u;
             int tile, kb0, kb1;
@@ -653,6 +658,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     continue;
                 }
                 __threadfence();
+                if (c_last - c_first == 1) {
+                    // one other piece: one bulk copy of its slot into shared memory
+                    const int c = c_first == cme ? c_last : c_first;
+                    const int which = (c == c_first && sk_start(c) < (long long)ts * nk) ? 1 : 0;
+                    const int32_t* src = p.sk_slots + (size_t)(2 * c + which) * slot_elems;
+                    const uint32_t bytes = (uint32_t)(slot_elems * 4), quarter = bytes / 4;
+                    if (et == 0) {
+                        tc::fence_proxy_async_global();
+                        tc::mbar_arrive_expect_tx(bar_part, bytes);
+                        for (int i = 0; i < 4; ++i)
+                            tc::bulk_g2s(sbase + OFF_ACT + kPartOff + i * quarter,
+                                         reinterpret_cast<const uint8_t*>(src) + (size_t)i * quarter,
+                                         quarter, bar_part);
+                    }
+                    const bool landed = tc::bar_and(
+                        1, kEpiThreads, tc::mbar_wait(bar_part, nfin & 1, p.flags, kWaitLimitNs));
+                    if (!landed) {
+                        // the flag is set; let the copy land before shared memory goes away
+                        if (et == 0) tc::mbar_wait(bar_part, nfin & 1, p.flags, kWaitLimitNs);
+                        break;
+                    }
+                    ++nfin;
+                }
             }
 
             // The fp16 tile is staged in the activation ring as [token][128
@@ -664,6 +692,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             // add the other pieces' partial accumulators of chunk cc (exact in int32)
             auto add_parts = [&](uint32_t (&d)[32], int cc) {
                 if (whole) return;
+                if (c_last - c_first == 1) {
+                    const int4* src = reinterpret_cast<const int4*>(smem + OFF_ACT + kPartOff) +
+                                      (size_t)cc * 8 * BW + r;
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const int4 v = src[i4 * BW];
+                        d[4 * i4] += (uint32_t)v.x;
+                        d[4 * i4 + 1] += (uint32_t)v.y;
+                        d[4 * i4 + 2] += (uint32_t)v.z;
+                        d[4 * i4 + 3] += (uint32_t)v.w;
+                    }
+                    return;
+                }
                 for (int c = c_first; c <= c_last; ++c) {
                     if (c == cme) continue;
                     const int which = (c == c_first && sk_start(c) < (long long)ts * nk) ? 1 : 0;
@@ -690,6 +731,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::tmem_ld_wait();
 #pragma unroll 1
             for (int cc = hsel; cc < nch; cc += 4) {
+                // 256-row tiles: the staging of chunks 4-7 reuses the space of
+                // the partial's chunks 0-1, read in the first round
+                if (cc >= 4 && nch == 8 && !whole && c_last - c_first == 1)
+                    asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
                 if (cc + 2 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 2), db);
                 add_parts(da, cc);
                 convert_chunk<FORM>(da, cc, stage, tok_scale, tok_rsum, p, r, n, t0, hn);

@@ -103,6 +103,12 @@ __device__ __forceinline__ void bulk_commit_group() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
+// Orders this thread's generic-proxy accesses of global memory with its later
+// async-proxy (bulk copy) accesses, and the other way round.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // wait until every committed bulk group of this thread has finished reading shared memory
 __device__ __forceinline__ void bulk_wait_group_read0() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
