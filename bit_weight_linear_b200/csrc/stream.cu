@@ -71,16 +71,25 @@ struct StreamParams {
     int off_act, astride, off_red, off_tok, off_h, off_bar, off_cnt;
 };
 
+// Round-to-nearest-even of an fp32 value t with |t| < 2^22, as the bit
+// pattern of rn(t + 1.5 * 2^23): that sum has an ulp of 1, so its low mantissa
+// bits hold rne(t) (ties go to the even sum, i.e. the even integer) and its
+// low byte is rne(t) mod 256.  One full-rate add instead of a float-to-int
+// conversion.  The add is separately rounded (__fadd_rn is never contracted
+// with the preceding __fmul_rn), which keeps the two-step rounding.
+__device__ __forceinline__ int rne_bits(float t) { return __float_as_int(__fadd_rn(t, 12582912.0f)); }
+constexpr int kRneBias = 0x4B400000;   // the bit pattern of 1.5 * 2^23
+
 // Quantise one 16-element ternary group (fp16 in a, b) into the permuted
 // activation tile; returns the group's sum of q.
 // |x * inv| <= 127 (1 + 2^-24) for inv = rn(127/amax), so the rounded value
 // never leaves [-127, 127] and no clamp is needed.
 __device__ __forceinline__ int quant_group_t(uint4 a, uint4 b, float inv, uint8_t* dst) {
     const uint32_t hv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    int qv[16];
+    int qv[16];   // low bytes = q
 #pragma unroll
     for (int e = 0; e < 16; ++e)
-        qv[e] = __float2int_rn(__fmul_rn(hbits(hv[e >> 1] >> (16 * (e & 1))), inv));
+        qv[e] = rne_bits(__fmul_rn(hbits(hv[e >> 1] >> (16 * (e & 1))), inv));
     uint4 o;
     o.x = pack4(qv[0], qv[4], qv[8], qv[12]);
     o.y = pack4(qv[1], qv[5], qv[9], qv[13]);
@@ -127,7 +136,7 @@ __device__ __forceinline__ int quant_group_s(const uint4 (&xa)[4], const uint4 (
         for (int e = 0; e < 8; ++e) {
             const float pr = __fmul_rn(hbits(av[e >> 1] >> (16 * (e & 1))),
                                        hbits(gv[e >> 1] >> (16 * (e & 1))));
-            const int X = __float2int_rn(__fmul_rn(pr, inv));
+            const int X = rne_bits(__fmul_rn(pr, inv)) - kRneBias;   // |X| <= 32639
             const int hi = (X + 128) >> 8;
             // element 8v+e goes to byte v of word e
             ho[e] |= ((uint32_t)hi & 0xffu) << (8 * v);
