@@ -51,6 +51,15 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+// Round-to-nearest-even of an fp32 value t with |t| < 2^22, as the bit
+// pattern of rn(t + 1.5 * 2^23): that sum has an ulp of 1, so its low mantissa
+// bits hold rne(t) (ties go to the even sum, i.e. the even integer) and its
+// low byte is rne(t) mod 256.  One full-rate add instead of a float-to-int
+// conversion.  The add is separately rounded (__fadd_rn is never contracted
+// with the preceding __fmul_rn), which keeps the two-step rounding.
+__device__ __forceinline__ int rne_bits(float t) { return __float_as_int(__fadd_rn(t, 12582912.0f)); }
+constexpr int kRneBias = 0x4B400000;   // the bit pattern of 1.5 * 2^23
+
 __device__ __forceinline__ int warp_sum(int v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -62,9 +62,10 @@ __device__ __forceinline__ float half_bits_to_float(uint32_t bits) {
     return __half2float(__ushort_as_half((unsigned short)(bits & 0xffffu)));
 }
 
+// |x * inv| <= 127 (1 + 2^-24) for inv = rn(127/amax): the code never leaves
+// [-127, 127], so no clamp is needed
 __device__ __forceinline__ int quant127(float xv, float inv) {
-    int r = __float2int_rn(__fmul_rn(xv, inv));
-    return min(127, max(-127, r));
+    return rne_bits(__fmul_rn(xv, inv)) - kRneBias;
 }
 
 // Layout 0: natural order.  Layout 1: the decode kernel's order, a 4x4 byte
@@ -283,8 +284,7 @@ __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* _
             for (int e = 0; e < 8; ++e) {
                 float p = __fmul_rn(half_bits_to_float(xs[e >> 1] >> (16 * (e & 1))),
                                     half_bits_to_float(gs[e >> 1] >> (16 * (e & 1))));
-                int X = __float2int_rn(__fmul_rn(p, inv));
-                X = min(kFixMax, max(-kFixMax, X));
+                const int X = rne_bits(__fmul_rn(p, inv)) - kRneBias;   // |X| <= 32639
                 int hi = (X + 128) >> 8;  // arithmetic shift = floor
                 hv[8 * part + e] = hi;
                 lv[8 * part + e] = X - 256 * hi;
