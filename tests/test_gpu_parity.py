@@ -284,6 +284,47 @@ def test_ternary_prefill_balanced_round(blw, oref, M, K, N):
     assert np.array_equal(y.cpu().numpy()[:, rows].view(np.uint16), y_ref.view(np.uint16))
 
 
+# Small token counts on the tensor-core path (ternary from M = 9, OneBit from
+# M = 5): 32-row activation tiles with four 128-k blocks per ring stage.  The
+# 13824-long layers have 40 tiles, which the kernel shares out over all SMs.
+# Large layers are checked on 128 sampled weight rows (first and last
+# included, so every tile is likely hit), small ones whole.
+SMALL_M_TERNARY = [(9, 13824, 5120), (16, 13824, 5120), (12, 4096, 4096), (9, 2048, 1024)]
+SMALL_M_ONEBIT = [(5, 13824, 5120), (8, 13824, 5120), (8, 5120, 13824)]
+
+
+def _sample_rows(N, seed):
+    if N <= 4096:
+        return np.arange(N)
+    rows = np.sort(np.random.default_rng(seed).choice(N, size=128, replace=False))
+    rows[0], rows[-1] = 0, N - 1
+    return rows
+
+
+@pytest.mark.parametrize("M,K,N", SMALL_M_TERNARY)
+def test_ternary_prefill_small_token_counts(blw, oref, M, K, N):
+    x = synth.activations(M, K, seed=3_200_000 + M + N, outlier_frac=0.01)
+    w = synth.ternary_weights(N, K, seed=3_200_001 + M + N)
+    y, acc = blw.bl_ternary_linear(x.cuda(), blw.bl_pack_ternary(w.cuda()), 0.02, return_acc=True)
+    torch.cuda.synchronize()
+    assert blw.bl_device_status() == 0
+    rows = _sample_rows(N, seed=M)
+    y_ref, acc_ref = oref.ternary_linear(x.numpy(), oref.pack_ternary(w.numpy()[rows]), 0.02)
+    assert np.array_equal(acc.cpu().numpy()[:, rows], acc_ref)
+    assert np.array_equal(y.cpu().numpy()[:, rows].view(np.uint16), y_ref.view(np.uint16))
+
+
+@pytest.mark.parametrize("M,K,N", SMALL_M_ONEBIT)
+def test_onebit_prefill_small_token_counts(blw, oref, M, K, N):
+    x, ws, g, h = _onebit_inputs(M, K, N, seed=4_100_000 + M + N)
+    y = blw.ob_linear(x.cuda(), blw.ob_pack_sign(ws.cuda()), g.cuda(), h.cuda())
+    torch.cuda.synchronize()
+    assert blw.bl_device_status() == 0
+    rows = _sample_rows(N, seed=M + 1)
+    _, z_ref = oref.ob_linear(x.numpy(), oref.pack_sign(ws.numpy()[rows]), g.numpy(), h.numpy()[rows])
+    assert _rel_err(y.cpu().numpy()[:, rows], z_ref) <= OB_TOL
+
+
 def test_onebit_prefill_13b_full_size_sampled_rows(blw, oref):
     """The 13B-shaped down layer (K=13824, N=5120) at M=256, sampled rows."""
     M, K, N = 256, 13824, 5120
