@@ -107,6 +107,47 @@ struct PrefillParams {
     int32_t* sk_slots;     // [2 * sk_ctas][bt * BW] partial accumulators
 };
 
+// Expand one weight row's 128 k of packed codes (32 B ternary / 16 B sign at
+// bp) to 128 int8 bytes and store them as 32 TMEM columns of this thread's
+// lane.  The byte order inside each 16-k (32-k) group is the order the byte
+// SIMD unpack produces: byte 4j+b holds element 4b+j (8b+j for sign).
+template <int FORM>
+__device__ __forceinline__ void expand_row_block(const uint8_t* bp, uint32_t taddr) {
+    uint32_t e[32];
+    if (FORM == 0) {
+        const uint4 w0 = *reinterpret_cast<const uint4*>(bp);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(bp + 16);
+        const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int o = 0; o < 8; ++o)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) e[4 * o + j] = (ws[o] >> (2 * j)) & 0x03030303u;
+    } else {
+        const uint4 w0 = *reinterpret_cast<const uint4*>(bp);
+        const uint32_t ws[4] = {w0.x, w0.y, w0.z, w0.w};
+#pragma unroll
+        for (int o = 0; o < 4; ++o)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) e[8 * o + j] = (ws[o] >> j) & 0x01010101u;
+    }
+    tc::tmem_st_32x32b_x32(taddr, e);
+}
+
+// Per-token scale and row sum of the activation rows [t0, t0 + bt) (token rows
+// for ternary, limb-row pairs for OneBit), zero past M; filled by the
+// epilogue threads et = 0 .. kEpiThreads-1.
+template <int FORM>
+__device__ __forceinline__ void fill_token_table(const PrefillParams& p, int t0, int bt, int et,
+                                                 float* tok_scale, int* tok_rsum) {
+    for (int i = et; i < bt; i += kEpiThreads) {
+        const int row = t0 + i;
+        const int tok = FORM == 0 ? row : row >> 1;
+        const bool in = FORM == 0 ? row < p.M : tok < p.M;
+        tok_scale[i] = in ? p.scale[tok] : 0.f;
+        tok_rsum[i] = in ? p.rsum[tok] : 0;
+    }
+}
+
 // Epilogue of one 32-token chunk of accumulators d (TMEM lane = weight row r,
 // output column n): bias by the token row sums, scale, round to fp16 and stage
 // as [token][128 columns]; optionally also store the int32 accumulators.
@@ -287,24 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int b = 0; b < KB; ++b) {
                 const uint8_t* bp = smem + OFF_BP + s * BP_STAGE + r * kRowBytes +
                                     b * PF<FORM>::kPackedRowBytes;
-                uint32_t e[32];
-                if (FORM == 0) {
-                    const uint4 w0 = *reinterpret_cast<const uint4*>(bp);
-                    const uint4 w1 = *reinterpret_cast<const uint4*>(bp + 16);
-                    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                    for (int o = 0; o < 8; ++o)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) e[4 * o + j] = (ws[o] >> (2 * j)) & 0x03030303u;
-                } else {
-                    const uint4 w0 = *reinterpret_cast<const uint4*>(bp);
-                    const uint32_t ws[4] = {w0.x, w0.y, w0.z, w0.w};
-#pragma unroll
-                    for (int o = 0; o < 4; ++o)
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) e[8 * o + j] = (ws[o] >> j) & 0x01010101u;
-                }
-                tc::tmem_st_32x32b_x32(lane_base + kWCol + 32 * KB * u + 32 * b, e);
+                expand_row_block<FORM>(bp, lane_base + kWCol + 32 * KB * u + 32 * b);
             }
             tc::tmem_st_wait();
             tc::tc_fence_before();
@@ -317,13 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int* tok_rsum = reinterpret_cast<int*>(tok_scale + BT);
         const int et = threadIdx.x - 64;        // 0..kEpiThreads-1
         tc::pdl_wait();                          // scale / row sums come from the previous kernel
-        for (int i = et; i < bt; i += kEpiThreads) {
-            const int row = t0 + i;
-            const int tok = FORM == 0 ? row : row >> 1;
-            const bool in = FORM == 0 ? row < p.M : tok < p.M;
-            tok_scale[i] = in ? p.scale[tok] : 0.f;
-            tok_rsum[i] = in ? p.rsum[tok] : 0;
-        }
+        fill_token_table<FORM>(p, t0, bt, et, tok_scale, tok_rsum);
         const bool acc_ok = tc::mbar_wait(bar_acc, 0, p.flags, kWaitLimitNs);
         // one decision for the eight epilogue warps; also publishes the token table
         const bool good = tc::bar_and(1, kEpiThreads, ok && acc_ok);
@@ -584,24 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int b = 0; b < KB; ++b) {
                     const uint8_t* bp = smem + OFF_BP + s * BP_STAGE + r * kRowBytes +
                                         b * PF<FORM>::kPackedRowBytes;
-                    uint32_t e[32];
-                    if (FORM == 0) {
-                        const uint4 w0 = *reinterpret_cast<const uint4*>(bp);
-                        const uint4 w1 = *reinterpret_cast<const uint4*>(bp + 16);
-                        const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                        for (int o = 0; o < 8; ++o)
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) e[4 * o + j] = (ws[o] >> (2 * j)) & 0x03030303u;
-                    } else {
-                        const uint4 w0 = *reinterpret_cast<const uint4*>(bp);
-                        const uint32_t ws[4] = {w0.x, w0.y, w0.z, w0.w};
-#pragma unroll
-                        for (int o = 0; o < 4; ++o)
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) e[8 * o + j] = (ws[o] >> j) & 0x01010101u;
-                    }
-                    tc::tmem_st_32x32b_x32(lane_base + kWCol + 32 * KB * uu + 32 * b, e);
+                    expand_row_block<FORM>(bp, lane_base + kWCol + 32 * KB * uu + 32 * b);
                 }
                 tc::tmem_st_wait();
                 tc::tc_fence_before();
@@ -611,13 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---------------- epilogue (warps 2-9) ----------------------------
             if (item == 0) tc::pdl_wait();       // scale / row sums come from the previous kernel
             // per-token scale and row sum of this activation tile
-            for (int i = et; i < bt; i += kEpiThreads) {
-                const int row = t0 + i;
-                const int tok = FORM == 0 ? row : row >> 1;
-                const bool in = FORM == 0 ? row < p.M : tok < p.M;
-                tok_scale[i] = in ? p.scale[tok] : 0.f;
-                tok_rsum[i] = in ? p.rsum[tok] : 0;
-            }
+            fill_token_table<FORM>(p, t0, bt, et, tok_scale, tok_rsum);
             const bool acc_ok = tc::mbar_wait(bar_acc, item & 1, p.flags, kWaitLimitNs);
             // one decision for the eight epilogue warps; also publishes the token table
             const bool good = tc::bar_and(1, kEpiThreads, ok && acc_ok);
