@@ -319,6 +319,85 @@ __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* _
     }
 }
 
+// Register-resident OneBit preparation: a 512-thread CTA per token keeps the
+// fp32 products x*g of up to NCH 32-element groups per thread in registers,
+// takes amax, then forms the fixed-point limbs from registers (x and g read
+// once).  Same arithmetic and output order as prep_onebit_kernel.
+template <int NCH>
+__global__ void __launch_bounds__(kRegThreads, 1)
+    prep_onebit_reg_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g, int K,
+                           int8_t* __restrict__ planes, float* __restrict__ step,
+                           int32_t* __restrict__ tsum, unsigned int* zero, int n_zero) {
+    constexpr int NW = kRegThreads / 32;
+    __shared__ uint32_t redu[NW];
+    __shared__ int redi[NW];
+    const int m = blockIdx.x;
+    const int ng = K / 32;
+    const uint16_t* row = x + (size_t)m * K;
+    tc::pdl_trigger();
+    tc::pdl_wait();
+    zero_words(zero, n_zero);
+
+    float pr[NCH][32];
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+        const int c = threadIdx.x + i * kRegThreads;
+        if (c < ng) {
+#pragma unroll
+            for (int part = 0; part < 4; ++part) {
+                const uint4 v = tc::ld_v4(row + 32 * c + 8 * part);
+                const uint4 gv = ld_ro_v4(g + 32 * c + 8 * part);
+                const uint32_t xs[4] = {v.x, v.y, v.z, v.w}, gs[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    pr[i][8 * part + e] = __fmul_rn(half_bits_to_float(xs[e >> 1] >> (16 * (e & 1))),
+                                                    half_bits_to_float(gs[e >> 1] >> (16 * (e & 1))));
+                    mx = fmaxf(mx, fabsf(pr[i][8 * part + e]));
+                }
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pr[i][e] = 0.f;
+        }
+    }
+    const float amax = __uint_as_float(block_max_u32_n<NW>(__float_as_uint(mx), redu));
+    const float inv = amax > 0.f ? __fdiv_rn((float)kFixMax, amax) : 0.f;
+
+    int sum = 0;
+    int8_t* hi_row = planes + (size_t)m * 2 * K;
+    int8_t* lo_row = hi_row + K;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+        const int c = threadIdx.x + i * kRegThreads;
+        if (c >= ng) break;
+        // byte 4j+b of the 32-byte group holds element 8b+j, the order the
+        // 1-bit unpack (w >> j) & 0x01010101 produces
+        uint32_t ho[8], lo[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ho[j] = lo[j] = 0u;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int X = rne_bits(__fmul_rn(pr[i][e], inv)) - kRneBias;   // |X| <= 32639
+            const int hi = (X + 128) >> 8;  // arithmetic shift = floor
+            ho[e & 7] |= ((uint32_t)hi & 0xffu) << (8 * (e >> 3));
+            lo[e & 7] |= ((uint32_t)(X - 256 * hi) & 0xffu) << (8 * (e >> 3));
+            sum += X;
+        }
+        uint4* hd = reinterpret_cast<uint4*>(hi_row + 32 * c);
+        uint4* ld = reinterpret_cast<uint4*>(lo_row + 32 * c);
+        hd[0] = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+        hd[1] = make_uint4(ho[4], ho[5], ho[6], ho[7]);
+        ld[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        ld[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+    }
+    const int tot = block_sum_i32_n<NW>(sum, redi);
+    if (threadIdx.x == 0) {
+        tsum[m] = tot;
+        step[m] = amax > 0.f ? __fdiv_rn(amax, (float)kFixMax) : 0.f;
+    }
+}
+
 template <auto KERN, int THREADS = kThreads, typename... Args>
 cudaError_t launch_pdl(int blocks, cudaStream_t s, Args... args) {
     static bool attr_set = false;  // one flag per kernel
@@ -378,6 +457,11 @@ cudaError_t launch_prep_onebit(const uint16_t* x, const uint16_t* g, int M, int 
                                int8_t* planes, float* step, int32_t* tsum, cudaStream_t s,
                                unsigned int* zero, int n_zero) {
     if (M == 0) return cudaSuccess;
+    const int groups = K / 32;
+    if (groups <= kRegThreads)
+        return launch_pdl<prep_onebit_reg_kernel<1>, kRegThreads>(M, s, x, g, K, planes, step, tsum, zero, n_zero);
+    if (groups <= 2 * kRegThreads)
+        return launch_pdl<prep_onebit_reg_kernel<2>, kRegThreads>(M, s, x, g, K, planes, step, tsum, zero, n_zero);
     return launch_pdl<prep_onebit_kernel>(M, s, x, g, K, planes, step, tsum, zero, n_zero);
 }
 
