@@ -45,6 +45,7 @@ ABI = {
     "ob_workspace_bytes": ([_I, _I, _I], _SZ),
     "ob_linear": ([_P, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P], _I),
     "bl_device_status": ([_P], _I),
+    "bl_prefill_plan": ([_I, _I, _I, _I, _I, _P], _I),
     "bl_ternary_linear_noalloc": ([_P, _I, _I, _I, _P, ctypes.c_float, _P, _P, _P], _I),
 }
 

@@ -254,6 +254,16 @@ bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
     return from_cuda(e);
 }
 
+bl_status bl_prefill_plan(int form, int M, int K, int N, int sm_count, int* plan) {
+    if (!plan) return BL_ERR_NULL;
+    if (form != 0 && form != 1) return BL_ERR_SHAPE;
+    if (bl_status st = check_mk(M, K)) return st;
+    if (bl_status st = check_nk(N, K)) return st;
+    if (M == 0 || N == 0 || sm_count <= 0) return BL_ERR_SHAPE;
+    bl::prefill_plan_info(form, M, K, N, sm_count, plan);
+    return BL_OK;
+}
+
 bl_status bl_device_status(bl_stream_t stream) {
     if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return BL_ERR_CUDA;
     unsigned int flags = 0;

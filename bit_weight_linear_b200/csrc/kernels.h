@@ -48,6 +48,10 @@ cudaError_t launch_onebit_skinny(const uint32_t* s1, const int8_t* planes, const
 // (the activation preparation kernel zeroes them).  Without it (NULL or too
 // small) every tile runs whole.
 size_t prefill_split_bytes(int form, int M, int K, int N, int* n_counters);
+// The same plan for an explicit SM count (host arithmetic only): activation
+// rows per tile, ring stages per tile, tiles, tiles computed whole, tiles of
+// the balanced round.
+void prefill_plan_info(int form, int M, int K, int N, int sm_count, int plan[5]);
 cudaError_t launch_ternary_prefill(const uint32_t* w2, const int8_t* qp, const float* scale,
                                    const int32_t* qsum, int M, int K, int N, float w_scale,
                                    uint16_t* y, int32_t* acc_out, unsigned int* flags,

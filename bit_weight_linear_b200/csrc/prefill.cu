@@ -901,6 +901,16 @@ cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, PrefillParams p
 
 }  // namespace
 
+void prefill_plan_info(int form, int M, int K, int N, int sm_count, int plan[5]) {
+    const Geometry g = geometry(form == 0 ? M : 2 * M, K, N);
+    const SplitPlan pl = plan_split(g, sm_count);
+    plan[0] = g.bt;
+    plan[1] = g.nk;
+    plan[2] = g.tiles;
+    plan[3] = pl.dp_tiles;
+    plan[4] = pl.sk_tiles;
+}
+
 size_t prefill_split_bytes(int form, int M, int K, int N, int* n_counters) {
     *n_counters = 0;
     if (M <= 0 || N <= 0) return 0;

@@ -198,6 +198,19 @@ bl_status bl_ternary_linear_noalloc(const uint16_t *x, int M, int K, int N, cons
                                     bl_stream_t stream);
 
 /*
+ * bl_prefill_plan -- diagnostic: how the tensor-core (prefill) path would run
+ * a call of this shape on a device with `sm_count` SMs (form 0 = ternary,
+ * 1 = OneBit, whose tiles hold two limb rows per token).  Fills plan[5]:
+ *   plan[0] activation rows per tile, plan[1] ring stages per tile,
+ *   plan[2] tiles, plan[3] tiles computed whole (one CTA each),
+ *   plan[4] tiles shared out in k-stages over sm_count CTAs in a balanced
+ *           last round (0: none).
+ * Host arithmetic only (no CUDA call).  BL_ERR_NULL without plan,
+ * BL_ERR_SHAPE for an invalid form or shape, M = 0, N = 0 or sm_count <= 0.
+ */
+bl_status bl_prefill_plan(int form, int M, int K, int N, int sm_count, int *plan);
+
+/*
  * bl_device_status -- synchronise `stream` and report (then clear) any
  * device-side condition the library's kernels recorded since the last call:
  * BL_ERR_TIMEOUT if a bounded wait inside a kernel gave up, else BL_OK
