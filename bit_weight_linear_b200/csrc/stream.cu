@@ -735,16 +735,23 @@ bool stream_plan(StreamParams& p, int prep, StreamPlan& pl, int nw = kSWarps) {
     // the reduced rows, when the first does not fit beside the activations
     const int red_full = nw * p.t_max * 16 * cols * 4;
     const int red_compact = (nw * 16 + p.t_max * 16) * cols * 4;
-    p.compact = cols * p.astride + red_full > kStreamSmemPair / 2 ? 1 : 0;
+    p.compact = act + red_full > kStreamSmemPair / 2 ? 1 : 0;
+    // A CTA that would need the compact reduction to fit beside a second CTA
+    // takes the SM alone instead, with the full per-warp reduction: the
+    // compact mode's two CTA barriers per tile cost more than the lost overlap
+    // with the next call (M = 4 on 13824-long rows: 17.8 -> 13.7 us).
+    const bool alone = p.compact && act + red_full <= kDecodeMaxSmem / 2;
+    if (alone) p.compact = 0;
     const int red = p.compact ? red_compact : red_full;
     const int tok = prep ? 0 : 2 * nw * M * 4;
     const int hbytes = FORM == 1 ? p.t_max * 16 * 2 : 0;
     auto up16 = [](int v) { return (v + 15) & ~15; };
     const int fixed = up16(act) + up16(red) + up16(tok) + up16(hbytes) + 16 * kMaxSlots + 8 * kMaxSlots;
     for (int cand = 0; cand < 4; ++cand) {
-        // (depth, budget): two CTAs per SM with 48-, 32- then 16-step boxes, else one
+        // (depth, budget): two CTAs per SM with 48-, 32- then 16-step boxes, else
+        // one (from the start for a CTA that takes the SM alone)
         const int depth = cand == 0 ? 48 : cand == 1 ? 32 : 16;
-        const int budget = cand < 3 ? kStreamSmemPair : kDecodeMaxSmem;
+        const int budget = alone || cand == 3 ? kDecodeMaxSmem : kStreamSmemPair;
         set_depth(depth);
         const int nst = p.t_max * p.nch;
         int S = (budget - fixed) / p.slot_bytes;
