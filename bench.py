@@ -560,6 +560,11 @@ def main():
                                                 layers=[("q", 4096, 4096)], ms_list=[8])
         extras["onebit_4096"] = run_sweep(blw, synth, dev, peaks, forms=("onebit",),
                                           layers=[("q", 4096, 4096)], ms_list=[1, 16])
+        # the decode sweep per layer shape: each 7B-shaped layer alone at M=1, in a
+        # chain of calls over rotating weight copies larger than L2
+        extras["decode_layers_7b"] = run_sweep(blw, synth, dev, peaks, forms=("ternary", "onebit"),
+                                               layers=[("q/k/v/o", 4096, 4096), ("gate/up", 4096, 11008),
+                                                       ("down", 11008, 4096)], ms_list=[1])
         if not args.no_sweep:
             extras["batch_sweep_13b"] = run_sweep(blw, synth, dev, peaks)
 
