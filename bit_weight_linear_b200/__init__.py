@@ -47,6 +47,7 @@ ABI = {
     "bl_device_status": ([_P], _I),
     "bl_prefill_plan": ([_I, _I, _I, _I, _I, _P], _I),
     "bl_ternary_linear_noalloc": ([_P, _I, _I, _I, _P, ctypes.c_float, _P, _P, _P], _I),
+    "bl_debug_stall_next_launch": ([ctypes.c_ulonglong], _I),
 }
 
 

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI (include/bitlinear.h): argument validation, workspace
 // layout and shape dispatch.  No allocation happens here; all buffers are the
 // caller's.
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -44,7 +45,7 @@ bl_status check_nk(int N, int K) {
 
 // Workspace layouts (offsets in bytes, each region 256-byte aligned):
 //   ternary: [0] permuted q  M*K int8 | scale M fp32 | row sums M int32 | split
-//   onebit : [0] limb planes 2*M*K int8 | step M fp32 | row sums M int32 | split
+//   onebit : [0] limb planes 3*M*K int8 | step M fp32 | image sums M int64 | split
 // `split` is the prefill kernel's scratch for sharing out its last round
 // (arrival counters + partial accumulators); empty unless the call takes the
 // prefill path and its tiles leave SMs idle in the last round.
@@ -56,9 +57,9 @@ struct WsLayout {
 WsLayout ws_layout(int form, int M, int K, int N) {
     WsLayout l;
     l.act = 0;
-    l.scale = align_up((size_t)M * (size_t)K * (size_t)(form == 0 ? 1 : 2));
+    l.scale = align_up((size_t)M * (size_t)K * (size_t)(form == 0 ? 1 : 3));
     l.rsum = l.scale + align_up((size_t)M * sizeof(float));
-    l.split = l.rsum + align_up((size_t)M * sizeof(int32_t));
+    l.split = l.rsum + align_up((size_t)M * (form == 0 ? sizeof(int32_t) : sizeof(long long)));
     l.split_bytes = 0;
     l.n_ctr = 0;
     const int min_m = form == 0 ? bl::kTernaryPrefillMinM : bl::kOnebitPrefillMinM;
@@ -112,6 +113,64 @@ int bl::device_sm_count() {
     return cached[dev];
 }
 
+// Host-side fault injection for callers' error paths: with the environment
+// variable BL_FAULT_INJECT set to "cuda" or "timeout", every entry point that
+// would launch work returns BL_ERR_CUDA or BL_ERR_TIMEOUT after validating its
+// arguments and before any CUDA call.  Read on every call (a test may change
+// it between calls).  Nothing on the device is touched.
+bl_status bl::fault_injected() {
+    const char* v = std::getenv("BL_FAULT_INJECT");
+    if (v == nullptr || *v == 0) return BL_OK;
+    if (std::strcmp(v, "cuda") == 0) return BL_ERR_CUDA;
+    if (std::strcmp(v, "timeout") == 0) return BL_ERR_TIMEOUT;
+    return BL_OK;
+}
+
+namespace {
+// Pending stall of the next streamed-decode or whole-tile tensor-core launch
+// (bl_debug_stall_next_launch); 0 = none.
+std::atomic<unsigned long long> g_stall_next{0};
+}  // namespace
+
+unsigned long long bl::take_stall() {
+    if (g_stall_next.load(std::memory_order_relaxed) == 0) return 0;
+    return g_stall_next.exchange(0);
+}
+
+size_t bl::ternary_act_bytes(int M, int K) { return ws_layout(0, M, K, 0).split; }
+
+bl_status bl::ternary_linear_on(const uint16_t* x, int M, int K, int N, const uint32_t* w2,
+                                float w_scale, uint16_t* y, int32_t* acc_out, void* workspace,
+                                size_t workspace_bytes, cudaStream_t s) {
+    if (bl_status st = bl::fault_injected()) return st;
+    unsigned int* flags = device_flags();
+    if (!flags) return BL_ERR_CUDA;
+    if (M <= bl::kStreamFusedMaxM && bl::stream_fits(0, M, K, N, 0))
+        return from_cuda(bl::launch_ternary_stream(x, w2, M, K, N, w_scale, y, acc_out, flags, s));
+    WsLayout l = ws_layout(0, M, K, N);
+    if (workspace_bytes < l.total) {   // room for the activations only: whole prefill tiles
+        l.split_bytes = 0;
+        l.n_ctr = 0;
+    }
+    char* ws = static_cast<char*>(workspace);
+    int8_t* qp = reinterpret_cast<int8_t*>(ws + l.act);
+    float* sc = reinterpret_cast<float*>(ws + l.scale);
+    int32_t* qs = reinterpret_cast<int32_t*>(ws + l.rsum);
+    unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + l.split);
+    cudaError_t e = bl::launch_quant_ternary_perm(x, M, K, qp, sc, qs, s, ctr, l.n_ctr);
+    if (e != cudaSuccess) return BL_ERR_CUDA;
+    if (M >= bl::kTernaryPrefillMinM) {
+        e = bl::launch_ternary_prefill(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, flags, s,
+                                       l.split_bytes ? ws + l.split : nullptr, l.split_bytes);
+    } else {
+        e = bl::stream_fits(0, M, K, N, 1)
+                ? bl::launch_ternary_stream_prepared(qp, sc, qs, w2, M, K, N, w_scale, y, acc_out,
+                                                     flags, s)
+                : bl::launch_ternary_skinny(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, s);
+    }
+    return from_cuda(e);
+}
+
 extern "C" {
 
 const char* bl_status_string(int status) {
@@ -137,6 +196,7 @@ bl_status bl_pack_ternary(const int8_t* w, int N, int K, uint32_t* w2, bl_stream
     if (N == 0) return BL_OK;
     if (!w || !w2) return BL_ERR_NULL;
     if (misaligned(w) || misaligned(w2)) return BL_ERR_ALIGN;
+    if (bl_status st = bl::fault_injected()) return st;
     unsigned int* flag = nullptr;
     if (bl_status st = pack_begin(&flag, cs(stream))) return st;
     return pack_finish(bl::launch_pack_ternary(w, N, K, w2, flag, cs(stream)), cs(stream));
@@ -147,6 +207,7 @@ bl_status ob_pack_sign(const uint16_t* w, int N, int K, uint32_t* s1, bl_stream_
     if (N == 0) return BL_OK;
     if (!w || !s1) return BL_ERR_NULL;
     if (misaligned(w) || misaligned(s1)) return BL_ERR_ALIGN;
+    if (bl_status st = bl::fault_injected()) return st;
     unsigned int* flag = nullptr;
     if (bl_status st = pack_begin(&flag, cs(stream))) return st;
     return pack_finish(bl::launch_pack_sign(w, N, K, s1, flag, cs(stream)), cs(stream));
@@ -158,6 +219,7 @@ bl_status bl_quant_act(const uint16_t* x, int M, int K, int8_t* q, float* scale,
     if (M == 0) return BL_OK;
     if (!x || !q || !scale) return BL_ERR_NULL;
     if (misaligned(x) || misaligned(q) || misaligned(scale)) return BL_ERR_ALIGN;
+    if (bl_status st = bl::fault_injected()) return st;
     return from_cuda(bl::launch_quant_plain(x, M, K, q, scale, cs(stream)));
 }
 
@@ -178,34 +240,8 @@ bl_status bl_ternary_linear(const uint16_t* x, int M, int K, int N, const uint32
     const WsLayout l = ws_layout(0, M, K, N);
     if (!workspace || workspace_bytes < l.total) return BL_ERR_WORKSPACE;
     if (misaligned(workspace)) return BL_ERR_ALIGN;
-    unsigned int* flags = device_flags();
-    if (!flags) return BL_ERR_CUDA;
-    if (M <= bl::kStreamFusedMaxM && bl::stream_fits(0, M, K, N, 0))
-        return from_cuda(
-            bl::launch_ternary_stream(x, w2, M, K, N, w_scale, y, acc_out, flags, cs(stream)));
-    if (M <= bl::kFusedMaxM && bl::decode_fused_fits(0, M, K))
-        return from_cuda(
-            bl::launch_ternary_decode(x, w2, M, K, N, w_scale, y, acc_out, flags, cs(stream)));
-    char* ws = static_cast<char*>(workspace);
-    int8_t* qp = reinterpret_cast<int8_t*>(ws + l.act);
-    float* sc = reinterpret_cast<float*>(ws + l.scale);
-    int32_t* qs = reinterpret_cast<int32_t*>(ws + l.rsum);
-    unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + l.split);
-    cudaError_t e = bl::launch_quant_ternary_perm(x, M, K, qp, sc, qs, cs(stream), ctr, l.n_ctr);
-    if (e != cudaSuccess) return BL_ERR_CUDA;
-    if (M >= bl::kTernaryPrefillMinM) {
-        e = bl::launch_ternary_prefill(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, flags,
-                                       cs(stream), ws + l.split, l.split_bytes);
-    } else {
-        e = bl::stream_fits(0, M, K, N, 1)
-                ? bl::launch_ternary_stream_prepared(qp, sc, qs, w2, M, K, N, w_scale, y, acc_out,
-                                                     flags, cs(stream))
-            : bl::decode_prepared_fits(0, M, K)
-                ? bl::launch_ternary_decode_prepared(qp, sc, qs, w2, M, K, N, w_scale, y, acc_out,
-                                                     flags, cs(stream))
-                : bl::launch_ternary_skinny(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, cs(stream));
-    }
-    return from_cuda(e);
+    return bl::ternary_linear_on(x, M, K, N, w2, w_scale, y, acc_out, workspace, workspace_bytes,
+                                 cs(stream));
 }
 
 size_t ob_workspace_bytes(int M, int K, int N) {
@@ -226,16 +262,15 @@ bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
     const WsLayout l = ws_layout(1, M, K, N);
     if (!workspace || workspace_bytes < l.total) return BL_ERR_WORKSPACE;
     if (misaligned(workspace)) return BL_ERR_ALIGN;
+    if (bl_status st = bl::fault_injected()) return st;
     unsigned int* flags = device_flags();
     if (!flags) return BL_ERR_CUDA;
-    if (M <= bl::kStreamFusedMaxM / 2 && bl::stream_fits(1, M, K, N, 0))
+    if (M <= bl::kStreamFusedMaxMOnebit && bl::stream_fits(1, M, K, N, 0))
         return from_cuda(bl::launch_onebit_stream(x, g, h, s1, M, K, N, y, flags, cs(stream)));
-    if (M <= bl::kFusedMaxM && bl::decode_fused_fits(1, M, K))
-        return from_cuda(bl::launch_onebit_decode(x, g, h, s1, M, K, N, y, flags, cs(stream)));
     char* ws = static_cast<char*>(workspace);
     int8_t* planes = reinterpret_cast<int8_t*>(ws + l.act);
     float* step = reinterpret_cast<float*>(ws + l.scale);
-    int32_t* ts = reinterpret_cast<int32_t*>(ws + l.rsum);
+    long long* ts = reinterpret_cast<long long*>(ws + l.rsum);
     unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + l.split);
     cudaError_t e = bl::launch_prep_onebit(x, g, M, K, planes, step, ts, cs(stream), ctr, l.n_ctr);
     if (e != cudaSuccess) return BL_ERR_CUDA;
@@ -245,9 +280,6 @@ bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
     } else {
         e = bl::stream_fits(1, M, K, N, 1)
                 ? bl::launch_onebit_stream_prepared(planes, step, ts, h, s1, M, K, N, y, flags,
-                                                    cs(stream))
-            : bl::decode_prepared_fits(1, M, K)
-                ? bl::launch_onebit_decode_prepared(planes, step, ts, h, s1, M, K, N, y, flags,
                                                     cs(stream))
                 : bl::launch_onebit_skinny(s1, planes, step, ts, h, M, K, N, y, cs(stream));
     }
@@ -261,6 +293,11 @@ bl_status bl_prefill_plan(int form, int M, int K, int N, int sm_count, int* plan
     if (bl_status st = check_nk(N, K)) return st;
     if (M == 0 || N == 0 || sm_count <= 0) return BL_ERR_SHAPE;
     bl::prefill_plan_info(form, M, K, N, sm_count, plan);
+    return BL_OK;
+}
+
+bl_status bl_debug_stall_next_launch(unsigned long long wait_limit_ns) {
+    g_stall_next.store(wait_limit_ns);
     return BL_OK;
 }
 

@@ -66,4 +66,37 @@ __device__ __forceinline__ int warp_sum(int v) {
     return v;
 }
 
+__device__ __forceinline__ long long warp_sum64(long long v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// OneBit fixed-point image of a token's x*g (fp32 products, exact for fp16
+// inputs): X = rne(x*g * rn(kImgMax / amax')), amax' = max_k |x*g|, so
+// |X| <= kImgMax = 2^22 - 1.  The fp32 product exceeds kImgMax by at most
+// kImgMax * 2^-24 < 0.25 and rounds back to kImgMax; and |t| < 2^22 is the
+// range in which rne_bits is exact.  The image's error is at most
+// amax' / (2 kImgMax) ~ 1.2e-7 amax' per element.
+constexpr int kImgMax = 4194303;
+constexpr float kImgMaxF = 4194303.0f;
+
+// Balanced base-256 digits of an image value: X = 65536 hi + 256 mid + lo with
+// every digit in [-128, 127] (hi in [-64, 64] for |X| <= kImgMax), so each
+// digit is an int8 MMA operand and each limb's contraction is exact in int32.
+__device__ __forceinline__ void split_limbs(int X, int& hi, int& mid, int& lo) {
+    const int x1 = (X + 128) >> 8;   // arithmetic shift = floor
+    lo = X - 256 * x1;
+    hi = (x1 + 128) >> 8;
+    mid = x1 - 256 * hi;
+}
+
+// sum X*S from the three limbs' 0/1-bit contractions D_l = sum limb_l * b
+// (b = (S+1)/2) and the token's image sum sum X:
+//   sum X*S = 2 (65536 D_hi + 256 D_mid + D_lo) - sum X      (exact in int64)
+__device__ __forceinline__ long long limb_combine(int d_hi, int d_mid, int d_lo, long long xsum) {
+    const long long P = 65536ll * d_hi + 256ll * d_mid + (long long)d_lo;
+    return 2 * P - xsum;
+}
+
 }  // namespace bl

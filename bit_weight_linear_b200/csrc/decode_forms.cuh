@@ -22,9 +22,9 @@ struct DF<0> {  // ternary, 2-bit codes
     static constexpr uint32_t kMask = 0x03030303u;
 };
 template <>
-struct DF<1> {  // sign, 1 bit; two activation columns (int8 limbs) per token
+struct DF<1> {  // sign, 1 bit; three activation columns (int8 limbs hi, mid, lo) per token
     static constexpr int kPerWord = 32, kRegs = 8, kShift = 1, kStepK = 512, kChunkK = 128;
-    static constexpr int kCPT = 2, kGroup = 32;
+    static constexpr int kCPT = 3, kGroup = 32;
     static constexpr uint32_t kMask = 0x01010101u;
 };
 

@@ -2,9 +2,14 @@
 // the ABI layer in api.cu checks shapes, pointers and workspace first).
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
+
 #include <cuda_runtime.h>
+
+#include "bitlinear.h"
 
 namespace bl {
 
@@ -18,8 +23,8 @@ cudaError_t launch_pack_sign(const uint16_t* w, int N, int K, uint32_t* s1,
 // Activation preparation (quant.cu).
 //   plain   : q [M][K] in natural k order, scale [M]          (bl_quant_act)
 //   ternary : q [M][K] in the decode kernel's permuted order, scale, row sum
-//   onebit  : 16-bit fixed-point image of x*g split into two int8 limb planes
-//             [M][2][K] (permuted), fixed-point step [M], row sum of the image
+//   onebit  : 23-bit fixed-point image of x*g split into three int8 limb planes
+//             [M][3][K] (permuted), fixed-point step [M], sum of the image [M] (int64)
 cudaError_t launch_quant_plain(const uint16_t* x, int M, int K, int8_t* q, float* scale,
                                cudaStream_t s);
 // The ternary and onebit preparations also zero `n_zero` words at `zero` (the
@@ -28,7 +33,7 @@ cudaError_t launch_quant_ternary_perm(const uint16_t* x, int M, int K, int8_t* q
                                       float* scale, int32_t* qsum, cudaStream_t s,
                                       unsigned int* zero = nullptr, int n_zero = 0);
 cudaError_t launch_prep_onebit(const uint16_t* x, const uint16_t* g, int M, int K,
-                               int8_t* planes, float* step, int32_t* tsum, cudaStream_t s,
+                               int8_t* planes, float* step, long long* tsum, cudaStream_t s,
                                unsigned int* zero = nullptr, int n_zero = 0);
 
 // Decode-shaped (small M) packed-weight kernels on warp-level int8 MMA (skinny.cu).
@@ -36,7 +41,7 @@ cudaError_t launch_ternary_skinny(const uint32_t* w2, const int8_t* qp, const fl
                                   const int32_t* qsum, int M, int K, int N, float w_scale,
                                   uint16_t* y, int32_t* acc_out, cudaStream_t s);
 cudaError_t launch_onebit_skinny(const uint32_t* s1, const int8_t* planes, const float* step,
-                                 const int32_t* tsum, const uint16_t* h, int M, int K, int N,
+                                 const long long* tsum, const uint16_t* h, int M, int K, int N,
                                  uint16_t* y, cudaStream_t s);
 
 // Prefill-shaped (large M) GEMM on tcgen05 int8 tensor cores with TMEM
@@ -58,42 +63,35 @@ cudaError_t launch_ternary_prefill(const uint32_t* w2, const int8_t* qp, const f
                                    cudaStream_t s, void* split_ws = nullptr,
                                    size_t split_ws_bytes = 0);
 cudaError_t launch_onebit_prefill(const uint32_t* s1, const int8_t* planes, const float* step,
-                                  const int32_t* tsum, const uint16_t* h, int M, int K, int N,
+                                  const long long* tsum, const uint16_t* h, int M, int K, int N,
                                   uint16_t* y, unsigned int* flags, cudaStream_t s,
                                   void* split_ws = nullptr, size_t split_ws_bytes = 0);
 
 // Number of SMs of the current device (cached per device; 0 on error).
 int device_sm_count();
 
-// Per-16-row decode (decode.cu): activation preparation + contraction in one
-// kernel, one CTA per 16 weight rows, weights bulk-copied to shared memory
-// before the programmatic-dependent-launch wait.  The fallback for shapes the
-// streamed decode kernel (stream.cu) has no plan for.
+// Largest dynamic shared memory of a CTA (227 KB on sm_100a).
 constexpr int kDecodeMaxSmem = 227 * 1024;
-bool decode_fused_fits(int form, int M, int K);
-cudaError_t launch_ternary_decode(const uint16_t* x, const uint32_t* w2, int M, int K, int N,
-                                  float w_scale, uint16_t* y, int32_t* acc_out,
-                                  unsigned int* flags, cudaStream_t s);
-cudaError_t launch_onebit_decode(const uint16_t* x, const uint16_t* g, const uint16_t* h,
-                                 const uint32_t* s1, int M, int K, int N, uint16_t* y,
-                                 unsigned int* flags, cudaStream_t s);
 
 // Device address of the condition word bounded waits mark (nullptr on error).
 unsigned int* device_flags_address();
 
-// The same decode kernel on activations prepared by launch_quant_ternary_perm /
-// launch_prep_onebit (launched just before; both kernels use programmatic
-// dependent launch).  Used for small M > kFusedMaxM, where preparing the
-// activations once beats preparing them in every CTA.
-cudaError_t launch_ternary_decode_prepared(const int8_t* qp, const float* scale, const int32_t* qsum,
-                                           const uint32_t* w2, int M, int K, int N, float w_scale,
-                                           uint16_t* y, int32_t* acc_out, unsigned int* flags,
-                                           cudaStream_t s);
-cudaError_t launch_onebit_decode_prepared(const int8_t* planes, const float* step,
-                                          const int32_t* tsum, const uint16_t* h,
-                                          const uint32_t* s1, int M, int K, int N, uint16_t* y,
-                                          unsigned int* flags, cudaStream_t s);
-bool decode_prepared_fits(int form, int M, int K);
+// The BitLinear forward behind bl_ternary_linear and bl_ternary_linear_noalloc
+// (api.cu), with the ABI's argument checks already done.  The workspace holds
+// at least ternary_act_bytes(M, K) bytes (the prepared activations, scales and
+// row sums); the prefill kernel's balanced last round is used only when it
+// also holds that round's scratch (bl_ternary_workspace_bytes).
+size_t ternary_act_bytes(int M, int K);
+// BL_FAULT_INJECT ("cuda" / "timeout"): the error every launching entry point
+// returns after its argument checks, BL_OK when unset (api.cu).
+bl_status fault_injected();
+// The stall bl_debug_stall_next_launch asked for (its wait limit in ns), taken
+// by the next streamed-decode or whole-tile tensor-core launch; 0 = none.
+unsigned long long take_stall();
+bl_status ternary_linear_on(const uint16_t* x, int M, int K, int N, const uint32_t* w2,
+                            float w_scale, uint16_t* y, int32_t* acc_out, void* workspace,
+                            size_t workspace_bytes, cudaStream_t s);
+
 // Streamed decode (stream.cu): at most one 512-thread CTA per SM, each owning a
 // contiguous range of 16-row tiles streamed through a shared-memory ring that
 // is filled before the programmatic-dependent-launch wait.  prep = 0: the CTA
@@ -111,7 +109,7 @@ cudaError_t launch_ternary_stream_prepared(const int8_t* qp, const float* scale,
                                            uint16_t* y, int32_t* acc_out, unsigned int* flags,
                                            cudaStream_t s);
 cudaError_t launch_onebit_stream_prepared(const int8_t* planes, const float* step,
-                                          const int32_t* tsum, const uint16_t* h,
+                                          const long long* tsum, const uint16_t* h,
                                           const uint32_t* s1, int M, int K, int N, uint16_t* y,
                                           unsigned int* flags, cudaStream_t s);
 
@@ -126,16 +124,48 @@ inline cudaError_t use_max_shared_carveout(Kern kern) {
                                 (int)cudaSharedmemCarveoutMaxShared);
 }
 
-// Largest M for which the decode kernel prepares the activations itself.
-constexpr int kFusedMaxM = 2;
-// Largest M (ternary; half of it for OneBit, two columns per token) for which
-// the streamed decode CTA prepares the activations itself.
+// One-time setup of a kernel's launch attributes (maximum dynamic shared
+// memory, shared-memory carveout), done once per device: cudaFuncSetAttribute
+// acts on the current device's context only, so a process that runs the
+// library on several devices sets them on each.  Safe to call from several
+// host threads.  Each launcher keeps one function-local static instance per
+// kernel.
+class KernelAttrs {
+public:
+    template <typename Kern>
+    cudaError_t ensure(Kern kern, int max_dyn_smem) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+        if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        std::lock_guard<std::mutex> lk(mu_);
+        if (done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+        if (max_dyn_smem > 0) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn_smem);
+            if (e != cudaSuccess) return e;
+        }
+        e = use_max_shared_carveout(kern);
+        if (e != cudaSuccess) return e;
+        done_[dev].store(true, std::memory_order_release);
+        return cudaSuccess;
+    }
+
+private:
+    static constexpr int kMaxDev = 128;
+    std::mutex mu_;
+    std::atomic<bool> done_[kMaxDev] = {};
+};
+
+// Largest M for which the streamed decode CTA prepares the activations itself
+// (ternary; OneBit, three columns per token, up to M = 2).
 constexpr int kStreamFusedMaxM = 8;
+constexpr int kStreamFusedMaxMOnebit = 2;
 
 // Token counts at or above which the tensor-core prefill kernel is used
 // (measured crossovers on 13B-shaped layers: ternary M = 16 runs 26 % faster
 // there than in the prepared streamed kernel; OneBit M = 8 up to 56 % faster,
-// while OneBit M = 4 is still faster streamed on the 13824-long rows).
+// while OneBit M = 4 was still faster streamed on the 13824-long rows).
 constexpr int kTernaryPrefillMinM = 9;
 constexpr int kOnebitPrefillMinM = 5;
 

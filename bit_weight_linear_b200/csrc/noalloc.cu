@@ -7,9 +7,11 @@
 // loop whose rules forbid allocation because cudaMalloc can block on the whole
 // device.  For them this entry point needs only inputs and outputs: its scratch
 // (the prepared int8 activations, token scales and row sums) lives in a
-// fixed-size array compiled into this library.  The arithmetic and the kernels
-// are those of bl_ternary_linear's two-kernel path (activation preparation,
-// then the packed-weight contraction), so results are identical.
+// fixed-size array compiled into this library.  It runs the same forward as
+// bl_ternary_linear (same kernels, same dispatch by shape), so results are
+// identical; only the tensor-core path's balanced last round, whose scratch
+// grows with the layer, is left out when it would not fit in the array (every
+// tile then runs whole, with the same integers).
 //
 // The array is a file-scope __device__ variable: every GPU that loads this
 // library holds one copy of it until the process exits.  Host code cannot use
@@ -46,8 +48,6 @@ bl_status scratch_address(void** out) {
     return BL_OK;
 }
 
-inline size_t round256(size_t v) { return (v + 255) / 256 * 256; }
-
 inline bool misaligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
 }  // namespace
@@ -62,28 +62,15 @@ extern "C" bl_status bl_ternary_linear_noalloc(const uint16_t* x, int M, int K, 
     if (!x || !w2 || !y) return BL_ERR_NULL;
     if (misaligned16(x) || misaligned16(w2) || misaligned16(y) || misaligned16(acc_out))
         return BL_ERR_ALIGN;
-    // scratch layout: permuted q [M][K] | token scales [M] | row sums [M], each 256-aligned
-    const size_t off_scale = round256((size_t)M * (size_t)K);
-    const size_t off_rsum = off_scale + round256((size_t)M * sizeof(float));
-    const size_t need = off_rsum + round256((size_t)M * sizeof(int32_t));
-    if (need > kScratchBytes) return BL_ERR_SCRATCH_LIMIT;
-
+    // scratch layout: permuted q [M][K] | token scales [M] | row sums [M], each
+    // 256-byte aligned (the layout of bl_ternary_linear's workspace)
+    if (bl::ternary_act_bytes(M, K) > kScratchBytes) return BL_ERR_SCRATCH_LIMIT;
+    if (bl_status st = bl::fault_injected()) return st;
     void* base = nullptr;
     if (bl_status st = scratch_address(&base)) return st;
-    unsigned int* flags = bl::device_flags_address();
-    if (!flags) return BL_ERR_CUDA;
-    char* ws = static_cast<char*>(base);
-    int8_t* qp = reinterpret_cast<int8_t*>(ws);
-    float* sc = reinterpret_cast<float*>(ws + off_scale);
-    int32_t* qs = reinterpret_cast<int32_t*>(ws + off_rsum);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // Every scratch byte read below is first written by this call's preparation
-    // kernel, so nothing needs clearing between calls.
-    if (bl::launch_quant_ternary_perm(x, M, K, qp, sc, qs, s) != cudaSuccess) return BL_ERR_CUDA;
-    cudaError_t e;
-    if (M >= bl::kTernaryPrefillMinM)
-        e = bl::launch_ternary_prefill(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, flags, s);
-    else
-        e = bl::launch_ternary_skinny(w2, qp, sc, qs, M, K, N, w_scale, y, acc_out, s);
-    return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+    // Every scratch byte the kernels read is first written by this call's
+    // activation kernel (which also zeroes the balanced round's counters), so
+    // nothing needs clearing between calls.
+    return bl::ternary_linear_on(x, M, K, N, w2, w_scale, y, acc_out, base, kScratchBytes,
+                                 reinterpret_cast<cudaStream_t>(stream));
 }

@@ -6,9 +6,9 @@
 // "1. 新的 1bit 结构": the +-1 matrix between x*g and h), so the weights are
 // expanded on chip to int8 and run through the int8 tensor cores:
 //   ternary: code in {0,1,2} (= t + 1), D = code . q^T, acc = D - sum_k q
-//   OneBit : bit in {0,1}, activation rows = the two int8 limbs (hi, lo) of each
-//            token's 16-bit fixed-point image X of x*g, so
-//            sum X*S = 2 (256 D_hi + D_lo) - sum X
+//   OneBit : bit in {0,1}, activation rows = the three int8 limbs (hi, mid, lo)
+//            of each token's 23-bit fixed-point image X of x*g, so
+//            sum X*S = 2 (65536 D_hi + 256 D_mid + D_lo) - sum X
 // Both are exact in int32.
 //
 // The expanded weights never touch shared memory: they are the MMA's A
@@ -21,7 +21,9 @@
 // CTA tile: 128 weight rows (MMA M, TMEM lanes) x bt activation rows (MMA N:
 // tokens, or token limb rows; bt = the smallest multiple of 32 covering them,
 // at most 256), K in 128-byte stages; tiles ordered
-// activation-tile-fastest so CTAs sharing a weight tile run together.
+// activation-tile-fastest so CTAs sharing a weight tile run together.  A
+// OneBit tile holds tpt <= bt/3 whole tokens (3 tpt limb rows; the rows past
+// them are loaded but unused), so a token's limbs never straddle two tiles.
 // Warp roles (320 threads):
 //   warp 0     TMA producer: activation tile (256 x 128 B) and packed weight tile
 //              (128 rows x 32 B or 16 B) into a 5-stage shared-memory ring; the
@@ -87,11 +89,14 @@ struct PF<1> {  // sign
 };
 
 struct PrefillParams {
-    int rows_a;        // activation rows: M (ternary) or 2M (OneBit limb rows)
+    int rows_a;        // activation rows: M (ternary) or 3M (OneBit limb rows)
     int bt;            // activation rows per tile: multiple of 32, <= BT
+    int tpt;           // tokens per tile: bt (ternary), <= bt / 3 (OneBit)
+    int rpt;           // first activation row of token tile i is i * rpt (bt; 3 tpt)
     int M, K, N;
     const float* scale;   // per token: ternary scale / OneBit fixed-point step
-    const int32_t* rsum;  // per token: sum q / sum X
+    const int32_t* rsum;  // ternary, per token: sum q
+    const long long* xsum;  // OneBit, per token: sum X
     const uint16_t* h;    // OneBit output value vector
     float w_scale;
     uint16_t* y;
@@ -105,6 +110,11 @@ struct PrefillParams {
     int dp_tiles, sk_tiles, sk_ctas;
     unsigned int* sk_ctr;  // [sk_tiles] arrival counts, zero when the kernel starts
     int32_t* sk_slots;     // [2 * sk_ctas][bt * BW] partial accumulators
+    // Whole-tile kernel: the limit of a pipeline wait (2 s).  Test hook
+    // (bl_debug_stall_next_launch): stall = 1 leaves CTA 0's first activation
+    // stage unrequested, so the MMA's wait for it runs out after wait_ns.
+    uint64_t wait_ns;
+    int stall;
 };
 
 // Expand one weight row's 128 k of packed codes (32 B ternary / 16 B sign at
@@ -133,53 +143,64 @@ __device__ __forceinline__ void expand_row_block(const uint8_t* bp, uint32_t tad
     tc::tmem_st_32x32b_x32(taddr, e);
 }
 
-// Per-token scale and row sum of the activation rows [t0, t0 + bt) (token rows
-// for ternary, limb-row pairs for OneBit), zero past M; filled by the
-// epilogue threads et = 0 .. kEpiThreads-1.
+// Per-token scale and row sum of the tile's tokens [tok0, tok0 + tpt), zero
+// past M; filled by the epilogue threads et = 0 .. kEpiThreads-1.  The row
+// sums are int32 (ternary, tok_rsum) or int64 (OneBit, tok_xsum; the same
+// shared-memory bytes).
 template <int FORM>
-__device__ __forceinline__ void fill_token_table(const PrefillParams& p, int t0, int bt, int et,
+__device__ __forceinline__ void fill_token_table(const PrefillParams& p, int tok0, int et,
                                                  float* tok_scale, int* tok_rsum) {
-    for (int i = et; i < bt; i += kEpiThreads) {
-        const int row = t0 + i;
-        const int tok = FORM == 0 ? row : row >> 1;
-        const bool in = FORM == 0 ? row < p.M : tok < p.M;
+    long long* tok_xsum = reinterpret_cast<long long*>(tok_rsum);
+    for (int i = et; i < p.tpt; i += kEpiThreads) {
+        const int tok = tok0 + i;
+        const bool in = tok < p.M;
         tok_scale[i] = in ? p.scale[tok] : 0.f;
-        tok_rsum[i] = in ? p.rsum[tok] : 0;
+        if (FORM == 0) tok_rsum[i] = in ? p.rsum[tok] : 0;
+        else tok_xsum[i] = in ? p.xsum[tok] : 0ll;
     }
 }
 
-// Epilogue of one 32-token chunk of accumulators d (TMEM lane = weight row r,
-// output column n): bias by the token row sums, scale, round to fp16 and stage
-// as [token][128 columns]; optionally also store the int32 accumulators.
-template <int FORM>
+// Ternary epilogue of one 32-token chunk of accumulators d (TMEM lane = weight
+// row r, output column n): bias by the token row sums, scale, round to fp16
+// and stage as [token][128 columns]; optionally also store the int32
+// accumulators.
 __device__ __forceinline__ void convert_chunk(const uint32_t (&d)[32], int cc, uint16_t* stage,
                                               const float* tok_scale, const int* tok_rsum,
-                                              const PrefillParams& p, int r, int n, int t0,
-                                              float hn) {
-    if (FORM == 0) {
+                                              const PrefillParams& p, int r, int n, int t0) {
 #pragma unroll
-        for (int i4 = 0; i4 < 32; i4 += 4) {
-            const int tb = 32 * cc + i4;
-            const float4 sc = *reinterpret_cast<const float4*>(tok_scale + tb);
-            const int4 rs = *reinterpret_cast<const int4*>(tok_rsum + tb);
-            const float scs[4] = {sc.x, sc.y, sc.z, sc.w};
-            const int rss[4] = {rs.x, rs.y, rs.z, rs.w};
+    for (int i4 = 0; i4 < 32; i4 += 4) {
+        const int tb = 32 * cc + i4;
+        const float4 sc = *reinterpret_cast<const float4*>(tok_scale + tb);
+        const int4 rs = *reinterpret_cast<const int4*>(tok_rsum + tb);
+        const float scs[4] = {sc.x, sc.y, sc.z, sc.w};
+        const int rss[4] = {rs.x, rs.y, rs.z, rs.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int a = (int)d[i4 + j] - rss[j];
-                const float v = __fmul_rn(__fmul_rn((float)a, scs[j]), p.w_scale);
-                stage[(tb + j) * BW + r] = __half_as_ushort(__float2half_rn(v));
-                const int m = t0 + tb + j;
-                if (p.acc_out && m < p.M && n < p.N) p.acc_out[(size_t)m * p.N + n] = a;
-            }
+        for (int j = 0; j < 4; ++j) {
+            const int a = (int)d[i4 + j] - rss[j];
+            const float v = __fmul_rn(__fmul_rn((float)a, scs[j]), p.w_scale);
+            stage[(tb + j) * BW + r] = __half_as_ushort(__float2half_rn(v));
+            const int m = t0 + tb + j;
+            if (p.acc_out && m < p.M && n < p.N) p.acc_out[(size_t)m * p.N + n] = a;
         }
-    } else {
+    }
+}
+
+// OneBit epilogue of token group gi (tokens 32 gi .. 32 gi + 31 of the tile,
+// accumulator columns 96 gi .. 96 gi + 95 in d): combine each token's three
+// limb columns, scale by its step and h[n], round to fp16 and stage as
+// [token][128 columns].  Tokens past the tile's tpt are skipped.
+__device__ __forceinline__ void convert_onebit_group(const uint32_t (&d)[96], int gi,
+                                                     uint16_t* stage, const float* tok_scale,
+                                                     const long long* tok_xsum, int tpt, int r,
+                                                     float hn) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-            const int ti = 32 * cc + i;
-            const long long P = 256ll * (int)d[i] + (int)d[i + 1];
-            const float z = __fmul_rn(tok_scale[ti], (float)(2 * P - (long long)tok_rsum[ti]));
-            stage[(ti >> 1) * BW + r] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hn)));
+    for (int i = 0; i < 32; ++i) {
+        const int t = 32 * gi + i;
+        if (t < tpt) {
+            const long long Z = limb_combine((int)d[3 * i], (int)d[3 * i + 1], (int)d[3 * i + 2],
+                                             tok_xsum[t]);
+            const float z = __fmul_rn(tok_scale[t], (float)Z);
+            stage[t * BW + r] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hn)));
         }
     }
 }
@@ -208,9 +229,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bt = p.bt;
-    const int ttiles = (p.rows_a + bt - 1) / bt;
-    const int t0 = (blockIdx.x % ttiles) * bt;   // first activation row of the tile
-    const int n0 = (blockIdx.x / ttiles) * BW;   // first weight row of the tile
+    const int ttiles = (p.M + p.tpt - 1) / p.tpt;
+    const int a0 = (blockIdx.x % ttiles) * p.rpt;  // first activation row of the tile
+    const int t0 = (blockIdx.x % ttiles) * p.tpt;  // first token of the tile
+    const int n0 = (blockIdx.x / ttiles) * BW;     // first weight row of the tile
     const int nblk = p.K / BK;                 // 128-k blocks
     const int nk = (nblk + KB - 1) / KB;       // stages; the last may hold fewer blocks
     // blocks in stage kb; the weight box of a short last stage runs past the row
@@ -260,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kb = 0; kb < nk && ok; ++kb) {
                 const int s = kb % SS;
                 if (kb >= SS) {
-                    ok = tc::mbar_wait(bar_empty + 8 * s, ((kb / SS) - 1) & 1, p.flags, kWaitLimitNs);
+                    ok = tc::mbar_wait(bar_empty + 8 * s, ((kb / SS) - 1) & 1, p.flags, p.wait_ns);
                     if (!ok) break;
                     tc::mbar_arrive_expect_tx(bar_wfull + 8 * s, (uint32_t)(kRowBytes * BW));
                     tc::tma_load_2d(sbase + OFF_BP + s * BP_STAGE, &tmap_w, kb * kRowBytes, n0,
@@ -268,19 +290,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++wissued;
                 }
                 const int nb = blocks(kb);
+                ++issued;
+                if (p.stall && blockIdx.x == 0 && kb == 0) continue;   // test hook
                 tc::mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)(nb * bt * BK));
                 for (int b = 0; b < nb; ++b)
                     tc::tma_load_2d(sbase + OFF_ACT + s * ACT_STAGE + b * bt * BK, &tmap_act,
-                                    (kb * KB + b) * BK, t0, bar_full + 8 * s);
-                ++issued;
+                                    (kb * KB + b) * BK, a0, bar_full + 8 * s);
             }
-            if (!ok) {
-                // drain copies still in flight before the CTA's shared memory goes away
-                for (int kb = (issued > SS ? issued - SS : 0); kb < issued; ++kb)
+            // Every copy requested here lands before the CTA can exit: on the
+            // normal path the MMA has consumed them (these waits return at
+            // once); after a timeout some may still be in flight.
+            for (int kb = (issued > SS ? issued - SS : 0); kb < issued; ++kb)
+                if (!(p.stall && blockIdx.x == 0 && kb == 0))   // never requested
                     tc::mbar_wait(bar_full + 8 * (kb % SS), (kb / SS) & 1, p.flags, kWaitLimitNs);
-                for (int kb = (wissued > SS ? wissued - SS : 0); kb < wissued; ++kb)
-                    tc::mbar_wait(bar_wfull + 8 * (kb % SS), (kb / SS) & 1, p.flags, kWaitLimitNs);
-            }
+            for (int kb = (wissued > SS ? wissued - SS : 0); kb < wissued; ++kb)
+                tc::mbar_wait(bar_wfull + 8 * (kb % SS), (kb / SS) & 1, p.flags, kWaitLimitNs);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -288,8 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int kb = 0; kb < nk && ok; ++kb) {
                 const int s = kb % SS, u = kb % SU;
-                ok = tc::mbar_wait(bar_full + 8 * s, (kb / SS) & 1, p.flags, kWaitLimitNs) &&
-                     tc::mbar_wait(bar_ufull + 8 * u, (kb / SU) & 1, p.flags, kWaitLimitNs);
+                ok = tc::mbar_wait(bar_full + 8 * s, (kb / SS) & 1, p.flags, p.wait_ns) &&
+                     tc::mbar_wait(bar_ufull + 8 * u, (kb / SU) & 1, p.flags, p.wait_ns);
                 if (!ok) break;
                 tc::tc_fence_after();
                 const uint32_t act_s = sbase + OFF_ACT + s * ACT_STAGE;
@@ -319,9 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int kb = 0; hsel == 0 && kb < nk && ok; ++kb) {
             const int s = kb % SS, u = kb % SU;
-            ok = tc::mbar_wait(bar_wfull + 8 * s, (kb / SS) & 1, p.flags, kWaitLimitNs);
+            ok = tc::mbar_wait(bar_wfull + 8 * s, (kb / SS) & 1, p.flags, p.wait_ns);
             if (ok && kb >= SU)
-                ok = tc::mbar_wait(bar_uempty + 8 * u, ((kb / SU) - 1) & 1, p.flags, kWaitLimitNs);
+                ok = tc::mbar_wait(bar_uempty + 8 * u, ((kb / SU) - 1) & 1, p.flags, p.wait_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
 #pragma unroll
@@ -341,8 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int* tok_rsum = reinterpret_cast<int*>(tok_scale + BT);
         const int et = threadIdx.x - 64;        // 0..kEpiThreads-1
         tc::pdl_wait();                          // scale / row sums come from the previous kernel
-        fill_token_table<FORM>(p, t0, bt, et, tok_scale, tok_rsum);
-        const bool acc_ok = tc::mbar_wait(bar_acc, 0, p.flags, kWaitLimitNs);
+        fill_token_table<FORM>(p, t0, et, tok_scale, tok_rsum);
+        const bool acc_ok = tc::mbar_wait(bar_acc, 0, p.flags, p.wait_ns);
         // one decision for the eight epilogue warps; also publishes the token table
         const bool good = tc::bar_and(1, kEpiThreads, ok && acc_ok);
         tc::tc_fence_after();
@@ -353,26 +377,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint16_t* stage = reinterpret_cast<uint16_t*>(smem + OFF_ACT);
             const int n = n0 + r;                // output column held by this thread
             const float hn = (FORM == 1 && n < p.N) ? __half2float(__ushort_as_half(p.h[n])) : 0.f;
-            // chunks cc = hsel, hsel+2, ...; the TMEM load of the next chunk is
-            // in flight while this one is converted
             const int nch = bt / 32;
-            uint32_t da[32], db[32];
-            if (hsel < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * hsel, da);
-            tc::tmem_ld_wait();
+            if constexpr (FORM == 0) {
+                // chunks cc = hsel, hsel+2, ...; the TMEM load of the next chunk is
+                // in flight while this one is converted
+                uint32_t da[32], db[32];
+                if (hsel < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * hsel, da);
+                tc::tmem_ld_wait();
 #pragma unroll 1
-            for (int cc = hsel; cc < nch; cc += 4) {
-                if (cc + 2 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 2), db);
-                convert_chunk<FORM>(da, cc, stage, tok_scale, tok_rsum, p, r, n, t0, hn);
-                tc::tmem_ld_wait();
-                if (cc + 2 >= nch) break;
-                if (cc + 4 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 4), da);
-                convert_chunk<FORM>(db, cc + 2, stage, tok_scale, tok_rsum, p, r, n, t0, hn);
-                tc::tmem_ld_wait();
+                for (int cc = hsel; cc < nch; cc += 4) {
+                    if (cc + 2 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 2), db);
+                    convert_chunk(da, cc, stage, tok_scale, tok_rsum, p, r, n, t0);
+                    tc::tmem_ld_wait();
+                    if (cc + 2 >= nch) break;
+                    if (cc + 4 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 4), da);
+                    convert_chunk(db, cc + 2, stage, tok_scale, tok_rsum, p, r, n, t0);
+                    tc::tmem_ld_wait();
+                }
+            } else {
+                // token groups gi = hsel, hsel+2, ...: 32 tokens = 96 columns = 3 chunks
+                const long long* tok_xsum = reinterpret_cast<const long long*>(tok_rsum);
+#pragma unroll 1
+                for (int gi = hsel; gi < (p.tpt + 31) / 32; gi += 2) {
+                    uint32_t d[96];
+#pragma unroll
+                    for (int c = 0; c < 3; ++c)
+                        if (3 * gi + c < nch)
+                            tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (3 * gi + c),
+                                                   *reinterpret_cast<uint32_t(*)[32]>(d + 32 * c));
+                    tc::tmem_ld_wait();
+                    convert_onebit_group(d, gi, stage, tok_scale, tok_xsum, p.tpt, r, hn);
+                }
             }
             tc::fence_proxy_async_smem();
             asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
             if (et == 0) {
-                tc::tma_store_2d(&tmap_y, sbase + OFF_ACT, n0 * 2, FORM == 0 ? t0 : t0 >> 1);
+                tc::tma_store_2d(&tmap_y, sbase + OFF_ACT, n0 * 2, t0);
                 tc::bulk_commit_group();
                 tc::bulk_wait_group_read0();
             }
@@ -420,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bt = p.bt;
-    const int ttiles = (p.rows_a + bt - 1) / bt;
+    const int ttiles = (p.M + p.tpt - 1) / p.tpt;
     const int nblk = p.K / BK;                 // 128-k blocks
     const int nk = (nblk + KB - 1) / KB;       // stages; the last may hold fewer blocks
     // blocks in stage kb; the weight box of a short last stage runs past the row
@@ -497,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (long long u = ua; u < ub && ok; ++item) {
                 piece(u, tile, kb0, kb1);
                 u += kb1 - kb0;
-                const int t0 = (tile % ttiles) * bt, n0 = (tile / ttiles) * BW;
+                const int a0 = (tile % ttiles) * p.rpt, n0 = (tile / ttiles) * BW;
                 // the previous piece's epilogue stages its output in the ring
                 if (item > 0) ok = tc::mbar_wait(bar_stfree, (item - 1) & 1, p.flags, kWaitLimitNs);
                 for (int kb = kb0; kb < kb1 && ok; ++kb) {
@@ -516,17 +556,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)(nb * bt * BK));
                     for (int b = 0; b < nb; ++b)
                         tc::tma_load_2d(sbase + OFF_ACT + s * ACT_STAGE + b * bt * BK, &tmap_act,
-                                        (kb * KB + b) * BK, t0, bar_full + 8 * s);
+                                        (kb * KB + b) * BK, a0, bar_full + 8 * s);
                     ++ag;
                 }
             }
-            if (!ok) {
-                // drain copies still in flight before the CTA's shared memory goes away
-                for (int g = (ag > SS ? ag - SS : 0); g < ag; ++g)
-                    tc::mbar_wait(bar_full + 8 * (g % SS), (g / SS) & 1, p.flags, kWaitLimitNs);
-                for (int g = (wg > SS ? wg - SS : 0); g < wg; ++g)
-                    tc::mbar_wait(bar_wfull + 8 * (g % SS), (g / SS) & 1, p.flags, kWaitLimitNs);
-            }
+            // Every copy requested here lands before the CTA can exit (see
+            // prefill_kernel).
+            for (int g = (ag > SS ? ag - SS : 0); g < ag; ++g)
+                tc::mbar_wait(bar_full + 8 * (g % SS), (g / SS) & 1, p.flags, kWaitLimitNs);
+            for (int g = (wg > SS ? wg - SS : 0); g < wg; ++g)
+                tc::mbar_wait(bar_wfull + 8 * (g % SS), (g / SS) & 1, p.flags, kWaitLimitNs);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -588,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int tile, kb0, kb1;
             piece(u, tile, kb0, kb1);
             u += kb1 - kb0;
-            const int t0 = (tile % ttiles) * bt, n0 = (tile / ttiles) * BW;
+            const int t0 = (tile % ttiles) * p.tpt, n0 = (tile / ttiles) * BW;
 
             // ------- expand (warps 2-5): one thread per weight row -------
             for (int kb = kb0; hsel == 0 && kb < kb1 && ok; ++kb, ++g) {
@@ -612,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---------------- epilogue (warps 2-9) ----------------------------
             if (item == 0) tc::pdl_wait();       // scale / row sums come from the previous kernel
             // per-token scale and row sum of this activation tile
-            fill_token_table<FORM>(p, t0, bt, et, tok_scale, tok_rsum);
+            fill_token_table<FORM>(p, t0, et, tok_scale, tok_rsum);
             const bool acc_ok = tc::mbar_wait(bar_acc, item & 1, p.flags, kWaitLimitNs);
             // one decision for the eight epilogue warps; also publishes the token table
             const bool good = tc::bar_and(1, kEpiThreads, ok && acc_ok);
@@ -718,34 +757,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             };
-            // chunks cc = hsel, hsel+2, ...; the TMEM load of the next chunk is
-            // in flight while this one is finished
             const int nch = bt / 32;
-            uint32_t da[32], db[32];
-            if (hsel < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * hsel, da);
-            tc::tmem_ld_wait();
+            if constexpr (FORM == 0) {
+                // chunks cc = hsel, hsel+2, ...; the TMEM load of the next chunk is
+                // in flight while this one is finished
+                uint32_t da[32], db[32];
+                if (hsel < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * hsel, da);
+                tc::tmem_ld_wait();
 #pragma unroll 1
-            for (int cc = hsel; cc < nch; cc += 4) {
-                // 256-row tiles: the staging of chunks 4-7 reuses the space of
-                // the partial's chunks 0-1, read in the first round
-                if (cc >= 4 && nch == 8 && !whole && c_last - c_first == 1)
-                    asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
-                if (cc + 2 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 2), db);
-                add_parts(da, cc);
-                convert_chunk<FORM>(da, cc, stage, tok_scale, tok_rsum, p, r, n, t0, hn);
-                tc::tmem_ld_wait();
-                if (cc + 2 >= nch) break;
-                if (cc + 4 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 4), da);
-                add_parts(db, cc + 2);
-                convert_chunk<FORM>(db, cc + 2, stage, tok_scale, tok_rsum, p, r, n, t0, hn);
-                tc::tmem_ld_wait();
+                for (int cc = hsel; cc < nch; cc += 4) {
+                    // 256-row tiles: the staging of chunks 4-7 reuses the space of
+                    // the partial's chunks 0-1, read in the first round
+                    if (cc >= 4 && nch == 8 && !whole && c_last - c_first == 1)
+                        asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+                    if (cc + 2 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 2), db);
+                    add_parts(da, cc);
+                    convert_chunk(da, cc, stage, tok_scale, tok_rsum, p, r, n, t0);
+                    tc::tmem_ld_wait();
+                    if (cc + 2 >= nch) break;
+                    if (cc + 4 < nch) tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (cc + 4), da);
+                    add_parts(db, cc + 2);
+                    convert_chunk(db, cc + 2, stage, tok_scale, tok_rsum, p, r, n, t0);
+                    tc::tmem_ld_wait();
+                }
+            } else {
+                // token groups gi = hsel, hsel+2, ...: 32 tokens = 96 columns = 3
+                // chunks (the fp16 staging of at most 85 tokens stays below the
+                // partial slot's copy at kPartOff)
+                const long long* tok_xsum = reinterpret_cast<const long long*>(tok_rsum);
+#pragma unroll 1
+                for (int gi = hsel; gi < (p.tpt + 31) / 32; gi += 2) {
+                    uint32_t d[96];
+#pragma unroll
+                    for (int c = 0; c < 3; ++c)
+                        if (3 * gi + c < nch)
+                            tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (3 * gi + c),
+                                                   *reinterpret_cast<uint32_t(*)[32]>(d + 32 * c));
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 3; ++c)
+                        if (3 * gi + c < nch)
+                            add_parts(*reinterpret_cast<uint32_t(*)[32]>(d + 32 * c), 3 * gi + c);
+                    convert_onebit_group(d, gi, stage, tok_scale, tok_xsum, p.tpt, r, hn);
+                }
             }
             tc::tc_fence_before();
             tc::mbar_arrive(bar_accfree);
             tc::fence_proxy_async_smem();
             asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
             if (et == 0) {
-                tc::tma_store_2d(&tmap_y, sbase + OFF_ACT, n0 * 2, FORM == 0 ? t0 : t0 >> 1);
+                tc::tma_store_2d(&tmap_y, sbase + OFF_ACT, n0 * 2, t0);
                 tc::bulk_commit_group();
                 tc::bulk_wait_group_read0();
                 tc::mbar_arrive(bar_stfree);
@@ -771,25 +832,33 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
     return encode_u8_map(m, base, 2, dims, strides, box, swz);
 }
 
-// Activation rows per tile: the smallest multiple of 32 that covers them, at most
-// BT (a tile never computes more than 31 padding columns when rows_a <= BT).
-inline int choose_bt(int rows_a) {
-    const int r = (rows_a + 31) / 32 * 32;
+// Activation rows per tile: the smallest multiple of 32 that covers them, at most BT.
+inline int choose_bt(int rows) {
+    const int r = (rows + 31) / 32 * 32;
     return r < BT ? r : BT;
 }
 
-// Tile geometry of a call: activation rows per tile, k-blocks per stage,
-// stages per tile and the number of (weight-row, activation-row) tiles.
+// Tile geometry of a call: activation rows per tile, tokens per tile, k-blocks
+// per stage, stages per tile and the number of (weight-row, token) tiles.
+// The tokens are cut into the fewest tiles of at most BT activation rows (BT
+// tokens, or BT/3 OneBit tokens of three limb rows), of balanced size: 300
+// ternary tokens run as two 160-row tiles rather than 256 + 44.  A OneBit tile
+// loads bt >= 3 tpt rows; the rows past its tokens are computed but unused.
 struct Geometry {
-    int bt, kb, nk, tiles;
+    int bt, tpt, kb, nk, tiles;
 };
 
-Geometry geometry(int rows_a, int K, int N) {
+Geometry geometry(int form, int M, int K, int N) {
     Geometry g;
-    g.bt = choose_bt(rows_a);
+    const int cpt = form == 0 ? 1 : 3;           // activation rows per token
+    const int max_tpt = BT / cpt;
+    const int ttiles = (M + max_tpt - 1) / max_tpt;
+    const int tpt = (M + ttiles - 1) / ttiles;
+    g.bt = choose_bt(cpt * tpt);
+    g.tpt = form == 0 ? g.bt : tpt;
     g.kb = g.bt <= BT / 4 ? 4 : g.bt <= BT / 2 ? 2 : 1;
     g.nk = (K / BK + g.kb - 1) / g.kb;
-    g.tiles = ((N + BW - 1) / BW) * ((rows_a + g.bt - 1) / g.bt);
+    g.tiles = ((N + BW - 1) / BW) * ((M + g.tpt - 1) / g.tpt);
     return g;
 }
 
@@ -839,15 +908,8 @@ cudaError_t launch_prefill_kb(const int8_t* act, const uint32_t* w, PrefillParam
                               cudaStream_t s) {
     constexpr int smem = PS<KB>::SMEM_BYTES;
     constexpr auto kern = SPLIT ? prefill_split_kernel<FORM, KB> : prefill_kernel<FORM, KB>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        e = use_max_shared_carveout(kern);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static KernelAttrs kattrs;
+    if (cudaError_t e = kattrs.ensure(kern, smem)) return e;
     CUtensorMap ta, tw;
     if (!make_tmap(&ta, act, (uint64_t)p.rows_a, (uint64_t)p.K, BK, (uint32_t)p.bt,
                    CU_TENSOR_MAP_SWIZZLE_128B))
@@ -858,9 +920,18 @@ cudaError_t launch_prefill_kb(const int8_t* act, const uint32_t* w, PrefillParam
         return cudaErrorInvalidValue;
     // y as bytes: N * 2 per row; one box = 128 columns x the tile's tokens
     CUtensorMap ty;
-    if (!make_tmap(&ty, p.y, (uint64_t)p.M, (uint64_t)p.N * 2, BW * 2,
-                   (uint32_t)(FORM == 0 ? p.bt : p.bt / 2), CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!make_tmap(&ty, p.y, (uint64_t)p.M, (uint64_t)p.N * 2, BW * 2, (uint32_t)p.tpt,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
+    p.wait_ns = kWaitLimitNs;
+    p.stall = 0;
+    if (!SPLIT) {
+        const unsigned long long stall = take_stall();
+        if (stall) {
+            p.wait_ns = stall;
+            p.stall = 1;
+        }
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.dp_tiles + p.sk_ctas);
     cfg.blockDim = dim3(kThreads);
@@ -877,8 +948,10 @@ cudaError_t launch_prefill_kb(const int8_t* act, const uint32_t* w, PrefillParam
 template <int FORM>
 cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, PrefillParams p, void* split_ws,
                            size_t split_ws_bytes, cudaStream_t s) {
-    const Geometry g = geometry(p.rows_a, p.K, p.N);
+    const Geometry g = geometry(FORM, p.M, p.K, p.N);
     p.bt = g.bt;
+    p.tpt = g.tpt;
+    p.rpt = FORM == 0 ? g.bt : 3 * g.tpt;   // a token tile's first activation row
     SplitPlan pl = plan_split(g, device_sm_count());
     const size_t need = split_bytes(g, pl);
     if (need == 0 || split_ws == nullptr || split_ws_bytes < need) pl = SplitPlan{g.tiles, 0, 0};
@@ -902,7 +975,7 @@ cudaError_t launch_prefill(const int8_t* act, const uint32_t* w, PrefillParams p
 }  // namespace
 
 void prefill_plan_info(int form, int M, int K, int N, int sm_count, int plan[5]) {
-    const Geometry g = geometry(form == 0 ? M : 2 * M, K, N);
+    const Geometry g = geometry(form, M, K, N);
     const SplitPlan pl = plan_split(g, sm_count);
     plan[0] = g.bt;
     plan[1] = g.nk;
@@ -914,7 +987,7 @@ void prefill_plan_info(int form, int M, int K, int N, int sm_count, int plan[5])
 size_t prefill_split_bytes(int form, int M, int K, int N, int* n_counters) {
     *n_counters = 0;
     if (M <= 0 || N <= 0) return 0;
-    const Geometry g = geometry(form == 0 ? M : 2 * M, K, N);
+    const Geometry g = geometry(form, M, K, N);
     const SplitPlan pl = plan_split(g, device_sm_count());
     *n_counters = pl.sk_tiles;
     return split_bytes(g, pl);
@@ -925,18 +998,18 @@ cudaError_t launch_ternary_prefill(const uint32_t* w2, const int8_t* qp, const f
                                    uint16_t* y, int32_t* acc_out, unsigned int* flags,
                                    cudaStream_t s, void* split_ws, size_t split_ws_bytes) {
     if (M == 0 || N == 0) return cudaSuccess;
-    PrefillParams p{M, 0, M, K, N, scale, qsum, nullptr, w_scale, y, acc_out, flags,
-                    0, 0, 0, nullptr, nullptr};
+    PrefillParams p{M, 0, 0, 0, M, K, N, scale, qsum, nullptr, nullptr, w_scale, y, acc_out,
+                    flags, 0, 0, 0, nullptr, nullptr, 0, 0};
     return launch_prefill<0>(qp, w2, p, split_ws, split_ws_bytes, s);
 }
 
 cudaError_t launch_onebit_prefill(const uint32_t* s1, const int8_t* planes, const float* step,
-                                  const int32_t* tsum, const uint16_t* h, int M, int K, int N,
+                                  const long long* tsum, const uint16_t* h, int M, int K, int N,
                                   uint16_t* y, unsigned int* flags, cudaStream_t s,
                                   void* split_ws, size_t split_ws_bytes) {
     if (M == 0 || N == 0) return cudaSuccess;
-    PrefillParams p{2 * M, 0, M, K, N, step, tsum, h, 0.f, y, nullptr, flags,
-                    0, 0, 0, nullptr, nullptr};
+    PrefillParams p{3 * M, 0, 0, 0, M, K, N, step, nullptr, tsum, h, 0.f, y, nullptr, flags,
+                    0, 0, 0, nullptr, nullptr, 0, 0};
     return launch_prefill<1>(planes, s1, p, split_ws, split_ws_bytes, s);
 }
 

@@ -9,9 +9,10 @@
 // OneBit: OneBit page ("清华、哈工大把大模型压缩到了1bit…"), "1. 新的 1bit 结构":
 // the input-side value vector g multiplies x before the sign contraction.  The
 // product x*g (exact in fp32: two 11-bit significands) is turned into a
-// per-token 16-bit fixed-point image X = rne(x*g * 32639 / amax'), split into
-// two signed bytes X = 256*hi + lo (hi = floor((X+128)/256), lo in [-128,127]),
-// so that the contraction with the 0/1 sign bits runs exactly in int8 MMA.
+// per-token 23-bit fixed-point image X = rne(x*g * (2^22-1) / amax'), split
+// into three signed bytes X = 65536 hi + 256 mid + lo (balanced base-256
+// digits), so that the contraction with the 0/1 sign bits runs exactly in int8
+// MMA, one limb at a time.
 //
 // One CTA per token, two passes over the token (the second hits L1/L2).
 // HBM-bound: the plain/ternary kernels read 2 B and write 1 B per element.
@@ -239,16 +240,57 @@ __global__ void __launch_bounds__(kRegThreads, NCH <= 4 ? 2 : 1)
     if (threadIdx.x == 0) scale[m] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
 }
 
-constexpr int kFixMax = 32639;  // |X| <= 32639 keeps hi = floor((X+128)/256) in int8
+// Store one 32-element group's three limb bytes, permuted: byte 4j+b of the
+// 32-byte group holds element 8b+j, the order the 1-bit unpack
+// (w >> j) & 0x01010101 produces.  Plane stride K bytes: [hi][mid][lo].
+// Returns the group's sum of X.
+__device__ __forceinline__ int store_limbs_group(const int (&X)[32], int8_t* hi_dst, int K) {
+    uint32_t hw[8], mw[8], lw[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) hw[j] = mw[j] = lw[j] = 0u;
+    int sum = 0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        int hi, mid, lo;
+        split_limbs(X[e], hi, mid, lo);
+        hw[e & 7] |= ((uint32_t)hi & 0xffu) << (8 * (e >> 3));
+        mw[e & 7] |= ((uint32_t)mid & 0xffu) << (8 * (e >> 3));
+        lw[e & 7] |= ((uint32_t)lo & 0xffu) << (8 * (e >> 3));
+        sum += X[e];
+    }
+    uint4* hd = reinterpret_cast<uint4*>(hi_dst);
+    uint4* md = reinterpret_cast<uint4*>(hi_dst + K);
+    uint4* ld = reinterpret_cast<uint4*>(hi_dst + 2 * (size_t)K);
+    hd[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    hd[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+    md[0] = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+    md[1] = make_uint4(mw[4], mw[5], mw[6], mw[7]);
+    ld[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    ld[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+    return sum;
+}
 
+template <int NW>
+__device__ __forceinline__ long long block_sum_i64_n(long long v, long long* red) {
+    v = warp_sum64(v);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    return warp_sum64(lane < NW ? red[lane] : 0ll);
+}
+
+// OneBit preparation, general K (two passes over the token): the image of
+// x*g in three int8 limb planes [M][3][K], the fixed-point step amax'/kImgMax
+// and the token's image sum (int64; per thread at most 256 elements of
+// |X| <= 2^22, so the per-thread int32 sums cannot overflow).
 __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* __restrict__ x,
                                                                const uint16_t* __restrict__ g,
                                                                int K, int8_t* __restrict__ planes,
                                                                float* __restrict__ step,
-                                                               int32_t* __restrict__ tsum,
+                                                               long long* __restrict__ tsum,
                                                                unsigned int* zero, int n_zero) {
     __shared__ uint32_t redu[kWarps];
-    __shared__ int redi[kWarps];
+    __shared__ long long redl[kWarps];
     const int m = blockIdx.x;
     const uint16_t* row = x + (size_t)m * K;
     tc::pdl_trigger();
@@ -268,13 +310,12 @@ __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* _
         }
     }
     const float amax = __uint_as_float(block_max_u32(__float_as_uint(mx), redu));
-    const float inv = amax > 0.f ? __fdiv_rn((float)kFixMax, amax) : 0.f;
+    const float inv = amax > 0.f ? __fdiv_rn(kImgMaxF, amax) : 0.f;
 
     int sum = 0;
-    int8_t* hi_row = planes + (size_t)m * 2 * K;
-    int8_t* lo_row = hi_row + K;
+    int8_t* hi_row = planes + (size_t)m * 3 * K;
     for (int c = threadIdx.x; c < K / 32; c += kThreads) {
-        int hv[32], lv[32];
+        int X[32];
 #pragma unroll
         for (int part = 0; part < 4; ++part) {
             uint4 v = tc::ld_v4(row + 32 * c + 8 * part);
@@ -284,53 +325,30 @@ __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* _
             for (int e = 0; e < 8; ++e) {
                 float p = __fmul_rn(half_bits_to_float(xs[e >> 1] >> (16 * (e & 1))),
                                     half_bits_to_float(gs[e >> 1] >> (16 * (e & 1))));
-                const int X = rne_bits(__fmul_rn(p, inv)) - kRneBias;   // |X| <= 32639
-                int hi = (X + 128) >> 8;  // arithmetic shift = floor
-                hv[8 * part + e] = hi;
-                lv[8 * part + e] = X - 256 * hi;
-                sum += X;
+                X[8 * part + e] = rne_bits(__fmul_rn(p, inv)) - kRneBias;   // |X| <= kImgMax
             }
         }
-        // byte 4j+b of the 32-byte group holds element 8b+j, the order the
-        // 1-bit unpack (w >> j) & 0x01010101 produces
-        uint32_t ho[8], lo[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            uint32_t a = 0, b = 0;
-#pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                a |= ((uint32_t)hv[8 * bb + j] & 0xffu) << (8 * bb);
-                b |= ((uint32_t)lv[8 * bb + j] & 0xffu) << (8 * bb);
-            }
-            ho[j] = a;
-            lo[j] = b;
-        }
-        uint4* hd = reinterpret_cast<uint4*>(hi_row + 32 * c);
-        uint4* ld = reinterpret_cast<uint4*>(lo_row + 32 * c);
-        hd[0] = make_uint4(ho[0], ho[1], ho[2], ho[3]);
-        hd[1] = make_uint4(ho[4], ho[5], ho[6], ho[7]);
-        ld[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        ld[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+        sum += store_limbs_group(X, hi_row + 32 * c, K);
     }
-    int tot = block_sum_i32(sum, redi);
+    const long long tot = block_sum_i64_n<kWarps>((long long)sum, redl);
     if (threadIdx.x == 0) {
         tsum[m] = tot;
-        step[m] = amax > 0.f ? __fdiv_rn(amax, (float)kFixMax) : 0.f;
+        step[m] = amax > 0.f ? __fdiv_rn(amax, kImgMaxF) : 0.f;
     }
 }
 
 // Register-resident OneBit preparation: a 512-thread CTA per token keeps the
 // fp32 products x*g of up to NCH 32-element groups per thread in registers,
-// takes amax, then forms the fixed-point limbs from registers (x and g read
-// once).  Same arithmetic and output order as prep_onebit_kernel.
+// takes amax, then forms the limbs from registers (x and g read once).  Same
+// arithmetic and output as prep_onebit_kernel.
 template <int NCH>
 __global__ void __launch_bounds__(kRegThreads, 1)
     prep_onebit_reg_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g, int K,
                            int8_t* __restrict__ planes, float* __restrict__ step,
-                           int32_t* __restrict__ tsum, unsigned int* zero, int n_zero) {
+                           long long* __restrict__ tsum, unsigned int* zero, int n_zero) {
     constexpr int NW = kRegThreads / 32;
     __shared__ uint32_t redu[NW];
-    __shared__ int redi[NW];
+    __shared__ long long redl[NW];
     const int m = blockIdx.x;
     const int ng = K / 32;
     const uint16_t* row = x + (size_t)m * K;
@@ -362,50 +380,30 @@ __global__ void __launch_bounds__(kRegThreads, 1)
         }
     }
     const float amax = __uint_as_float(block_max_u32_n<NW>(__float_as_uint(mx), redu));
-    const float inv = amax > 0.f ? __fdiv_rn((float)kFixMax, amax) : 0.f;
+    const float inv = amax > 0.f ? __fdiv_rn(kImgMaxF, amax) : 0.f;
 
     int sum = 0;
-    int8_t* hi_row = planes + (size_t)m * 2 * K;
-    int8_t* lo_row = hi_row + K;
+    int8_t* hi_row = planes + (size_t)m * 3 * K;
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
         const int c = threadIdx.x + i * kRegThreads;
         if (c >= ng) break;
-        // byte 4j+b of the 32-byte group holds element 8b+j, the order the
-        // 1-bit unpack (w >> j) & 0x01010101 produces
-        uint32_t ho[8], lo[8];
+        int X[32];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) ho[j] = lo[j] = 0u;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const int X = rne_bits(__fmul_rn(pr[i][e], inv)) - kRneBias;   // |X| <= 32639
-            const int hi = (X + 128) >> 8;  // arithmetic shift = floor
-            ho[e & 7] |= ((uint32_t)hi & 0xffu) << (8 * (e >> 3));
-            lo[e & 7] |= ((uint32_t)(X - 256 * hi) & 0xffu) << (8 * (e >> 3));
-            sum += X;
-        }
-        uint4* hd = reinterpret_cast<uint4*>(hi_row + 32 * c);
-        uint4* ld = reinterpret_cast<uint4*>(lo_row + 32 * c);
-        hd[0] = make_uint4(ho[0], ho[1], ho[2], ho[3]);
-        hd[1] = make_uint4(ho[4], ho[5], ho[6], ho[7]);
-        ld[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        ld[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+        for (int e = 0; e < 32; ++e) X[e] = rne_bits(__fmul_rn(pr[i][e], inv)) - kRneBias;
+        sum += store_limbs_group(X, hi_row + 32 * c, K);
     }
-    const int tot = block_sum_i32_n<NW>(sum, redi);
+    const long long tot = block_sum_i64_n<NW>((long long)sum, redl);
     if (threadIdx.x == 0) {
         tsum[m] = tot;
-        step[m] = amax > 0.f ? __fdiv_rn(amax, (float)kFixMax) : 0.f;
+        step[m] = amax > 0.f ? __fdiv_rn(amax, kImgMaxF) : 0.f;
     }
 }
 
 template <auto KERN, int THREADS = kThreads, typename... Args>
 cudaError_t launch_pdl(int blocks, cudaStream_t s, Args... args) {
-    static bool attr_set = false;  // one flag per kernel
-    if (!attr_set) {
-        cudaError_t e = use_max_shared_carveout(KERN);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static KernelAttrs kattrs;  // one per kernel
+    if (cudaError_t e = kattrs.ensure(KERN, 0)) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(blocks);
     cfg.blockDim = dim3(THREADS);
@@ -454,7 +452,7 @@ cudaError_t launch_quant_ternary_perm(const uint16_t* x, int M, int K, int8_t* q
 }
 
 cudaError_t launch_prep_onebit(const uint16_t* x, const uint16_t* g, int M, int K,
-                               int8_t* planes, float* step, int32_t* tsum, cudaStream_t s,
+                               int8_t* planes, float* step, long long* tsum, cudaStream_t s,
                                unsigned int* zero, int n_zero) {
     if (M == 0) return cudaSuccess;
     const int groups = K / 32;

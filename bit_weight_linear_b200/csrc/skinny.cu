@@ -10,8 +10,9 @@
 // OneBit (OneBit page, "1. 新的 1bit 结构" and "讨论与分析 / 1. 效率": matrix
 // products become bit assignment and addition): with b = (S+1)/2 in {0,1},
 //     sum_k X*S = 2 sum_k X*b - sum_k X,
-// where X is the 16-bit fixed-point image of x*g split into two int8 limbs,
-// and the bits are unpacked as (w >> j) & 0x01010101.
+// where X is the 23-bit fixed-point image of x*g split into three int8 limbs
+// (each limb contracted exactly in int32), and the bits are unpacked as
+// (w >> j) & 0x01010101.
 //
 // Because integer sums are exact in any order, the k order inside the MMA is
 // free: the activation preparation kernels store each 16-byte (ternary) or
@@ -22,7 +23,7 @@
 // its 8 warps split K in steps (256 k ternary, 512 k sign, 16 words per row
 // per step, one 16-byte load per lane per row), then reduce through shared
 // memory.  The kernel is HBM-bound on the packed weights for M up to 8
-// (ternary) / 4 (OneBit) tokens per MMA column tile.
+// (ternary) / 2 (OneBit) tokens per MMA column tile.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -55,14 +56,15 @@ struct Form<1> {                         // sign, 1 bit
     static constexpr uint32_t kMask = 0x01010101u;
     static constexpr int kStepK = 512;
     static constexpr int kChunkK = 128;
-    static constexpr int kColsPerToken = 2;  // hi and lo limb of the fixed-point image
+    static constexpr int kColsPerToken = 3;  // hi, mid and lo limb of the fixed-point image
 };
 
 struct SkinnyParams {
     const uint32_t* w;      // packed weights [N][K / kPerWord]
     const int8_t* act;      // prepared activations [M][kColsPerToken][K] (permuted)
     const float* scale;     // ternary: token scale; onebit: fixed-point step
-    const int32_t* rsum;    // ternary: sum_k q; onebit: sum_k X
+    const int32_t* rsum;    // ternary: sum_k q
+    const long long* xsum;  // onebit: sum_k X
     const uint16_t* h;      // onebit output value vector [N]
     float w_scale;          // ternary per-tensor weight scale
     int M, K, N;
@@ -93,7 +95,8 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyParams p) 
         const int col = nt * 8 + g;
         const int tok = tok_base + col / F::kColsPerToken;
         const int plane = col % F::kColsPerToken;
-        bvalid[nt] = tok < p.M;
+        // (OneBit: the columns past the last whole token of the tile stay unused)
+        bvalid[nt] = tok < p.M && col < kTokPerCta * F::kColsPerToken;
         bsrc[nt] = p.act + ((size_t)(bvalid[nt] ? tok : 0) * F::kColsPerToken + plane) * K +
                    t * F::kChunkK;
     }
@@ -173,15 +176,16 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyParams p) 
             const int u = o >> 4, r = o & 15;
             const int tok = tok_base + u;
             if (tok >= p.M) continue;
-            const int chi = 2 * u, clo = 2 * u + 1;
-            long long phi = 0, plo = 0;
+            int d[3];
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) {
-                phi += red[w][chi >> 3][r][chi & 7];
-                plo += red[w][clo >> 3][r][clo & 7];
+            for (int l = 0; l < 3; ++l) {
+                const int c = 3 * u + l;
+                int v = 0;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) v += red[w][c >> 3][r][c & 7];
+                d[l] = v;
             }
-            const long long P = 256 * phi + plo;            // sum_k X * b
-            const long long Z = 2 * P - (long long)p.rsum[tok];  // sum_k X * S
+            const long long Z = limb_combine(d[0], d[1], d[2], p.xsum[tok]);  // sum_k X * S
             const int n = blockIdx.x * 16 + r;
             const float z = __fmul_rn(p.scale[tok], (float)Z);
             const float hv = __half2float(__ushort_as_half(p.h[n]));
@@ -194,12 +198,8 @@ template <int FORM, int NT>
 cudaError_t launch(const SkinnyParams& p, cudaStream_t s) {
     constexpr int kTokPerCta = NT * 8 / Form<FORM>::kColsPerToken;
     dim3 grid(p.N / 16, (p.M + kTokPerCta - 1) / kTokPerCta);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = use_max_shared_carveout(skinny_kernel<FORM, NT>);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static KernelAttrs kattrs;
+    if (cudaError_t e = kattrs.ensure(skinny_kernel<FORM, NT>, 0)) return e;
     skinny_kernel<FORM, NT><<<grid, kThreads, 0, s>>>(p);
     return cudaGetLastError();
 }
@@ -210,19 +210,19 @@ cudaError_t launch_ternary_skinny(const uint32_t* w2, const int8_t* qp, const fl
                                   const int32_t* qsum, int M, int K, int N, float w_scale,
                                   uint16_t* y, int32_t* acc_out, cudaStream_t s) {
     if (M == 0 || N == 0) return cudaSuccess;
-    SkinnyParams p{w2, qp, scale, qsum, nullptr, w_scale, M, K, N, y, acc_out};
+    SkinnyParams p{w2, qp, scale, qsum, nullptr, nullptr, w_scale, M, K, N, y, acc_out};
     if (M <= 8) return launch<0, 1>(p, s);
     if (M <= 16) return launch<0, 2>(p, s);
     return launch<0, 4>(p, s);
 }
 
 cudaError_t launch_onebit_skinny(const uint32_t* s1, const int8_t* planes, const float* step,
-                                 const int32_t* tsum, const uint16_t* h, int M, int K, int N,
+                                 const long long* tsum, const uint16_t* h, int M, int K, int N,
                                  uint16_t* y, cudaStream_t s) {
     if (M == 0 || N == 0) return cudaSuccess;
-    SkinnyParams p{s1, planes, step, tsum, h, 0.f, M, K, N, y, nullptr};
-    if (M <= 4) return launch<1, 1>(p, s);
-    if (M <= 8) return launch<1, 2>(p, s);
+    SkinnyParams p{s1, planes, step, nullptr, tsum, h, 0.f, M, K, N, y, nullptr};
+    if (M <= 2) return launch<1, 1>(p, s);
+    if (M <= 5) return launch<1, 2>(p, s);
     return launch<1, 4>(p, s);
 }
 

@@ -5,8 +5,8 @@
 // Arithmetic is that of the other decode kernels:
 //   BitLinear (BitNet b1.58 page, "BitNet b1.58 介绍"): per-token absmax int8
 //     q = rne(x * rn(127/amax)), acc = sum q*code - sum q, y = fp16((acc*s)*w_scale);
-//   OneBit (OneBit page, "1. 新的 1bit 结构"): 16-bit fixed-point image X of
-//     x*g in two int8 limbs, sum X*S = 2 sum X*b - sum X, y = fp16(step*Z*h).
+//   OneBit (OneBit page, "1. 新的 1bit 结构"): 23-bit fixed-point image X of
+//     x*g in three int8 limbs, sum X*S = 2 sum X*b - sum X, y = fp16(step*Z*h).
 //
 // Why this shape on B200.  At M = 1 a call is a chain: wait for the previous
 // grid, read x, reduce its absmax, quantise, contract, write y.  The weights
@@ -50,7 +50,8 @@ constexpr int kStreamSmemPair = 112 * 1024;
 struct StreamParams {
     const int8_t* prep;     // prepared activations [cols][K] (PREP kernels only)
     const float* pscale;    // per token: scale (ternary) / fixed-point step (OneBit)
-    const int32_t* prsum;   // per token: row sum of the prepared activations
+    const int32_t* prsum;   // ternary, per token: row sum of the prepared activations
+    const long long* prsum64;  // OneBit, per token: sum of the fixed-point image
     const uint16_t* x;
     const uint16_t* g;      // OneBit input value vector
     const uint16_t* h;      // OneBit output value vector
@@ -69,6 +70,11 @@ struct StreamParams {
     int slot_bytes;
     int compact;             // 1: per-tile reduction through one [16 warps][16][cols] scratch
     int off_act, astride, off_red, off_tok, off_h, off_bar, off_cnt;
+    // Bounded waits: the limit of a ring-stage wait (2 s).  Test hook
+    // (bl_debug_stall_next_launch): stall = 1 leaves CTA 0's first stage
+    // unrequested, so its wait runs out after wait_ns.
+    uint64_t wait_ns;
+    int stall;
 };
 
 // Quantise one 16-element ternary group (fp16 in a, b) into the permuted
@@ -110,15 +116,15 @@ __device__ __forceinline__ float absmax_prod(uint4 a, uint4 gg) {
     return mx;
 }
 
-// OneBit: one 32-element group of x*g -> X = rne(x*g*inv) in two int8 limbs,
-// hi = floor((X+128)/256), lo = X - 256 hi, written permuted into the two
-// limb rows; returns the group's sum of X.  |x*g*inv| <= 32639 (1 + 2^-24),
-// so no clamp is needed.
-__device__ __forceinline__ int quant_group_s(const uint4 (&xa)[4], const uint4 (&ga)[4], float inv,
-                                             uint8_t* dh, uint8_t* dl) {
-    uint32_t ho[8], lo[8];
+// OneBit: one 32-element group of x*g -> X = rne(x*g*inv), split into three
+// int8 limbs written permuted into the limb rows dh, dh + astride, dh + 2
+// astride (byte 4j+b of the group holds element 8b+j); ls receives the
+// group's sum of each limb.  |x*g*inv| < kImgMax + 0.25, so no clamp is needed.
+__device__ __forceinline__ void quant_group_s(const uint4 (&xa)[4], const uint4 (&ga)[4], float inv,
+                                              uint8_t* dh, int astride, int (&ls)[3]) {
+    uint32_t hw[8], mw[8], lw[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) ho[j] = lo[j] = 0;
+    for (int j = 0; j < 8; ++j) hw[j] = mw[j] = lw[j] = 0;
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
         const uint32_t av[4] = {xa[v].x, xa[v].y, xa[v].z, xa[v].w};
@@ -127,26 +133,34 @@ __device__ __forceinline__ int quant_group_s(const uint4 (&xa)[4], const uint4 (
         for (int e = 0; e < 8; ++e) {
             const float pr = __fmul_rn(hbits(av[e >> 1] >> (16 * (e & 1))),
                                        hbits(gv[e >> 1] >> (16 * (e & 1))));
-            const int X = rne_bits(__fmul_rn(pr, inv)) - kRneBias;   // |X| <= 32639
-            const int hi = (X + 128) >> 8;
+            const int X = rne_bits(__fmul_rn(pr, inv)) - kRneBias;   // |X| <= kImgMax
+            int hi, mid, lo;
+            split_limbs(X, hi, mid, lo);
             // element 8v+e goes to byte v of word e
-            ho[e] |= ((uint32_t)hi & 0xffu) << (8 * v);
-            lo[e] |= ((uint32_t)(X - 256 * hi) & 0xffu) << (8 * v);
+            hw[e] |= ((uint32_t)hi & 0xffu) << (8 * v);
+            mw[e] |= ((uint32_t)mid & 0xffu) << (8 * v);
+            lw[e] |= ((uint32_t)lo & 0xffu) << (8 * v);
         }
     }
-    int shi = 0, slo = 0;
+    int sh = 0, sm = 0, sl = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        shi = __dp4a((int)ho[j], 0x01010101, shi);
-        slo = __dp4a((int)lo[j], 0x01010101, slo);
+        sh = __dp4a((int)hw[j], 0x01010101, sh);
+        sm = __dp4a((int)mw[j], 0x01010101, sm);
+        sl = __dp4a((int)lw[j], 0x01010101, sl);
     }
     uint4* h4 = reinterpret_cast<uint4*>(dh);
-    uint4* l4 = reinterpret_cast<uint4*>(dl);
-    h4[0] = make_uint4(ho[0], ho[1], ho[2], ho[3]);
-    h4[1] = make_uint4(ho[4], ho[5], ho[6], ho[7]);
-    l4[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    l4[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-    return 256 * shi + slo;
+    uint4* m4 = reinterpret_cast<uint4*>(dh + astride);
+    uint4* l4 = reinterpret_cast<uint4*>(dh + 2 * astride);
+    h4[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    h4[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+    m4[0] = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+    m4[1] = make_uint4(mw[4], mw[5], mw[6], mw[7]);
+    l4[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    l4[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+    ls[0] = sh;
+    ls[1] = sm;
+    ls[2] = sl;
 }
 
 // Steps [s0, s1) of chunk c of a tile: chunks of bsteps steps, the last one
@@ -232,7 +246,8 @@ __global__ void __launch_bounds__(NW * 32, 2)
     uint8_t* act = smem + p.off_act;
     int* racc = reinterpret_cast<int*>(smem + p.off_red);             // [NW warps][t_max*16][ncols]
     float* red_max = reinterpret_cast<float*>(smem + p.off_tok);      // [NW][M]
-    int* red_sum = reinterpret_cast<int*>(red_max + kW * M);          // [NW][M]
+    constexpr int LS = FORM == 1 ? 3 : 1;                             // row sums per token
+    int* red_sum = reinterpret_cast<int*>(red_max + kW * M);          // [NW][M][LS]
     uint16_t* hs = reinterpret_cast<uint16_t*>(smem + p.off_h);       // [t_max*16]
     uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + p.off_cnt);    // [S] releases, [S] rounds issued
     const uint32_t cnt_sb = sb + p.off_cnt;
@@ -295,6 +310,7 @@ __global__ void __launch_bounds__(NW * 32, 2)
     if (tid == 0) {
         const int nfill = min(S, nstages);
         for (int u = 0; u < nfill; ++u) {
+            if (p.stall && cta == 0 && u == 0) continue;   // test hook: a stage that never comes
             tc::mbar_arrive_expect_tx(sb + p.off_bar + 8 * u, stage_bytes(p, u));
             issue_stage(p, &tm_main, &tm_tail, sb, tile0, u);
         }
@@ -362,28 +378,32 @@ __global__ void __launch_bounds__(NW * 32, 2)
             for (int w = 0; w < kW; ++w) amax_l = fmaxf(amax_l, red_max[w * Mx + lane]);
         }
         tok_amax = amax_l;
-        const float qmax = FORM == 0 ? 127.0f : 32639.0f;
+        const float qmax = FORM == 0 ? 127.0f : kImgMaxF;
         const float inv_l = amax_l > 0.f ? __fdiv_rn(qmax, amax_l) : 0.f;
-        int usum[U];
+        int usum[U][LS];
 #pragma unroll
         for (int i = 0; i < U; ++i) {
             const float inv = Mx == 1 ? inv_l : __shfl_sync(0xffffffffu, inv_l, um[i] < Mx ? um[i] : 0);
-            usum[i] = 0;
+#pragma unroll
+            for (int l = 0; l < LS; ++l) usum[i][l] = 0;
             if (!has[i]) continue;
             uint8_t* dst = act + (kOne ? 0 : um[i]) * F::kCPT * p.astride + uk[i];
             if constexpr (FORM == 0) {
-                usum[i] = quant_group_t(xa[i][0], xa[i][1], inv, dst);
+                usum[i][0] = quant_group_t(xa[i][0], xa[i][1], inv, dst);
             } else {
-                usum[i] = quant_group_s(xa[i], ga[UG > 1 ? i : 0], inv, dst, dst + p.astride);
+                quant_group_s(xa[i], ga[UG > 1 ? i : 0], inv, dst, p.astride, usum[i]);
             }
         }
         for (int m = 0; m < Mx; ++m) {
-            int v = 0;
 #pragma unroll
-            for (int i = 0; i < U; ++i)
-                if (has[i] && um[i] == m) v += usum[i];
-            v = __reduce_add_sync(0xffffffffu, v);
-            if (lane == 0) red_sum[warp * Mx + m] = v;
+            for (int l = 0; l < LS; ++l) {
+                int v = 0;
+#pragma unroll
+                for (int i = 0; i < U; ++i)
+                    if (has[i] && um[i] == m) v += usum[i][l];
+                v = __reduce_add_sync(0xffffffffu, v);
+                if (lane == 0) red_sum[(warp * Mx + m) * LS + l] = v;
+            }
         }
         __syncwarp();
     } else {
@@ -421,7 +441,8 @@ __global__ void __launch_bounds__(NW * 32, 2)
                     sum += quant_group_t(tc::ld_v4(xr + 16 * i), tc::ld_v4(xr + 16 * i + 8), inv,
                                          act + m * p.astride + 16 * i);
             } else {
-                const float inv = amax > 0.f ? __fdiv_rn(32639.0f, amax) : 0.f;
+                const float inv = amax > 0.f ? __fdiv_rn(kImgMaxF, amax) : 0.f;
+                int ls3[3] = {0, 0, 0};
                 for (int i = tid; i < ngroups; i += kT) {
                     uint4 xa[4], gg[4];
 #pragma unroll
@@ -429,12 +450,22 @@ __global__ void __launch_bounds__(NW * 32, 2)
                         xa[v] = tc::ld_v4(xr + 32 * i + 8 * v);
                         gg[v] = ld_ro_v4(p.g + 32 * i + 8 * v);
                     }
-                    sum += quant_group_s(xa, gg, inv, act + (2 * m) * p.astride + 32 * i,
-                                         act + (2 * m + 1) * p.astride + 32 * i);
+                    int gs[3];
+                    quant_group_s(xa, gg, inv, act + (3 * m) * p.astride + 32 * i, p.astride, gs);
+                    ls3[0] += gs[0];
+                    ls3[1] += gs[1];
+                    ls3[2] += gs[2];
+                }
+#pragma unroll
+                for (int l = 0; l < 3; ++l) {
+                    const int v = warp_sum(ls3[l]);
+                    if (lane == 0) red_sum[(warp * M + m) * LS + l] = v;
                 }
             }
-            sum = warp_sum(sum);
-            if (lane == 0) red_sum[warp * M + m] = sum;
+            if (FORM == 0) {
+                sum = warp_sum(sum);
+                if (lane == 0) red_sum[warp * M + m] = sum;
+            }
         }
         __syncthreads();
     }
@@ -469,11 +500,11 @@ __global__ void __launch_bounds__(NW * 32, 2)
         // the CTA agrees to stop
         if (!compact) {
             ok = __all_sync(0xffffffffu, tc::mbar_wait(sb + p.off_bar + 8 * slot, (uint32_t)phase,
-                                                       p.flags, kSWaitLimitNs));
+                                                       p.flags, p.wait_ns));
             if (!ok) break;
         } else if (ok) {
             ok = __all_sync(0xffffffffu, tc::mbar_wait(sb + p.off_bar + 8 * slot, (uint32_t)phase,
-                                                       p.flags, kSWaitLimitNs));
+                                                       p.flags, p.wait_ns));
         }
         const int s0 = chunk * p.bsteps, s1 = ok ? min(s0 + p.bsteps, p.steps) : s0;
         const uint8_t* slot_p = smem + slot * p.slot_bytes;
@@ -610,8 +641,10 @@ __global__ void __launch_bounds__(NW * 32, 2)
         // a stage never arrived: let the copies still in flight land before the
         // CTA's shared memory is released, then leave (the flag is set)
         if (tid == 0) {
-            for (int sl = 0; sl < min(S, nstages); ++sl)
+            for (int sl = 0; sl < min(S, nstages); ++sl) {
+                if (p.stall && cta == 0 && sl == 0) continue;   // nothing was ever requested there
                 tc::mbar_wait(sb + p.off_bar + 8 * sl, cnt[S + sl] & 1u, p.flags, kSDrainLimitNs);
+            }
         }
         __syncthreads();
         return;
@@ -658,29 +691,23 @@ __global__ void __launch_bounds__(NW * 32, 2)
             long long ts = 0;
             if (PREP) {
                 st = p.pscale[m];
-                ts = p.prsum[m];
+                ts = p.prsum64[m];
             } else {
-                float amax = tok_amax;
-                if (kOne) {  // M == 1: the 16 warp sums are contiguous
+                float amax = kOne ? tok_amax : 0.f;
 #pragma unroll
-                    for (int w = 0; w < kW; w += 4) {
-                        const int4 r4 = *reinterpret_cast<const int4*>(red_sum + w);
-                        ts += (r4.x + r4.y) + (r4.z + r4.w);
-                    }
-                } else {
-                    amax = 0.f;
-#pragma unroll
-                    for (int w = 0; w < kW; ++w) {
-                        amax = fmaxf(amax, red_max[w * M + m]);
-                        ts += red_sum[w * M + m];
-                    }
+                for (int w = 0; w < kW; ++w) {
+                    if (!kOne) amax = fmaxf(amax, red_max[w * M + m]);
+                    const int* rs = red_sum + (w * M + m) * LS;
+                    ts += 65536ll * rs[0] + 256ll * rs[1] + (long long)rs[2];
                 }
-                st = amax > 0.f ? __fdiv_rn(amax, 32639.0f) : 0.f;
+                st = amax > 0.f ? __fdiv_rn(amax, kImgMaxF) : 0.f;
             }
-            const long long P = 256ll * tile_sum<kW>(racc, p, r * ncols + 2 * m, ncols) +
-                                tile_sum<kW>(racc, p, r * ncols + 2 * m + 1, ncols);
+            const int c0 = r * ncols + 3 * m;
+            const long long Z = limb_combine(tile_sum<kW>(racc, p, c0, ncols),
+                                             tile_sum<kW>(racc, p, c0 + 1, ncols),
+                                             tile_sum<kW>(racc, p, c0 + 2, ncols), ts);
             const int n = tile0 * 16 + r;
-            const float z = __fmul_rn(st, (float)(2 * P - ts));
+            const float z = __fmul_rn(st, (float)Z);
             const float hv = __half2float(__ushort_as_half(hs[r]));
             p.y[(size_t)m * p.N + n] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hv)));
         }
@@ -743,7 +770,7 @@ bool stream_plan(StreamParams& p, int prep, StreamPlan& pl, int nw = kSWarps) {
     const bool alone = p.compact && act + red_full <= kDecodeMaxSmem / 2;
     if (alone) p.compact = 0;
     const int red = p.compact ? red_compact : red_full;
-    const int tok = prep ? 0 : 2 * nw * M * 4;
+    const int tok = prep ? 0 : (FORM == 1 ? 4 : 2) * nw * M * 4;  // [NW][M] max + [NW][M][LS] sums
     const int hbytes = FORM == 1 ? p.t_max * 16 * 2 : 0;
     auto up16 = [](int v) { return (v + 15) & ~15; };
     const int fixed = up16(act) + up16(red) + up16(tok) + up16(hbytes) + 16 * kMaxSlots + 8 * kMaxSlots;
@@ -796,15 +823,12 @@ template <int FORM, int NT, int PREP, int XREG, int NW = kSWarps>
 cudaError_t launch_stream(const CUtensorMap& tm_main, const CUtensorMap& tm_tail,
                           const StreamParams& p, const StreamPlan& pl, cudaStream_t s) {
     constexpr auto kern = stream_kernel<FORM, NT, PREP, XREG, NW>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kDecodeMaxSmem);
-        if (e != cudaSuccess) return e;
-        e = use_max_shared_carveout(kern);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static KernelAttrs kattrs;
+    if (cudaError_t e = kattrs.ensure(kern, kDecodeMaxSmem)) return e;
+    StreamParams q = p;
+    const unsigned long long stall = take_stall();
+    q.wait_ns = stall ? stall : kSWaitLimitNs;
+    q.stall = stall ? 1 : 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.grid);
     cfg.blockDim = dim3(NW * 32);
@@ -815,7 +839,7 @@ cudaError_t launch_stream(const CUtensorMap& tm_main, const CUtensorMap& tm_tail
     attrs[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tm_main, tm_tail, p);
+    return cudaLaunchKernelEx(&cfg, kern, tm_main, tm_tail, q);
 }
 
 template <int FORM, int PREP>
@@ -935,13 +959,13 @@ cudaError_t launch_ternary_stream_prepared(const int8_t* qp, const float* scale,
 }
 
 cudaError_t launch_onebit_stream_prepared(const int8_t* planes, const float* step,
-                                          const int32_t* tsum, const uint16_t* h,
+                                          const long long* tsum, const uint16_t* h,
                                           const uint32_t* s1, int M, int K, int N, uint16_t* y,
                                           unsigned int* flags, cudaStream_t s) {
     StreamParams p = {};
     p.prep = planes;
     p.pscale = step;
-    p.prsum = tsum;
+    p.prsum64 = tsum;
     p.h = h;
     p.w = s1;
     p.M = M;

@@ -36,6 +36,10 @@
  *     touching memory.
  *   - Errors are returned, never raised on the device: validation errors are
  *     detected before any launch; a failed launch returns BL_ERR_CUDA.
+ *   - Fault injection for callers' error paths: when the environment variable
+ *     BL_FAULT_INJECT is "cuda" or "timeout", every entry point that launches
+ *     work returns BL_ERR_CUDA or BL_ERR_TIMEOUT right after validating its
+ *     arguments, without any CUDA call (read on every call).
  *
  * Packed weight formats (bit-exact ABI; little-endian 32-bit words):
  *   w2 (ternary): uint32 [N][K/16]; weight (n,k) is the 2-bit field at bits
@@ -151,10 +155,10 @@ size_t ob_workspace_bytes(int M, int K, int N);
  * ob_linear -- OneBit linear forward.
  * OneBit page, "1. 新的 1bit 结构": y = ((x (.) g) . S^T) (.) h, with S = +-1
  * (packed s1) and fp16 value vectors g [K] and h [N].
- * The contraction is accumulated exactly in integers on a 16-bit per-token
- * fixed-point image of x (.) g (relative error of that image <= 2^-16 of the
- * token's max |x (.) g|), then scaled in fp32 and rounded once to fp16.
- * K <= 65536.
+ * The contraction is accumulated exactly in integers on a per-token
+ * fixed-point image of x (.) g with 2^22 - 1 levels (error of that image
+ * <= 2^-23 of the token's max |x (.) g| per element), contracted as three
+ * int8 limbs, then scaled in fp32 and rounded once to fp16.  K <= 65536.
  *   x, y      : fp16 [M, K] in, fp16 [M, N] out
  *   s1        : packed signs, uint32 [N, K/32]
  *   g, h      : fp16 [K], fp16 [N]
@@ -176,8 +180,10 @@ bl_status ob_linear(const uint16_t *x, int M, int K, int N, const uint32_t *s1,
  * forbids allocation because cudaMalloc can block the whole device.  This entry
  * point takes no workspace: its scratch is a fixed array of
  * BL_NOALLOC_SCRATCH_BYTES compiled into the library, held by every GPU that
- * loads the library until the process exits.  It computes exactly what
- * bl_ternary_linear computes (same arguments minus the workspace).
+ * loads the library until the process exits.  It runs the same kernels as
+ * bl_ternary_linear, chosen the same way by shape, and gives identical results
+ * (same arguments minus the workspace); only the tensor-core path's balanced
+ * last round is skipped when its scratch would not fit in the array.
  *   - Shapes needing more than the array, i.e. when
  *       round256(M*K) + round256(4*M) + round256(4*M) > BL_NOALLOC_SCRATCH_BYTES
  *     (M*K up to about 16.7 million int8 activations), return
@@ -209,6 +215,19 @@ bl_status bl_ternary_linear_noalloc(const uint16_t *x, int M, int K, int N, cons
  * BL_ERR_SHAPE for an invalid form or shape, M = 0, N = 0 or sm_count <= 0.
  */
 bl_status bl_prefill_plan(int form, int M, int K, int N, int sm_count, int *plan);
+
+/*
+ * bl_debug_stall_next_launch -- test hook for the bounded device-side waits
+ * (no counterpart on the pages).  The next launch in this process of the
+ * streamed decode kernel (small M) or of the whole-tile tensor-core kernel
+ * (prefill M) leaves the first pipeline stage of its CTA 0 unrequested, so a
+ * wait in that CTA never sees its data: it gives up after wait_limit_ns
+ * (instead of 2 s), the kernel records BL_ERR_TIMEOUT for bl_device_status,
+ * lets every copy it did request land, frees its tensor memory and returns.
+ * That launch's outputs are then incomplete.  Later launches are unaffected.
+ * 0 cancels a pending stall.  Host-side only; not for concurrent use.
+ */
+bl_status bl_debug_stall_next_launch(unsigned long long wait_limit_ns);
 
 /*
  * bl_device_status -- synchronise `stream` and report (then clear) any

@@ -30,57 +30,82 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "liboref.so")
+_OMP_LIB_PATH = os.path.join(_HERE, "liboref_omp.so")   # the same source with -fopenmp
 _SRC = os.path.join(_HERE, "oref.c")
 
 OREF_OK, OREF_ERR_SHAPE, OREF_ERR_VALUE, OREF_ERR_ALLOC = 0, -1, -2, -3
 
 CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
-          "-fno-unsafe-math-optimizations", "-Wall"]
+          "-fno-unsafe-math-optimizations", "-Wall", "-Wno-unknown-pragmas"]
+
+
+def _build_one(path: str, extra, force: bool) -> str:
+    if (not force and os.path.exists(path)
+            and os.path.getmtime(path) >= max(os.path.getmtime(_SRC),
+                                              os.path.getmtime(os.path.join(_HERE, "oref.h")))):
+        return path
+    tmp = path + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", *CFLAGS, *extra, "-o", tmp, _SRC, "-lm"], cwd=_HERE)
+    os.replace(tmp, path)
+    return path
 
 
 def build(force: bool = False) -> str:
-    """Compile ``oref.c`` into ``liboref.so`` (gcc); returns the library path."""
-    if (not force and os.path.exists(_LIB_PATH)
-            and os.path.getmtime(_LIB_PATH) >= max(os.path.getmtime(_SRC),
-                                                   os.path.getmtime(os.path.join(_HERE, "oref.h")))):
-        return _LIB_PATH
-    tmp = _LIB_PATH + f".tmp{os.getpid()}"
-    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"], cwd=_HERE)
-    os.replace(tmp, _LIB_PATH)
-    return _LIB_PATH
+    """Compile ``oref.c`` into ``liboref.so`` (one core) and ``liboref_omp.so``
+    (output rows on all host cores, OpenMP); returns the first library's path."""
+    _build_one(_OMP_LIB_PATH, ["-fopenmp"], force)
+    return _build_one(_LIB_PATH, [], force)
 
 
 _lib = None
+_omp_lib = None
 
 
-def lib() -> ctypes.CDLL:
-    global _lib
+def lib(parallel: bool = False) -> ctypes.CDLL:
+    """The oracle library: single-threaded, or (parallel=True) the OpenMP build
+    whose linear forms spread output rows over the host cores."""
+    global _lib, _omp_lib
+    if parallel:
+        if _omp_lib is None:
+            build()
+            _omp_lib = _declare(ctypes.CDLL(_OMP_LIB_PATH))
+        return _omp_lib
     if _lib is None:
         build()
-        L = ctypes.CDLL(_LIB_PATH)
-        P = ctypes.c_void_p
-        I = ctypes.c_int
-        L.oref_half_to_double.argtypes = [ctypes.c_uint16]
-        L.oref_half_to_double.restype = ctypes.c_double
-        L.oref_double_to_half.argtypes = [ctypes.c_double]
-        L.oref_double_to_half.restype = ctypes.c_uint16
-        L.oref_float_to_half.argtypes = [ctypes.c_float]
-        L.oref_float_to_half.restype = ctypes.c_uint16
-        L.oref_pack_ternary.argtypes = [P, I, I, P]
-        L.oref_pack_sign.argtypes = [P, I, I, P]
-        L.oref_quant_act.argtypes = [P, I, I, P, P]
-        L.oref_ternary_linear.argtypes = [P, I, I, I, P, ctypes.c_float, P, P]
-        L.oref_ob_linear.argtypes = [P, I, I, I, P, P, P, P, P]
-        L.oref_svid.argtypes = [P, I, I, P, P, P, P, I, ctypes.c_double]
-        L.oref_onebit_bits.argtypes = [ctypes.c_int64, ctypes.c_int64]
-        L.oref_onebit_bits.restype = ctypes.c_int64
-        L.oref_onebit_params.argtypes = [ctypes.c_int64, ctypes.c_int64]
-        L.oref_onebit_params.restype = ctypes.c_int64
-        for f in ("oref_pack_ternary", "oref_pack_sign", "oref_quant_act",
-                  "oref_ternary_linear", "oref_ob_linear", "oref_svid"):
-            getattr(L, f).restype = I
-        _lib = L
+        _lib = _declare(ctypes.CDLL(_LIB_PATH))
     return _lib
+
+
+def omp_threads() -> int:
+    """Threads the OpenMP build uses (OMP_NUM_THREADS, else the host's cores)."""
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v and v.isdigit() else (os.cpu_count() or 1)
+
+
+def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
+    """Declare the C signatures on a loaded oracle library."""
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    L.oref_half_to_double.argtypes = [ctypes.c_uint16]
+    L.oref_half_to_double.restype = ctypes.c_double
+    L.oref_double_to_half.argtypes = [ctypes.c_double]
+    L.oref_double_to_half.restype = ctypes.c_uint16
+    L.oref_float_to_half.argtypes = [ctypes.c_float]
+    L.oref_float_to_half.restype = ctypes.c_uint16
+    L.oref_pack_ternary.argtypes = [P, I, I, P]
+    L.oref_pack_sign.argtypes = [P, I, I, P]
+    L.oref_quant_act.argtypes = [P, I, I, P, P]
+    L.oref_ternary_linear.argtypes = [P, I, I, I, P, ctypes.c_float, P, P]
+    L.oref_ob_linear.argtypes = [P, I, I, I, P, P, P, P, P]
+    L.oref_svid.argtypes = [P, I, I, P, P, P, P, I, ctypes.c_double]
+    L.oref_onebit_bits.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    L.oref_onebit_bits.restype = ctypes.c_int64
+    L.oref_onebit_params.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    L.oref_onebit_params.restype = ctypes.c_int64
+    for f in ("oref_pack_ternary", "oref_pack_sign", "oref_quant_act",
+              "oref_ternary_linear", "oref_ob_linear", "oref_svid"):
+        getattr(L, f).restype = I
+    return L
 
 
 class OracleError(RuntimeError):
@@ -150,8 +175,9 @@ def quant_act(x: np.ndarray):
     return q, s
 
 
-def ternary_linear(x: np.ndarray, w2: np.ndarray, w_scale: float):
-    """BitLinear forward: returns (y fp16 [M,N], acc int32 [M,N])."""
+def ternary_linear(x: np.ndarray, w2: np.ndarray, w_scale: float, parallel: bool = False):
+    """BitLinear forward: returns (y fp16 [M,N], acc int32 [M,N]).  parallel:
+    the OpenMP build (output rows on all host cores, same results)."""
     xb = _half_bits(x)
     w2 = _c(w2, np.uint32)
     M, K = xb.shape
@@ -159,13 +185,15 @@ def ternary_linear(x: np.ndarray, w2: np.ndarray, w_scale: float):
     assert w2.shape[1] * 16 == K
     y = np.zeros((M, N), dtype=np.uint16)
     acc = np.zeros((M, N), dtype=np.int32)
-    _check(lib().oref_ternary_linear(_p(xb), M, K, N, _p(w2), float(w_scale), _p(y), _p(acc)),
+    _check(lib(parallel).oref_ternary_linear(_p(xb), M, K, N, _p(w2), float(w_scale), _p(y), _p(acc)),
            "ternary_linear")
     return y.view(np.float16), acc
 
 
-def ob_linear(x: np.ndarray, s1: np.ndarray, g: np.ndarray, h: np.ndarray):
-    """OneBit forward: returns (y fp16 [M,N], z fp64 [M,N] before fp16 rounding)."""
+def ob_linear(x: np.ndarray, s1: np.ndarray, g: np.ndarray, h: np.ndarray,
+              parallel: bool = False):
+    """OneBit forward: returns (y fp16 [M,N], z fp64 [M,N] before fp16 rounding).
+    parallel: the OpenMP build (output rows on all host cores, same results)."""
     xb = _half_bits(x)
     s1 = _c(s1, np.uint32)
     gb = _half_bits(g)
@@ -175,7 +203,7 @@ def ob_linear(x: np.ndarray, s1: np.ndarray, g: np.ndarray, h: np.ndarray):
     assert s1.shape[1] * 32 == K and gb.shape == (K,) and hb.shape == (N,)
     y = np.zeros((M, N), dtype=np.uint16)
     z = np.zeros((M, N), dtype=np.float64)
-    _check(lib().oref_ob_linear(_p(xb), M, K, N, _p(s1), _p(gb), _p(hb), _p(y), _p(z)),
+    _check(lib(parallel).oref_ob_linear(_p(xb), M, K, N, _p(s1), _p(gb), _p(hb), _p(y), _p(z)),
            "ob_linear")
     return y.view(np.float16), z
 

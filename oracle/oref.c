@@ -12,7 +12,11 @@
  *          "3. 通过知识蒸馏迁移原模型能力", "讨论与分析 / 1. 效率".
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math (float arithmetic
- * is IEEE binary32 with round-to-nearest-even; no fused multiply-add).
+ * is IEEE binary32 with round-to-nearest-even; no fused multiply-add).  A
+ * second build adds -fopenmp: the two linear forms then compute their output
+ * rows n in parallel on the host cores (each output is still the same scalar
+ * loop over k, in the same order, so the results are identical); the plain
+ * build ignores the pragmas and runs on one core.
  *
  * Readings where the pages are silent (each one is listed in the design notes):
  *   - activation range [-Qb, Qb] with Qb = 127, symmetric, no zero point;
@@ -195,21 +199,25 @@ int oref_ternary_linear(const uint16_t *x, int M, int K, int N, const uint32_t *
     oref_quant_act(x, M, K, q, s);
     int rc = OREF_OK;
     for (int m = 0; m < M && rc == OREF_OK; ++m) {
+        int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
         for (int n = 0; n < N; ++n) {
             int64_t acc = 0;
+            int row_bad = 0;
             for (int k = 0; k < K; ++k) {
                 int t = ternary_at(w2, K, n, k);
-                if (t == -2) { rc = OREF_ERR_VALUE; break; }
+                if (t == -2) { row_bad = 1; break; }
                 int qv = q[(size_t)m * K + k];
                 if (t == 1) acc += qv;
                 else if (t == -1) acc -= qv;
             }
-            if (rc != OREF_OK) break;
+            if (row_bad) { bad = 1; continue; }
             float a = (float)(int32_t)acc;      /* |acc| <= 127*K < 2^24 here */
             float v = (a * s[m]) * w_scale;
             if (acc_out) acc_out[(size_t)m * N + n] = (int32_t)acc;
             if (y) y[(size_t)m * N + n] = oref_float_to_half(v);
         }
+        if (bad) rc = OREF_ERR_VALUE;
     }
     free(q);
     free(s);
@@ -228,6 +236,7 @@ int oref_ob_linear(const uint16_t *x, int M, int K, int N, const uint32_t *s1,
 {
     if (M < 0 || N < 0 || K < 0 || K % 32 != 0) return OREF_ERR_SHAPE;
     for (int m = 0; m < M; ++m) {
+#pragma omp parallel for schedule(static)
         for (int n = 0; n < N; ++n) {
             double z = 0.0;
             for (int k = 0; k < K; ++k) {

@@ -48,7 +48,7 @@ def test_status_strings(L):
 def test_workspace_sizes(L):
     assert L.bl_ternary_workspace_bytes(1, 4096, 4096) == 4096 + 256 + 256
     assert L.bl_ternary_workspace_bytes(8, 4096, 4096) == 8 * 4096 + 256 + 256
-    assert L.ob_workspace_bytes(16, 4096, 4096) == 2 * 16 * 4096 + 256 + 256
+    assert L.ob_workspace_bytes(16, 4096, 4096) == 3 * 16 * 4096 + 256 + 256   # three limb planes
     assert L.bl_ternary_workspace_bytes(1, 100, 16) == 0       # bad K
     assert L.bl_ternary_workspace_bytes(1, 128, 24) == 0       # bad N (not a multiple of 16)
     assert L.ob_workspace_bytes(1, 128, -16) == 0
@@ -103,3 +103,24 @@ def test_python_binding_refuses_cpu_tensors():
     import bit_weight_linear_b200 as blw
     with pytest.raises(ValueError):
         blw.bl_quant_act(torch.zeros((1, 128), dtype=torch.float16))
+
+
+@pytest.mark.parametrize("mode,code", [("cuda", 5), ("timeout", 6)])
+def test_fault_injection_hook(L, monkeypatch, mode, code):
+    """BL_FAULT_INJECT makes every launching entry point return the injected
+    error after its argument checks and before any CUDA call (so this runs
+    without a GPU); bad arguments still win, and unsetting it restores the
+    normal behaviour."""
+    monkeypatch.setenv("BL_FAULT_INJECT", mode)
+    assert L.bl_ternary_linear(A, 1, 128, 16, A, 1.0, A, None, A, 1 << 20, None) == code
+    assert L.ob_linear(A, 1, 128, 16, A, A, A, A, A, 1 << 20, None) == code
+    assert L.bl_quant_act(A, 1, 128, A, A, None) == code
+    assert L.bl_pack_ternary(A, 16, 128, A, None) == code
+    assert L.ob_pack_sign(A, 16, 128, A, None) == code
+    assert L.bl_ternary_linear_noalloc(A, 1, 128, 16, A, 1.0, A, None, None) == code
+    assert L.bl_ternary_linear(A, 1, 100, 16, A, 1.0, A, None, A, 1 << 20, None) == 2
+    assert L.bl_ternary_linear(None, 0, 128, 16, None, 1.0, None, None, None, 0, None) == 0
+    monkeypatch.setenv("BL_FAULT_INJECT", "")
+    # with no GPU the call now fails in the CUDA runtime, not in the hook
+    if not __import__("torch").cuda.is_available():
+        assert L.bl_ternary_linear(A, 1, 128, 16, A, 1.0, A, None, A, 1 << 20, None) == 5

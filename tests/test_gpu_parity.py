@@ -328,8 +328,7 @@ def test_onebit_prefill_small_token_counts(blw, oref, M, K, N):
 def test_onebit_prefill_13b_full_size_sampled_rows(blw, oref):
     """The 13B-shaped down layer (K=13824, N=5120) at M=256, sampled rows."""
     M, K, N = 256, 13824, 5120
-    # 80 tiles of 256 limb rows: shared out over all SMs in k-stages
-    assert blw.ob_workspace_bytes(M, K, N) > 2 * M * K + 1_000_000
+    assert blw.ob_workspace_bytes(M, K, N) >= 3 * M * K   # three limb planes
     x, ws, g, h = _onebit_inputs(M, K, N, seed=4_000_000)
     y = blw.ob_linear(x.cuda(), blw.ob_pack_sign(ws.cuda()), g.cuda(), h.cuda())
     torch.cuda.synchronize()
@@ -489,3 +488,78 @@ def test_quant_two_step_rounding_on_every_path(blw, oref, M):
     q, s = blw.bl_quant_act(x.cuda())
     torch.cuda.synchronize()
     assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+# ------------------------------------- OneBit tokens dominated by one value --
+
+def _per_token_rel_err(y, z_ref):
+    """max over tokens of max_n |y - z_ref| / max_n |z_ref| (each token against
+    its own scale: stricter than one max over the whole output)."""
+    y = np.asarray(y, dtype=np.float64)
+    den = np.max(np.abs(z_ref), axis=1)
+    den[den == 0] = 1.0
+    return float(np.max(np.max(np.abs(y - z_ref), axis=1) / den))
+
+
+# (M, K, N) reaching every OneBit path: M = 1 and 2 prepare the activations in
+# the streamed decode kernel (warp-local), M = 4 through the activation kernel
+# and the prepared streamed kernel, M = 16 the small-token tensor-core tiles,
+# M = 256 the full tensor-core tiles; K = 65536 (M = 1, 4) takes the two-pass
+# activation kernel and the skinny fallback.
+OUTLIER_SHAPES = [(M, K, N) for (K, N) in [(4096, 4096), (13824, 5120)] for M in (1, 2, 4, 16, 256)]
+OUTLIER_SHAPES += [(1, 65536, 32), (4, 65536, 32)]
+
+
+@pytest.mark.parametrize("val", [2000.0, -60000.0])
+@pytest.mark.parametrize("M,K,N", OUTLIER_SHAPES)
+def test_onebit_outlier_tokens_every_path(blw, oref, M, K, N, val):
+    """A token holding one activation of 2000 or -60000 among N(0,1) values:
+    that element sets the token's fixed-point step, so the rest of the token
+    is resolved at step = max|x*g| / (2^22 - 1).  Every token must stay within
+    2e-3 of its own largest output."""
+    x, ws, g, h = _onebit_inputs(M, K, N, seed=4_200_000 + M + K + int(val))
+    x[0, 17] = val
+    if M > 1:
+        x[M - 1, K - 3] = -val
+        x[M // 2, K // 2 + 1] = val / 3
+    y = blw.ob_linear(x.cuda(), blw.ob_pack_sign(ws.cuda()), g.cuda(), h.cuda())
+    torch.cuda.synchronize()
+    assert blw.bl_device_status() == 0
+    rows = np.arange(N)
+    if M * N * K > 2e8:   # 128 sampled rows, first and last included
+        rows = np.sort(np.random.default_rng(M + 3).choice(N, size=128, replace=False))
+        rows[0], rows[-1] = 0, N - 1
+    _, z_ref = oref.ob_linear(x.numpy(), oref.pack_sign(ws.numpy()[rows]), g.numpy(), h.numpy()[rows])
+    assert _per_token_rel_err(y.cpu().numpy()[:, rows], z_ref) <= OB_TOL
+
+
+# ------------------------------------------- largest sweep and 70B shapes ----
+
+@pytest.mark.parametrize("K,N", [(5120, 13824), (13824, 5120)])
+def test_ternary_m1024_13b_sampled_rows(blw, oref, K, N):
+    """The batch sweep's largest token count (M = 1024) on both 13B-shaped
+    layers: int32 accumulators and y bit-exact on sampled rows (first and last
+    included)."""
+    M = 1024
+    x = synth.activations(M, K, seed=4_300_000 + K, outlier_frac=0.01)
+    w = synth.ternary_weights(N, K, seed=4_300_001 + K)
+    y, acc = blw.bl_ternary_linear(x.cuda(), blw.bl_pack_ternary(w.cuda()), 0.02, return_acc=True)
+    torch.cuda.synchronize()
+    assert blw.bl_device_status() == 0
+    rows = _sample_rows(N, seed=11)
+    y_ref, acc_ref = oref.ternary_linear(x.numpy(), oref.pack_ternary(w.numpy()[rows]), 0.02)
+    assert np.array_equal(acc.cpu().numpy()[:, rows], acc_ref)
+    assert np.array_equal(y.cpu().numpy()[:, rows].view(np.uint16), y_ref.view(np.uint16))
+
+
+@pytest.mark.parametrize("M,K,N", [(1024, 5120, 13824), (1024, 13824, 5120), (512, 8192, 28672)])
+def test_onebit_large_m_sampled_rows(blw, oref, M, K, N):
+    """OneBit at the batch sweep's M = 1024 on both 13B-shaped layers and at
+    M = 512 on the 70B-shaped 8192->28672 layer, sampled rows."""
+    x, ws, g, h = _onebit_inputs(M, K, N, seed=4_400_000 + M + K)
+    y = blw.ob_linear(x.cuda(), blw.ob_pack_sign(ws.cuda()), g.cuda(), h.cuda())
+    torch.cuda.synchronize()
+    assert blw.bl_device_status() == 0
+    rows = _sample_rows(N, seed=13)
+    _, z_ref = oref.ob_linear(x.numpy(), oref.pack_sign(ws.numpy()[rows]), g.numpy(), h.numpy()[rows])
+    assert _per_token_rel_err(y.cpu().numpy()[:, rows], z_ref) <= OB_TOL

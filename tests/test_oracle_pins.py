@@ -318,3 +318,20 @@ def test_svid_drives_onebit_layer_by_order_swap(oref):
     Wd = S * np.outer(h.astype(np.float64), g.astype(np.float64))
     ref = x.astype(np.float64) @ Wd.T
     assert np.max(np.abs(z - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_openmp_build_gives_identical_results(oref):
+    """The all-cores oracle build (output rows spread over OpenMP threads) is
+    the same scalar loop per output: bit-identical y, accumulators and z."""
+    from bit_weight_linear_b200 import synth
+    x = synth.activations(3, 640, seed=77, outlier_frac=0.01).numpy()
+    w2 = oref.pack_ternary(synth.ternary_weights(272, 640, seed=78).numpy())
+    y1, a1 = oref.ternary_linear(x, w2, 0.02)
+    y2, a2 = oref.ternary_linear(x, w2, 0.02, parallel=True)
+    assert np.array_equal(a1, a2) and np.array_equal(y1.view(np.uint16), y2.view(np.uint16))
+    s1 = oref.pack_sign(synth.sign_weights(96, 640, seed=79).numpy())
+    g = synth.value_vector(640, seed=80).numpy()
+    h = synth.value_vector(96, seed=81).numpy()
+    _, z1 = oref.ob_linear(x, s1, g, h)
+    _, z2 = oref.ob_linear(x, s1, g, h, parallel=True)
+    assert np.array_equal(z1, z2)

@@ -41,21 +41,35 @@ def test_small_token_counts_share_few_tiles(L):
         p = plan(L, 0, M, 13824, 5120)
         assert (p["bt"], p["stages"], p["tiles"], p["whole"], p["shared"]) == \
             ({9: 32, 16: 32, 64: 64}[M], 27, 40, 0, 40)
-    # OneBit doubles the activation rows (two limbs per token)
-    assert plan(L, 1, 16, 13824, 5120)["bt"] == 32
-    assert plan(L, 1, 64, 13824, 5120)["bt"] == 128
+    # OneBit triples the activation rows (three limbs per token)
+    assert plan(L, 1, 10, 13824, 5120)["bt"] == 32
+    assert plan(L, 1, 16, 13824, 5120)["bt"] == 64
+    assert plan(L, 1, 64, 13824, 5120)["bt"] == 192
     # 108 tiles of a 5120->13824 layer stay whole at M = 16
     assert plan(L, 0, 16, 5120, 13824)["shared"] == 0
 
 
 def test_tile_geometry(L):
-    # activation rows per tile: the smallest multiple of 32 covering the
-    # rows, at most 256; k-blocks per stage 4 / 2 / 1 for <= 64 / <= 128 / more
-    for M, bt, kb in [(9, 32, 4), (33, 64, 4), (100, 128, 2), (129, 160, 1), (300, 256, 1), (512, 256, 1)]:
+    # tokens cut into the fewest tiles of at most 256 activation rows, of
+    # balanced size; activation rows per tile: the smallest multiple of 32
+    # covering a tile's tokens; k-blocks per stage 4 / 2 / 1 for <= 64 / <= 128 / more
+    for M, bt, kb in [(9, 32, 4), (33, 64, 4), (100, 128, 2), (129, 160, 1), (300, 160, 1),
+                      (512, 256, 1), (513, 192, 1), (1024, 256, 1)]:
         p = plan(L, 0, M, 4096, 4096)
         assert p["bt"] == bt
         assert p["stages"] == (4096 // 128 + kb - 1) // kb
         assert p["tiles"] == (4096 // 128) * ((M + bt - 1) // bt)
+
+
+def test_onebit_tile_geometry(L):
+    # OneBit: three limb rows per token, at most 85 tokens (255 rows) per
+    # tile, the token tiles balanced; a tile never splits a token's limbs
+    for M, ttiles in [(5, 1), (10, 1), (11, 1), (85, 1), (86, 2), (256, 4), (512, 7), (1024, 13)]:
+        tpt = -(-M // ttiles)
+        assert tpt <= 85
+        p = plan(L, 1, M, 5120, 13824)
+        assert p["bt"] == min(256, -(-3 * tpt // 32) * 32), M
+        assert p["tiles"] == (13824 // 128) * ttiles, M
 
 
 @pytest.mark.parametrize("sms", [148, 132, 64, 7, 1])
