@@ -54,10 +54,11 @@ def int8_peak(peaks):
     return 2.0 * peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
 
 
-# DRAM bytes per launch of the M = 1 decode kernel over one 7-call LLaMA-7B block
-# (4 x 4096->4096, 2 x 4096->11008, 11008->4096), from one ncu capture of the
-# current (8-warp) kernel: 50.93 MB / 7 launches, i.e. 1.006 x the packed-weight bytes.
-DECODE_TRAFFIC_PER_LAUNCH = 7.275e6
+# DRAM bytes (read + write) per packed-weight byte of the chain kernel, from an
+# ncu capture of a shorter chain of the same blocks (traffic grows with the
+# weights streamed); None until that capture has been taken on this kernel.
+CHAIN_TRAFFIC_PER_WEIGHT_BYTE = None
+CHAIN_TRAFFIC_SOURCE = "not yet captured for this kernel"
 
 
 def load_peaks():
@@ -191,6 +192,64 @@ def run_calls(blw, calls, form):
     else:
         for c in calls:
             blw.ob_linear(c["x"], c["w"], c["g"], c["h"], workspace=c["ws"], out=c["y"])
+
+
+def block_sources(blocks: int):
+    """Dependency pattern of a LLaMA-like decode step through the 7-layer block,
+    each elementwise step between two linears taken as the identity: q, k, v
+    read the block input (block 0: a given x; later: the previous block's down
+    output), o reads v's output (attention's place), gate and up read o's
+    output (the residual/norm's place), down reads gate's output (SwiGLU's)."""
+    src = []
+    for b in range(blocks):
+        base = 7 * b
+        blk_in = -1 if b == 0 else base - 1
+        src += [blk_in, blk_in, blk_in, base + 2, base + 3, base + 3, base + 4]
+    return src
+
+
+def chain_stack(blw, synth, dev, form: str, dependent: bool, layers: int = LLAMA7B_LAYERS):
+    """The 7B-shaped stack as decode-chain layers (M = 1).  dependent: the
+    decode step's dependency pattern (one given input); else every layer reads
+    its own given input.  Returns (layer dicts, weight bytes, given-input
+    buffer, output buffer); every layer's given x and y are views into those
+    two buffers.  Ternary w_scale is 1/sqrt(2K/3) per layer, which keeps the
+    activations O(1) along a dependent chain (timing does not depend on it)."""
+    shapes = [(K, N) for _ in range(layers) for (_, K, N) in LLAMA7B_BLOCK]
+    srcs = block_sources(layers) if dependent else [-1] * len(shapes)
+    x_all = torch.empty((sum(K for (K, _), s in zip(shapes, srcs) if s < 0),), dtype=torch.float16,
+                        device=dev)
+    y_all = torch.empty((sum(N for _, N in shapes),), dtype=torch.float16, device=dev)
+    out, wbytes, xo, yo = [], 0, 0, 0
+    prev_x = None
+    for j, ((K, N), s) in enumerate(zip(shapes, srcs)):
+        seed = 2_000_000 + (j // 7) * 16 + j % 7
+        d = dict(K=K, N=N, src=s, y=y_all[yo:yo + N])
+        yo += N
+        if s < 0:
+            if dependent and prev_x is not None and j % 7 in (1, 2):
+                d["x"] = prev_x            # k and v read q's input
+            else:
+                d["x"] = x_all[xo:xo + K]
+                d["x"].copy_(synth.activations(1, K, seed=seed, device=dev)[0])
+                xo += K
+            prev_x = d["x"]
+        if form == "ternary":
+            w = synth.ternary_weights(N, K, seed=seed + 7, device=dev)
+            d["w"] = blw.bl_pack_ternary(w)
+            d["w_scale"] = float(1.0 / (2.0 * K / 3.0) ** 0.5)
+        else:
+            w = synth.sign_weights(N, K, seed=seed + 7, device=dev)
+            d["w"] = blw.ob_pack_sign(w)
+            d["g"] = synth.value_vector(K, seed=seed + 8, device=dev)
+            d["h"] = synth.value_vector(N, seed=seed + 9, device=dev)
+            wbytes += 2 * (K + N)
+        del w
+        wbytes += d["w"].numel() * 4
+        out.append(d)
+    x_all = x_all[:xo]
+    torch.cuda.synchronize()
+    return out, wbytes, x_all, y_all
 
 
 def capture(fn):
@@ -480,37 +539,39 @@ def main():
             torch.distributed.destroy_process_group()
         return 0
 
-    # ---- headline: ternary decode stack, M=1
-    calls, wbytes, x_all, y_all = decode_stack(blw, synth, dev, "ternary", layers=args.layers)
+    # ---- headline: the ternary 7B-shaped stack at M = 1 as ONE decode-chain launch per step,
+    # with a decode step's dependency pattern
+    chain_layers, wbytes, x_all, y_all = chain_stack(blw, synth, dev, "ternary", dependent=True,
+                                                     layers=args.layers)
     in_b, out_b = x_all.numel() * 2, y_all.numel() * 2
-    g = capture(lambda: run_calls(blw, calls, "ternary"))
+    chain = blw.Chain(0, chain_layers)
+    g = capture(chain.run)
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
     ms = time_replays(g, args.steps, args.warmup, dist_on, dev, clocks)
     time.sleep(0.3)
     clocks.stop()
-    n_calls = len(calls)
+    n_layers = len(chain_layers)
     value = wbytes * world / (ms * 1e-3) / 1e9
 
-    # roofline of the dominant kernel: the packed-weight decode contraction
-    alg_bytes_per_launch = (wbytes + in_b + out_b) / n_calls
-    launch_ms = ms / n_calls          # upper bound: includes the per-call activation quant
-    achieved = alg_bytes_per_launch / (launch_ms * 1e-3) / 1e9
-    roofline = {"kernel": "streamed ternary decode (stream_kernel<0,1,0,2,8>; the 11008-long "
-                          "down rows use stream_kernel<0,1,0,4,8>)", "bound": "hbm",
-                "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": DECODE_TRAFFIC_PER_LAUNCH, "traffic_unit": "bytes",
-                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one 7-call block "
-                                  "(cold caches), averaged per launch",
+    # roofline of the one kernel of the step: the persistent chain kernel
+    alg_bytes = wbytes + in_b + out_b
+    achieved = alg_bytes / (ms * 1e-3) / 1e9
+    roofline = {"kernel": "chain_kernel<0> (one persistent launch per step; all 224 layers)",
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "algorithmic_bytes_per_launch": alg_bytes,
+                "traffic": CHAIN_TRAFFIC_PER_WEIGHT_BYTE * wbytes if CHAIN_TRAFFIC_PER_WEIGHT_BYTE else None,
+                "traffic_unit": "bytes",
+                "traffic_source": CHAIN_TRAFFIC_SOURCE,
                 "peak_source": peaks["_source"],
-                "note": "launch duration = timed region / launches (one kernel per call; includes launch gaps)"}
+                "note": "launch duration = timed region / steps (one chain kernel and one "
+                        f"{4 * n_layers}-byte counter memset per step)"}
 
-    # ---- e2e: host buffers, H2D of every call's input and D2H of every output inside the timed
-    # region.  Two device buffer sets are used in turn, so step i+1's inputs upload and step i-1's
-    # outputs download on a copy stream while step i computes (each step's copies stay in the
-    # timed region; the first upload and the last download are not overlapped).
+    # ---- e2e: host buffers.  Every step uploads the step's given input from pinned host memory
+    # and downloads every layer's output, inside the timed region.  Two device buffer sets (two
+    # chains, two graphs) alternate, so step i+1's upload and step i-1's download overlap step i.
     xin = x_all.cpu().pin_memory()
     youts = [torch.empty(y_all.shape, dtype=torch.float16).pin_memory() for _ in range(2)]
     x_all2, y_all2 = torch.empty_like(x_all), torch.empty_like(y_all)
@@ -519,8 +580,10 @@ def main():
         off = t.storage_offset() - base.storage_offset()
         return other[off:off + t.numel()].view(t.shape)
 
-    calls2 = [dict(c, x=rebased(c["x"], x_all, x_all2), y=rebased(c["y"], y_all, y_all2)) for c in calls]
-    g2 = capture(lambda: run_calls(blw, calls2, "ternary"))
+    layers2 = [dict(d, y=rebased(d["y"], y_all, y_all2),
+                    **({"x": rebased(d["x"], x_all, x_all2)} if "x" in d else {})) for d in chain_layers]
+    chain2 = blw.Chain(0, layers2)
+    g2 = capture(chain2.run)
     sets = [(x_all, y_all, g), (x_all2, y_all2, g2)]
     comp = torch.cuda.current_stream()
     upl, dnl = torch.cuda.Stream(), torch.cuda.Stream()  # uploads and downloads do not queue behind each other
@@ -566,47 +629,67 @@ def main():
     torch.cuda.synchronize()
     barrier(dist_on)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist_on, dev) / e2e_steps
+    assert blw.bl_device_status() == 0, "a bounded wait expired in the chain kernel"
     assert torch.equal(youts[(e2e_steps - 1) % 2], y_all.cpu()), "e2e outputs differ from the device run"
     e2e = {"value": round(wbytes * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
            "h2d_bytes_per_step": xin.numel() * 2, "d2h_bytes_per_step": youts[0].numel() * 2,
            "ms_per_step": round(e2e_ms, 4),
-           "overlap": "double-buffered: uploads/downloads of neighbouring steps overlap the graph"}
-    del g2, calls2, x_all2, y_all2
-    del g, calls, x_all, y_all
+           "overlap": "double-buffered: uploads/downloads of neighbouring steps overlap the launch"}
+    del g2, chain2, layers2, x_all2, y_all2
+    del g, chain, chain_layers, x_all, y_all
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
 
     extras = {}
     if not args.no_extras:
-        # ---- same stack with fused QKV and gate+up projections (4 calls per block)
-        fcalls, fwbytes, _fx, _fy = decode_stack(blw, synth, dev, "ternary", layers=args.layers,
-                                                 block=LLAMA7B_BLOCK_FUSED)
-        fg = capture(lambda: run_calls(blw, fcalls, "ternary"))
-        fms = time_replays(fg, args.steps, args.warmup, dist_on, dev)
-        fval = fwbytes * world / (fms * 1e-3) / 1e9
-        extras["decode_fused_projections"] = {
-            "workload": "llama7b-decode-M1-ternary, qkv (4096->12288) and gate+up (4096->22016) fused",
-            "calls_per_step": len(fcalls), "value": round(fval, 2), "unit": "GB/s",
-            "ms_per_step": round(fms, 4), "weight_bytes_per_step": fwbytes,
-            "roofline": {"bound": "hbm", "achieved": round(fval / world, 1), "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": round(fval / world / peaks["hbm_gbs"], 4)}}
-        del fg, fcalls, _fx, _fy
+        # ---- the same stack as one chain launch whose layers all read their own given input
+        ilayers, iwbytes, _ix, _iy = chain_stack(blw, synth, dev, "ternary", dependent=False,
+                                                 layers=args.layers)
+        ich = blw.Chain(0, ilayers)
+        ig = capture(ich.run)
+        ims = time_replays(ig, args.steps, args.warmup, dist_on, dev)
+        ival = iwbytes * world / (ims * 1e-3) / 1e9
+        extras["decode_chain_independent"] = {
+            "workload": "llama7b-decode-M1-ternary-32x7, one chain launch, every layer its own input",
+            "value": round(ival, 2), "unit": "GB/s", "ms_per_step": round(ims, 4),
+            "roofline": {"bound": "hbm", "achieved": round(ival / world, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(ival / world / peaks["hbm_gbs"], 4)}}
+        del ig, ich, ilayers, _ix, _iy
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
 
-        # ---- OneBit decode stack, M=1
-        ocalls, owbytes, _ox, _oy = decode_stack(blw, synth, dev, "onebit", layers=args.layers)
-        og = capture(lambda: run_calls(blw, ocalls, "onebit"))
-        oms = time_replays(og, max(10, args.steps // 2), args.warmup, dist_on, dev)
+        # ---- OneBit: the same dependent decode-chain step
+        olayers, owbytes, _ox, _oy = chain_stack(blw, synth, dev, "onebit", dependent=True,
+                                                 layers=args.layers)
+        och = blw.Chain(1, olayers)
+        og = capture(och.run)
+        oms = time_replays(og, args.steps, args.warmup, dist_on, dev)
         oval = owbytes * world / (oms * 1e-3) / 1e9
         extras["onebit_decode"] = {
-            "workload": "llama7b-decode-M1-onebit-32x7", "value": round(oval, 2), "unit": "GB/s",
-            "ms_per_step": round(oms, 4), "weight_bytes_per_step": owbytes,
+            "workload": "llama7b-decode-M1-onebit-32x7, one chain launch, decode-step dependencies",
+            "value": round(oval, 2), "unit": "GB/s", "ms_per_step": round(oms, 4),
+            "weight_bytes_per_step": owbytes,
             "roofline": {"bound": "hbm", "achieved": round(oval / world, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(oval / world / peaks["hbm_gbs"], 4)}}
-        del og, ocalls, _ox, _oy
+        del og, och, olayers, _ox, _oy
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
+
+        # ---- the per-call path: 224 bl_ternary_linear / ob_linear calls per step in a graph
+        for form in ("ternary", "onebit"):
+            pcalls, pwbytes, _px, _py = decode_stack(blw, synth, dev, form, layers=args.layers)
+            pg = capture(lambda: run_calls(blw, pcalls, form))
+            pms = time_replays(pg, max(10, args.steps // 2), args.warmup, dist_on, dev)
+            pval = pwbytes * world / (pms * 1e-3) / 1e9
+            extras[f"decode_per_call_{form}"] = {
+                "workload": f"llama7b-decode-M1-{form}-32x7, one library call per layer (CUDA graph)",
+                "value": round(pval, 2), "unit": "GB/s", "ms_per_step": round(pms, 4),
+                "roofline": {"bound": "hbm", "achieved": round(pval / world, 1),
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": round(pval / world / peaks["hbm_gbs"], 4)}}
+            del pg, pcalls, _px, _py
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
 
         extras["prefill"] = run_prefill(blw, synth, dev, args, dist_on, world, peaks)
         # the two small configurations: BitLinear M=8 and OneBit M=1 / M=16 on 4096x4096
@@ -629,12 +712,15 @@ def main():
         "data": "synthetic",
         "config": {"workload": "llama7b-decode-M1-ternary-bitlinear-32x7", "M": 1,
                    "layers": args.layers, "shapes_KxN": [[K, N] for _, K, N in LLAMA7B_BLOCK],
-                   "weight_bytes_per_step": wbytes, "w_scale": W_SCALE,
+                   "weight_bytes_per_step": wbytes, "w_scale": "1/sqrt(2K/3) per layer",
+                   "dependencies": "decode step: q,k,v <- block input; o <- v; gate,up <- o; "
+                                   "down <- gate; next block input <- down",
                    "l2": "inputs larger than L2 (1.62 GB packed weights per step, 126 MB L2)",
-                   "parallelism": f"replicas x{world}", "graph": "CUDA graph of 224 calls"},
+                   "parallelism": f"replicas x{world}",
+                   "graph": "CUDA graph of one bl_chain_run (counter memset + one kernel)"},
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": args.steps * n_calls,
+        "gpu_launches": args.steps,
         "clocks": clocks.summary(),
     }
     line.update(extras)

@@ -34,6 +34,18 @@ STATUS_NAMES = {0: "BL_OK", 1: "BL_ERR_NULL", 2: "BL_ERR_SHAPE", 3: "BL_ERR_ALIG
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _SZ = ctypes.c_size_t
+
+
+class ChainLayer(ctypes.Structure):
+    """bl_chain_layer (include/bitlinear.h)."""
+    _fields_ = [("x", _P), ("src", _I), ("K", _I), ("N", _I), ("w", _P), ("w_scale", ctypes.c_float),
+                ("g", _P), ("h", _P), ("y", _P), ("acc_out", _P)]
+
+
+class ChainPlan(ctypes.Structure):
+    """bl_chain_plan (include/bitlinear.h)."""
+    _fields_ = [("form", _I), ("n_layers", _I), ("sm_count", _I), ("kmax", _I), ("slots", _I),
+                ("smem_bytes", _I)]
 ABI = {
     "bl_status_string": ([_I], ctypes.c_char_p),
     "bl_abi_version": ([], _I),
@@ -48,6 +60,9 @@ ABI = {
     "bl_prefill_plan": ([_I, _I, _I, _I, _I, _P], _I),
     "bl_ternary_linear_noalloc": ([_P, _I, _I, _I, _P, ctypes.c_float, _P, _P, _P], _I),
     "bl_debug_stall_next_launch": ([ctypes.c_ulonglong], _I),
+    "bl_chain_bytes": ([_I], _SZ),
+    "bl_chain_build": ([_I, _P, _I, _P, _SZ, _P, _P], _I),
+    "bl_chain_run": ([_P, _P, _P], _I),
 }
 
 
@@ -197,10 +212,51 @@ def bl_ternary_linear_noalloc(x: torch.Tensor, w2: torch.Tensor, w_scale: float,
     return (y, acc) if return_acc else y
 
 
+class Chain:
+    """A decode chain built on the device (bl_chain_build): the single-token
+    forward of a list of layers in one persistent launch per run().  Holds the
+    device descriptor buffer and the plan; keeps the layers' tensors alive."""
+
+    def __init__(self, form: int, layers: list[dict]):
+        """layers: dicts with K, N, w (packed, CUDA), y (fp16 [N] or [1, N],
+        CUDA), and either x (fp16 [K], CUDA) or src (index of an earlier
+        layer); ternary: w_scale, optional acc_out (int32 [N]); OneBit: g, h."""
+        n = len(layers)
+        arr = (ChainLayer * n)()
+        self._keep = []
+        dev = None
+        for j, d in enumerate(layers):
+            ts = [d.get(k) for k in ("x", "w", "g", "h", "y", "acc_out")]
+            _need_cuda(*[t for t in ts if t is not None])
+            self._keep.extend(t for t in ts if t is not None)
+            dev = dev or d["w"].device
+            arr[j].x = None if d.get("x") is None else d["x"].data_ptr()
+            arr[j].src = int(d.get("src", -1))
+            arr[j].K, arr[j].N = int(d["K"]), int(d["N"])
+            arr[j].w = d["w"].data_ptr()
+            arr[j].w_scale = float(d.get("w_scale", 0.0))
+            arr[j].g = None if d.get("g") is None else d["g"].data_ptr()
+            arr[j].h = None if d.get("h") is None else d["h"].data_ptr()
+            arr[j].y = d["y"].data_ptr()
+            arr[j].acc_out = None if d.get("acc_out") is None else d["acc_out"].data_ptr()
+        nbytes = int(lib().bl_chain_bytes(n))
+        if nbytes == 0:
+            raise ValueError("chain length out of range")
+        self.buf = torch.empty((nbytes,), dtype=torch.uint8, device=dev)
+        self.plan = ChainPlan()
+        _check("bl_chain_build", lib().bl_chain_build(form, arr, n, _ptr(self.buf), nbytes,
+                                                      ctypes.byref(self.plan), _stream()))
+
+    def run(self):
+        """One decode step over the chain on torch's current stream."""
+        _check("bl_chain_run", lib().bl_chain_run(ctypes.byref(self.plan), _ptr(self.buf),
+                                                  _stream()))
+
+
 def bl_device_status() -> int:
     return int(lib().bl_device_status(_stream()))
 
 
 __all__ = ["bl_pack_ternary", "ob_pack_sign", "bl_quant_act", "bl_ternary_linear",
            "ob_linear", "bl_ternary_workspace_bytes", "ob_workspace_bytes",
-           "bl_device_status", "bl_ternary_linear_noalloc", "BitLinearError", "lib", "ABI"]
+           "bl_device_status", "bl_ternary_linear_noalloc", "Chain", "BitLinearError", "lib", "ABI"]

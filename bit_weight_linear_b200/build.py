@@ -14,8 +14,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libbitlinear.so")
-SOURCES = ["api.cu", "pack.cu", "quant.cu", "skinny.cu", "prefill.cu", "stream.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "decode_forms.cuh", "kernels.h", "tc_prims.cuh", "tmap.cuh"]
+SOURCES = ["api.cu", "pack.cu", "quant.cu", "skinny.cu", "prefill.cu", "stream.cu", "chain.cu",
+           "noalloc.cu"]
+HEADERS = ["act_groups.cuh", "common.cuh", "decode_forms.cuh", "kernels.h", "tc_prims.cuh", "tmap.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -19,6 +19,7 @@ __device__ unsigned int g_pack_error = 0;
 namespace {
 
 constexpr size_t kAlign = 256;
+constexpr int kMaxChainLayers = 65536;
 
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
@@ -294,6 +295,45 @@ bl_status bl_prefill_plan(int form, int M, int K, int N, int sm_count, int* plan
     if (M == 0 || N == 0 || sm_count <= 0) return BL_ERR_SHAPE;
     bl::prefill_plan_info(form, M, K, N, sm_count, plan);
     return BL_OK;
+}
+
+size_t bl_chain_bytes(int n_layers) {
+    if (n_layers <= 0 || n_layers > kMaxChainLayers) return 0;
+    return bl::chain_bytes(n_layers);
+}
+
+bl_status bl_chain_build(int form, const bl_chain_layer* layers, int n_layers, void* chain,
+                         size_t chain_bytes, bl_chain_plan* plan, bl_stream_t stream) {
+    if (!layers || !chain || !plan) return BL_ERR_NULL;
+    if ((form != 0 && form != 1) || n_layers <= 0 || n_layers > kMaxChainLayers) return BL_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(chain) & 255u) != 0) return BL_ERR_ALIGN;
+    for (int j = 0; j < n_layers; ++j) {
+        const bl_chain_layer& L = layers[j];
+        if (L.K <= 0 || L.K % 128 != 0 || L.K > bl::chain_max_k(form) || L.N <= 0 || L.N % 16 != 0 ||
+            L.N > (1 << 24))
+            return BL_ERR_SHAPE;
+        if (L.src < -1 || L.src >= j) return BL_ERR_SHAPE;
+        if (L.src >= 0 && layers[L.src].N != L.K) return BL_ERR_SHAPE;
+        if ((L.src < 0 && !L.x) || !L.w || !L.y || (form == 1 && (!L.g || !L.h))) return BL_ERR_NULL;
+        if ((L.src < 0 && misaligned(L.x)) || misaligned(L.w) || misaligned(L.y) ||
+            misaligned(L.acc_out) || misaligned(L.g) || misaligned(L.h))
+            return BL_ERR_ALIGN;
+    }
+    if (chain_bytes < bl::chain_bytes(n_layers)) return BL_ERR_WORKSPACE;
+    if (bl_status st = bl::fault_injected()) return st;
+    return bl::chain_build(form, layers, n_layers, chain, chain_bytes, plan, cs(stream));
+}
+
+bl_status bl_chain_run(const bl_chain_plan* plan, const void* chain, bl_stream_t stream) {
+    if (!plan || !chain) return BL_ERR_NULL;
+    if ((plan->form != 0 && plan->form != 1) || plan->n_layers <= 0 ||
+        plan->n_layers > kMaxChainLayers)
+        return BL_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(chain) & 255u) != 0) return BL_ERR_ALIGN;
+    if (bl_status st = bl::fault_injected()) return st;
+    unsigned int* flags = device_flags();
+    if (!flags) return BL_ERR_CUDA;
+    return bl::chain_run(plan, chain, flags, cs(stream));
 }
 
 bl_status bl_debug_stall_next_launch(unsigned long long wait_limit_ns) {

@@ -1,0 +1,758 @@
+// chain.cu -- persistent single-token (M = 1) forward of a whole list of
+// layers in ONE launch: the decode step of a stack of extreme-low-bit linear
+// layers (BitNet b1.58 page, "内存和延迟": at decode sizes the time of the
+// model goes to its nn.Linear layers, whose cost is reading their weights).
+//
+// Arithmetic per layer is that of the other decode kernels (stream.cu):
+//   BitLinear (BitNet b1.58 page, "BitNet b1.58 介绍"): per-token absmax int8
+//     q = rne(x * rn(127/amax)), acc = sum q*code - sum q, y = fp16((acc*s)*w_scale);
+//   OneBit (OneBit page, "1. 新的 1bit 结构"): 23-bit fixed-point image X of
+//     x*g in three int8 limbs, sum X*S = 2 sum X*b - sum X, y = fp16(step*Z*h).
+//
+// A layer's input is either given (x) or the output y of an earlier layer of
+// the list.  Why one launch: a separate launch per layer costs a kernel
+// boundary and then a dependent chain (read x, reduce its absmax, quantise,
+// contract, write y) in front of every layer; here the weights of the next
+// layers keep streaming while the current one finishes, and the activations
+// of the next layer are prepared while the current one is contracted.
+//
+// One CTA per SM (all co-resident: cooperative launch), three warp roles:
+//   warp 0      producer: one thread streams the CTA's weight stages, layer
+//               after layer, through an S-slot shared-memory ring (one 3-D TMA
+//               box of 16 rows x up to 16 64-byte steps per stage, plus a 2-D
+//               box for a partial last step), limited only by free slots;
+//   warps 1-8   contraction: u8 x s8 warp MMA (m16n8k32) over the steps of
+//               each stage they own, per-tile partial sums added into shared
+//               memory with integer atomics (exact in any order);
+//   warps 9-12  activations and epilogue: for layer j+1 (while warps 1-8
+//               contract layer j; two buffers) the per-token absmax and the
+//               quantisation into the permuted int8 tile; for layer j the
+//               fp16 outputs, and, when a later layer reads them, one arrival
+//               per CTA on the layer's completion counter (release fence).
+// A layer whose input is another layer's output waits (bounded, acquire)
+// until every CTA has arrived on that layer's counter, then reads its y
+// through L2.  A layer with the same input as the layer before it reuses that
+// layer's prepared activations.  The tiles of a layer are dealt to the CTAs
+// round-robin from a per-layer rotation, so every CTA carries the same share
+// of the whole list.
+//
+// Every wait is bounded (2 s): on expiry the kernel sets the device condition
+// word (BL_ERR_TIMEOUT through bl_device_status), and the producer lets every
+// copy it requested land before its CTA can exit.
+#include "act_groups.cuh"
+#include "common.cuh"
+#include "decode_forms.cuh"
+#include "kernels.h"
+#include "tc_prims.cuh"
+#include "tmap.cuh"
+
+#include <cstring>
+#include <vector>
+
+namespace bl {
+
+namespace {
+
+constexpr int kMmaWarps = 8;
+constexpr int kPrepWarps = 4;
+constexpr int kPrepThreads = kPrepWarps * 32;
+constexpr int kThreads = (1 + kMmaWarps + kPrepWarps) * 32;   // 416
+constexpr int kFirstPrepWarp = 1 + kMmaWarps;
+constexpr int kMaxTiles = 16;              // tiles of one layer per CTA
+constexpr int kMaxSlots = 12;
+constexpr int kStageSteps = 16;            // 64-byte steps of a row per stage: 16 KB for 16 rows
+// + the [16 rows][<= 48 B] tail box, and room for the 16 bytes past it that lanes
+// of a partial step read (they meet zero activations)
+constexpr int kSlotBytes = 16 * kStageSteps * 64 + 1024;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr int kBarPrep = 1;                // named barrier of the activation/epilogue warps
+
+// One layer of a chain in device memory (written by bl_chain_build, read-only
+// in the kernel).  384 bytes, 64-byte aligned: the tensor maps come first.
+struct alignas(64) ChainLayer {
+    CUtensorMap tm_main;   // [step][row][64 B] boxes of 16 rows x bsteps steps
+    CUtensorMap tm_tail;   // [row][tail B] box of a partial last step
+    const uint16_t* x;     // given input (src < 0)
+    const uint32_t* w;     // packed weights
+    uint16_t* y;
+    int32_t* acc_out;      // optional (ternary)
+    const uint16_t* g;     // OneBit input value vector
+    const uint16_t* h;     // OneBit output value vector
+    float w_scale;
+    int src;               // -1: x given; else the layer whose y is the input
+    int K, N;
+    int steps, nfull, tail, ragged, bsteps, nch, ntile, rot;
+    int has_dep;           // a later layer reads y: arrive on done[] after the epilogue
+    int reuse;             // same input as the previous layer: copy its prepared activations
+    int pad[6];
+};
+static_assert(sizeof(ChainLayer) == 384, "chain layer descriptor size");
+
+struct ChainParams {
+    const ChainLayer* layers;
+    int n;
+    unsigned int* done;    // [n] arrivals of CTAs that finished a layer's epilogue
+    unsigned int* flags;   // device condition word
+    int S;                 // ring slots
+    int astride;           // bytes between activation rows (Kmax + 16)
+    int off_act, off_part, off_tok, off_bar;
+    uint64_t wait_ns;
+};
+
+// Tiles of layer L taken by CTA c of G: first, first + G, ... < ntile.
+__device__ __forceinline__ int first_tile(const ChainLayer& L, int c, int G) {
+    const int r = (c - L.rot) % G;
+    return r < 0 ? r + G : r;
+}
+__device__ __forceinline__ int tiles_of(const ChainLayer& L, int first, int G) {
+    return first < L.ntile ? (L.ntile - 1 - first) / G + 1 : 0;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned int* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// 16-byte load through L2 only (another CTA's output, after an acquire).
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void bar_prep() {
+    asm volatile("bar.sync %0, %1;" ::"r"(kBarPrep), "r"(kPrepThreads) : "memory");
+}
+
+// Per-layer shared state of the activation/epilogue warps.
+struct TokStats {
+    float scale[2];        // ternary amax/127, OneBit amax'/kImgMax; per buffer
+    int qsum[2];           // ternary sum q
+    long long xsum[2];     // OneBit sum X
+    uint32_t red[3][kPrepWarps];
+    int redi[3][kPrepWarps];
+};
+
+// Rows up to this many elements are prepared from registers in one read.
+constexpr int kRegK = 16384;
+constexpr int kRegChunks = kRegK / 8 / kPrepThreads;   // 16-byte chunks of x per thread
+
+// Activations of layer L into buffer act ([cols][astride] bytes) for a single
+// token.  K <= kRegK: x is read once into registers (every load in flight at
+// once), then its absmax is reduced and it is quantised from registers
+// (OneBit re-reads g, a parameter, for the products).  Longer rows: two passes
+// over x (the second from L1 or L2).  `cg`: x is another CTA's output, read
+// through L2.
+template <int FORM>
+__device__ void prep_layer(const ChainLayer& L, const uint16_t* x, bool cg, uint8_t* act,
+                           int astride, TokStats* ts, int b, int et) {
+    const int K = L.K;
+    const int pw = et >> 5, lane = et & 31;
+    auto ld = [&](const uint16_t* p) { return cg ? ld_cg_v4(p) : tc::ld_v4(p); };
+    const bool in_regs = K <= kRegK;
+    uint4 xr[kRegChunks];
+    float amax;
+    if constexpr (FORM == 0) {
+        // chunk c of thread et covers elements 8 (et + c P) .. +8, P = kPrepThreads
+        uint32_t mx = 0;
+        // chunks of this thread: c < nc (8 (et + c P) < K)
+        const int nc = (K / 8 - et + kPrepThreads - 1) / kPrepThreads;
+        if (in_regs) {
+#pragma unroll
+            for (int c = 0; c < kRegChunks; ++c) {
+                if (c >= nc) break;
+                xr[c] = ld(x + 8 * (et + c * kPrepThreads));
+            }
+#pragma unroll
+            for (int c = 0; c < kRegChunks; ++c) {
+                if (c >= nc) break;
+                mx = max(mx, absmax_bits_t(xr[c]));
+            }
+        } else {
+#pragma unroll 4
+            for (int c = et; c < K / 8; c += kPrepThreads) mx = max(mx, absmax_bits_t(ld(x + 8 * c)));
+        }
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if (lane == 0) ts->red[0][pw] = mx;
+        bar_prep();
+        uint32_t m = 0;
+#pragma unroll
+        for (int w = 0; w < kPrepWarps; ++w) m = max(m, ts->red[0][w]);
+        amax = hbits(m);
+        const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+        int sum = 0;
+        if (in_regs) {
+            // a 16-element group is two 8-element chunks: chunk pairs (c, c+1)
+            // of a thread cover elements 8 (et + c P) and 8 (et + (c+1) P), not
+            // adjacent, so quantise 8-element halves into the permuted group:
+            // byte 4j+b of the group of element e holds element 4b+j
+#pragma unroll
+            for (int c = 0; c < kRegChunks; ++c) {
+                if (c >= nc) break;
+                const int e = 8 * (et + c * kPrepThreads);
+                sum += quant_half_group_t(xr[c], inv, act + (e & ~15), (e >> 3) & 1);
+            }
+        } else {
+#pragma unroll 2
+            for (int gi = et; gi < K / 16; gi += kPrepThreads)
+                sum += quant_group_t(ld(x + 16 * gi), ld(x + 16 * gi + 8), inv, act + 16 * gi);
+        }
+        sum = __reduce_add_sync(0xffffffffu, sum);
+        if (lane == 0) ts->redi[0][pw] = sum;
+        bar_prep();
+        if (et == 0) {
+            int s = 0;
+#pragma unroll
+            for (int w = 0; w < kPrepWarps; ++w) s += ts->redi[0][w];
+            ts->qsum[b] = s;
+            ts->scale[b] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
+        }
+    } else {
+        // chunk c of thread et: the 32-element group et + c P, as 4 x 8 halves
+        // (OneBit rows are at most kRegK / 4 groups per thread in registers)
+        constexpr int kG = kRegChunks / 4;
+        float mx = 0.f;
+        const int ng = (K / 32 - et + kPrepThreads - 1) / kPrepThreads;   // groups of this thread
+        if (in_regs) {
+#pragma unroll
+            for (int c = 0; c < kG; ++c) {
+                if (c >= ng) break;
+                const int e = 32 * (et + c * kPrepThreads);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) xr[4 * c + v] = ld(x + e + 8 * v);
+            }
+#pragma unroll
+            for (int c = 0; c < kG; ++c) {
+                if (c >= ng) break;
+                const int e = 32 * (et + c * kPrepThreads);
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                    mx = fmaxf(mx, absmax_prod(xr[4 * c + v], ld_ro_v4(L.g + e + 8 * v)));
+            }
+        } else {
+            for (int c = et; c < K / 8; c += kPrepThreads)
+                mx = fmaxf(mx, absmax_prod(ld(x + 8 * c), ld_ro_v4(L.g + 8 * c)));
+        }
+        const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
+        if (lane == 0) ts->red[0][pw] = mb;
+        bar_prep();
+        uint32_t m = 0;
+#pragma unroll
+        for (int w = 0; w < kPrepWarps; ++w) m = max(m, ts->red[0][w]);
+        amax = __uint_as_float(m);
+        const float inv = amax > 0.f ? __fdiv_rn(kImgMaxF, amax) : 0.f;
+        int ls[3] = {0, 0, 0};
+        auto group = [&](const uint4 (&xa)[4], int gi) {
+            uint4 ga[4];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) ga[v] = ld_ro_v4(L.g + 32 * gi + 8 * v);
+            int gs[3];
+            quant_group_s(xa, ga, inv, act + 32 * gi, astride, gs);
+            ls[0] += gs[0];
+            ls[1] += gs[1];
+            ls[2] += gs[2];
+        };
+        if (in_regs) {
+#pragma unroll
+            for (int c = 0; c < kG; ++c) {
+                if (c >= ng) break;
+                const uint4 xa[4] = {xr[4 * c], xr[4 * c + 1], xr[4 * c + 2], xr[4 * c + 3]};
+                group(xa, et + c * kPrepThreads);
+            }
+        } else {
+            for (int gi = et; gi < K / 32; gi += kPrepThreads) {
+                uint4 xa[4];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) xa[v] = ld(x + 32 * gi + 8 * v);
+                group(xa, gi);
+            }
+        }
+#pragma unroll
+        for (int l = 0; l < 3; ++l) {
+            const int v = __reduce_add_sync(0xffffffffu, ls[l]);
+            if (lane == 0) ts->redi[l][pw] = v;
+        }
+        bar_prep();
+        if (et == 0) {
+            long long s = 0;
+#pragma unroll
+            for (int w = 0; w < kPrepWarps; ++w)
+                s += 65536ll * ts->redi[0][w] + 256ll * ts->redi[1][w] + (long long)ts->redi[2][w];
+            ts->xsum[b] = s;
+            ts->scale[b] = amax > 0.f ? __fdiv_rn(amax, kImgMaxF) : 0.f;
+        }
+    }
+}
+
+template <int FORM>
+__global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p) {
+    using F = DF<FORM>;
+    constexpr int COLS = F::kCPT;          // activation columns of the single token
+    constexpr int CH = 4;                  // independent accumulator chains
+    constexpr bool kMasked = FORM == 0;    // ternary: in-place masked 2-bit unpack
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, G = gridDim.x, S = p.S, n = p.n;
+    const uint32_t sb = tc::smem_u32(smem);
+    int* part = reinterpret_cast<int*>(smem + p.off_part);          // [2][kMaxTiles*16][COLS]
+    TokStats* ts = reinterpret_cast<TokStats*>(smem + p.off_tok);
+    const uint32_t bar_full = sb + p.off_bar;                         // [S] stage landed
+    const uint32_t bar_empty = bar_full + 8 * S;                      // [S] 8 warps done with it
+    const uint32_t bar_act = bar_empty + 8 * S;                       // [2] activations ready
+    const uint32_t bar_mma = bar_act + 16;                            // [2] layer contracted
+    constexpr int kPartInts = 2 * kMaxTiles * 16 * COLS;
+
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) {
+            tc::mbar_init(bar_full + 8 * i, 1);
+            tc::mbar_init(bar_empty + 8 * i, kMmaWarps);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(bar_act + 8 * i, 1);
+            tc::mbar_init(bar_mma + 8 * i, kMmaWarps);
+        }
+        tc::mbar_fence_init();
+    }
+    for (int i = tid; i < kPartInts; i += kThreads) part[i] = 0;
+    __syncthreads();
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer --
+        if (lane != 0) return;
+        int u = 0;
+        bool ok = true;
+        for (int j = 0; j < n && ok; ++j) {
+            const ChainLayer& L = p.layers[j];
+            if (j + 1 < n) {
+                tc::prefetch_tmap(&p.layers[j + 1].tm_main);
+                if (p.layers[j + 1].ragged) tc::prefetch_tmap(&p.layers[j + 1].tm_tail);
+            }
+            // a given input two layers ahead: into L2 before its activations are prepared
+            if (j + 2 < n && p.layers[j + 2].src < 0 && !p.layers[j + 2].reuse)
+                tc::bulk_prefetch_l2(p.layers[j + 2].x, (uint32_t)(2 * p.layers[j + 2].K));
+            const int first = first_tile(L, c, G), T = tiles_of(L, first, G);
+            const int steps = L.steps, nfull = L.nfull, bsteps = L.bsteps, nch = L.nch;
+            const bool ragged = L.ragged != 0;
+            for (int k = 0; k < T && ok; ++k) {
+                const int row0 = (first + k * G) * 16;
+                for (int ch = 0; ch < nch; ++ch, ++u) {
+                    const int slot = u % S;
+                    if (u >= S) {
+                        ok = tc::mbar_wait(bar_empty + 8 * slot, ((u / S) - 1) & 1, p.flags, p.wait_ns);
+                        if (!ok) break;
+                    }
+                    const int s0 = ch * bsteps, s1 = min(s0 + bsteps, steps);
+                    uint32_t bytes = s0 < nfull ? (uint32_t)bsteps * 1024u : 0u;
+                    if (ragged && s1 == steps) bytes += 16u * (uint32_t)L.tail;
+                    const uint32_t dst = sb + slot * kSlotBytes, bar = bar_full + 8 * slot;
+                    tc::mbar_arrive_expect_tx(bar, bytes);
+                    if (s0 < nfull) tc::tma_load_3d(dst, &L.tm_main, 0, row0, s0, bar);
+                    if (ragged && s1 == steps) tc::tma_load_2d(dst + bsteps * 1024, &L.tm_tail, 0, row0, bar);
+                }
+            }
+        }
+        // Every copy requested lands before the CTA can exit (on the normal
+        // path the contraction has consumed them and these waits return at once).
+        for (int v = (u > S ? u - S : 0); v < u; ++v)
+            tc::mbar_wait(bar_full + 8 * (v % S), (v / S) & 1, p.flags, kWaitNs);
+        return;
+    }
+
+    if (warp <= kMmaWarps) {
+        // --------------------------------------------------- contraction --
+        // A stage holds at most kStageSteps = 2 x kMmaWarps steps: warp mw owns
+        // steps s0 + mw and s0 + mw + kMmaWarps of every stage.
+        const int mw = warp - 1;
+        const int g8 = lane >> 2, t = lane & 3;
+        const uint8_t* act_base = smem + p.off_act;
+        int slot = 0;
+        uint32_t phase = 0;
+        for (int j = 0; j < n; ++j) {
+            const ChainLayer& L = p.layers[j];
+            const int first = first_tile(L, c, G), T = tiles_of(L, first, G);
+            const int steps = L.steps, nfull = L.nfull, bsteps = L.bsteps, nch = L.nch;
+            const int K = L.K, tail = L.tail;
+            const int b = j & 1;
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_act + 8 * b, (j >> 1) & 1, p.flags, p.wait_ns)))
+                return;
+            // B operand source of this lane's column (token limb row); lanes of the
+            // unused columns read row 0
+            const uint8_t* bsrc = act_base + b * COLS * p.astride + (g8 < COLS ? g8 : 0) * p.astride +
+                                  t * F::kChunkK;
+            int* pb = part + b * kMaxTiles * 16 * COLS;
+            for (int k = 0; k < T; ++k) {
+                int acc[CH][4];
+#pragma unroll
+                for (int cc = 0; cc < CH; ++cc) acc[cc][0] = acc[cc][1] = acc[cc][2] = acc[cc][3] = 0;
+                for (int ch = 0; ch < nch; ++ch) {
+                    const int s0 = ch * bsteps, s1 = min(s0 + bsteps, steps);
+                    // This warp's (at most) two steps.  No lane is masked: columns
+                    // >= COLS of the MMA are never read, so lanes of other columns
+                    // may load any activation bytes (row 0); and the activation rows
+                    // are zero past K to a whole step, so the weight bytes a partial
+                    // last step reads past its row end meet zeros.
+                    constexpr int BW_ = F::kRegs * 4;       // activation words per step and lane
+                    const bool has0 = s0 + mw < s1, has1 = s0 + mw + kMmaWarps < s1;
+                    uint32_t bw[2][BW_];
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const uint8_t* src = bsrc + (s0 + mw + kMmaWarps * i) * F::kStepK;
+                        if (i == 0 ? has0 : has1) {
+#pragma unroll
+                            for (int q = 0; q < BW_ / 4; ++q) {
+                                const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * q);
+                                bw[i][4 * q + 0] = v.x;
+                                bw[i][4 * q + 1] = v.y;
+                                bw[i][4 * q + 2] = v.z;
+                                bw[i][4 * q + 3] = v.w;
+                            }
+                        }
+                    }
+                    if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_full + 8 * slot, phase, p.flags, p.wait_ns)))
+                        return;
+                    const uint8_t* slot_p = smem + slot * kSlotBytes;
+                    uint4 a0[2], a1[2];
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const int s = s0 + mw + kMmaWarps * i;
+                        if (i == 0 ? has0 : has1) {
+                            if (s < nfull) {   // whole step: [step][row][64 B]
+                                const uint8_t* w0 = slot_p + (s - s0) * 1024 + 64 * g8 + 16 * t;
+                                a0[i] = *reinterpret_cast<const uint4*>(w0);
+                                a1[i] = *reinterpret_cast<const uint4*>(w0 + 512);
+                            } else {           // partial last step: tail box [row][tail B]
+                                const uint8_t* w0 = slot_p + bsteps * 1024 + tail * g8 + 16 * t;
+                                a0[i] = *reinterpret_cast<const uint4*>(w0);
+                                a1[i] = *reinterpret_cast<const uint4*>(w0 + 8 * tail);
+                            }
+                        }
+                    }
+                    // the stage's bytes are in registers: release the slot to the producer
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar_empty + 8 * slot);
+                    if (++slot == S) {
+                        slot = 0;
+                        phase ^= 1u;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        if (!(i == 0 ? has0 : has1)) continue;
+                        const uint32_t r0[4] = {a0[i].x, a0[i].y, a0[i].z, a0[i].w};
+                        const uint32_t r1[4] = {a1[i].x, a1[i].y, a1[i].z, a1[i].w};
+                        if constexpr (kMasked) {
+                            // field jj of every byte masked in place (code * 4^jj) against
+                            // activation word jj; the two words of a pair share jj, so chain
+                            // jj holds 4^jj times its sum
+#pragma unroll
+                            for (int op = 0; op < 4; op += 2)
+#pragma unroll
+                                for (int jj = 0; jj < 4; ++jj) {
+                                    const uint32_t m = 0x03030303u << (2 * jj);
+                                    mma_u8s8_16832(acc[jj], r0[op] & m, r1[op] & m, r0[op + 1] & m,
+                                                   r1[op + 1] & m, bw[i][4 * op + jj], bw[i][4 * op + 4 + jj]);
+                                }
+                        } else {
+#pragma unroll
+                            for (int om = 0; om < 4; ++om) {
+                                uint32_t u0r[F::kRegs], u1r[F::kRegs];
+#pragma unroll
+                                for (int jj = 0; jj < F::kRegs; ++jj) {
+                                    u0r[jj] = (r0[om] >> (F::kShift * jj)) & F::kMask;
+                                    u1r[jj] = (r1[om] >> (F::kShift * jj)) & F::kMask;
+                                }
+#pragma unroll
+                                for (int jj = 0; jj < F::kRegs; jj += 2)
+                                    mma_u8s8_16832(acc[om % CH], u0r[jj], u1r[jj], u0r[jj + 1],
+                                                   u1r[jj + 1], bw[i][om * F::kRegs + jj],
+                                                   bw[i][om * F::kRegs + jj + 1]);
+                            }
+                        }
+                    }
+                }
+                // tile done: fold the chains and add this warp's share into the tile's rows
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    int v = 0;
+#pragma unroll
+                    for (int cc = 0; cc < CH; ++cc) v += kMasked ? (acc[cc][e] >> (2 * cc)) : acc[cc][e];
+                    const int row = g8 + 8 * (e >> 1), col = 2 * t + (e & 1);
+                    if (col < COLS) atomicAdd(pb + (k * 16 + row) * COLS + col, v);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar_mma + 8 * b);
+        }
+        return;
+    }
+
+    // ---------------------------------------- activations and epilogue --
+    const int et = tid - kFirstPrepWarp * 32;     // 0 .. kPrepThreads-1
+    uint8_t* act_base = smem + p.off_act;
+    bool ok = true;
+    bool prev_prepared = false;   // layer next_prep-1's activations are in its buffer
+    int next_prep = 0, next_epi = 0;
+    while (next_epi < n && ok) {
+        const bool can_prep = next_prep < n && next_prep < next_epi + 2 &&
+                              p.layers[next_prep].src < next_epi;
+        if (can_prep) {
+            // ---- activations of layer j into buffer j % 2
+            const int j = next_prep++;
+            const ChainLayer& L = p.layers[j];
+            const int b = j & 1;
+            const int T = tiles_of(L, first_tile(L, c, G), G);
+            uint8_t* act = act_base + b * COLS * p.astride;
+            const bool prepare = T > 0;
+            if (prepare) {
+                if (L.reuse && prev_prepared) {
+                    // same input as layer j-1: copy its prepared activations
+                    const uint8_t* prev = act_base + (b ^ 1) * COLS * p.astride;
+                    for (int r = 0; r < COLS; ++r)
+                        for (int i = et; i < L.K / 16; i += kPrepThreads)
+                            *reinterpret_cast<uint4*>(act + r * p.astride + 16 * i) =
+                                *reinterpret_cast<const uint4*>(prev + r * p.astride + 16 * i);
+                    if (et == 0) {
+                        ts->scale[b] = ts->scale[b ^ 1];
+                        ts->qsum[b] = ts->qsum[b ^ 1];
+                        ts->xsum[b] = ts->xsum[b ^ 1];
+                    }
+                } else {
+                    const uint16_t* x = L.x;
+                    if (L.src >= 0) {
+                        // wait until every CTA has finished the producing layer
+                        bool got = true;
+                        if (et == 0) {
+                            const unsigned int* d = p.done + L.src;
+                            if (ld_acquire_u32(d) < (unsigned)G) {
+                                const uint64_t t0 = tc::globaltimer_ns();
+                                while (ld_acquire_u32(d) < (unsigned)G) {
+                                    if (tc::globaltimer_ns() - t0 > p.wait_ns) {
+                                        atomicOr(p.flags, kFlagTimeout);
+                                        got = false;
+                                        break;
+                                    }
+                                    __nanosleep(64);
+                                }
+                            }
+                        }
+                        if (!tc::bar_and(kBarPrep, kPrepThreads, got)) {
+                            ok = false;
+                            break;
+                        }
+                        x = p.layers[L.src].y;
+                    }
+                    prep_layer<FORM>(L, x, L.src >= 0, act, p.astride, ts, b, et);
+                }
+            }
+            if (prepare) {
+                // zeros from K to a whole step in every row (a partial last step's
+                // lanes past the row end multiply them)
+                const int kp = (L.K + F::kStepK - 1) / F::kStepK * F::kStepK;
+                for (int r = 0; r < COLS; ++r)
+                    for (int i = L.K + 16 * et; i < kp; i += 16 * kPrepThreads)
+                        *reinterpret_cast<uint4*>(act + r * p.astride + i) = make_uint4(0, 0, 0, 0);
+            }
+            prev_prepared = prepare;
+            bar_prep();   // activations and token scalars written (and the scratch reads done)
+            if (et == 0) tc::mbar_arrive(bar_act + 8 * b);
+        } else {
+            // ---- epilogue of layer j from buffer j % 2
+            const int j = next_epi++;
+            const ChainLayer& L = p.layers[j];
+            const int b = j & 1;
+            const int first = first_tile(L, c, G), T = tiles_of(L, first, G);
+            if (!tc::bar_and(kBarPrep, kPrepThreads,
+                             tc::mbar_wait(bar_mma + 8 * b, (j >> 1) & 1, p.flags, p.wait_ns))) {
+                ok = false;
+                break;
+            }
+            int* pb = part + b * kMaxTiles * 16 * COLS;
+            const float sc = ts->scale[b];
+            for (int o = et; o < T * 16; o += kPrepThreads) {
+                const int k = o >> 4, r = o & 15;
+                const int nrow = (first + k * G) * 16 + r;
+                if constexpr (FORM == 0) {
+                    const int a = pb[o] - ts->qsum[b];
+                    pb[o] = 0;
+                    L.y[nrow] = __half_as_ushort(__float2half_rn(__fmul_rn(__fmul_rn((float)a, sc), L.w_scale)));
+                    if (L.acc_out) L.acc_out[nrow] = a;
+                } else {
+                    const long long Z = limb_combine(pb[3 * o], pb[3 * o + 1], pb[3 * o + 2], ts->xsum[b]);
+                    pb[3 * o] = pb[3 * o + 1] = pb[3 * o + 2] = 0;
+                    const float z = __fmul_rn(sc, (float)Z);
+                    const float hv = __half2float(__ushort_as_half(L.h[nrow]));
+                    L.y[nrow] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hv)));
+                }
+            }
+            bar_prep();   // every output of this CTA written, partials cleared
+            if (L.has_dep && et == 0) {
+                __threadfence();
+                atomicAdd(p.done + j, 1u);
+            }
+        }
+    }
+}
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Shared-memory layout of a launch: ring [S][kSlotBytes] | activations
+// [2][COLS][astride] | partial sums [2][kMaxTiles*16][COLS] int32 | token
+// scalars | barriers.
+struct ChainSmem {
+    int S, astride, off_act, off_part, off_tok, off_bar, total;
+};
+
+bool chain_smem(int form, int kmax, ChainSmem& m) {
+    const int cols = form == 0 ? 1 : 3;
+    // rows padded to a whole step (256 / 512 k), +16 bytes between rows
+    m.astride = (kmax + 511) / 512 * 512 + 16;
+    const int act = 2 * cols * m.astride;
+    const int partb = 2 * kMaxTiles * 16 * cols * 4;
+    const int tok = (int)round_up(sizeof(TokStats), 16);
+    for (int S = kMaxSlots; S >= 3; --S) {
+        int off = S * kSlotBytes;
+        m.off_act = off;
+        off += (int)round_up((size_t)act, 16);
+        m.off_part = off;
+        off += partb;
+        m.off_tok = off;
+        off += tok;
+        m.off_bar = off;
+        off += 8 * (2 * S + 4);
+        if (off <= kDecodeMaxSmem) {
+            m.S = S;
+            m.total = off;
+            return true;
+        }
+    }
+    return false;
+}
+
+template <int FORM>
+cudaError_t launch_chain(const ChainParams& p, int smem, cudaStream_t s) {
+    static KernelAttrs kattrs;
+    if (cudaError_t e = kattrs.ensure(chain_kernel<FORM>, kDecodeMaxSmem)) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(device_sm_count());
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    // every CTA must be resident at once: layers wait on other CTAs' results
+    cudaLaunchAttribute attrs[1];
+    attrs[0].id = cudaLaunchAttributeCooperative;
+    attrs[0].val.cooperative = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, chain_kernel<FORM>, p);
+}
+
+}  // namespace
+
+size_t chain_bytes(int n_layers) {
+    return round_up((size_t)n_layers * sizeof(ChainLayer), 256) + round_up((size_t)n_layers * 4, 256);
+}
+
+int chain_max_k(int form) { return form == 0 ? 32768 : 16384; }
+
+bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain, size_t bytes,
+                      bl_chain_plan* plan, cudaStream_t s) {
+    const int G = device_sm_count();
+    if (G <= 0) return BL_ERR_CUDA;
+    std::vector<ChainLayer> host((size_t)n);
+    int kmax = 0;
+    long long tiles_before = 0;
+    for (int j = 0; j < n; ++j) {
+        const bl_chain_layer& in = layers[j];
+        ChainLayer& L = host[(size_t)j];
+        std::memset(&L, 0, sizeof(L));
+        L.K = in.K;
+        L.N = in.N;
+        L.src = in.src;
+        L.x = in.x;
+        L.w = in.w;
+        L.y = in.y;
+        L.acc_out = in.acc_out;
+        L.g = in.g;
+        L.h = in.h;
+        L.w_scale = in.w_scale;
+        L.ntile = in.N / 16;
+        L.rot = (int)(tiles_before % G);
+        tiles_before += L.ntile;
+        if (in.src >= 0) host[(size_t)in.src].has_dep = 1;
+        if (j > 0 && in.K == layers[j - 1].K && in.src == layers[j - 1].src &&
+            (in.src >= 0 || in.x == layers[j - 1].x) && (form == 0 || in.g == layers[j - 1].g))
+            L.reuse = 1;
+        // k-steps of 64 packed bytes per row; stages of at most 16 steps, a
+        // multiple of 16 when a row takes several (a warp owns the same steps
+        // in every stage)
+        const int wbytes = form == 0 ? in.K / 4 : in.K / 8;   // packed bytes per row
+        L.nfull = wbytes / 64;
+        L.tail = wbytes % 64;
+        L.ragged = L.tail != 0;
+        L.steps = L.nfull + L.ragged;
+        L.nch = (L.steps + kStageSteps - 1) / kStageSteps;
+        L.bsteps = L.nch > 1 ? kStageSteps : L.steps;
+        if (L.nfull > 0) {
+            const cuuint64_t dims[3] = {64, (cuuint64_t)in.N, (cuuint64_t)L.nfull};
+            const cuuint64_t strides[2] = {(cuuint64_t)wbytes, 64};
+            const cuuint32_t box[3] = {64, 16, (cuuint32_t)L.bsteps};
+            if (!encode_u8_map(&L.tm_main, in.w, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+                return BL_ERR_CUDA;
+        }
+        if (L.ragged) {
+            const cuuint64_t dims[2] = {(cuuint64_t)L.tail, (cuuint64_t)in.N};
+            const cuuint64_t strides[1] = {(cuuint64_t)wbytes};
+            const cuuint32_t box[2] = {(cuuint32_t)L.tail, 16};
+            const uint8_t* tailp = reinterpret_cast<const uint8_t*>(in.w) + 64 * (size_t)L.nfull;
+            if (!encode_u8_map(&L.tm_tail, tailp, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+                return BL_ERR_CUDA;
+        }
+        if (in.K > kmax) kmax = in.K;
+        if (L.ntile > kMaxTiles * G) return BL_ERR_SHAPE;
+    }
+    ChainSmem m;
+    if (!chain_smem(form, kmax, m)) return BL_ERR_SHAPE;
+    if (bytes < chain_bytes(n)) return BL_ERR_WORKSPACE;
+    if (cudaMemcpyAsync(chain, host.data(), (size_t)n * sizeof(ChainLayer), cudaMemcpyHostToDevice,
+                        s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return BL_ERR_CUDA;
+    plan->form = form;
+    plan->n_layers = n;
+    plan->sm_count = G;
+    plan->kmax = kmax;
+    plan->slots = m.S;
+    plan->smem_bytes = m.total;
+    return BL_OK;
+}
+
+bl_status chain_run(const bl_chain_plan* plan, const void* chain, unsigned int* flags,
+                    cudaStream_t s) {
+    ChainSmem m;
+    if (!chain_smem(plan->form, plan->kmax, m) || m.S != plan->slots || m.total != plan->smem_bytes)
+        return BL_ERR_SHAPE;
+    if (device_sm_count() != plan->sm_count) return BL_ERR_SHAPE;
+    const int n = plan->n_layers;
+    ChainParams p;
+    p.layers = static_cast<const ChainLayer*>(chain);
+    p.n = n;
+    p.done = reinterpret_cast<unsigned int*>(static_cast<char*>(const_cast<void*>(chain)) +
+                                             round_up((size_t)n * sizeof(ChainLayer), 256));
+    p.flags = flags;
+    p.S = m.S;
+    p.astride = m.astride;
+    p.off_act = m.off_act;
+    p.off_part = m.off_part;
+    p.off_tok = m.off_tok;
+    p.off_bar = m.off_bar;
+    p.wait_ns = kWaitNs;
+    // the completion counters start at zero on every run
+    if (cudaMemsetAsync(p.done, 0, (size_t)n * 4, s) != cudaSuccess) return BL_ERR_CUDA;
+    const cudaError_t e = plan->form == 0 ? launch_chain<0>(p, m.total, s) : launch_chain<1>(p, m.total, s);
+    return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+}  // namespace bl

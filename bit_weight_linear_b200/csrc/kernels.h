@@ -113,6 +113,16 @@ cudaError_t launch_onebit_stream_prepared(const int8_t* planes, const float* ste
                                           const uint32_t* s1, int M, int K, int N, uint16_t* y,
                                           unsigned int* flags, cudaStream_t s);
 
+// Persistent single-token decode over a list of layers (chain.cu): device
+// descriptors (tensor maps, tile plan) written by chain_build into the caller's
+// `chain` buffer of chain_bytes(n) bytes, one cooperative launch per run.
+size_t chain_bytes(int n_layers);
+int chain_max_k(int form);
+bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain, size_t bytes,
+                      bl_chain_plan* plan, cudaStream_t s);
+bl_status chain_run(const bl_chain_plan* plan, const void* chain, unsigned int* flags,
+                    cudaStream_t s);
+
 // Every kernel of the library runs with the whole L1/shared-memory carveout
 // given to shared memory.  An SM changes its carveout only when it is idle, so
 // kernels with differing carveouts could not share an SM: the next call's CTAs

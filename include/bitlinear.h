@@ -204,6 +204,72 @@ bl_status bl_ternary_linear_noalloc(const uint16_t *x, int M, int K, int N, cons
                                     bl_stream_t stream);
 
 /*
+ * Decode chains: the single-token (M = 1) forward of a whole list of layers
+ * in ONE persistent launch -- the decode step of a stack of BitLinear or
+ * OneBit layers (BitNet b1.58 page, "内存和延迟": at decode sizes the model's
+ * time goes to its linear layers).  Per layer the arithmetic is exactly that
+ * of bl_ternary_linear / ob_linear at M = 1 (same outputs, bit for bit).
+ *
+ * A layer's input is either given (x) or the output y of an EARLIER layer of
+ * the list (src): the kernel then waits, inside the launch, until every part
+ * of that layer's y is written.  Layers whose inputs do not depend on each
+ * other overlap; the weights of later layers stream while earlier ones finish.
+ *
+ * Usage: describe the layers, call bl_chain_build once (it writes the device
+ * descriptors, including TMA tensor maps, into the caller's `chain` buffer and
+ * fills `plan`), then bl_chain_run as often as needed (graph-capturable: one
+ * 4*n-byte memset node and one kernel node).  Weights, g, h and the pointers
+ * are baked into the chain: rebuild it if any of them changes; the CONTENTS of
+ * given inputs x may change between runs.  Runs of the same chain must not
+ * overlap on the GPU (they share its counters).
+ */
+typedef struct {
+    const uint16_t *x;     /* fp16 [K] input, or NULL when src >= 0 */
+    int src;               /* -1: x is given; else the index (< this layer's) of
+                              the layer whose output y is this layer's input
+                              (its N must equal this layer's K) */
+    int K, N;              /* K % 128 == 0, K <= 32768 (ternary) / 16384
+                              (OneBit); N % 16 == 0 */
+    const uint32_t *w;     /* packed weights: w2 [N, K/16] or s1 [N, K/32] */
+    float w_scale;         /* ternary per-tensor weight scale */
+    const uint16_t *g;     /* OneBit input value vector fp16 [K] (else NULL) */
+    const uint16_t *h;     /* OneBit output value vector fp16 [N] (else NULL) */
+    uint16_t *y;           /* fp16 [N] output */
+    int32_t *acc_out;      /* optional int32 [N] accumulators (ternary), or NULL */
+} bl_chain_layer;
+
+typedef struct {           /* filled by bl_chain_build; pass unchanged to bl_chain_run */
+    int form;              /* 0 = BitLinear (ternary), 1 = OneBit */
+    int n_layers;
+    int sm_count;          /* the device's SM count the plan was made for */
+    int kmax;              /* largest K of the chain */
+    int slots;             /* weight-ring slots per CTA */
+    int smem_bytes;        /* shared memory per CTA */
+} bl_chain_plan;
+
+/* Device bytes of the chain buffer for n_layers layers (0 if out of range). */
+size_t bl_chain_bytes(int n_layers);
+
+/*
+ * bl_chain_build -- validate the layers and write the chain into `chain`
+ * (caller-owned device memory, 256-byte aligned, >= bl_chain_bytes(n_layers)).
+ * Synchronises `stream` (a host-to-device copy of the descriptors).  Errors:
+ * BL_ERR_NULL / BL_ERR_ALIGN for pointers (16-byte alignment as everywhere),
+ * BL_ERR_SHAPE for a shape or src outside the rules above or a layer too wide
+ * for one launch (N/16 tiles > 16 per SM), BL_ERR_WORKSPACE if the buffer is
+ * too small.  Make the device that will run the chain current.
+ */
+bl_status bl_chain_build(int form, const bl_chain_layer *layers, int n_layers, void *chain,
+                         size_t chain_bytes, bl_chain_plan *plan, bl_stream_t stream);
+
+/*
+ * bl_chain_run -- one decode step over the chain, asynchronous on `stream`:
+ * zeroes the chain's completion counters, then one cooperative launch of one
+ * CTA per SM.  BL_ERR_SHAPE if `plan` does not match the current device.
+ */
+bl_status bl_chain_run(const bl_chain_plan *plan, const void *chain, bl_stream_t stream);
+
+/*
  * bl_prefill_plan -- diagnostic: how the tensor-core (prefill) path would run
  * a call of this shape on a device with `sm_count` SMs (form 0 = ternary,
  * 1 = OneBit, whose tiles hold two limb rows per token).  Fills plan[5]:

@@ -124,3 +124,34 @@ def test_fault_injection_hook(L, monkeypatch, mode, code):
     # with no GPU the call now fails in the CUDA runtime, not in the hook
     if not __import__("torch").cuda.is_available():
         assert L.bl_ternary_linear(A, 1, 128, 16, A, 1.0, A, None, A, 1 << 20, None) == 5
+
+
+def test_chain_build_rejects_bad_layers(L):
+    """bl_chain_build validates every layer before any CUDA call."""
+    import bit_weight_linear_b200 as blw
+    n = 2
+    arr = (blw.ChainLayer * n)()
+    for j in range(n):
+        arr[j].x, arr[j].src, arr[j].K, arr[j].N = 0x10000, -1, 128, 16
+        arr[j].w, arr[j].y = 0x10000, 0x10000
+    plan = blw.ChainPlan()
+    buf = ctypes.c_void_p(0x100000)
+    nb = L.bl_chain_bytes(n)
+    assert nb > 0 and L.bl_chain_bytes(0) == 0
+    assert L.bl_chain_build(0, None, n, buf, nb, ctypes.byref(plan), None) == 1
+    assert L.bl_chain_build(2, arr, n, buf, nb, ctypes.byref(plan), None) == 2       # bad form
+    assert L.bl_chain_build(0, arr, n, ctypes.c_void_p(0x100010), nb, ctypes.byref(plan), None) == 3
+    arr[1].src = 1                                  # not an earlier layer
+    assert L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None) == 2
+    arr[1].src, arr[1].K = 0, 256                   # K must equal the source's N
+    assert L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None) == 2
+    arr[1].K, arr[1].N, arr[1].src = 128, 16, -1
+    arr[0].K = 100                                  # K % 128
+    assert L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None) == 2
+    arr[0].K, arr[0].x = 128, None                  # a given input needs x
+    assert L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None) == 1
+    arr[0].x = 0x10004                              # misaligned
+    assert L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None) == 3
+    arr[0].x = 0x10000
+    assert L.bl_chain_build(1, arr, n, buf, nb, ctypes.byref(plan), None) == 1       # OneBit needs g, h
+    assert L.bl_chain_build(0, arr, n, buf, nb - 1, ctypes.byref(plan), None) == 7
