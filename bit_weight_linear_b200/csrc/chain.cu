@@ -24,8 +24,8 @@
 //   warps 1-8   contraction: u8 x s8 warp MMA (m16n8k32) over the steps of
 //               each stage they own, per-tile partial sums added into shared
 //               memory with integer atomics (exact in any order);
-//   warps 9-12  activations and epilogue: for layer j+1 (while warps 1-8
-//               contract layer j; two buffers) the per-token absmax and the
+//   warps 9-15  activations and epilogue: for layers j+1.. (while warps 1-8
+//               contract layer j; up to four buffers) the per-token absmax and the
 //               quantisation into the permuted int8 tile; for layer j the
 //               fp16 outputs, and, when a later layer reads them, one arrival
 //               per CTA on the layer's completion counter (release fence).
@@ -54,9 +54,11 @@ namespace bl {
 namespace {
 
 constexpr int kMmaWarps = 8;
-constexpr int kPrepWarps = 4;
+// 16 warps: four per SM sub-partition, whose register file then allows 128
+// registers per thread (a 17th warp would put five on one and cap them at 96)
+constexpr int kPrepWarps = 7;
 constexpr int kPrepThreads = kPrepWarps * 32;
-constexpr int kThreads = (1 + kMmaWarps + kPrepWarps) * 32;   // 416
+constexpr int kThreads = (1 + kMmaWarps + kPrepWarps) * 32;   // 512
 constexpr int kFirstPrepWarp = 1 + kMmaWarps;
 constexpr int kMaxTiles = 16;              // tiles of one layer per CTA
 constexpr int kMaxSlots = 12;
@@ -66,6 +68,7 @@ constexpr int kStageSteps = 16;            // 64-byte steps of a row per stage: 
 constexpr int kSlotBytes = 16 * kStageSteps * 64 + 1024;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kBarPrep = 1;                // named barrier of the activation/epilogue warps
+constexpr int kMaxBufs = 4;                // activation buffers: layers prepared ahead
 
 // One layer of a chain in device memory (written by bl_chain_build, read-only
 // in the kernel).  384 bytes, 64-byte aligned: the tensor maps come first.
@@ -88,23 +91,42 @@ struct alignas(64) ChainLayer {
 };
 static_assert(sizeof(ChainLayer) == 384, "chain layer descriptor size");
 
+// The per-layer fields every warp role reads, 32 bytes per layer: written by
+// the host next to the descriptors and copied into shared memory at launch.
+// A descriptor field read from global memory costs an L2 round trip per layer
+// and warp -- for the producer thread, a stall of every stage it issues.
+struct alignas(16) LayerInfo {
+    uint16_t ntile, rot;    // 16-row tiles; rotation of their deal over the CTAs
+    uint16_t k16;           // K / 16
+    int16_t src;            // -1: x given; else the producing layer
+    uint8_t steps, nfull, tail, bsteps, nch;
+    uint8_t flags;          // kInfoRagged | kInfoHasDep | kInfoReuse
+    uint16_t pad;
+    const uint16_t* x;      // given input (src < 0)
+    uint16_t* y;            // output
+};
+static_assert(sizeof(LayerInfo) == 32, "layer info size");
+constexpr uint8_t kInfoRagged = 1, kInfoHasDep = 2, kInfoReuse = 4;
+
 struct ChainParams {
     const ChainLayer* layers;
+    const LayerInfo* info;  // [n] in global memory
     int n;
     unsigned int* done;    // [n] arrivals of CTAs that finished a layer's epilogue
     unsigned int* flags;   // device condition word
     int S;                 // ring slots
+    int nbuf;              // activation buffers (2..kMaxBufs): layer j uses buffer j % nbuf
     int astride;           // bytes between activation rows (Kmax + 16)
-    int off_act, off_part, off_tok, off_bar;
+    int off_act, off_part, off_tok, off_bar, off_tab;
     uint64_t wait_ns;
 };
 
 // Tiles of layer L taken by CTA c of G: first, first + G, ... < ntile.
-__device__ __forceinline__ int first_tile(const ChainLayer& L, int c, int G) {
-    const int r = (c - L.rot) % G;
+__device__ __forceinline__ int first_tile(const LayerInfo& L, int c, int G) {
+    const int r = (c - (int)L.rot) % G;
     return r < 0 ? r + G : r;
 }
-__device__ __forceinline__ int tiles_of(const ChainLayer& L, int first, int G) {
+__device__ __forceinline__ int tiles_of(const LayerInfo& L, int first, int G) {
     return first < L.ntile ? (L.ntile - 1 - first) / G + 1 : 0;
 }
 
@@ -130,16 +152,17 @@ __device__ __forceinline__ void bar_prep() {
 
 // Per-layer shared state of the activation/epilogue warps.
 struct TokStats {
-    float scale[2];        // ternary amax/127, OneBit amax'/kImgMax; per buffer
-    int qsum[2];           // ternary sum q
-    long long xsum[2];     // OneBit sum X
+    float scale[kMaxBufs];       // ternary amax/127, OneBit amax'/kImgMax; per buffer
+    int qsum[kMaxBufs];          // ternary sum q
+    long long xsum[kMaxBufs];    // OneBit sum X
     uint32_t red[3][kPrepWarps];
     int redi[3][kPrepWarps];
 };
 
-// Rows up to this many elements are prepared from registers in one read.
-constexpr int kRegK = 16384;
-constexpr int kRegChunks = kRegK / 8 / kPrepThreads;   // 16-byte chunks of x per thread
+// 16-byte chunks of x per thread held in registers: rows up to kRegChunks x 8 x
+// kPrepThreads elements (ternary; OneBit: whole 32-element groups, a quarter
+// as many) are prepared from registers in one read.
+constexpr int kRegChunks = 10;
 
 // Activations of layer L into buffer act ([cols][astride] bytes) for a single
 // token.  K <= kRegK: x is read once into registers (every load in flight at
@@ -148,12 +171,12 @@ constexpr int kRegChunks = kRegK / 8 / kPrepThreads;   // 16-byte chunks of x pe
 // over x (the second from L1 or L2).  `cg`: x is another CTA's output, read
 // through L2.
 template <int FORM>
-__device__ void prep_layer(const ChainLayer& L, const uint16_t* x, bool cg, uint8_t* act,
+__device__ void prep_layer(int K, const uint16_t* x, const uint16_t* gvec, bool cg, uint8_t* act,
                            int astride, TokStats* ts, int b, int et) {
-    const int K = L.K;
     const int pw = et >> 5, lane = et & 31;
     auto ld = [&](const uint16_t* p) { return cg ? ld_cg_v4(p) : tc::ld_v4(p); };
-    const bool in_regs = K <= kRegK;
+    const bool in_regs = FORM == 0 ? K <= 8 * kRegChunks * kPrepThreads
+                                   : K <= 32 * (kRegChunks / 4) * kPrepThreads;
     uint4 xr[kRegChunks];
     float amax;
     if constexpr (FORM == 0) {
@@ -231,11 +254,11 @@ __device__ void prep_layer(const ChainLayer& L, const uint16_t* x, bool cg, uint
                 const int e = 32 * (et + c * kPrepThreads);
 #pragma unroll
                 for (int v = 0; v < 4; ++v)
-                    mx = fmaxf(mx, absmax_prod(xr[4 * c + v], ld_ro_v4(L.g + e + 8 * v)));
+                    mx = fmaxf(mx, absmax_prod(xr[4 * c + v], ld_ro_v4(gvec + e + 8 * v)));
             }
         } else {
             for (int c = et; c < K / 8; c += kPrepThreads)
-                mx = fmaxf(mx, absmax_prod(ld(x + 8 * c), ld_ro_v4(L.g + 8 * c)));
+                mx = fmaxf(mx, absmax_prod(ld(x + 8 * c), ld_ro_v4(gvec + 8 * c)));
         }
         const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
         if (lane == 0) ts->red[0][pw] = mb;
@@ -249,7 +272,7 @@ __device__ void prep_layer(const ChainLayer& L, const uint16_t* x, bool cg, uint
         auto group = [&](const uint4 (&xa)[4], int gi) {
             uint4 ga[4];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) ga[v] = ld_ro_v4(L.g + 32 * gi + 8 * v);
+            for (int v = 0; v < 4; ++v) ga[v] = ld_ro_v4(gvec + 32 * gi + 8 * v);
             int gs[3];
             quant_group_s(xa, ga, inv, act + 32 * gi, astride, gs);
             ls[0] += gs[0];
@@ -298,62 +321,91 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, G = gridDim.x, S = p.S, n = p.n;
     const uint32_t sb = tc::smem_u32(smem);
-    int* part = reinterpret_cast<int*>(smem + p.off_part);          // [2][kMaxTiles*16][COLS]
+    const int NB = p.nbuf;
+    int* part = reinterpret_cast<int*>(smem + p.off_part);          // [NB][kMaxTiles*16][COLS]
     TokStats* ts = reinterpret_cast<TokStats*>(smem + p.off_tok);
     const uint32_t bar_full = sb + p.off_bar;                         // [S] stage landed
     const uint32_t bar_empty = bar_full + 8 * S;                      // [S] 8 warps done with it
-    const uint32_t bar_act = bar_empty + 8 * S;                       // [2] activations ready
-    const uint32_t bar_mma = bar_act + 16;                            // [2] layer contracted
-    constexpr int kPartInts = 2 * kMaxTiles * 16 * COLS;
+    const uint32_t bar_act = bar_empty + 8 * S;                       // [NB] activations ready
+    const uint32_t bar_mma = bar_act + 8 * kMaxBufs;                  // [NB] layer contracted
+    const int kPartInts = NB * kMaxTiles * 16 * COLS;
 
     if (tid == 0) {
         for (int i = 0; i < S; ++i) {
             tc::mbar_init(bar_full + 8 * i, 1);
             tc::mbar_init(bar_empty + 8 * i, kMmaWarps);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NB; ++i) {
             tc::mbar_init(bar_act + 8 * i, 1);
             tc::mbar_init(bar_mma + 8 * i, kMmaWarps);
         }
         tc::mbar_fence_init();
     }
     for (int i = tid; i < kPartInts; i += kThreads) part[i] = 0;
+    LayerInfo* tab = reinterpret_cast<LayerInfo*>(smem + p.off_tab);
+    for (int i = tid; i < 2 * n; i += kThreads)
+        reinterpret_cast<uint4*>(tab)[i] = reinterpret_cast<const uint4*>(p.info)[i];
     __syncthreads();
 
     if (warp == 0) {
         // ------------------------------------------------------ producer --
         if (lane != 0) return;
-        int u = 0;
+        // Stages of this CTA in order: (layer j, tile k, chunk ch).  (A second
+        // cursor that brought the stages 16 ahead of the ring into L2 with TMA
+        // prefetches measured slower: 0.57 -> 0.64 ms on the 7B-shaped stack.)
+        struct Cursor {
+            int j, k, ch, first, T;
+        };
+        auto enter = [&](Cursor& q) {   // first stage at or after layer q.j
+            for (; q.j < n; ++q.j) {
+                q.first = first_tile(tab[q.j], c, G);
+                q.T = tiles_of(tab[q.j], q.first, G);
+                if (q.T > 0) break;
+            }
+            q.k = q.ch = 0;
+        };
+        auto next = [&](Cursor& q) {
+            if (++q.ch < tab[q.j].nch) return;
+            q.ch = 0;
+            if (++q.k < q.T) return;
+            ++q.j;
+            enter(q);
+        };
+        Cursor ld{0, 0, 0, 0, 0};
+        enter(ld);
+        int u = 0, jprev = -1;
         bool ok = true;
-        for (int j = 0; j < n && ok; ++j) {
-            const ChainLayer& L = p.layers[j];
-            if (j + 1 < n) {
-                tc::prefetch_tmap(&p.layers[j + 1].tm_main);
-                if (p.layers[j + 1].ragged) tc::prefetch_tmap(&p.layers[j + 1].tm_tail);
-            }
-            // a given input two layers ahead: into L2 before its activations are prepared
-            if (j + 2 < n && p.layers[j + 2].src < 0 && !p.layers[j + 2].reuse)
-                tc::bulk_prefetch_l2(p.layers[j + 2].x, (uint32_t)(2 * p.layers[j + 2].K));
-            const int first = first_tile(L, c, G), T = tiles_of(L, first, G);
-            const int steps = L.steps, nfull = L.nfull, bsteps = L.bsteps, nch = L.nch;
-            const bool ragged = L.ragged != 0;
-            for (int k = 0; k < T && ok; ++k) {
-                const int row0 = (first + k * G) * 16;
-                for (int ch = 0; ch < nch; ++ch, ++u) {
-                    const int slot = u % S;
-                    if (u >= S) {
-                        ok = tc::mbar_wait(bar_empty + 8 * slot, ((u / S) - 1) & 1, p.flags, p.wait_ns);
-                        if (!ok) break;
-                    }
-                    const int s0 = ch * bsteps, s1 = min(s0 + bsteps, steps);
-                    uint32_t bytes = s0 < nfull ? (uint32_t)bsteps * 1024u : 0u;
-                    if (ragged && s1 == steps) bytes += 16u * (uint32_t)L.tail;
-                    const uint32_t dst = sb + slot * kSlotBytes, bar = bar_full + 8 * slot;
-                    tc::mbar_arrive_expect_tx(bar, bytes);
-                    if (s0 < nfull) tc::tma_load_3d(dst, &L.tm_main, 0, row0, s0, bar);
-                    if (ragged && s1 == steps) tc::tma_load_2d(dst + bsteps * 1024, &L.tm_tail, 0, row0, bar);
+        while (ld.j < n) {
+            const int j = ld.j;
+            const LayerInfo& L = tab[j];
+            if (j != jprev) {
+                jprev = j;
+                if (j + 1 < n) {
+                    tc::prefetch_tmap(&p.layers[j + 1].tm_main);
+                    if (tab[j + 1].flags & kInfoRagged) tc::prefetch_tmap(&p.layers[j + 1].tm_tail);
                 }
+                // a given input two layers ahead: into L2 before its activations are prepared
+                if (j + 2 < n && tab[j + 2].src < 0 && !(tab[j + 2].flags & kInfoReuse))
+                    tc::bulk_prefetch_l2(tab[j + 2].x, (uint32_t)(32 * tab[j + 2].k16));
             }
+            const int slot = u % S;
+            if (u >= S) {
+                ok = tc::mbar_wait(bar_empty + 8 * slot, ((u / S) - 1) & 1, p.flags, p.wait_ns);
+                if (!ok) break;
+            }
+            const int steps = L.steps, nfull = L.nfull, bsteps = L.bsteps;
+            const bool ragged = (L.flags & kInfoRagged) != 0;
+            const int row0 = (ld.first + ld.k * G) * 16;
+            const int s0 = ld.ch * bsteps, s1 = min(s0 + bsteps, steps);
+            uint32_t bytes = s0 < nfull ? (uint32_t)bsteps * 1024u : 0u;
+            if (ragged && s1 == steps) bytes += 16u * (uint32_t)L.tail;
+            const uint32_t dst = sb + slot * kSlotBytes, bar = bar_full + 8 * slot;
+            tc::mbar_arrive_expect_tx(bar, bytes);
+            if (s0 < nfull) tc::tma_load_3d(dst, &p.layers[j].tm_main, 0, row0, s0, bar);
+            if (ragged && s1 == steps)
+                tc::tma_load_2d(dst + bsteps * 1024, &p.layers[j].tm_tail, 0, row0, bar);
+            ++u;
+            next(ld);
         }
         // Every copy requested lands before the CTA can exit (on the normal
         // path the contraction has consumed them and these waits return at once).
@@ -371,47 +423,54 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
         const uint8_t* act_base = smem + p.off_act;
         int slot = 0;
         uint32_t phase = 0;
+        int b = 0;            // activation buffer of layer j (= j % NB), its phase bphase
+        uint32_t bphase = 0;
         for (int j = 0; j < n; ++j) {
-            const ChainLayer& L = p.layers[j];
+            const LayerInfo L = tab[j];
             const int first = first_tile(L, c, G), T = tiles_of(L, first, G);
             const int steps = L.steps, nfull = L.nfull, bsteps = L.bsteps, nch = L.nch;
-            const int K = L.K, tail = L.tail;
-            const int b = j & 1;
-            if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_act + 8 * b, (j >> 1) & 1, p.flags, p.wait_ns)))
+            const int tail = L.tail;
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_act + 8 * b, bphase, p.flags, p.wait_ns)))
                 return;
             // B operand source of this lane's column (token limb row); lanes of the
             // unused columns read row 0
             const uint8_t* bsrc = act_base + b * COLS * p.astride + (g8 < COLS ? g8 : 0) * p.astride +
                                   t * F::kChunkK;
             int* pb = part + b * kMaxTiles * 16 * COLS;
+            // This warp's (at most) two steps of a stage.  No lane is masked:
+            // columns >= COLS of the MMA are never read, so lanes of other columns
+            // may load any activation bytes (row 0); and the activation rows are
+            // zero past K to a whole step, so the weight bytes a partial last step
+            // reads past its row end meet zeros.  A layer of one stage per tile
+            // uses the same activation words for every tile: they are loaded once.
+            constexpr int BW_ = F::kRegs * 4;       // activation words per step and lane
+            uint32_t bw[2][BW_];
+            auto load_b = [&](int s0, int s1) {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int s = s0 + mw + kMmaWarps * i;
+                    if (s < s1) {
+                        const uint8_t* src = bsrc + s * F::kStepK;
+#pragma unroll
+                        for (int q = 0; q < BW_ / 4; ++q) {
+                            const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * q);
+                            bw[i][4 * q + 0] = v.x;
+                            bw[i][4 * q + 1] = v.y;
+                            bw[i][4 * q + 2] = v.z;
+                            bw[i][4 * q + 3] = v.w;
+                        }
+                    }
+                }
+            };
+            if (nch == 1 && T > 0) load_b(0, steps);
             for (int k = 0; k < T; ++k) {
                 int acc[CH][4];
 #pragma unroll
                 for (int cc = 0; cc < CH; ++cc) acc[cc][0] = acc[cc][1] = acc[cc][2] = acc[cc][3] = 0;
                 for (int ch = 0; ch < nch; ++ch) {
                     const int s0 = ch * bsteps, s1 = min(s0 + bsteps, steps);
-                    // This warp's (at most) two steps.  No lane is masked: columns
-                    // >= COLS of the MMA are never read, so lanes of other columns
-                    // may load any activation bytes (row 0); and the activation rows
-                    // are zero past K to a whole step, so the weight bytes a partial
-                    // last step reads past its row end meet zeros.
-                    constexpr int BW_ = F::kRegs * 4;       // activation words per step and lane
                     const bool has0 = s0 + mw < s1, has1 = s0 + mw + kMmaWarps < s1;
-                    uint32_t bw[2][BW_];
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const uint8_t* src = bsrc + (s0 + mw + kMmaWarps * i) * F::kStepK;
-                        if (i == 0 ? has0 : has1) {
-#pragma unroll
-                            for (int q = 0; q < BW_ / 4; ++q) {
-                                const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * q);
-                                bw[i][4 * q + 0] = v.x;
-                                bw[i][4 * q + 1] = v.y;
-                                bw[i][4 * q + 2] = v.z;
-                                bw[i][4 * q + 3] = v.w;
-                            }
-                        }
-                    }
+                    if (nch > 1) load_b(s0, s1);
                     if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_full + 8 * slot, phase, p.flags, p.wait_ns)))
                         return;
                     const uint8_t* slot_p = smem + slot * kSlotBytes;
@@ -485,6 +544,10 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
             }
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar_mma + 8 * b);
+            if (++b == NB) {
+                b = 0;
+                bphase ^= 1u;
+            }
         }
         return;
     }
@@ -496,31 +559,33 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
     bool prev_prepared = false;   // layer next_prep-1's activations are in its buffer
     int next_prep = 0, next_epi = 0;
     while (next_epi < n && ok) {
-        const bool can_prep = next_prep < n && next_prep < next_epi + 2 &&
-                              p.layers[next_prep].src < next_epi;
+        const bool can_prep = next_prep < n && next_prep < next_epi + NB && tab[next_prep].src < next_epi;
         if (can_prep) {
-            // ---- activations of layer j into buffer j % 2
+            // ---- activations of layer j into buffer j % NB
             const int j = next_prep++;
-            const ChainLayer& L = p.layers[j];
-            const int b = j & 1;
+            const LayerInfo L = tab[j];
+            const int K = 16 * L.k16;
+            const int b = j % NB, bprev = (j + NB - 1) % NB;
             const int T = tiles_of(L, first_tile(L, c, G), G);
             uint8_t* act = act_base + b * COLS * p.astride;
             const bool prepare = T > 0;
             if (prepare) {
-                if (L.reuse && prev_prepared) {
+                if ((L.flags & kInfoReuse) && prev_prepared) {
                     // same input as layer j-1: copy its prepared activations
-                    const uint8_t* prev = act_base + (b ^ 1) * COLS * p.astride;
+                    const uint8_t* prev = act_base + bprev * COLS * p.astride;
                     for (int r = 0; r < COLS; ++r)
-                        for (int i = et; i < L.K / 16; i += kPrepThreads)
+                        for (int i = et; i < K / 16; i += kPrepThreads)
                             *reinterpret_cast<uint4*>(act + r * p.astride + 16 * i) =
                                 *reinterpret_cast<const uint4*>(prev + r * p.astride + 16 * i);
                     if (et == 0) {
-                        ts->scale[b] = ts->scale[b ^ 1];
-                        ts->qsum[b] = ts->qsum[b ^ 1];
-                        ts->xsum[b] = ts->xsum[b ^ 1];
+                        ts->scale[b] = ts->scale[bprev];
+                        ts->qsum[b] = ts->qsum[bprev];
+                        ts->xsum[b] = ts->xsum[bprev];
                     }
                 } else {
-                    const uint16_t* x = L.x;
+                    // the input and g pointers, loaded before the dependency wait
+                    const uint16_t* x = L.src >= 0 ? tab[L.src].y : L.x;
+                    const uint16_t* gvec = FORM == 1 ? p.layers[j].g : nullptr;
                     if (L.src >= 0) {
                         // wait until every CTA has finished the producing layer
                         bool got = true;
@@ -534,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
                                         got = false;
                                         break;
                                     }
-                                    __nanosleep(64);
+                                    __nanosleep(32);
                                 }
                             }
                         }
@@ -542,30 +607,34 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
                             ok = false;
                             break;
                         }
-                        x = p.layers[L.src].y;
                     }
-                    prep_layer<FORM>(L, x, L.src >= 0, act, p.astride, ts, b, et);
+                    prep_layer<FORM>(K, x, gvec, L.src >= 0, act, p.astride, ts, b, et);
                 }
-            }
-            if (prepare) {
                 // zeros from K to a whole step in every row (a partial last step's
                 // lanes past the row end multiply them)
-                const int kp = (L.K + F::kStepK - 1) / F::kStepK * F::kStepK;
+                const int kp = (K + F::kStepK - 1) / F::kStepK * F::kStepK;
                 for (int r = 0; r < COLS; ++r)
-                    for (int i = L.K + 16 * et; i < kp; i += 16 * kPrepThreads)
+                    for (int i = K + 16 * et; i < kp; i += 16 * kPrepThreads)
                         *reinterpret_cast<uint4*>(act + r * p.astride + i) = make_uint4(0, 0, 0, 0);
             }
             prev_prepared = prepare;
             bar_prep();   // activations and token scalars written (and the scratch reads done)
             if (et == 0) tc::mbar_arrive(bar_act + 8 * b);
         } else {
-            // ---- epilogue of layer j from buffer j % 2
+            // ---- epilogue of layer j from buffer j % NB
             const int j = next_epi++;
-            const ChainLayer& L = p.layers[j];
-            const int b = j & 1;
+            const LayerInfo L = tab[j];
+            const int b = j % NB;
             const int first = first_tile(L, c, G), T = tiles_of(L, first, G);
-            if (!tc::bar_and(kBarPrep, kPrepThreads,
-                             tc::mbar_wait(bar_mma + 8 * b, (j >> 1) & 1, p.flags, p.wait_ns))) {
+            // the output pointers, loaded before the wait for the contraction
+            uint16_t* y = L.y;
+            int32_t* acc_out = FORM == 0 ? p.layers[j].acc_out : nullptr;
+            const float w_scale = p.layers[j].w_scale;
+            const uint16_t* h = FORM == 1 ? p.layers[j].h : nullptr;
+            // one thread waits (asleep) for the contraction; the others in the barrier
+            bool got = true;
+            if (et == 0) got = tc::mbar_wait(bar_mma + 8 * b, (uint32_t)((j / NB) & 1), p.flags, p.wait_ns);
+            if (!tc::bar_and(kBarPrep, kPrepThreads, got)) {
                 ok = false;
                 break;
             }
@@ -577,18 +646,18 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
                 if constexpr (FORM == 0) {
                     const int a = pb[o] - ts->qsum[b];
                     pb[o] = 0;
-                    L.y[nrow] = __half_as_ushort(__float2half_rn(__fmul_rn(__fmul_rn((float)a, sc), L.w_scale)));
-                    if (L.acc_out) L.acc_out[nrow] = a;
+                    y[nrow] = __half_as_ushort(__float2half_rn(__fmul_rn(__fmul_rn((float)a, sc), w_scale)));
+                    if (acc_out) acc_out[nrow] = a;
                 } else {
                     const long long Z = limb_combine(pb[3 * o], pb[3 * o + 1], pb[3 * o + 2], ts->xsum[b]);
                     pb[3 * o] = pb[3 * o + 1] = pb[3 * o + 2] = 0;
                     const float z = __fmul_rn(sc, (float)Z);
-                    const float hv = __half2float(__ushort_as_half(L.h[nrow]));
-                    L.y[nrow] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hv)));
+                    const float hv = __half2float(__ushort_as_half(h[nrow]));
+                    y[nrow] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hv)));
                 }
             }
             bar_prep();   // every output of this CTA written, partials cleared
-            if (L.has_dep && et == 0) {
+            if ((L.flags & kInfoHasDep) && et == 0) {
                 __threadfence();
                 atomicAdd(p.done + j, 1u);
             }
@@ -599,35 +668,41 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Shared-memory layout of a launch: ring [S][kSlotBytes] | activations
-// [2][COLS][astride] | partial sums [2][kMaxTiles*16][COLS] int32 | token
-// scalars | barriers.
+// [NB][COLS][astride] | partial sums [NB][kMaxTiles*16][COLS] int32 | token
+// scalars | barriers | layer table [n].  S (ring slots) is the largest that
+// fits, then NB (activation buffers, 2..4).
 struct ChainSmem {
-    int S, astride, off_act, off_part, off_tok, off_bar, total;
+    int S, NB, astride, off_act, off_part, off_tok, off_bar, off_tab, total;
 };
 
-bool chain_smem(int form, int kmax, ChainSmem& m) {
+bool chain_smem(int form, int kmax, int n, ChainSmem& m) {
     const int cols = form == 0 ? 1 : 3;
     // rows padded to a whole step (256 / 512 k), +16 bytes between rows
     m.astride = (kmax + 511) / 512 * 512 + 16;
-    const int act = 2 * cols * m.astride;
-    const int partb = 2 * kMaxTiles * 16 * cols * 4;
     const int tok = (int)round_up(sizeof(TokStats), 16);
-    for (int S = kMaxSlots; S >= 3; --S) {
+    auto layout = [&](int NB, int S) {
         int off = S * kSlotBytes;
         m.off_act = off;
-        off += (int)round_up((size_t)act, 16);
+        off += (int)round_up((size_t)NB * cols * m.astride, 16);
         m.off_part = off;
-        off += partb;
+        off += NB * kMaxTiles * 16 * cols * 4;
         m.off_tok = off;
         off += tok;
         m.off_bar = off;
-        off += 8 * (2 * S + 4);
-        if (off <= kDecodeMaxSmem) {
-            m.S = S;
-            m.total = off;
-            return true;
-        }
-    }
+        off += 8 * (2 * S + 2 * kMaxBufs);
+        off = (int)round_up((size_t)off, 16);
+        m.off_tab = off;
+        off += (int)sizeof(LayerInfo) * n;
+        m.S = S;
+        m.NB = NB;
+        m.total = off;
+        return off <= kDecodeMaxSmem;
+    };
+    // the most ring slots first (bytes in flight set the streaming rate), then
+    // the most activation buffers
+    for (int S = kMaxSlots; S >= 3; --S)
+        for (int NB = kMaxBufs; NB >= 2; --NB)
+            if (layout(NB, S)) return true;
     return false;
 }
 
@@ -651,9 +726,10 @@ cudaError_t launch_chain(const ChainParams& p, int smem, cudaStream_t s) {
 
 }  // namespace
 
-size_t chain_bytes(int n_layers) {
-    return round_up((size_t)n_layers * sizeof(ChainLayer), 256) + round_up((size_t)n_layers * 4, 256);
-}
+// Chain buffer: descriptors [n] | layer table [n] | completion counters [n].
+size_t chain_info_offset(int n) { return round_up((size_t)n * sizeof(ChainLayer), 256); }
+size_t chain_done_offset(int n) { return chain_info_offset(n) + round_up((size_t)n * sizeof(LayerInfo), 256); }
+size_t chain_bytes(int n_layers) { return chain_done_offset(n_layers) + round_up((size_t)n_layers * 4, 256); }
 
 int chain_max_k(int form) { return form == 0 ? 32768 : 16384; }
 
@@ -662,6 +738,7 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
     const int G = device_sm_count();
     if (G <= 0) return BL_ERR_CUDA;
     std::vector<ChainLayer> host((size_t)n);
+    std::vector<LayerInfo> info((size_t)n);
     int kmax = 0;
     long long tiles_before = 0;
     for (int j = 0; j < n; ++j) {
@@ -713,11 +790,32 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
         if (in.K > kmax) kmax = in.K;
         if (L.ntile > kMaxTiles * G) return BL_ERR_SHAPE;
     }
+    for (int j = 0; j < n; ++j) {
+        const ChainLayer& L = host[(size_t)j];
+        LayerInfo& I = info[(size_t)j];
+        I.ntile = (uint16_t)L.ntile;
+        I.rot = (uint16_t)L.rot;
+        I.k16 = (uint16_t)(L.K / 16);
+        I.src = (int16_t)L.src;
+        I.steps = (uint8_t)L.steps;
+        I.nfull = (uint8_t)L.nfull;
+        I.tail = (uint8_t)L.tail;
+        I.bsteps = (uint8_t)L.bsteps;
+        I.nch = (uint8_t)L.nch;
+        I.flags = (uint8_t)((L.ragged ? kInfoRagged : 0) | (L.has_dep ? kInfoHasDep : 0) |
+                            (L.reuse ? kInfoReuse : 0));
+        I.pad = 0;
+        I.x = L.src < 0 ? L.x : nullptr;
+        I.y = L.y;
+    }
     ChainSmem m;
-    if (!chain_smem(form, kmax, m)) return BL_ERR_SHAPE;
+    if (!chain_smem(form, kmax, n, m)) return BL_ERR_SHAPE;
     if (bytes < chain_bytes(n)) return BL_ERR_WORKSPACE;
-    if (cudaMemcpyAsync(chain, host.data(), (size_t)n * sizeof(ChainLayer), cudaMemcpyHostToDevice,
+    char* cb = static_cast<char*>(chain);
+    if (cudaMemcpyAsync(cb, host.data(), (size_t)n * sizeof(ChainLayer), cudaMemcpyHostToDevice,
                         s) != cudaSuccess ||
+        cudaMemcpyAsync(cb + chain_info_offset(n), info.data(), (size_t)n * sizeof(LayerInfo),
+                        cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
         return BL_ERR_CUDA;
     plan->form = form;
@@ -732,22 +830,26 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
 bl_status chain_run(const bl_chain_plan* plan, const void* chain, unsigned int* flags,
                     cudaStream_t s) {
     ChainSmem m;
-    if (!chain_smem(plan->form, plan->kmax, m) || m.S != plan->slots || m.total != plan->smem_bytes)
+    if (!chain_smem(plan->form, plan->kmax, plan->n_layers, m) || m.S != plan->slots ||
+        m.total != plan->smem_bytes)
         return BL_ERR_SHAPE;
     if (device_sm_count() != plan->sm_count) return BL_ERR_SHAPE;
     const int n = plan->n_layers;
     ChainParams p;
-    p.layers = static_cast<const ChainLayer*>(chain);
+    char* cb = static_cast<char*>(const_cast<void*>(chain));
+    p.layers = reinterpret_cast<const ChainLayer*>(cb);
+    p.info = reinterpret_cast<const LayerInfo*>(cb + chain_info_offset(n));
     p.n = n;
-    p.done = reinterpret_cast<unsigned int*>(static_cast<char*>(const_cast<void*>(chain)) +
-                                             round_up((size_t)n * sizeof(ChainLayer), 256));
+    p.done = reinterpret_cast<unsigned int*>(cb + chain_done_offset(n));
     p.flags = flags;
     p.S = m.S;
+    p.nbuf = m.NB;
     p.astride = m.astride;
     p.off_act = m.off_act;
     p.off_part = m.off_part;
     p.off_tok = m.off_tok;
     p.off_bar = m.off_bar;
+    p.off_tab = m.off_tab;
     p.wait_ns = kWaitNs;
     // the completion counters start at zero on every run
     if (cudaMemsetAsync(p.done, 0, (size_t)n * 4, s) != cudaSuccess) return BL_ERR_CUDA;
