@@ -98,12 +98,14 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oref_ternary_linear.argtypes = [P, I, I, I, P, ctypes.c_float, P, P]
     L.oref_ob_linear.argtypes = [P, I, I, I, P, P, P, P, P]
     L.oref_svid.argtypes = [P, I, I, P, P, P, P, I, ctypes.c_double]
+    L.oref_rmsnorm.argtypes = [P, I, I, P, ctypes.c_double, P]
+    L.oref_swiglu.argtypes = [P, P, I, P]
     L.oref_onebit_bits.argtypes = [ctypes.c_int64, ctypes.c_int64]
     L.oref_onebit_bits.restype = ctypes.c_int64
     L.oref_onebit_params.argtypes = [ctypes.c_int64, ctypes.c_int64]
     L.oref_onebit_params.restype = ctypes.c_int64
     for f in ("oref_pack_ternary", "oref_pack_sign", "oref_quant_act",
-              "oref_ternary_linear", "oref_ob_linear", "oref_svid"):
+              "oref_ternary_linear", "oref_ob_linear", "oref_svid", "oref_rmsnorm", "oref_swiglu"):
         getattr(L, f).restype = I
     return L
 
@@ -219,6 +221,27 @@ def svid(W: np.ndarray, max_iter: int = 1000, tol: float = 1e-12):
     it = _check(lib().oref_svid(_p(W), N, K, _p(S), _p(a), _p(b), ctypes.byref(sig),
                                 int(max_iter), float(tol)), "svid")
     return S, a, b, sig.value, it
+
+
+def rmsnorm(x: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
+    """RMSNorm of each token (row) of fp16 x [M,K] with fp16 weight gamma [K] -> fp16 [M,K]."""
+    xb = _half_bits(np.atleast_2d(x))
+    gb = _half_bits(gamma)
+    M, K = xb.shape
+    assert gb.shape == (K,)
+    y = np.zeros((M, K), dtype=np.uint16)
+    _check(lib().oref_rmsnorm(_p(xb), M, K, _p(gb), float(eps), _p(y)), "rmsnorm")
+    return y.view(np.float16)
+
+
+def swiglu(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """fp16((a / (1 + exp(-a))) * b), elementwise over fp16 arrays of one shape."""
+    ab = _half_bits(a).reshape(-1)
+    bb = _half_bits(b).reshape(-1)
+    assert ab.shape == bb.shape
+    y = np.zeros(ab.shape, dtype=np.uint16)
+    _check(lib().oref_swiglu(_p(ab), _p(bb), ab.size, _p(y)), "swiglu")
+    return y.view(np.float16).reshape(np.asarray(a).shape)
 
 
 def onebit_bits(N: int, K: int) -> int:

@@ -305,6 +305,73 @@ int oref_svid(const float *W, int N, int K, int8_t *S, double *a, double *b,
     return it;
 }
 
+/* ---------------------------------------------------------------------
+ * [B158] "BitNet b1.58 介绍": the model keeps LLaMA's components, RMSNorm and
+ * SwiGLU, around its BitLinear layers.  Reading used here (the page gives no
+ * formulas): RMSNorm of one token
+ *     r = 1 / sqrt(sum_k x_k^2 / K + eps),   y_k = fp16((x_k * r) * gamma_k)
+ * and SwiGLU  y = fp16((a / (1 + exp(-a))) * b).
+ * Precision: fp64.  The sum of squares is exact (integers) and rounded once
+ * to fp64; every later operation is one IEEE fp64 rounding, then one
+ * rounding to fp16.  So a result is fixed by its inputs alone (SwiGLU up to
+ * the accuracy of exp).
+ * ------------------------------------------------------------------- */
+
+/* nearest double (ties to even) of the 128-bit integer hi * 2^64 + lo */
+static double u128_to_double(uint64_t hi, uint64_t lo)
+{
+    if (hi == 0) return (double)lo;             /* one IEEE conversion */
+    int nbits = 64;                             /* bit length of hi */
+    while (!(hi >> (nbits - 1))) --nbits;
+    int sh = nbits;                             /* drop the low sh bits: keep 64 */
+    uint64_t top = sh == 64 ? hi : (hi << (64 - sh)) | (lo >> sh);
+    uint64_t rest = sh == 64 ? lo : lo & ((((uint64_t)1) << sh) - 1);
+    /* top has 64 significant bits, 53 are kept: a set bit 0 stands for any
+     * nonzero rest (it lies below the rounding position) */
+    double d = (double)(top | (rest ? 1u : 0u));
+    return ldexp(d, sh);
+}
+
+int oref_rmsnorm(const uint16_t *x, int M, int K, const uint16_t *gamma, double eps, uint16_t *y)
+{
+    if (M < 0 || K <= 0) return OREF_ERR_SHAPE;
+    for (int m = 0; m < M; ++m) {
+        const uint16_t *row = x + (size_t)m * K;
+        /* x = mant * 2^e exactly (mant < 2^11, e in [-24, 5]); x^2 * 2^48 is an
+         * integer below 2^80; the sum of K of them fits 128 bits */
+        uint64_t hi = 0, lo = 0;
+        for (int k = 0; k < K; ++k) {
+            int ex = (row[k] >> 10) & 31, f = row[k] & 1023;
+            if (ex == 31) return OREF_ERR_VALUE;
+            uint64_t mant = ex ? (uint64_t)(1024 | f) : (uint64_t)f;
+            int e = (ex ? ex : 1) - 25;
+            int sh = 2 * e + 48;                 /* 0 .. 58 */
+            uint64_t sq = mant * mant;           /* < 2^22 */
+            uint64_t add_lo = sh < 64 ? sq << sh : 0, add_hi = sh == 0 ? 0 : sq >> (64 - sh);
+            uint64_t nlo = lo + add_lo;
+            hi += add_hi + (nlo < lo ? 1u : 0u);
+            lo = nlo;
+        }
+        double ss = ldexp(u128_to_double(hi, lo), -48);
+        double r = 1.0 / sqrt(ss / (double)K + eps);
+        for (int k = 0; k < K; ++k)
+            y[(size_t)m * K + k] = oref_double_to_half((oref_half_to_double(row[k]) * r) *
+                                                       oref_half_to_double(gamma[k]));
+    }
+    return OREF_OK;
+}
+
+int oref_swiglu(const uint16_t *a, const uint16_t *b, int n, uint16_t *y)
+{
+    if (n < 0) return OREF_ERR_SHAPE;
+    for (int i = 0; i < n; ++i) {
+        double av = oref_half_to_double(a[i]);
+        double silu = av / (1.0 + exp(-av));
+        y[i] = oref_double_to_half(silu * oref_half_to_double(b[i]));
+    }
+    return OREF_OK;
+}
+
 /* [ONEBIT] "1. 新的 1bit 结构" worked example: storage of an N x K OneBit
  * layer = N*K one-bit signs + (N + K) fp16 values. */
 int64_t oref_onebit_bits(int64_t N, int64_t K) { return N * K + 16 * (N + K); }

@@ -27,6 +27,8 @@ int oref_ob_linear(const uint16_t *x, int M, int K, int N, const uint32_t *s1,
                    const uint16_t *g, const uint16_t *h, uint16_t *y, double *z_out);
 int oref_svid(const float *W, int N, int K, int8_t *S, double *a, double *b,
               double *sigma_out, int max_iter, double tol);
+int oref_rmsnorm(const uint16_t *x, int M, int K, const uint16_t *gamma, double eps, uint16_t *y);
+int oref_swiglu(const uint16_t *a, const uint16_t *b, int n, uint16_t *y);
 int64_t oref_onebit_bits(int64_t N, int64_t K);
 int64_t oref_onebit_params(int64_t N, int64_t K);
 

@@ -335,3 +335,77 @@ def test_openmp_build_gives_identical_results(oref):
     _, z1 = oref.ob_linear(x, s1, g, h)
     _, z2 = oref.ob_linear(x, s1, g, h, parallel=True)
     assert np.array_equal(z1, z2)
+
+
+# ------------------------------------------------ RMSNorm and SwiGLU -----
+
+def _golden_rows(name):
+    rows = {}
+    for line in open(os.path.join(os.path.dirname(__file__), "golden", name)):
+        if line.strip() and not line.startswith("#"):
+            k, *v = line.split()
+            rows[k] = v
+    return rows
+
+
+def test_rmsnorm_hand_worked_token(oref):
+    g = _golden_rows("rmsnorm_3_4.txt")
+    x = np.array([[float(v) for v in g["x"]]], dtype=np.float16)
+    y = oref.rmsnorm(x, np.ones(2, dtype=np.float16), 0.0)
+    assert [int(b) for b in y.view(np.uint16)[0]] == [int(v, 16) for v in g["y_bits"]]
+
+
+@pytest.mark.parametrize("K", [64, 640, 4096])
+def test_rmsnorm_against_exactly_rounded_sum(oref, K):
+    """The definition evaluated independently: math.fsum is the exactly rounded
+    sum of the squares (each exact in fp64 for fp16 inputs), then the same
+    fp64 steps in numpy, then numpy's fp16 rounding."""
+    import math
+    rng = np.random.default_rng(K)
+    x = (rng.standard_normal((3, K)) * np.array([[1.0], [1e-3], [300.0]])).astype(np.float16)
+    x[1, 5] = np.float16(6e-8)          # a subnormal
+    gamma = rng.uniform(0.5, 1.5, K).astype(np.float16)
+    eps = 1e-6
+    y = oref.rmsnorm(x, gamma, eps)
+    for m in range(3):
+        xd = x[m].astype(np.float64)
+        ss = math.fsum(float(v) * float(v) for v in xd)
+        r = 1.0 / math.sqrt(ss / K + eps)
+        ref = ((xd * r) * gamma.astype(np.float64)).astype(np.float16)
+        assert np.array_equal(y[m].view(np.uint16), ref.view(np.uint16)), m
+
+
+def test_rmsnorm_scale_invariance_and_unit_rms(oref):
+    """With eps = 0 the output does not change when x is scaled by a power of
+    two (the mean square scales by its square, exactly); with gamma = 1 the
+    output's mean square is 1 up to fp16 rounding."""
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((2, 1024)).astype(np.float16)
+    one = np.ones(1024, dtype=np.float16)
+    y = oref.rmsnorm(x, one, 0.0)
+    for j in (1, 3):
+        xs = (x.astype(np.float64) * 2.0 ** j).astype(np.float16)
+        assert np.array_equal(xs.astype(np.float64), x.astype(np.float64) * 2.0 ** j)  # exact scaling
+        ys = oref.rmsnorm(xs, one, 0.0)
+        assert np.array_equal(ys.view(np.uint16), y.view(np.uint16))
+    ms = np.mean(y.astype(np.float64) ** 2, axis=1)
+    assert np.all(np.abs(ms - 1.0) < 2e-3)
+
+
+def test_swiglu_identities(oref):
+    """silu(a) - silu(-a) = a exactly (1/(1+e^-a) + 1/(1+e^a) = 1), silu(0) = 0,
+    silu(a) -> a for large a and -> 0 for very negative a; b scales the output."""
+    a = np.linspace(-12, 12, 481).astype(np.float16)
+    one = np.ones_like(a)
+    yp = oref.swiglu(a, one).astype(np.float64)
+    yn = oref.swiglu(-a, one).astype(np.float64)
+    diff = yp - yn
+    # each side carries one fp16 rounding: at most half an fp16 spacing of |silu|
+    tol = 2.0 ** -10 * np.maximum(np.abs(yp), np.abs(yn)) + 2.0 ** -24
+    assert np.all(np.abs(diff - a.astype(np.float64)) <= tol)
+    assert oref.swiglu(np.zeros(1, np.float16), np.ones(1, np.float16))[0] == 0
+    big = np.array([30.0, -30.0], dtype=np.float16)
+    yb = oref.swiglu(big, np.ones(2, np.float16))
+    assert yb[0] == np.float16(30.0) and abs(float(yb[1])) < 1e-10
+    b = np.full_like(a, 2.0)
+    assert np.array_equal(oref.swiglu(a, b).astype(np.float64), 2 * oref.swiglu(a, one).astype(np.float64))
