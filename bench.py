@@ -208,10 +208,14 @@ def block_sources(blocks: int):
     return src
 
 
-def chain_stack(blw, synth, dev, form: str, dependent: bool, layers: int = LLAMA7B_LAYERS):
+def chain_stack(blw, synth, dev, form: str, dependent: bool, layers: int = LLAMA7B_LAYERS,
+                fused: bool = False):
     """The 7B-shaped stack as decode-chain layers (M = 1).  dependent: the
     decode step's dependency pattern (one given input); else every layer reads
-    its own given input.  Returns (layer dicts, weight bytes, given-input
+    its own given input.  fused (with dependent): q, k, v and gate, up read an
+    RMSNorm of their input (one weight per block and place, counted in the
+    weight bytes) and down reads SwiGLU(gate, up) -- the block's elementwise
+    steps run inside the chain launch.  Returns (layer dicts, weight bytes, given-input
     buffer, output buffer); every layer's given x and y are views into those
     two buffers.  Ternary w_scale is 1/sqrt(2K/3) per layer, which keeps the
     activations O(1) along a dependent chain (timing does not depend on it)."""
@@ -222,9 +226,18 @@ def chain_stack(blw, synth, dev, form: str, dependent: bool, layers: int = LLAMA
     y_all = torch.empty((sum(N for _, N in shapes),), dtype=torch.float16, device=dev)
     out, wbytes, xo, yo = [], 0, 0, 0
     prev_x = None
+    norm_w = None
     for j, ((K, N), s) in enumerate(zip(shapes, srcs)):
         seed = 2_000_000 + (j // 7) * 16 + j % 7
         d = dict(K=K, N=N, src=s, y=y_all[yo:yo + N])
+        if fused and dependent:
+            if j % 7 in (0, 4):            # attention and MLP RMSNorm weights of the block
+                norm_w = synth.norm_weight(K, seed=seed + 10, device=dev)
+                wbytes += 2 * K
+            if j % 7 in (0, 1, 2, 4, 5):
+                d["norm_w"], d["norm_eps"] = norm_w, 1e-5
+            if j % 7 == 6:
+                d["src2"] = j - 1          # down reads SwiGLU(gate, up)
         yo += N
         if s < 0:
             if dependent and prev_x is not None and j % 7 in (1, 2):
@@ -655,6 +668,25 @@ def main():
             "roofline": {"bound": "hbm", "achieved": round(ival / world, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(ival / world / peaks["hbm_gbs"], 4)}}
         del ig, ich, ilayers, _ix, _iy
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+        # ---- the dependent step with RMSNorm and SwiGLU fused into the chain
+        flayers, fwbytes, _fx, _fy = chain_stack(blw, synth, dev, "ternary", dependent=True,
+                                                 layers=args.layers, fused=True)
+        fch = blw.Chain(0, flayers)
+        fg = capture(fch.run)
+        fms = time_replays(fg, args.steps, args.warmup, dist_on, dev)
+        assert blw.bl_device_status() == 0, "a bounded wait expired in the chain kernel"
+        fval = fwbytes * world / (fms * 1e-3) / 1e9
+        extras["decode_chain_fused"] = {
+            "workload": "llama7b-decode-M1-ternary-32x7, one chain launch, decode-step dependencies, "
+                        "RMSNorm (q,k,v; gate,up) and SwiGLU (down) fused",
+            "value": round(fval, 2), "unit": "GB/s", "ms_per_step": round(fms, 4),
+            "weight_bytes_per_step": fwbytes,
+            "roofline": {"bound": "hbm", "achieved": round(fval / world, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(fval / world / peaks["hbm_gbs"], 4)}}
+        del fg, fch, flayers, _fx, _fy
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
 

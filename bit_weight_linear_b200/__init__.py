@@ -39,7 +39,8 @@ _SZ = ctypes.c_size_t
 class ChainLayer(ctypes.Structure):
     """bl_chain_layer (include/bitlinear.h)."""
     _fields_ = [("x", _P), ("src", _I), ("K", _I), ("N", _I), ("w", _P), ("w_scale", ctypes.c_float),
-                ("g", _P), ("h", _P), ("y", _P), ("acc_out", _P)]
+                ("g", _P), ("h", _P), ("y", _P), ("acc_out", _P), ("src2", _I), ("norm_w", _P),
+                ("norm_eps", ctypes.c_float)]
 
 
 class ChainPlan(ctypes.Structure):
@@ -220,13 +221,15 @@ class Chain:
     def __init__(self, form: int, layers: list[dict]):
         """layers: dicts with K, N, w (packed, CUDA), y (fp16 [N] or [1, N],
         CUDA), and either x (fp16 [K], CUDA) or src (index of an earlier
-        layer); ternary: w_scale, optional acc_out (int32 [N]); OneBit: g, h."""
+        layer); optional src2 (SwiGLU of the outputs of src and src2), norm_w
+        (fp16 [K] RMSNorm weight) and norm_eps; ternary: w_scale, optional
+        acc_out (int32 [N]); OneBit: g, h."""
         n = len(layers)
         arr = (ChainLayer * n)()
         self._keep = []
         dev = None
         for j, d in enumerate(layers):
-            ts = [d.get(k) for k in ("x", "w", "g", "h", "y", "acc_out")]
+            ts = [d.get(k) for k in ("x", "w", "g", "h", "y", "acc_out", "norm_w")]
             _need_cuda(*[t for t in ts if t is not None])
             self._keep.extend(t for t in ts if t is not None)
             dev = dev or d["w"].device
@@ -239,6 +242,9 @@ class Chain:
             arr[j].h = None if d.get("h") is None else d["h"].data_ptr()
             arr[j].y = d["y"].data_ptr()
             arr[j].acc_out = None if d.get("acc_out") is None else d["acc_out"].data_ptr()
+            arr[j].src2 = int(d.get("src2", -1))
+            arr[j].norm_w = None if d.get("norm_w") is None else d["norm_w"].data_ptr()
+            arr[j].norm_eps = float(d.get("norm_eps", 0.0))
         nbytes = int(lib().bl_chain_bytes(n))
         if nbytes == 0:
             raise ValueError("chain length out of range")

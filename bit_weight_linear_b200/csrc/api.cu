@@ -19,7 +19,9 @@ __device__ unsigned int g_pack_error = 0;
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr int kMaxChainLayers = 65536;
+// chain length: the layer table lives in shared memory (32 bytes a layer) and
+// layer indexes are 16-bit there
+constexpr int kMaxChainLayers = 2048;
 
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
@@ -314,9 +316,14 @@ bl_status bl_chain_build(int form, const bl_chain_layer* layers, int n_layers, v
             return BL_ERR_SHAPE;
         if (L.src < -1 || L.src >= j) return BL_ERR_SHAPE;
         if (L.src >= 0 && layers[L.src].N != L.K) return BL_ERR_SHAPE;
+        if (L.src2 < -1 || L.src2 >= j || (L.src2 >= 0 && (L.src < 0 || layers[L.src2].N != L.K)))
+            return BL_ERR_SHAPE;
+        // the fused prologues work on a row held in registers
+        if ((L.src2 >= 0 || L.norm_w) && L.K > bl::chain_max_fused_k(form)) return BL_ERR_SHAPE;
+        if (L.norm_w && !(L.norm_eps >= 0.f)) return BL_ERR_SHAPE;
         if ((L.src < 0 && !L.x) || !L.w || !L.y || (form == 1 && (!L.g || !L.h))) return BL_ERR_NULL;
         if ((L.src < 0 && misaligned(L.x)) || misaligned(L.w) || misaligned(L.y) ||
-            misaligned(L.acc_out) || misaligned(L.g) || misaligned(L.h))
+            misaligned(L.acc_out) || misaligned(L.g) || misaligned(L.h) || misaligned(L.norm_w))
             return BL_ERR_ALIGN;
     }
     if (chain_bytes < bl::chain_bytes(n_layers)) return BL_ERR_WORKSPACE;

@@ -81,13 +81,16 @@ struct alignas(64) ChainLayer {
     int32_t* acc_out;      // optional (ternary)
     const uint16_t* g;     // OneBit input value vector
     const uint16_t* h;     // OneBit output value vector
+    const uint16_t* norm_w;  // RMSNorm weight of the input (nullptr: none)
     float w_scale;
     int src;               // -1: x given; else the layer whose y is the input
     int K, N;
+    int src2;              // -1, or SwiGLU input: silu(y_src) * y_src2
+    float norm_eps;
     int steps, nfull, tail, ragged, bsteps, nch, ntile, rot;
     int has_dep;           // a later layer reads y: arrive on done[] after the epilogue
     int reuse;             // same input as the previous layer: copy its prepared activations
-    int pad[6];
+    int pad[2];
 };
 static_assert(sizeof(ChainLayer) == 384, "chain layer descriptor size");
 
@@ -101,12 +104,12 @@ struct alignas(16) LayerInfo {
     int16_t src;            // -1: x given; else the producing layer
     uint8_t steps, nfull, tail, bsteps, nch;
     uint8_t flags;          // kInfoRagged | kInfoHasDep | kInfoReuse
-    uint16_t pad;
+    int16_t src2;           // -1, or the second input of a SwiGLU prologue
     const uint16_t* x;      // given input (src < 0)
     uint16_t* y;            // output
 };
 static_assert(sizeof(LayerInfo) == 32, "layer info size");
-constexpr uint8_t kInfoRagged = 1, kInfoHasDep = 2, kInfoReuse = 4;
+constexpr uint8_t kInfoRagged = 1, kInfoHasDep = 2, kInfoReuse = 4, kInfoNorm = 8;
 
 struct ChainParams {
     const ChainLayer* layers;
@@ -157,7 +160,135 @@ struct TokStats {
     long long xsum[kMaxBufs];    // OneBit sum X
     uint32_t red[3][kPrepWarps];
     int redi[3][kPrepWarps];
+    unsigned long long ss[kPrepWarps][2];   // RMSNorm: per-warp exact sums of squares
+    double norm_r;                          // RMSNorm: 1 / sqrt(mean square + eps)
 };
+
+// ---- fused prologues of a layer's input (the BitNet b1.58 page keeps LLaMA's
+// RMSNorm and SwiGLU around BitLinear; definitions in include/bitlinear.h)
+
+__device__ __forceinline__ double half_bits_d(uint32_t v) {
+    return (double)__half2float(__ushort_as_half((unsigned short)(v & 0xffffu)));   // exact
+}
+__device__ __forceinline__ uint32_t pack_half2(double lo, double hi) {
+    return (uint32_t)__half_as_ushort(__double2half(lo)) |
+           ((uint32_t)__half_as_ushort(__double2half(hi)) << 16);
+}
+
+// SwiGLU of 8 elements: fp16((a / (1 + exp(-a))) * b) in fp64
+__device__ __forceinline__ uint4 swiglu8(uint4 a, uint4 b) {
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        double r[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const double x = half_bits_d(av[i] >> (16 * h)), y = half_bits_d(bv[i] >> (16 * h));
+            r[h] = __dmul_rn(__ddiv_rn(x, __dadd_rn(1.0, exp(-x))), y);
+        }
+        o[i] = pack_half2(r[0], r[1]);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// exact sum of squares of 8 fp16 elements, as a 128-bit integer in units of
+// 2^-48: x = mant 2^e (mant < 2^11, e >= -24) gives x^2 2^48 < 2^80
+__device__ __forceinline__ void sumsq8(uint4 a, unsigned long long& hi, unsigned long long& lo) {
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int e8 = 0; e8 < 8; ++e8) {
+        const uint32_t hb = (av[e8 >> 1] >> (16 * (e8 & 1))) & 0xffffu;
+        const int ex = (hb >> 10) & 31;
+        const unsigned long long mant = ex ? (1024u | (hb & 1023u)) : (hb & 1023u);
+        const int sh = 2 * ((ex ? ex : 1) - 25) + 48;            // 0 .. 58
+        const unsigned long long sq = mant * mant;
+        const unsigned long long add_lo = sq << sh, add_hi = sh ? sq >> (64 - sh) : 0ull;
+        const unsigned long long nlo = lo + add_lo;
+        hi += add_hi + (nlo < lo ? 1ull : 0ull);
+        lo = nlo;
+    }
+}
+
+// nearest double (ties to even) of the 128-bit integer hi 2^64 + lo
+__device__ __forceinline__ double u128_to_double(unsigned long long hi, unsigned long long lo) {
+    if (hi == 0) return __ull2double_rn(lo);
+    const int sh = 64 - __clzll((long long)hi);   // drop the low sh bits, keep 64
+    const unsigned long long top = sh == 64 ? hi : (hi << (64 - sh)) | (lo >> sh);
+    const unsigned long long rest = sh == 64 ? lo : lo & ((1ull << sh) - 1);
+    // 53 of top's 64 bits are kept: bit 0 set stands for any nonzero rest
+    return ldexp(__ull2double_rn(top | (rest ? 1ull : 0ull)), sh);
+}
+
+// RMSNorm of 8 elements with r and the weight chunk: fp16((x r) gamma), fp64
+__device__ __forceinline__ uint4 norm8(uint4 a, double r, uint4 gq) {
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {gq.x, gq.y, gq.z, gq.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        o[i] = pack_half2(__dmul_rn(__dmul_rn(half_bits_d(av[i]), r), half_bits_d(gv[i])),
+                          __dmul_rn(__dmul_rn(half_bits_d(av[i] >> 16), r), half_bits_d(gv[i] >> 16)));
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+struct Prologue {
+    const uint16_t* x2;      // SwiGLU: the second input (another CTA's output; nullptr: none)
+    const uint16_t* gamma;   // RMSNorm weight (nullptr: none)
+    double eps;
+};
+
+// Apply the prologue to the row held in registers: chunk c (c < nch) holds
+// the 8 elements at off(c).
+template <int NCH, typename Off>
+__device__ __forceinline__ void apply_prologue(uint4 (&xr)[NCH], int nch, Off off, int K,
+                                               const Prologue& pro, TokStats* ts, int et) {
+    if (pro.x2) {
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            if (c >= nch) break;
+            xr[c] = swiglu8(xr[c], ld_cg_v4(pro.x2 + off(c)));
+        }
+    }
+    if (pro.gamma) {
+        const int pw = et >> 5, lane = et & 31;
+        unsigned long long hi = 0, lo = 0;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            if (c >= nch) break;
+            sumsq8(xr[c], hi, lo);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long h2 = __shfl_xor_sync(0xffffffffu, hi, o);
+            const unsigned long long l2 = __shfl_xor_sync(0xffffffffu, lo, o);
+            const unsigned long long nlo = lo + l2;
+            hi += h2 + (nlo < lo ? 1ull : 0ull);
+            lo = nlo;
+        }
+        if (lane == 0) {
+            ts->ss[pw][0] = hi;
+            ts->ss[pw][1] = lo;
+        }
+        bar_prep();
+        if (et == 0) {
+            unsigned long long H = 0, Lo = 0;
+            for (int w = 0; w < kPrepWarps; ++w) {
+                const unsigned long long nlo = Lo + ts->ss[w][1];
+                H += ts->ss[w][0] + (nlo < Lo ? 1ull : 0ull);
+                Lo = nlo;
+            }
+            const double ssq = ldexp(u128_to_double(H, Lo), -48);
+            ts->norm_r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ssq, (double)K), pro.eps)));
+        }
+        bar_prep();
+        const double r = ts->norm_r;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            if (c >= nch) break;
+            xr[c] = norm8(xr[c], r, ld_ro_v4(pro.gamma + off(c)));
+        }
+    }
+}
 
 // 16-byte chunks of x per thread held in registers: rows up to kRegChunks x 8 x
 // kPrepThreads elements (ternary; OneBit: whole 32-element groups, a quarter
@@ -171,8 +302,8 @@ constexpr int kRegChunks = 10;
 // over x (the second from L1 or L2).  `cg`: x is another CTA's output, read
 // through L2.
 template <int FORM>
-__device__ void prep_layer(int K, const uint16_t* x, const uint16_t* gvec, bool cg, uint8_t* act,
-                           int astride, TokStats* ts, int b, int et) {
+__device__ void prep_layer(int K, const uint16_t* x, const uint16_t* gvec, bool cg, const Prologue& pro,
+                           uint8_t* act, int astride, TokStats* ts, int b, int et) {
     const int pw = et >> 5, lane = et & 31;
     auto ld = [&](const uint16_t* p) { return cg ? ld_cg_v4(p) : tc::ld_v4(p); };
     const bool in_regs = FORM == 0 ? K <= 8 * kRegChunks * kPrepThreads
@@ -190,6 +321,7 @@ __device__ void prep_layer(int K, const uint16_t* x, const uint16_t* gvec, bool 
                 if (c >= nc) break;
                 xr[c] = ld(x + 8 * (et + c * kPrepThreads));
             }
+            apply_prologue(xr, nc, [&](int c) { return 8 * (et + c * kPrepThreads); }, K, pro, ts, et);
 #pragma unroll
             for (int c = 0; c < kRegChunks; ++c) {
                 if (c >= nc) break;
@@ -248,6 +380,9 @@ __device__ void prep_layer(int K, const uint16_t* x, const uint16_t* gvec, bool 
 #pragma unroll
                 for (int v = 0; v < 4; ++v) xr[4 * c + v] = ld(x + e + 8 * v);
             }
+            apply_prologue(xr, 4 * ng,
+                           [&](int c) { return 32 * (et + (c >> 2) * kPrepThreads) + 8 * (c & 3); }, K,
+                           pro, ts, et);
 #pragma unroll
             for (int c = 0; c < kG; ++c) {
                 if (c >= ng) break;
@@ -559,7 +694,8 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
     bool prev_prepared = false;   // layer next_prep-1's activations are in its buffer
     int next_prep = 0, next_epi = 0;
     while (next_epi < n && ok) {
-        const bool can_prep = next_prep < n && next_prep < next_epi + NB && tab[next_prep].src < next_epi;
+        const bool can_prep = next_prep < n && next_prep < next_epi + NB &&
+                              tab[next_prep].src < next_epi && tab[next_prep].src2 < next_epi;
         if (can_prep) {
             // ---- activations of layer j into buffer j % NB
             const int j = next_prep++;
@@ -583,15 +719,22 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
                         ts->xsum[b] = ts->xsum[bprev];
                     }
                 } else {
-                    // the input and g pointers, loaded before the dependency wait
+                    // the input, g and prologue pointers, loaded before the dependency wait
                     const uint16_t* x = L.src >= 0 ? tab[L.src].y : L.x;
                     const uint16_t* gvec = FORM == 1 ? p.layers[j].g : nullptr;
+                    Prologue pro;
+                    pro.x2 = L.src2 >= 0 ? tab[L.src2].y : nullptr;
+                    pro.gamma = (L.flags & kInfoNorm) ? p.layers[j].norm_w : nullptr;
+                    pro.eps = (double)p.layers[j].norm_eps;
                     if (L.src >= 0) {
-                        // wait until every CTA has finished the producing layer
+                        // wait until every CTA has finished the producing layer(s)
                         bool got = true;
                         if (et == 0) {
-                            const unsigned int* d = p.done + L.src;
-                            if (ld_acquire_u32(d) < (unsigned)G) {
+                            for (int dsrc = 0; dsrc < 2 && got; ++dsrc) {
+                                const int sj = dsrc == 0 ? L.src : L.src2;
+                                if (sj < 0) continue;
+                                const unsigned int* d = p.done + sj;
+                                if (ld_acquire_u32(d) >= (unsigned)G) continue;
                                 const uint64_t t0 = tc::globaltimer_ns();
                                 while (ld_acquire_u32(d) < (unsigned)G) {
                                     if (tc::globaltimer_ns() - t0 > p.wait_ns) {
@@ -608,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
                             break;
                         }
                     }
-                    prep_layer<FORM>(K, x, gvec, L.src >= 0, act, p.astride, ts, b, et);
+                    prep_layer<FORM>(K, x, gvec, L.src >= 0, pro, act, p.astride, ts, b, et);
                 }
                 // zeros from K to a whole step in every row (a partial last step's
                 // lanes past the row end multiply them)
@@ -732,6 +875,9 @@ size_t chain_done_offset(int n) { return chain_info_offset(n) + round_up((size_t
 size_t chain_bytes(int n_layers) { return chain_done_offset(n_layers) + round_up((size_t)n_layers * 4, 256); }
 
 int chain_max_k(int form) { return form == 0 ? 32768 : 16384; }
+int chain_max_fused_k(int form) {
+    return form == 0 ? 8 * kRegChunks * kPrepThreads : 32 * (kRegChunks / 4) * kPrepThreads;
+}
 
 bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain, size_t bytes,
                       bl_chain_plan* plan, cudaStream_t s) {
@@ -748,6 +894,9 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
         L.K = in.K;
         L.N = in.N;
         L.src = in.src;
+        L.src2 = in.src2;
+        L.norm_w = in.norm_w;
+        L.norm_eps = in.norm_eps;
         L.x = in.x;
         L.w = in.w;
         L.y = in.y;
@@ -759,8 +908,13 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
         L.rot = (int)(tiles_before % G);
         tiles_before += L.ntile;
         if (in.src >= 0) host[(size_t)in.src].has_dep = 1;
+        if (in.src2 >= 0) host[(size_t)in.src2].has_dep = 1;
+        // the same prepared input as the layer before: same source(s), same
+        // prologue, same g (OneBit)
         if (j > 0 && in.K == layers[j - 1].K && in.src == layers[j - 1].src &&
-            (in.src >= 0 || in.x == layers[j - 1].x) && (form == 0 || in.g == layers[j - 1].g))
+            in.src2 == layers[j - 1].src2 && (in.src >= 0 || in.x == layers[j - 1].x) &&
+            in.norm_w == layers[j - 1].norm_w && (!in.norm_w || in.norm_eps == layers[j - 1].norm_eps) &&
+            (form == 0 || in.g == layers[j - 1].g))
             L.reuse = 1;
         // k-steps of 64 packed bytes per row; stages of at most 16 steps, a
         // multiple of 16 when a row takes several (a warp owns the same steps
@@ -803,8 +957,8 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
         I.bsteps = (uint8_t)L.bsteps;
         I.nch = (uint8_t)L.nch;
         I.flags = (uint8_t)((L.ragged ? kInfoRagged : 0) | (L.has_dep ? kInfoHasDep : 0) |
-                            (L.reuse ? kInfoReuse : 0));
-        I.pad = 0;
+                            (L.reuse ? kInfoReuse : 0) | (L.norm_w ? kInfoNorm : 0));
+        I.src2 = (int16_t)L.src2;
         I.x = L.src < 0 ? L.x : nullptr;
         I.y = L.y;
     }

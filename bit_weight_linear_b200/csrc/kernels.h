@@ -118,6 +118,7 @@ cudaError_t launch_onebit_stream_prepared(const int8_t* planes, const float* ste
 // `chain` buffer of chain_bytes(n) bytes, one cooperative launch per run.
 size_t chain_bytes(int n_layers);
 int chain_max_k(int form);
+int chain_max_fused_k(int form);   // longest row the RMSNorm / SwiGLU prologues take
 bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain, size_t bytes,
                       bl_chain_plan* plan, cudaStream_t s);
 bl_status chain_run(const bl_chain_plan* plan, const void* chain, unsigned int* flags,

@@ -12,7 +12,8 @@ Distributions:
 * sign weights: iid +-1 with p = 0.5, as fp16 (the dense matrix whose sign
   is packed);
 * OneBit value vectors g, h: U(0.5, 1.5) * 0.02, rounded to fp16;
-* SVID input: N(0, 0.02) fp32.
+* SVID input: N(0, 0.02) fp32;
+* RMSNorm weights: 1 + 0.1 N(0, 1), rounded to fp16.
 """
 from __future__ import annotations
 
@@ -51,6 +52,11 @@ def value_vector(n: int, seed: int, device="cpu") -> torch.Tensor:
     g = _gen(seed, device)
     u = torch.rand((n,), generator=g, device=device, dtype=torch.float32)
     return ((u + 0.5) * 0.02).to(torch.float16)
+
+
+def norm_weight(n: int, seed: int, device="cpu") -> torch.Tensor:
+    g = _gen(seed, device)
+    return (1.0 + 0.1 * torch.randn((n,), generator=g, device=device, dtype=torch.float32)).to(torch.float16)
 
 
 def svid_weights(N: int, K: int, seed: int, device="cpu") -> torch.Tensor:

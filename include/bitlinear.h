@@ -215,6 +215,12 @@ bl_status bl_ternary_linear_noalloc(const uint16_t *x, int M, int K, int N, cons
  * of that layer's y is written.  Layers whose inputs do not depend on each
  * other overlap; the weights of later layers stream while earlier ones finish.
  *
+ * The fused steps of a LLaMA-like block (the BitNet b1.58 page keeps RMSNorm
+ * and SwiGLU around BitLinear) run inside the launch: an RMSNorm of a layer's
+ * input (norm_w) and SwiGLU of two earlier outputs (src2) -- on rows of at
+ * most 17920 (ternary) / 14336 (OneBit) elements.  Consecutive layers with the
+ * same input (q, k, v; gate, up) prepare it once.
+ *
  * Usage: describe the layers, call bl_chain_build once (it writes the device
  * descriptors, including TMA tensor maps, into the caller's `chain` buffer and
  * fills `plan`), then bl_chain_run as often as needed (graph-capturable: one
@@ -236,6 +242,15 @@ typedef struct {
     const uint16_t *h;     /* OneBit output value vector fp16 [N] (else NULL) */
     uint16_t *y;           /* fp16 [N] output */
     int32_t *acc_out;      /* optional int32 [N] accumulators (ternary), or NULL */
+    int src2;              /* -1, or (with src >= 0) the index of a second earlier
+                              layer: the input is then SwiGLU of the two outputs,
+                              fp16(silu(y_src) * y_src2), silu(a) = a/(1+exp(-a)),
+                              in fp64 (its N must equal this layer's K too) */
+    const uint16_t *norm_w; /* NULL, or the fp16 [K] weight of an RMSNorm of the
+                              input before it is quantised:
+                              fp16((x * r) * norm_w), r = 1/sqrt(sum x^2/K + eps),
+                              the sum of squares exact, the rest in fp64 */
+    float norm_eps;        /* eps of that RMSNorm */
 } bl_chain_layer;
 
 typedef struct {           /* filled by bl_chain_build; pass unchanged to bl_chain_run */
@@ -247,7 +262,8 @@ typedef struct {           /* filled by bl_chain_build; pass unchanged to bl_cha
     int smem_bytes;        /* shared memory per CTA */
 } bl_chain_plan;
 
-/* Device bytes of the chain buffer for n_layers layers (0 if out of range). */
+/* Device bytes of the chain buffer for n_layers layers, 1 <= n_layers <= 2048
+ * (0 if out of range). */
 size_t bl_chain_bytes(int n_layers);
 
 /*

@@ -133,11 +133,11 @@ def test_chain_build_rejects_bad_layers(L):
     arr = (blw.ChainLayer * n)()
     for j in range(n):
         arr[j].x, arr[j].src, arr[j].K, arr[j].N = 0x10000, -1, 128, 16
-        arr[j].w, arr[j].y = 0x10000, 0x10000
+        arr[j].w, arr[j].y, arr[j].src2 = 0x10000, 0x10000, -1
     plan = blw.ChainPlan()
     buf = ctypes.c_void_p(0x100000)
     nb = L.bl_chain_bytes(n)
-    assert nb > 0 and L.bl_chain_bytes(0) == 0
+    assert nb > 0 and L.bl_chain_bytes(0) == 0 and L.bl_chain_bytes(2049) == 0
     assert L.bl_chain_build(0, None, n, buf, nb, ctypes.byref(plan), None) == 1
     assert L.bl_chain_build(2, arr, n, buf, nb, ctypes.byref(plan), None) == 2       # bad form
     assert L.bl_chain_build(0, arr, n, ctypes.c_void_p(0x100010), nb, ctypes.byref(plan), None) == 3
@@ -155,3 +155,20 @@ def test_chain_build_rejects_bad_layers(L):
     arr[0].x = 0x10000
     assert L.bl_chain_build(1, arr, n, buf, nb, ctypes.byref(plan), None) == 1       # OneBit needs g, h
     assert L.bl_chain_build(0, arr, n, buf, nb - 1, ctypes.byref(plan), None) == 7
+    # fused prologues: SwiGLU needs src >= 0 and an earlier src2 of the same width
+    arr[1].src2 = 0                                 # src2 without src
+    assert L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None) == 2
+    arr[1].src, arr[1].x, arr[1].src2 = 0, None, 1  # src2 not an earlier layer
+    arr[0].N = 128
+    assert L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None) == 2
+    arr[1].src2, arr[1].norm_w, arr[1].norm_eps = 0, 0x20000, -1.0    # eps < 0
+    assert L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None) == 2
+    arr[1].norm_eps, arr[1].norm_w = 1e-6, 0x20002                    # misaligned weight
+    assert L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None) == 3
+    # a fused row must fit the registers of the prologue: 17920 ternary
+    arr[0].N = arr[1].K = 18048
+    arr[1].norm_w, arr[1].src2 = 0x20000, -1
+    assert L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None) == 2
+    arr[1].norm_w = None                            # unfused, the same row is fine
+    r = L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None)
+    assert r != 2

@@ -153,3 +153,118 @@ def test_chain_onebit_dependent_and_edge_shapes(blw, oref):
                                   h.numpy(), parallel=True)
         y = d["y"].cpu().numpy().astype(np.float64)
         assert np.max(np.abs(y - z_ref[0])) <= OB_TOL * np.max(np.abs(z_ref[0])), j
+
+
+def fused_block_layers(blocks):
+    """The LLaMA-like decode step with its fused steps: q, k, v read
+    RMSNorm(block input); o reads v's output (attention's place, identity);
+    gate and up read RMSNorm(o's output); down reads SwiGLU(gate, up).
+    Returns (src, src2, has_norm) per layer."""
+    out = []
+    for b in range(blocks):
+        base = 7 * b
+        blk_in = -1 if b == 0 else base - 1
+        out += [(blk_in, -1, True), (blk_in, -1, True), (blk_in, -1, True), (base + 2, -1, False),
+                (base + 3, -1, True), (base + 3, -1, True), (base + 4, base + 5, False)]
+    return out
+
+
+def _fused_input(oref, layers, d):
+    """The fp16 input a fused layer quantises, from the oracle's RMSNorm and
+    SwiGLU applied to what the GPU layer read."""
+    xin = (d["x"] if d["src"] < 0 else layers[d["src"]]["y"]).cpu().numpy()
+    if d.get("src2", -1) >= 0:
+        xin = oref.swiglu(xin, layers[d["src2"]]["y"].cpu().numpy())
+    if d.get("norm_w") is not None:
+        xin = oref.rmsnorm(xin[None, :], d["norm_w"].cpu().numpy(), d["norm_eps"])[0]
+    return xin
+
+
+EPS = float(np.float32(1e-5))
+
+
+def test_chain_fused_llama7b_blocks_bit_exact(blw, oref):
+    """Four LLaMA-7B blocks with RMSNorm and SwiGLU fused into the chain: every
+    layer's accumulators and outputs equal the oracle's RMSNorm / SwiGLU /
+    BitLinear applied to the GPU's own inputs, bit for bit."""
+    blocks = 4
+    shapes = [(K, N) for _ in range(blocks) for (_, K, N) in BLOCK_7B]
+    plan = fused_block_layers(blocks)
+    layers, host = ternary_chain(blw, shapes, [s for s, _, _ in plan], seed=640_000)
+    for j, (d, (_, s2, norm)) in enumerate(zip(layers, plan)):
+        d["src2"] = s2
+        if norm:
+            # q, k, v (and gate, up) share one RMSNorm weight: prepared once
+            d["norm_w"] = synth.norm_weight(d["K"], seed=641_000 + (j // 7) * 2 + (j % 7 >= 4)).cuda()
+            d["norm_eps"] = EPS
+    for j in range(1, len(layers)):
+        if plan[j][2] and plan[j - 1][2] and plan[j][0] == plan[j - 1][0]:
+            layers[j]["norm_w"] = layers[j - 1]["norm_w"]
+    ch = blw.Chain(0, layers)
+    for _ in range(2):
+        for d in layers:
+            d["y"].zero_()
+        ch.run()
+        torch.cuda.synchronize()
+        assert blw.bl_device_status() == 0
+    for j, (d, w) in enumerate(zip(layers, host)):
+        xin = _fused_input(oref, layers, d)
+        assert np.isfinite(xin.astype(np.float32)).all(), j
+        y_ref, acc_ref = oref.ternary_linear(xin[None, :], oref.pack_ternary(w.numpy()), d["w_scale"],
+                                             parallel=True)
+        assert np.array_equal(d["acc_out"].cpu().numpy(), acc_ref[0]), j
+        assert np.array_equal(d["y"].cpu().numpy().view(np.uint16), y_ref[0].view(np.uint16)), j
+
+
+def test_chain_fused_prologue_edge_rows(blw, oref):
+    """RMSNorm at the largest fused row (17920) and on a zero row (r =
+    1/sqrt(eps)); SwiGLU of a row whose gate values reach +-5e3 (exp(-a)
+    overflows to inf: silu -> -0) and of two rows in either order."""
+    K1 = 17920
+    shapes = [(K1, 256), (1024, 128), (1024, 1024), (128, 1024), (1024, 64), (1024, 64)]
+    layers, host = ternary_chain(blw, shapes, [-1, -1, -1, -1, 2, 3], seed=650_000)
+    layers[0]["norm_w"], layers[0]["norm_eps"] = synth.norm_weight(K1, seed=650_100).cuda(), EPS
+    layers[1]["x"].zero_()
+    layers[1]["norm_w"], layers[1]["norm_eps"] = synth.norm_weight(1024, seed=650_101).cuda(), 0.25
+    # y2 large (|y2| ~ 2e3, beyond exp overflow at 709) but silu(y2) * y3 finite
+    x2 = layers[2]["x"].float()
+    x2[::7] = 60000.0
+    x2[1::7] = -60000.0
+    layers[2]["x"].copy_(x2.half())
+    layers[2]["w_scale"] = 0.002
+    layers[4]["src2"] = 3                   # SwiGLU(y2, y3)
+    layers[5]["src2"] = 2                   # SwiGLU(y3, y2), then RMSNorm
+    layers[5]["norm_w"], layers[5]["norm_eps"] = synth.norm_weight(1024, seed=650_102).cuda(), EPS
+    blw.Chain(0, layers).run()
+    torch.cuda.synchronize()
+    assert blw.bl_device_status() == 0
+    y2 = layers[2]["y"].float()
+    assert torch.isfinite(y2).all() and y2.abs().max() > 1000.0
+    for j, (d, w) in enumerate(zip(layers, host)):
+        xin = _fused_input(oref, layers, d)
+        assert np.isfinite(xin.astype(np.float32)).all(), j
+        y_ref, acc_ref = oref.ternary_linear(xin[None, :], oref.pack_ternary(w.numpy()), d["w_scale"],
+                                             parallel=True)
+        assert np.array_equal(d["acc_out"].cpu().numpy(), acc_ref[0]), j
+        assert np.array_equal(d["y"].cpu().numpy().view(np.uint16), y_ref[0].view(np.uint16)), j
+
+
+def test_chain_fused_onebit_block(blw, oref):
+    """The fused block on OneBit layers (row widths up to 11008 < 14336)."""
+    shapes = [(K, N) for (_, K, N) in BLOCK_7B]
+    plan = fused_block_layers(1)
+    layers, host = _onebit_chain(blw, shapes, [s for s, _, _ in plan], seed=660_000)
+    nw = [synth.norm_weight(4096, seed=660_100 + i).cuda() for i in range(2)]
+    for j, (d, (_, s2, norm)) in enumerate(zip(layers, plan)):
+        d["src2"] = s2
+        if norm:
+            d["norm_w"], d["norm_eps"] = nw[j >= 4], EPS
+    blw.Chain(1, layers).run()
+    torch.cuda.synchronize()
+    assert blw.bl_device_status() == 0
+    for j, (d, (w, g, h)) in enumerate(zip(layers, host)):
+        xin = _fused_input(oref, layers, d)
+        _, z_ref = oref.ob_linear(xin[None, :], oref.pack_sign(w.numpy()), g.numpy(), h.numpy(),
+                                  parallel=True)
+        y = d["y"].cpu().numpy().astype(np.float64)
+        assert np.max(np.abs(y - z_ref[0])) <= OB_TOL * np.max(np.abs(z_ref[0])), j
