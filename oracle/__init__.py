@@ -100,12 +100,15 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oref_svid.argtypes = [P, I, I, P, P, P, P, I, ctypes.c_double]
     L.oref_rmsnorm.argtypes = [P, I, I, P, ctypes.c_double, P]
     L.oref_swiglu.argtypes = [P, P, I, P]
+    L.oref_billm_binarize.argtypes = [P, I, I, P, P, P, P]
+    L.oref_billm_linear.argtypes = [P, I, I, I, P, P, P, P, P, P]
     L.oref_onebit_bits.argtypes = [ctypes.c_int64, ctypes.c_int64]
     L.oref_onebit_bits.restype = ctypes.c_int64
     L.oref_onebit_params.argtypes = [ctypes.c_int64, ctypes.c_int64]
     L.oref_onebit_params.restype = ctypes.c_int64
     for f in ("oref_pack_ternary", "oref_pack_sign", "oref_quant_act",
-              "oref_ternary_linear", "oref_ob_linear", "oref_svid", "oref_rmsnorm", "oref_swiglu"):
+              "oref_ternary_linear", "oref_ob_linear", "oref_svid", "oref_rmsnorm", "oref_swiglu",
+              "oref_billm_binarize", "oref_billm_linear"):
         getattr(L, f).restype = I
     return L
 
@@ -221,6 +224,36 @@ def svid(W: np.ndarray, max_iter: int = 1000, tol: float = 1e-12):
     it = _check(lib().oref_svid(_p(W), N, K, _p(S), _p(a), _p(b), ctypes.byref(sig),
                                 int(max_iter), float(tol)), "svid")
     return S, a, b, sig.value, it
+
+
+def billm_binarize(W: np.ndarray):
+    """BiLLM binary residual approximation of fp32 W [N,K]:
+    returns (B_o int8 +-1 [N,K], B_r int8 +-1 [N,K], alpha_o fp64 [N], alpha_r fp64 [N])."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    Bo = np.zeros((N, K), dtype=np.int8)
+    Br = np.zeros((N, K), dtype=np.int8)
+    ao = np.zeros((N,), dtype=np.float64)
+    ar = np.zeros((N,), dtype=np.float64)
+    _check(lib().oref_billm_binarize(_p(W), N, K, _p(Bo), _p(Br), _p(ao), _p(ar)), "billm_binarize")
+    return Bo, Br, ao, ar
+
+
+def billm_linear(x: np.ndarray, bo1: np.ndarray, br1: np.ndarray, alpha_o: np.ndarray,
+                 alpha_r: np.ndarray, parallel: bool = False):
+    """Two-plane binary linear: returns (y fp16 [M,N], z fp64 [M,N]) for fp16 x
+    [M,K], packed sign planes [N, K/32] and fp16 scales [N]."""
+    xb = _half_bits(np.atleast_2d(x))
+    bo1, br1 = _c(bo1, np.uint32), _c(br1, np.uint32)
+    aob, arb = _half_bits(alpha_o), _half_bits(alpha_r)
+    M, K = xb.shape
+    N = bo1.shape[0]
+    assert bo1.shape == (N, K // 32) and br1.shape == bo1.shape and aob.shape == (N,) and arb.shape == (N,)
+    y = np.zeros((M, N), dtype=np.uint16)
+    z = np.zeros((M, N), dtype=np.float64)
+    _check(lib(parallel).oref_billm_linear(_p(xb), M, K, N, _p(bo1), _p(br1), _p(aob), _p(arb), _p(y),
+                                           _p(z)), "billm_linear")
+    return y.view(np.float16), z
 
 
 def rmsnorm(x: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:

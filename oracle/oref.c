@@ -10,6 +10,9 @@
  *   [ONEBIT] "清华、哈工大把大模型压缩到了1bit，把大模型放在手机里跑的愿望就快要实现了！"
  *          (OneBit), sections "1. 新的 1bit 结构", "2. 基于 SVID 初始化量化模型",
  *          "3. 通过知识蒸馏迁移原模型能力", "讨论与分析 / 1. 效率".
+ *   [BILLM] "BiLLM: Pushing the Limit of Post-Training Quantization for LLMs",
+ *          section "方法细节：残差近似与最优断点拆分", step 2 (binary residual
+ *          approximation).
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math (float arithmetic
  * is IEEE binary32 with round-to-nearest-even; no fused multiply-add).  A
@@ -376,3 +379,68 @@ int oref_swiglu(const uint16_t *a, const uint16_t *b, int n, uint16_t *y)
  * layer = N*K one-bit signs + (N + K) fp16 values. */
 int64_t oref_onebit_bits(int64_t N, int64_t K) { return N * K + 16 * (N + K); }
 int64_t oref_onebit_params(int64_t N, int64_t K) { return N * K + N + K; }
+
+/* ---------------------------------------------------------------------
+ * [BILLM] step 2, binary residual approximation: binarise W (alpha_o B_o),
+ * binarise what is left (alpha_r B_r), and use W ~ alpha_o B_o + alpha_r B_r.
+ * Readings (the page gives neither the granularity nor the formula of the
+ * scales): one scale per output row n; B = sign(.) with sign(0) = +1; alpha =
+ * the mean absolute value of the row being binarised, which is the scale that
+ * minimises || row - alpha B ||_2 once B = sign(row).  fp64 throughout.
+ * ------------------------------------------------------------------- */
+int oref_billm_binarize(const float *W, int N, int K, int8_t *Bo, int8_t *Br, double *alpha_o,
+                        double *alpha_r)
+{
+    if (N < 0 || K <= 0) return OREF_ERR_SHAPE;
+    for (int n = 0; n < N; ++n) {
+        const float *row = W + (size_t)n * K;
+        double so = 0.0;
+        for (int k = 0; k < K; ++k) so += fabs((double)row[k]);
+        const double ao = so / (double)K;
+        double sr = 0.0;
+        for (int k = 0; k < K; ++k) {
+            int8_t b = row[k] < 0.0f ? -1 : 1;
+            Bo[(size_t)n * K + k] = b;
+            sr += fabs((double)row[k] - ao * (double)b);
+        }
+        const double ar = sr / (double)K;
+        for (int k = 0; k < K; ++k) {
+            double r = (double)row[k] - ao * (double)Bo[(size_t)n * K + k];
+            Br[(size_t)n * K + k] = r < 0.0 ? -1 : 1;
+        }
+        alpha_o[n] = ao;
+        alpha_r[n] = ar;
+    }
+    return OREF_OK;
+}
+
+/* The two-plane binary linear layer: y = x W~^T with
+ *     W~[n][k] = alpha_o[n] B_o[n][k] + alpha_r[n] B_r[n][k],
+ * B_o and B_r as packed sign planes (the s1 format), alpha_o and alpha_r as
+ * fp16 [N] (the stored scales), activations fp16 and not quantised (the page:
+ * only the weights are binarised).  z = sum_k x_k W~[n][k] in fp64, in k
+ * order, y = fp16(z). */
+int oref_billm_linear(const uint16_t *x, int M, int K, int N, const uint32_t *bo1,
+                      const uint32_t *br1, const uint16_t *alpha_o, const uint16_t *alpha_r,
+                      uint16_t *y, double *z_out)
+{
+    if (M < 0 || N < 0 || K <= 0 || K % 32 != 0) return OREF_ERR_SHAPE;
+    const int words = K / 32;
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        const double ao = oref_half_to_double(alpha_o[n]);
+        const double ar = oref_half_to_double(alpha_r[n]);
+        for (int m = 0; m < M; ++m) {
+            double z = 0.0;
+            for (int k = 0; k < K; ++k) {
+                const int so = (bo1[(size_t)n * words + k / 32] >> (k % 32)) & 1 ? 1 : -1;
+                const int sr = (br1[(size_t)n * words + k / 32] >> (k % 32)) & 1 ? 1 : -1;
+                const double w = ao * (double)so + ar * (double)sr;
+                z += oref_half_to_double(x[(size_t)m * K + k]) * w;
+            }
+            y[(size_t)m * N + n] = oref_double_to_half(z);
+            if (z_out) z_out[(size_t)m * N + n] = z;
+        }
+    }
+    return OREF_OK;
+}

@@ -29,6 +29,11 @@ int oref_svid(const float *W, int N, int K, int8_t *S, double *a, double *b,
               double *sigma_out, int max_iter, double tol);
 int oref_rmsnorm(const uint16_t *x, int M, int K, const uint16_t *gamma, double eps, uint16_t *y);
 int oref_swiglu(const uint16_t *a, const uint16_t *b, int n, uint16_t *y);
+int oref_billm_binarize(const float *W, int N, int K, int8_t *Bo, int8_t *Br, double *alpha_o,
+                        double *alpha_r);
+int oref_billm_linear(const uint16_t *x, int M, int K, int N, const uint32_t *bo1,
+                      const uint32_t *br1, const uint16_t *alpha_o, const uint16_t *alpha_r,
+                      uint16_t *y, double *z_out);
 int64_t oref_onebit_bits(int64_t N, int64_t K);
 int64_t oref_onebit_params(int64_t N, int64_t K);
 

@@ -409,3 +409,77 @@ def test_swiglu_identities(oref):
     assert yb[0] == np.float16(30.0) and abs(float(yb[1])) < 1e-10
     b = np.full_like(a, 2.0)
     assert np.array_equal(oref.swiglu(a, b).astype(np.float64), 2 * oref.swiglu(a, one).astype(np.float64))
+
+
+# ---- BiLLM binary residual approximation (oracle.billm_binarize / billm_linear)
+
+def _pad32(rows):
+    """Pad int8 +-1 rows to 32 columns with +1 (zero x there) for the s1 packing."""
+    out = np.ones((rows.shape[0], 32), dtype=np.int8)
+    out[:, :rows.shape[1]] = rows
+    return out
+
+
+def test_billm_hand_worked_rows(oref):
+    g = _golden_rows("billm_residual_2x4.txt")
+    W = np.array([[float(v) for v in g["w0"]], [float(v) for v in g["w1"]]], dtype=np.float32)
+    Bo, Br, ao, ar = oref.billm_binarize(W)
+    assert Bo.tolist() == [[int(v) for v in g["bo0"]], [int(v) for v in g["bo1"]]]
+    assert Br.tolist() == [[int(v) for v in g["br0"]], [int(v) for v in g["br1"]]]
+    assert ao.tolist() == [float(v) for v in g["alpha_o"]]
+    assert ar.tolist() == [float(v) for v in g["alpha_r"]]
+    assert (ao[0] * Bo[0] + ar[0] * Br[0]).tolist() == [float(v) for v in g["approx0"]]
+    # the linear layer on those planes (zero-padded to one 32-bit word)
+    x = np.zeros((1, 32), dtype=np.float16)
+    x[0, :4] = [float(v) for v in g["x"]]
+    bo1 = oref.pack_sign(_pad32(Bo).astype(np.float16))
+    br1 = oref.pack_sign(_pad32(Br).astype(np.float16))
+    y, z = oref.billm_linear(x, bo1, br1, ao.astype(np.float16), ar.astype(np.float16))
+    assert z[0].tolist() == [float(v) for v in g["y"]]
+
+
+def test_billm_residual_never_worse_and_scales_optimal(oref):
+    """The page's property: the residual approximation's error is at most that
+    of plain binarisation.  And each alpha is the least-squares scale of its
+    sign plane: moving it either way increases the row's error."""
+    rng = np.random.default_rng(9)
+    W = (rng.standard_normal((16, 512)) * 0.02).astype(np.float32)
+    W[3] = rng.laplace(size=512).astype(np.float32)            # heavier tails
+    Bo, Br, ao, ar = oref.billm_binarize(W)
+    Wd = W.astype(np.float64)
+    e1 = np.sum((Wd - ao[:, None] * Bo) ** 2, axis=1)
+    e2 = np.sum((Wd - ao[:, None] * Bo - ar[:, None] * Br) ** 2, axis=1)
+    assert (e2 <= e1).all() and (e2 < 0.6 * e1).all()
+    assert np.array_equal(Bo, np.where(W < 0, -1, 1))
+    R = Wd - ao[:, None] * Bo
+    assert np.array_equal(Br, np.where(R < 0, -1, 1))
+    for f in (1 - 1e-3, 1 + 1e-3):
+        assert (np.sum((Wd - f * ao[:, None] * Bo) ** 2, axis=1) > e1).all()
+        assert (np.sum((R - f * ar[:, None] * Br) ** 2, axis=1) >
+                np.sum((R - ar[:, None] * Br) ** 2, axis=1)).all()
+
+
+def test_billm_linear_against_dense_and_special_cases(oref):
+    """z equals the dense fp64 product with alpha_o B_o + alpha_r B_r; with
+    B_r = B_o it is (alpha_o + alpha_r) x B_o^T; with alpha_r = 0 it is the
+    OneBit layer with g = 1 and h = alpha_o."""
+    rng = np.random.default_rng(11)
+    M, K, N = 3, 256, 48
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    Bo = np.where(rng.random((N, K)) < 0.5, -1, 1).astype(np.int8)
+    Br = np.where(rng.random((N, K)) < 0.5, -1, 1).astype(np.int8)
+    ao = rng.uniform(0.01, 0.03, N).astype(np.float16)
+    ar = rng.uniform(0.002, 0.01, N).astype(np.float16)
+    bo1, br1 = oref.pack_sign(Bo.astype(np.float16)), oref.pack_sign(Br.astype(np.float16))
+    y, z = oref.billm_linear(x, bo1, br1, ao, ar)
+    dense = ao.astype(np.float64)[:, None] * Bo + ar.astype(np.float64)[:, None] * Br
+    ref = x.astype(np.float64) @ dense.T
+    assert np.max(np.abs(z - ref)) <= 1e-12 * np.max(np.abs(ref))
+    assert np.array_equal(y, ref.astype(np.float16)) or \
+        np.max(np.abs(y.astype(np.float64) - ref)) <= 2.0 ** -10 * np.max(np.abs(ref))
+    _, z_same = oref.billm_linear(x, bo1, bo1, ao, ar)
+    ref_same = (ao.astype(np.float64) + ar.astype(np.float64)) * (x.astype(np.float64) @ Bo.T.astype(np.float64))
+    assert np.max(np.abs(z_same - ref_same)) <= 1e-12 * np.max(np.abs(ref_same))
+    _, z_zero = oref.billm_linear(x, bo1, br1, ao, np.zeros(N, dtype=np.float16))
+    _, z_ob = oref.ob_linear(x, bo1, np.ones(K, dtype=np.float16), ao)
+    assert np.max(np.abs(z_zero - z_ob)) <= 1e-12 * np.max(np.abs(z_ob))
