@@ -434,7 +434,8 @@ def run_sweep(blw, synth, dev, peaks, reps=10, forms=("ternary", "onebit"), laye
     out = []
     for form in forms:
         for (name, K, N) in layers:
-            wb = N * K // (4 if form == "ternary" else 8)
+            planes = 2 if form == "billm" else 1        # BiLLM: two stacked sign planes
+            wb = planes * N * K // (4 if form == "ternary" else 8)
             copies = max(2, -(-2 * l2_bytes // wb) + 1)
             ws, gs, hs = [], None, None
             for c in range(copies):
@@ -443,29 +444,35 @@ def run_sweep(blw, synth, dev, peaks, reps=10, forms=("ternary", "onebit"), laye
                     w = synth.ternary_weights(N, K, seed=seed, device=dev)
                     ws.append(blw.bl_pack_ternary(w))
                 else:
-                    w = synth.sign_weights(N, K, seed=seed, device=dev)
+                    w = synth.sign_weights(planes * N, K, seed=seed, device=dev)
                     ws.append(blw.ob_pack_sign(w))
                 del w
             if form == "onebit":
                 gs = synth.value_vector(K, seed=4_000_900, device=dev)
                 hs = synth.value_vector(N, seed=4_000_901, device=dev)
+            if form == "billm":
+                hs = synth.value_vector(2 * N, seed=4_000_902, device=dev)    # alpha_o, alpha_r
             for M in ms_list:
                 x = synth.activations(M, K, seed=4_001_000 + M, device=dev)
                 y = torch.empty((M, N), dtype=torch.float16, device=dev)
-                nws = (blw.bl_ternary_workspace_bytes if form == "ternary" else blw.ob_workspace_bytes)(M, K, N)
+                nws = {"ternary": blw.bl_ternary_workspace_bytes, "onebit": blw.ob_workspace_bytes,
+                       "billm": blw.billm_workspace_bytes}[form](M, K, N)
                 wsp = torch.empty((nws,), dtype=torch.uint8, device=dev)
 
                 def step():
                     for w2 in ws:
                         if form == "ternary":
                             blw.bl_ternary_linear(x, w2, W_SCALE, workspace=wsp, out=y)
+                        elif form == "billm":
+                            blw.billm_linear(x, w2, hs, workspace=wsp, out=y)
                         else:
                             blw.ob_linear(x, w2, gs, hs, workspace=wsp, out=y)
 
                 g = capture(step)
                 ms = time_replays(g, reps, 3, False, dev) / copies
-                gbs = (wb + (2 * (K + N) if form == "onebit" else 0)) / (ms * 1e-3) / 1e9
-                tops = 2 * M * K * N / (ms * 1e-3) / 1e12
+                vec = {"ternary": 0, "onebit": 2 * (K + N), "billm": 4 * N}[form]
+                gbs = (wb + vec) / (ms * 1e-3) / 1e9
+                tops = 2 * planes * M * K * N / (ms * 1e-3) / 1e12
                 out.append({"form": form, "layer": f"{name} {K}->{N}", "M": M, "us_per_call": round(ms * 1e3, 2),
                             "weight_GBs": round(gbs, 1), "TOPS": round(tops, 2),
                             "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
@@ -707,6 +714,30 @@ def main():
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
 
+        # ---- SVID initialisation of the OneBit 4096x4096 layer on the device
+        W = synth.svid_weights(4096, 4096, seed=1_000_001, device=dev)
+        for _ in range(3):
+            blw.ob_svid(W)
+        sv_ms = []
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            _s1, _g, _h, sv_sigma, sv_it = blw.ob_svid(W)
+            e1.record()
+            torch.cuda.synchronize()
+            sv_ms.append(e0.elapsed_time(e1))
+        sv_med = sorted(sv_ms)[len(sv_ms) // 2]
+        sv_passes = 1 + 2 * sv_it                   # sign pass + a row and a column pass per iteration
+        extras["svid_4096x4096"] = {
+            "workload": "ob_svid of a 4096x4096 N(0, 0.02) fp32 W (sign pack + rank-1 power iteration "
+                        "of |W| in fp64, tol 1e-12)",
+            "ms": round(sv_med, 4), "iterations": sv_it, "sigma": sv_sigma,
+            "w_passes": sv_passes,
+            "w_GBs": round(sv_passes * W.numel() * 4 / (sv_med * 1e-3) / 1e9, 1),
+            "note": "includes the call's host read-backs of the convergence flag; W (64 MB) stays in L2"}
+        del W, _s1, _g, _h
+        torch.cuda.synchronize()
+
         # ---- the per-call path: 224 bl_ternary_linear / ob_linear calls per step in a graph
         for form in ("ternary", "onebit"):
             pcalls, pwbytes, _px, _py = decode_stack(blw, synth, dev, form, layers=args.layers)
@@ -729,6 +760,10 @@ def main():
                                                 layers=[("q", 4096, 4096)], ms_list=[8])
         extras["onebit_4096"] = run_sweep(blw, synth, dev, peaks, forms=("onebit",),
                                           layers=[("q", 4096, 4096)], ms_list=[1, 16])
+        # the two-plane binary layer (BiLLM residual approximation) on the same shapes
+        extras["billm_4096"] = run_sweep(blw, synth, dev, peaks, forms=("billm",),
+                                         layers=[("q", 4096, 4096), ("up", 4096, 11008)],
+                                         ms_list=[1, 16, 256])
         # the decode sweep per layer shape: each 7B-shaped layer alone at M=1, in a
         # chain of calls over rotating weight copies larger than L2
         extras["decode_layers_7b"] = run_sweep(blw, synth, dev, peaks, forms=("ternary", "onebit"),

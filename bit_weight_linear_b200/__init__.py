@@ -61,6 +61,11 @@ ABI = {
     "bl_prefill_plan": ([_I, _I, _I, _I, _I, _P], _I),
     "bl_ternary_linear_noalloc": ([_P, _I, _I, _I, _P, ctypes.c_float, _P, _P, _P], _I),
     "bl_debug_stall_next_launch": ([ctypes.c_ulonglong], _I),
+    "ob_svid_workspace_bytes": ([_I, _I], _SZ),
+    "ob_svid": ([_P, _I, _I, _I, ctypes.c_double, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "billm_workspace_bytes": ([_I, _I, _I], _SZ),
+    "billm_linear": ([_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P], _I),
+    "billm_binarize": ([_P, _I, _I, _P, _P, _P, _P, _P], _I),
     "bl_chain_bytes": ([_I], _SZ),
     "bl_chain_build": ([_I, _P, _I, _P, _SZ, _P, _P], _I),
     "bl_chain_run": ([_P, _P, _P], _I),
@@ -131,6 +136,65 @@ def ob_pack_sign(w: torch.Tensor) -> torch.Tensor:
     s1 = torch.empty((N, K // 32), dtype=torch.int32, device=w.device)
     _check("ob_pack_sign", lib().ob_pack_sign(_ptr(w), N, K, _ptr(s1), _stream()))
     return s1
+
+
+def ob_svid(W: torch.Tensor, max_iter: int = 1000, tol: float = 1e-12, return_ab: bool = False):
+    """SVID of fp32 W [N,K] (CUDA) on the device: returns (s1 packed signs
+    [N, K/32], g fp16 [K], h fp16 [N], sigma, iterations), plus fp64 a [N] and
+    b [K] when return_ab."""
+    _need_cuda(W)
+    assert W.dtype == torch.float32 and W.dim() == 2
+    N, K = W.shape
+    dev = W.device
+    s1 = torch.empty((N, K // 32), dtype=torch.int32, device=dev)
+    g = torch.empty((K,), dtype=torch.float16, device=dev)
+    h = torch.empty((N,), dtype=torch.float16, device=dev)
+    a = torch.empty((N,), dtype=torch.float64, device=dev) if return_ab else None
+    b = torch.empty((K,), dtype=torch.float64, device=dev) if return_ab else None
+    nws = int(lib().ob_svid_workspace_bytes(N, K))
+    if nws == 0:
+        raise BitLinearError("ob_svid", 2)
+    ws = torch.empty((nws,), dtype=torch.uint8, device=dev)
+    sigma, iters = ctypes.c_double(0.0), ctypes.c_int(0)
+    _check("ob_svid", lib().ob_svid(_ptr(W), N, K, int(max_iter), float(tol), _ptr(s1), _ptr(g), _ptr(h),
+                                    _ptr(a), _ptr(b), ctypes.byref(sigma), ctypes.byref(iters), _ptr(ws),
+                                    nws, _stream()))
+    out = (s1, g, h, sigma.value, iters.value)
+    return out + (a, b) if return_ab else out
+
+
+def billm_binarize(W: torch.Tensor, return_alpha64: bool = False):
+    """Residual binarisation of fp32 W [N,K] (CUDA): returns (b2 stacked sign
+    planes [2N, K/32], alpha fp16 [2N]), plus fp64 alpha_o, alpha_r [N] when
+    return_alpha64."""
+    _need_cuda(W)
+    assert W.dtype == torch.float32 and W.dim() == 2
+    N, K = W.shape
+    b2 = torch.empty((2 * N, K // 32), dtype=torch.int32, device=W.device)
+    alpha = torch.empty((2 * N,), dtype=torch.float16, device=W.device)
+    ao = torch.empty((N,), dtype=torch.float64, device=W.device) if return_alpha64 else None
+    ar = torch.empty((N,), dtype=torch.float64, device=W.device) if return_alpha64 else None
+    _check("billm_binarize", lib().billm_binarize(_ptr(W), N, K, _ptr(b2), _ptr(alpha), _ptr(ao), _ptr(ar),
+                                                  _stream()))
+    return (b2, alpha, ao, ar) if return_alpha64 else (b2, alpha)
+
+
+def billm_linear(x: torch.Tensor, b2: torch.Tensor, alpha: torch.Tensor, *,
+                 workspace: torch.Tensor | None = None, out: torch.Tensor | None = None):
+    """Two-plane binary forward: y = alpha_o * (x B_o^T) + alpha_r * (x B_r^T),
+    fp16 in/out; b2 = [B_o; B_r] packed [2N, K/32], alpha = [alpha_o; alpha_r]."""
+    _need_cuda(x, b2, alpha)
+    M, K = x.shape
+    N = b2.shape[0] // 2
+    nws = int(lib().billm_workspace_bytes(M, K, N))
+    if nws == 0 and M > 0 and N > 0:
+        raise BitLinearError("billm_linear", 2)
+    ws = workspace if workspace is not None else torch.empty((max(nws, 1),), dtype=torch.uint8,
+                                                             device=x.device)
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _check("billm_linear", lib().billm_linear(_ptr(x), M, K, N, _ptr(b2), _ptr(alpha), _ptr(y), _ptr(ws),
+                                              ws.numel(), _stream()))
+    return y
 
 
 def bl_quant_act(x: torch.Tensor):

@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libbitlinear.so")
 SOURCES = ["api.cu", "pack.cu", "quant.cu", "skinny.cu", "prefill.cu", "stream.cu", "chain.cu",
-           "noalloc.cu"]
+           "noalloc.cu", "svid.cu", "billm.cu"]
 HEADERS = ["act_groups.cuh", "common.cuh", "decode_forms.cuh", "kernels.h", "tc_prims.cuh", "tmap.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

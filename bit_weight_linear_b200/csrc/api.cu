@@ -252,6 +252,33 @@ size_t ob_workspace_bytes(int M, int K, int N) {
     return ws_layout(1, M, K, N).total;
 }
 
+// The OneBit forward (argument checks done): the fused streamed kernel for the
+// smallest M, else activation preparation and then the streamed, skinny or
+// tensor-core contraction.  zf: optional fp32 copy of the output.
+static bl_status onebit_forward(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
+                                const uint16_t* g, const uint16_t* h, uint16_t* y, float* zf,
+                                char* ws, const WsLayout& l, cudaStream_t s) {
+    unsigned int* flags = device_flags();
+    if (!flags) return BL_ERR_CUDA;
+    if (M <= bl::kStreamFusedMaxMOnebit && bl::stream_fits(1, M, K, N, 0))
+        return from_cuda(bl::launch_onebit_stream(x, g, h, s1, M, K, N, y, flags, s, zf));
+    int8_t* planes = reinterpret_cast<int8_t*>(ws + l.act);
+    float* step = reinterpret_cast<float*>(ws + l.scale);
+    long long* ts = reinterpret_cast<long long*>(ws + l.rsum);
+    unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + l.split);
+    cudaError_t e = bl::launch_prep_onebit(x, g, M, K, planes, step, ts, s, ctr, l.n_ctr);
+    if (e != cudaSuccess) return BL_ERR_CUDA;
+    if (M >= bl::kOnebitPrefillMinM) {
+        e = bl::launch_onebit_prefill(s1, planes, step, ts, h, M, K, N, y, flags, s, ws + l.split,
+                                      l.split_bytes, zf);
+    } else {
+        e = bl::stream_fits(1, M, K, N, 1)
+                ? bl::launch_onebit_stream_prepared(planes, step, ts, h, s1, M, K, N, y, flags, s, zf)
+                : bl::launch_onebit_skinny(s1, planes, step, ts, h, M, K, N, y, s, zf);
+    }
+    return from_cuda(e);
+}
+
 bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
                     const uint16_t* g, const uint16_t* h, uint16_t* y, void* workspace,
                     size_t workspace_bytes, bl_stream_t stream) {
@@ -266,27 +293,100 @@ bl_status ob_linear(const uint16_t* x, int M, int K, int N, const uint32_t* s1,
     if (!workspace || workspace_bytes < l.total) return BL_ERR_WORKSPACE;
     if (misaligned(workspace)) return BL_ERR_ALIGN;
     if (bl_status st = bl::fault_injected()) return st;
-    unsigned int* flags = device_flags();
-    if (!flags) return BL_ERR_CUDA;
-    if (M <= bl::kStreamFusedMaxMOnebit && bl::stream_fits(1, M, K, N, 0))
-        return from_cuda(bl::launch_onebit_stream(x, g, h, s1, M, K, N, y, flags, cs(stream)));
+    return onebit_forward(x, M, K, N, s1, g, h, y, nullptr, static_cast<char*>(workspace), l,
+                          cs(stream));
+}
+
+// Two-plane binary layer: the OneBit forward over the stacked planes (2N rows,
+// g = 1, h = alpha) writes fp32 products zf [M][2N] (and an fp16 copy in
+// scratch), then y = fp16(zf[:, :N] + zf[:, N:]).
+//   workspace: OneBit layout for (M, K, 2N) | zf M*2N fp32 | scratch y M*2N fp16
+struct BillmWs {
+    WsLayout ob;
+    size_t zf, ysc, total;
+};
+
+static BillmWs billm_ws(int M, int K, int N) {
+    BillmWs b;
+    b.ob = ws_layout(1, M, K, 2 * N);
+    b.zf = b.ob.total;
+    b.ysc = b.zf + align_up((size_t)M * 2 * N * sizeof(float));
+    b.total = b.ysc + align_up((size_t)M * 2 * N * sizeof(uint16_t));
+    return b;
+}
+
+static bl_status check_billm_shape(int M, int K, int N) {
+    if (bl_status st = check_mk(M, K)) return st;
+    if (bl_status st = check_nk(N, K)) return st;
+    if (K > 65536 || N > (1 << 23)) return BL_ERR_SHAPE;
+    return BL_OK;
+}
+
+size_t billm_workspace_bytes(int M, int K, int N) {
+    if (check_billm_shape(M, K, N) != BL_OK) return 0;
+    return billm_ws(M, K, N).total;
+}
+
+bl_status billm_linear(const uint16_t* x, int M, int K, int N, const uint32_t* b2,
+                       const uint16_t* alpha, uint16_t* y, void* workspace, size_t workspace_bytes,
+                       bl_stream_t stream) {
+    if (bl_status st = check_billm_shape(M, K, N)) return st;
+    if (M == 0 || N == 0) return BL_OK;
+    if (!x || !b2 || !alpha || !y) return BL_ERR_NULL;
+    if (misaligned(x) || misaligned(b2) || misaligned(alpha) || misaligned(y)) return BL_ERR_ALIGN;
+    const BillmWs l = billm_ws(M, K, N);
+    if (!workspace || workspace_bytes < l.total) return BL_ERR_WORKSPACE;
+    if (misaligned(workspace)) return BL_ERR_ALIGN;
+    if (bl_status st = bl::fault_injected()) return st;
     char* ws = static_cast<char*>(workspace);
-    int8_t* planes = reinterpret_cast<int8_t*>(ws + l.act);
-    float* step = reinterpret_cast<float*>(ws + l.scale);
-    long long* ts = reinterpret_cast<long long*>(ws + l.rsum);
-    unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + l.split);
-    cudaError_t e = bl::launch_prep_onebit(x, g, M, K, planes, step, ts, cs(stream), ctr, l.n_ctr);
-    if (e != cudaSuccess) return BL_ERR_CUDA;
-    if (M >= bl::kOnebitPrefillMinM) {
-        e = bl::launch_onebit_prefill(s1, planes, step, ts, h, M, K, N, y, flags, cs(stream),
-                                      ws + l.split, l.split_bytes);
-    } else {
-        e = bl::stream_fits(1, M, K, N, 1)
-                ? bl::launch_onebit_stream_prepared(planes, step, ts, h, s1, M, K, N, y, flags,
-                                                    cs(stream))
-                : bl::launch_onebit_skinny(s1, planes, step, ts, h, M, K, N, y, cs(stream));
-    }
-    return from_cuda(e);
+    float* zf = reinterpret_cast<float*>(ws + l.zf);
+    uint16_t* ysc = reinterpret_cast<uint16_t*>(ws + l.ysc);
+    if (bl_status st = onebit_forward(x, M, K, 2 * N, b2, nullptr, alpha, ysc, zf, ws, l.ob, cs(stream)))
+        return st;
+    return from_cuda(bl::launch_billm_combine(zf, M, N, y, cs(stream)));
+}
+
+bl_status billm_binarize(const float* W, int N, int K, uint32_t* b2, uint16_t* alpha,
+                         double* alpha_o, double* alpha_r, bl_stream_t stream) {
+    if (bl_status st = check_nk(N, K)) return st;
+    if (N > (1 << 23)) return BL_ERR_SHAPE;
+    if (N == 0) return BL_OK;
+    if (!W || !b2 || !alpha) return BL_ERR_NULL;
+    if (misaligned(W) || misaligned(b2) || misaligned(alpha) || misaligned(alpha_o) ||
+        misaligned(alpha_r))
+        return BL_ERR_ALIGN;
+    if (bl_status st = bl::fault_injected()) return st;
+    unsigned int* flag = nullptr;
+    if (bl_status st = pack_begin(&flag, cs(stream))) return st;
+    return pack_finish(bl::launch_billm_binarize(W, N, K, b2, alpha, alpha_o, alpha_r, flag, cs(stream)),
+                       cs(stream));
+}
+
+static bl_status check_svid_shape(int N, int K) {
+    if (bl_status st = check_nk(N, K)) return st;
+    if (N > bl::svid_max_n()) return BL_ERR_SHAPE;
+    return BL_OK;
+}
+
+size_t ob_svid_workspace_bytes(int N, int K) {
+    if (check_svid_shape(N, K) != BL_OK || N == 0) return 0;
+    return bl::svid_workspace_bytes(N, K);
+}
+
+bl_status ob_svid(const float* W, int N, int K, int max_iter, double tol, uint32_t* s1, uint16_t* g,
+                  uint16_t* h, double* a, double* b, double* sigma, int* iters, void* workspace,
+                  size_t workspace_bytes, bl_stream_t stream) {
+    if (bl_status st = check_svid_shape(N, K)) return st;
+    if (max_iter < 1 || !(tol >= 0.0)) return BL_ERR_SHAPE;
+    if (N == 0) return BL_OK;
+    if (!W || !s1 || !g || !h) return BL_ERR_NULL;
+    if (misaligned(W) || misaligned(s1) || misaligned(g) || misaligned(h) || misaligned(a) ||
+        misaligned(b))
+        return BL_ERR_ALIGN;
+    if (!workspace || workspace_bytes < bl::svid_workspace_bytes(N, K)) return BL_ERR_WORKSPACE;
+    if (misaligned(workspace)) return BL_ERR_ALIGN;
+    if (bl_status st = bl::fault_injected()) return st;
+    return bl::svid_run(W, N, K, max_iter, tol, s1, g, h, a, b, sigma, iters, workspace, cs(stream));
 }
 
 bl_status bl_prefill_plan(int form, int M, int K, int N, int sm_count, int* plan) {

@@ -45,6 +45,12 @@ __device__ __forceinline__ uint4 ld_ro_v4(const void* p) {
     return __ldg(reinterpret_cast<const uint4*>(p));
 }
 
+// A chunk of 8 elements of a OneBit input value vector; g == nullptr stands
+// for g = 1 (the two-plane binary layer, whose inputs are not scaled).
+__device__ __forceinline__ uint4 ld_gvec(const uint16_t* g, size_t off) {
+    return g ? ld_ro_v4(g + off) : make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

@@ -40,9 +40,11 @@ cudaError_t launch_prep_onebit(const uint16_t* x, const uint16_t* g, int M, int 
 cudaError_t launch_ternary_skinny(const uint32_t* w2, const int8_t* qp, const float* scale,
                                   const int32_t* qsum, int M, int K, int N, float w_scale,
                                   uint16_t* y, int32_t* acc_out, cudaStream_t s);
+// OneBit launchers take an optional zf: an fp32 [M][N] copy of the output
+// (z (.) h) before its fp16 rounding, for the two-plane binary layer.
 cudaError_t launch_onebit_skinny(const uint32_t* s1, const int8_t* planes, const float* step,
                                  const long long* tsum, const uint16_t* h, int M, int K, int N,
-                                 uint16_t* y, cudaStream_t s);
+                                 uint16_t* y, cudaStream_t s, float* zf = nullptr);
 
 // Prefill-shaped (large M) GEMM on tcgen05 int8 tensor cores with TMEM
 // accumulators (prefill.cu).  `flags` is the device condition word that bounded
@@ -65,7 +67,8 @@ cudaError_t launch_ternary_prefill(const uint32_t* w2, const int8_t* qp, const f
 cudaError_t launch_onebit_prefill(const uint32_t* s1, const int8_t* planes, const float* step,
                                   const long long* tsum, const uint16_t* h, int M, int K, int N,
                                   uint16_t* y, unsigned int* flags, cudaStream_t s,
-                                  void* split_ws = nullptr, size_t split_ws_bytes = 0);
+                                  void* split_ws = nullptr, size_t split_ws_bytes = 0,
+                                  float* zf = nullptr);
 
 // Number of SMs of the current device (cached per device; 0 on error).
 int device_sm_count();
@@ -103,7 +106,7 @@ cudaError_t launch_ternary_stream(const uint16_t* x, const uint32_t* w2, int M, 
                                   cudaStream_t s);
 cudaError_t launch_onebit_stream(const uint16_t* x, const uint16_t* g, const uint16_t* h,
                                  const uint32_t* s1, int M, int K, int N, uint16_t* y,
-                                 unsigned int* flags, cudaStream_t s);
+                                 unsigned int* flags, cudaStream_t s, float* zf = nullptr);
 cudaError_t launch_ternary_stream_prepared(const int8_t* qp, const float* scale, const int32_t* qsum,
                                            const uint32_t* w2, int M, int K, int N, float w_scale,
                                            uint16_t* y, int32_t* acc_out, unsigned int* flags,
@@ -111,14 +114,28 @@ cudaError_t launch_ternary_stream_prepared(const int8_t* qp, const float* scale,
 cudaError_t launch_onebit_stream_prepared(const int8_t* planes, const float* step,
                                           const long long* tsum, const uint16_t* h,
                                           const uint32_t* s1, int M, int K, int N, uint16_t* y,
-                                          unsigned int* flags, cudaStream_t s);
+                                          unsigned int* flags, cudaStream_t s, float* zf = nullptr);
 
 // Persistent single-token decode over a list of layers (chain.cu): device
 // descriptors (tensor maps, tile plan) written by chain_build into the caller's
 // `chain` buffer of chain_bytes(n) bytes, one cooperative launch per run.
 size_t chain_bytes(int n_layers);
 int chain_max_k(int form);
-int chain_max_fused_k(int form);   // longest row the RMSNorm / SwiGLU prologues take
+int chain_max_fused_k(int form);
+
+// Two-plane binary layer (billm.cu): y = fp16(zf[:, :N] + zf[:, N:]) from the
+// OneBit forward's fp32 outputs over the stacked planes, and the residual
+// binarisation of a weight into those planes and scales.
+cudaError_t launch_billm_combine(const float* zf, int M, int N, uint16_t* y, cudaStream_t s);
+cudaError_t launch_billm_binarize(const float* W, int N, int K, uint32_t* b2, uint16_t* alpha,
+                                  double* ao, double* ar, unsigned int* bad_flag, cudaStream_t s);
+
+// SVID initialisation of a OneBit layer (svid.cu)
+int svid_max_n();
+size_t svid_workspace_bytes(int N, int K);
+bl_status svid_run(const float* W, int N, int K, int max_iter, double tol, uint32_t* s1, uint16_t* g,
+                   uint16_t* h, double* a, double* b, double* sigma, int* iters, void* workspace,
+                   cudaStream_t s);   // longest row the RMSNorm / SwiGLU prologues take
 bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain, size_t bytes,
                       bl_chain_plan* plan, cudaStream_t s);
 bl_status chain_run(const bl_chain_plan* plan, const void* chain, unsigned int* flags,

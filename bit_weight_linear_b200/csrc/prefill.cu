@@ -102,6 +102,7 @@ struct PrefillParams {
     uint16_t* y;
     int32_t* acc_out;
     unsigned int* flags;
+    float* zf;            // OneBit: optional fp32 [M][N] copy of y before fp16 rounding
     // Work split.  CTAs [0, dp_tiles) each compute one whole tile.  The
     // remaining sk_tiles tiles form one balanced round: CTA dp_tiles + c
     // (c < sk_ctas) takes the (tile, k-stage) units [c U / G, (c+1) U / G) of
@@ -192,7 +193,7 @@ __device__ __forceinline__ void convert_chunk(const uint32_t (&d)[32], int cc, u
 __device__ __forceinline__ void convert_onebit_group(const uint32_t (&d)[96], int gi,
                                                      uint16_t* stage, const float* tok_scale,
                                                      const long long* tok_xsum, int tpt, int r,
-                                                     float hn) {
+                                                     float hn, const PrefillParams& p, int n, int t0) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const int t = 32 * gi + i;
@@ -200,7 +201,9 @@ __device__ __forceinline__ void convert_onebit_group(const uint32_t (&d)[96], in
             const long long Z = limb_combine((int)d[3 * i], (int)d[3 * i + 1], (int)d[3 * i + 2],
                                              tok_xsum[t]);
             const float z = __fmul_rn(tok_scale[t], (float)Z);
-            stage[t * BW + r] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hn)));
+            const float zh = __fmul_rn(z, hn);
+            stage[t * BW + r] = __half_as_ushort(__float2half_rn(zh));
+            if (p.zf && t0 + t < p.M && n < p.N) p.zf[(size_t)(t0 + t) * p.N + n] = zh;
         }
     }
 }
@@ -406,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc::tmem_ld_32x32b_x32(lane_base + kAccCol + 32 * (3 * gi + c),
                                                    *reinterpret_cast<uint32_t(*)[32]>(d + 32 * c));
                     tc::tmem_ld_wait();
-                    convert_onebit_group(d, gi, stage, tok_scale, tok_xsum, p.tpt, r, hn);
+                    convert_onebit_group(d, gi, stage, tok_scale, tok_xsum, p.tpt, r, hn, p, n, t0);
                 }
             }
             tc::fence_proxy_async_smem();
@@ -798,7 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < 3; ++c)
                         if (3 * gi + c < nch)
                             add_parts(*reinterpret_cast<uint32_t(*)[32]>(d + 32 * c), 3 * gi + c);
-                    convert_onebit_group(d, gi, stage, tok_scale, tok_xsum, p.tpt, r, hn);
+                    convert_onebit_group(d, gi, stage, tok_scale, tok_xsum, p.tpt, r, hn, p, n, t0);
                 }
             }
             tc::tc_fence_before();
@@ -999,16 +1002,16 @@ cudaError_t launch_ternary_prefill(const uint32_t* w2, const int8_t* qp, const f
                                    cudaStream_t s, void* split_ws, size_t split_ws_bytes) {
     if (M == 0 || N == 0) return cudaSuccess;
     PrefillParams p{M, 0, 0, 0, M, K, N, scale, qsum, nullptr, nullptr, w_scale, y, acc_out,
-                    flags, 0, 0, 0, nullptr, nullptr, 0, 0};
+                    flags, nullptr, 0, 0, 0, nullptr, nullptr, 0, 0};
     return launch_prefill<0>(qp, w2, p, split_ws, split_ws_bytes, s);
 }
 
 cudaError_t launch_onebit_prefill(const uint32_t* s1, const int8_t* planes, const float* step,
                                   const long long* tsum, const uint16_t* h, int M, int K, int N,
                                   uint16_t* y, unsigned int* flags, cudaStream_t s,
-                                  void* split_ws, size_t split_ws_bytes) {
+                                  void* split_ws, size_t split_ws_bytes, float* zf) {
     if (M == 0 || N == 0) return cudaSuccess;
-    PrefillParams p{3 * M, 0, 0, 0, M, K, N, step, nullptr, tsum, h, 0.f, y, nullptr, flags,
+    PrefillParams p{3 * M, 0, 0, 0, M, K, N, step, nullptr, tsum, h, 0.f, y, nullptr, flags, zf,
                     0, 0, 0, nullptr, nullptr, 0, 0};
     return launch_prefill<1>(planes, s1, p, split_ws, split_ws_bytes, s);
 }

@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* _
     float mx = 0.f;
     for (int c = threadIdx.x; c < K / 8; c += kThreads) {
         uint4 v = tc::ld_v4(row + 8 * c);
-        uint4 gv = ld_ro_v4(g + 8 * c);
+        uint4 gv = ld_gvec(g, 8 * c);
         uint32_t xs[4] = {v.x, v.y, v.z, v.w}, gs[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(kThreads) prep_onebit_kernel(const uint16_t* _
 #pragma unroll
         for (int part = 0; part < 4; ++part) {
             uint4 v = tc::ld_v4(row + 32 * c + 8 * part);
-            uint4 gv = ld_ro_v4(g + 32 * c + 8 * part);
+            uint4 gv = ld_gvec(g, 32 * c + 8 * part);
             uint32_t xs[4] = {v.x, v.y, v.z, v.w}, gs[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -365,7 +365,7 @@ __global__ void __launch_bounds__(kRegThreads, 1)
 #pragma unroll
             for (int part = 0; part < 4; ++part) {
                 const uint4 v = tc::ld_v4(row + 32 * c + 8 * part);
-                const uint4 gv = ld_ro_v4(g + 32 * c + 8 * part);
+                const uint4 gv = ld_gvec(g, 32 * c + 8 * part);
                 const uint32_t xs[4] = {v.x, v.y, v.z, v.w}, gs[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {

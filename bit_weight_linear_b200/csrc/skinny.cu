@@ -70,6 +70,7 @@ struct SkinnyParams {
     int M, K, N;
     uint16_t* y;            // fp16 [M][N]
     int32_t* acc_out;       // ternary optional int32 [M][N]
+    float* zf;              // onebit optional fp32 [M][N] copy of y before fp16 rounding
 };
 
 template <int FORM, int NT>
@@ -189,7 +190,9 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyParams p) 
             const int n = blockIdx.x * 16 + r;
             const float z = __fmul_rn(p.scale[tok], (float)Z);
             const float hv = __half2float(__ushort_as_half(p.h[n]));
-            p.y[(size_t)tok * p.N + n] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hv)));
+            const float zh = __fmul_rn(z, hv);
+            p.y[(size_t)tok * p.N + n] = __half_as_ushort(__float2half_rn(zh));
+            if (p.zf) p.zf[(size_t)tok * p.N + n] = zh;
         }
     }
 }
@@ -210,7 +213,7 @@ cudaError_t launch_ternary_skinny(const uint32_t* w2, const int8_t* qp, const fl
                                   const int32_t* qsum, int M, int K, int N, float w_scale,
                                   uint16_t* y, int32_t* acc_out, cudaStream_t s) {
     if (M == 0 || N == 0) return cudaSuccess;
-    SkinnyParams p{w2, qp, scale, qsum, nullptr, nullptr, w_scale, M, K, N, y, acc_out};
+    SkinnyParams p{w2, qp, scale, qsum, nullptr, nullptr, w_scale, M, K, N, y, acc_out, nullptr};
     if (M <= 8) return launch<0, 1>(p, s);
     if (M <= 16) return launch<0, 2>(p, s);
     return launch<0, 4>(p, s);
@@ -218,9 +221,9 @@ cudaError_t launch_ternary_skinny(const uint32_t* w2, const int8_t* qp, const fl
 
 cudaError_t launch_onebit_skinny(const uint32_t* s1, const int8_t* planes, const float* step,
                                  const long long* tsum, const uint16_t* h, int M, int K, int N,
-                                 uint16_t* y, cudaStream_t s) {
+                                 uint16_t* y, cudaStream_t s, float* zf) {
     if (M == 0 || N == 0) return cudaSuccess;
-    SkinnyParams p{s1, planes, step, nullptr, tsum, h, 0.f, M, K, N, y, nullptr};
+    SkinnyParams p{s1, planes, step, nullptr, tsum, h, 0.f, M, K, N, y, nullptr, zf};
     if (M <= 2) return launch<1, 1>(p, s);
     if (M <= 5) return launch<1, 2>(p, s);
     return launch<1, 4>(p, s);

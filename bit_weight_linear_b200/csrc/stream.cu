@@ -61,6 +61,7 @@ struct StreamParams {
     int M, K, N;
     uint16_t* y;
     int32_t* acc_out;
+    float* zf;              // OneBit: optional fp32 [M][N] copy of the output before fp16 rounding
     unsigned int* flags;
     // plan (host-computed)
     int t_lo, t_rem, t_max;  // tiles per CTA: t_lo + (cta < t_rem)
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(NW * 32, 2)
         for (int i = 0; i < UG; ++i) {
             if (has[i]) {
 #pragma unroll
-                for (int v = 0; v < 4; ++v) ga[i][v] = ld_ro_v4(p.g + uk[i] + 8 * v);
+                for (int v = 0; v < 4; ++v) ga[i][v] = ld_gvec(p.g, uk[i] + 8 * v);
             }
         }
     }
@@ -337,7 +338,7 @@ __global__ void __launch_bounds__(NW * 32, 2)
 #pragma unroll
                     for (int v = 0; v < 4; ++v)
                         mx = fmaxf(mx, absmax_prod(tc::ld_v4(xr + 32 * i + 8 * v),
-                                                   ld_ro_v4(p.g + 32 * i + 8 * v)));
+                                                   ld_gvec(p.g, 32 * i + 8 * v)));
                 }
             }
             mx = warp_max(mx);
@@ -363,7 +364,7 @@ __global__ void __launch_bounds__(NW * 32, 2)
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         xa[v] = tc::ld_v4(xr + 32 * i + 8 * v);
-                        gg[v] = ld_ro_v4(p.g + 32 * i + 8 * v);
+                        gg[v] = ld_gvec(p.g, 32 * i + 8 * v);
                     }
                     int gs[3];
                     quant_group_s(xa, gg, inv, act + (3 * m) * p.astride + 32 * i, p.astride, gs);
@@ -624,7 +625,9 @@ __global__ void __launch_bounds__(NW * 32, 2)
             const int n = tile0 * 16 + r;
             const float z = __fmul_rn(st, (float)Z);
             const float hv = __half2float(__ushort_as_half(hs[r]));
-            p.y[(size_t)m * p.N + n] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hv)));
+            const float zh = __fmul_rn(z, hv);
+            p.y[(size_t)m * p.N + n] = __half_as_ushort(__float2half_rn(zh));
+            if (p.zf) p.zf[(size_t)m * p.N + n] = zh;
         }
     }
 }
@@ -840,8 +843,9 @@ cudaError_t launch_ternary_stream(const uint16_t* x, const uint32_t* w2, int M, 
 
 cudaError_t launch_onebit_stream(const uint16_t* x, const uint16_t* g, const uint16_t* h,
                                  const uint32_t* s1, int M, int K, int N, uint16_t* y,
-                                 unsigned int* flags, cudaStream_t s) {
+                                 unsigned int* flags, cudaStream_t s, float* zf) {
     StreamParams p = {};
+    p.zf = zf;
     p.x = x;
     p.g = g;
     p.h = h;
@@ -876,8 +880,9 @@ cudaError_t launch_ternary_stream_prepared(const int8_t* qp, const float* scale,
 cudaError_t launch_onebit_stream_prepared(const int8_t* planes, const float* step,
                                           const long long* tsum, const uint16_t* h,
                                           const uint32_t* s1, int M, int K, int N, uint16_t* y,
-                                          unsigned int* flags, cudaStream_t s) {
+                                          unsigned int* flags, cudaStream_t s, float* zf) {
     StreamParams p = {};
+    p.zf = zf;
     p.prep = planes;
     p.pscale = step;
     p.prsum64 = tsum;

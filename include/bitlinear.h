@@ -170,6 +170,70 @@ bl_status ob_linear(const uint16_t *x, int M, int K, int N, const uint32_t *s1,
                     void *workspace, size_t workspace_bytes, bl_stream_t stream);
 
 /*
+ * Two-plane binary layer (BiLLM page, "BiLLM: Pushing the Limit of
+ * Post-Training Quantization for LLMs", section "方法细节：残差近似与最优断点拆分",
+ * step 2, binary residual approximation): W ~ alpha_o (.) B_o + alpha_r (.) B_r,
+ * both B = +-1, one scale per output row (the reading taken here), fp16
+ * activations not quantised:
+ *     y = fp16( alpha_o (.) (x B_o^T) + alpha_r (.) (x B_r^T) )
+ * Stored form (a OneBit layer of 2N rows with g = 1):
+ *   b2    : uint32 [2N, K/32] in the s1 format: rows 0..N-1 = B_o,
+ *           rows N..2N-1 = B_r
+ *   alpha : fp16 [2N]: alpha_o, then alpha_r
+ * Arithmetic: each plane's contraction is exact in integers on the 23-bit
+ * fixed-point image of x (as ob_linear with g = 1); each plane's product
+ * s * Z * alpha is formed in fp32, the two are added in fp32 and rounded once
+ * to fp16.  K <= 65536, N <= 2^23.
+ */
+size_t billm_workspace_bytes(int M, int K, int N);
+bl_status billm_linear(const uint16_t *x, int M, int K, int N, const uint32_t *b2,
+                       const uint16_t *alpha, uint16_t *y, void *workspace,
+                       size_t workspace_bytes, bl_stream_t stream);
+
+/*
+ * billm_binarize -- the residual binarisation of a weight, on the device:
+ * per row n, alpha_o = mean_k |W[n][k]|, B_o = sign(W[n]), R = W[n] - alpha_o
+ * B_o, alpha_r = mean_k |R[k]|, B_r = sign(R) (sign(0) = +1), in fp64 (the
+ * mean absolute value is the least-squares scale of a sign plane).  Writes b2
+ * and alpha (fp16, rounded to nearest even) in the stored form above, and
+ * optionally fp64 [N] copies of alpha_o and alpha_r (device, or NULL).
+ * W is fp32 [N, K] (a NaN or inf -> BL_ERR_INVALID_VALUE).  Synchronises
+ * `stream` like the packers, and shares their error word.
+ */
+bl_status billm_binarize(const float *W, int N, int K, uint32_t *b2, uint16_t *alpha,
+                         double *alpha_o, double *alpha_r, bl_stream_t stream);
+
+/* Workspace bytes ob_svid needs (a multiple of 256), 0 for an invalid shape. */
+size_t ob_svid_workspace_bytes(int N, int K);
+
+/*
+ * ob_svid -- SVID initialisation of a OneBit layer from a trained weight.
+ * OneBit page, "2. 基于 SVID 初始化量化模型": W ~ sign(W) (.) (a b^T) with a b^T
+ * a rank-1 approximation of |W|; the layer's value vectors are then h = a and
+ * g = b (the order swap of the same section makes ob_linear compute x W^T
+ * with this approximation).  Reading taken here: the rank-1 factor is the
+ * leading singular pair (sigma, u, v) of |W| (the SVD choice of "SVD or
+ * NMF"), a = sqrt(sigma) u, b = sqrt(sigma) v, found by power iteration from
+ * v = 1/sqrt(K):
+ *     u = |W| v / || |W| v ||,  v' = |W|^T u,  sigma = ||v'||,  v = v' / sigma
+ * stopping after iteration i >= 2 when |sigma_i - sigma_{i-1}| <= tol * sigma_i,
+ * or after max_iter iterations.  Arithmetic in fp64 (u, v >= 0 throughout).
+ *   W         : fp32 [N, K], finite (a NaN or inf -> BL_ERR_INVALID_VALUE)
+ *   s1        : packed sign(W), uint32 [N, K/32] (the s1 format; +-0 -> +1)
+ *   g, h      : fp16 [K] = fp16(b), fp16 [N] = fp16(a), round to nearest even
+ *   a, b      : optional device fp64 [N], [K] copies of a and b (NULL: skipped)
+ *   sigma     : optional HOST double: the last sigma
+ *   iters     : optional HOST int: iterations run
+ *   workspace : device scratch of at least ob_svid_workspace_bytes(N, K) bytes
+ * N % 16 == 0 and N <= 524288, K % 128 == 0, max_iter >= 1, tol >= 0, else
+ * BL_ERR_SHAPE.  Synchronises `stream` (it reads the convergence test back
+ * every few iterations).  A weight-preparation call, not a layer forward.
+ */
+bl_status ob_svid(const float *W, int N, int K, int max_iter, double tol, uint32_t *s1,
+                  uint16_t *g, uint16_t *h, double *a, double *b, double *sigma, int *iters,
+                  void *workspace, size_t workspace_bytes, bl_stream_t stream);
+
+/*
  * bl_ternary_linear_noalloc -- bl_ternary_linear for callers that cannot
  * allocate device memory.  (No counterpart on the pages: this is a calling
  * convention, not part of the method.)

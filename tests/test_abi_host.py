@@ -172,3 +172,43 @@ def test_chain_build_rejects_bad_layers(L):
     arr[1].norm_w = None                            # unfused, the same row is fine
     r = L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None)
     assert r != 2
+
+
+def test_svid_rejects_bad_arguments(L):
+    """ob_svid validates shape, iteration limits, pointers and workspace before
+    any CUDA call."""
+    ws = L.ob_svid_workspace_bytes(64, 256)
+    assert ws > 0 and ws % 256 == 0
+    assert L.ob_svid_workspace_bytes(24, 256) == 0               # N % 16
+    assert L.ob_svid_workspace_bytes(64, 100) == 0               # K % 128
+    assert L.ob_svid_workspace_bytes(524288 + 16, 128) == 0      # N limit
+    args = lambda **kw: [kw.get("W", A), kw.get("N", 64), kw.get("K", 256), kw.get("it", 10),
+                         kw.get("tol", 1e-12), kw.get("s1", A), kw.get("g", A), kw.get("h", A),
+                         kw.get("a", None), kw.get("b", None), None, None, kw.get("ws", A),
+                         kw.get("nws", ws), None]
+    assert L.ob_svid(*args(N=0)) == 0                             # empty: no-op
+    assert L.ob_svid(*args(K=100)) == 2
+    assert L.ob_svid(*args(it=0)) == 2
+    assert L.ob_svid(*args(tol=-1.0)) == 2
+    assert L.ob_svid(*args(tol=float("nan"))) == 2
+    assert L.ob_svid(*args(W=None)) == 1
+    assert L.ob_svid(*args(g=None)) == 1
+    assert L.ob_svid(*args(h=ctypes.c_void_p(0x10002))) == 3
+    assert L.ob_svid(*args(a=ctypes.c_void_p(0x10008))) == 3
+    assert L.ob_svid(*args(nws=ws - 1)) == 7
+    assert L.ob_svid(*args(ws=None)) == 7
+
+
+def test_billm_rejects_bad_arguments(L):
+    ws = L.billm_workspace_bytes(4, 256, 32)
+    assert ws > 0 and ws % 256 == 0
+    assert L.billm_workspace_bytes(4, 100, 32) == 0
+    assert L.billm_workspace_bytes(4, 65536 + 128, 32) == 0
+    assert L.billm_linear(A, 4, 256, 24, A, A, A, A, ws, None) == 2           # N % 16
+    assert L.billm_linear(A, 0, 256, 32, A, A, A, A, ws, None) == 0           # empty
+    assert L.billm_linear(None, 4, 256, 32, A, A, A, A, ws, None) == 1
+    assert L.billm_linear(A, 4, 256, 32, A, ctypes.c_void_p(0x10002), A, A, ws, None) == 3
+    assert L.billm_linear(A, 4, 256, 32, A, A, A, A, ws - 1, None) == 7
+    assert L.billm_binarize(A, 32, 100, A, A, None, None, None) == 2
+    assert L.billm_binarize(A, 32, 128, None, A, None, None, None) == 1
+    assert L.billm_binarize(A, 32, 128, A, A, ctypes.c_void_p(0x10008), None, None) == 3
