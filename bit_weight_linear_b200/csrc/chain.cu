@@ -167,28 +167,48 @@ struct TokStats {
 // ---- fused prologues of a layer's input (the BitNet b1.58 page keeps LLaMA's
 // RMSNorm and SwiGLU around BitLinear; definitions in include/bitlinear.h)
 
-__device__ __forceinline__ double half_bits_d(uint32_t v) {
-    return (double)__half2float(__ushort_as_half((unsigned short)(v & 0xffffu)));   // exact
-}
-__device__ __forceinline__ uint32_t pack_half2(double lo, double hi) {
-    return (uint32_t)__half_as_ushort(__double2half(lo)) |
-           ((uint32_t)__half_as_ushort(__double2half(hi)) << 16);
+// fp16 bits of an fp32 result t whose error is below 16 units in t's last
+// place, when that error cannot change the rounding: t lies in the fp16
+// normal range and at least 16 fp32 units from the midpoint between two fp16
+// values (the 13 mantissa bits fp16 drops are not within 16 of 0x1000).  An
+// exact zero is safe too.  Otherwise 0xffffffff: the caller takes the fp64
+// definition.
+__device__ __forceinline__ uint32_t half_if_safe(float t) {
+    const uint32_t b = __float_as_uint(t);
+    if ((b & 0x7fffffffu) == 0) return b >> 16;                  // +-0
+    const uint32_t e = (b >> 23) & 0xffu;
+    if (e < 113 || e > 141) return 0xffffffffu;                  // outside [2^-14, 2^15)
+    const int rem = (int)(b & 0x1fffu) - 0x1000;
+    if (rem >= -16 && rem <= 16) return 0xffffffffu;
+    return __half_as_ushort(__float2half_rn(t));
 }
 
-// SwiGLU of 8 elements: fp16((a / (1 + exp(-a))) * b) in fp64
-__device__ __forceinline__ uint4 swiglu8(uint4 a, uint4 b) {
+// SwiGLU of one element pair of fp16 bits, the definition fp16((a / (1 +
+// exp(-a))) * b) in fp64.  First in fp32: expf is within 2 units in the last
+// place, the add, divide and multiply within half a unit each, and 1 + e >= 1
+// adds no cancellation, so the fp32 value is within 4 units of the exact one
+// and the fp64 definition's value within 2^-50 of it: where half_if_safe
+// accepts the fp32 value, both round to the same fp16.
+// the fp64 definition, out of line: one copy of the code for every caller
+__device__ __noinline__ uint32_t swiglu1_f64(float a, float b) {
+    const double x = (double)a, y = (double)b;
+    return __half_as_ushort(__double2half(__dmul_rn(__ddiv_rn(x, __dadd_rn(1.0, exp(-x))), y)));
+}
+
+__device__ __forceinline__ uint32_t swiglu1(uint32_t ah, uint32_t bh) {
+    const float a = __half2float(__ushort_as_half((unsigned short)ah));
+    const float b = __half2float(__ushort_as_half((unsigned short)bh));
+    const uint32_t f = half_if_safe(__fmul_rn(__fdiv_rn(a, __fadd_rn(1.0f, expf(-a))), b));
+    return f != 0xffffffffu ? f : swiglu1_f64(a, b);
+}
+
+// out of line: the chunk loops that call it are unrolled
+__device__ __noinline__ uint4 swiglu8(uint4 a, uint4 b) {
     const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
     uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        double r[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const double x = half_bits_d(av[i] >> (16 * h)), y = half_bits_d(bv[i] >> (16 * h));
-            r[h] = __dmul_rn(__ddiv_rn(x, __dadd_rn(1.0, exp(-x))), y);
-        }
-        o[i] = pack_half2(r[0], r[1]);
-    }
+    for (int i = 0; i < 4; ++i)
+        o[i] = swiglu1(av[i] & 0xffffu, bv[i] & 0xffffu) | (swiglu1(av[i] >> 16, bv[i] >> 16) << 16);
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
@@ -220,14 +240,28 @@ __device__ __forceinline__ double u128_to_double(unsigned long long hi, unsigned
     return ldexp(__ull2double_rn(top | (rest ? 1ull : 0ull)), sh);
 }
 
-// RMSNorm of 8 elements with r and the weight chunk: fp16((x r) gamma), fp64
-__device__ __forceinline__ uint4 norm8(uint4 a, double r, uint4 gq) {
+// RMSNorm of one element, the definition fp16((x r) gamma) in fp64 with r the
+// row's fp64 factor.  First in fp32 with r rounded to fp32: three roundings of
+// half a unit each, so within 2 units of the exact value; half_if_safe decides
+// as for SwiGLU.
+__device__ __noinline__ uint32_t norm1_f64(float x, double r, float gm) {
+    return __half_as_ushort(__double2half(__dmul_rn(__dmul_rn((double)x, r), (double)gm)));
+}
+
+__device__ __forceinline__ uint32_t norm1(uint32_t xh, double r, float r32, uint32_t gh) {
+    const float x = __half2float(__ushort_as_half((unsigned short)xh));
+    const float gm = __half2float(__ushort_as_half((unsigned short)gh));
+    const uint32_t f = half_if_safe(__fmul_rn(__fmul_rn(x, r32), gm));
+    return f != 0xffffffffu ? f : norm1_f64(x, r, gm);
+}
+
+__device__ __noinline__ uint4 norm8(uint4 a, double r, float r32, uint4 gq) {
     const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {gq.x, gq.y, gq.z, gq.w};
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        o[i] = pack_half2(__dmul_rn(__dmul_rn(half_bits_d(av[i]), r), half_bits_d(gv[i])),
-                          __dmul_rn(__dmul_rn(half_bits_d(av[i] >> 16), r), half_bits_d(gv[i] >> 16)));
+        o[i] = norm1(av[i] & 0xffffu, r, r32, gv[i] & 0xffffu) |
+               (norm1(av[i] >> 16, r, r32, gv[i] >> 16) << 16);
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
@@ -239,14 +273,20 @@ struct Prologue {
 
 // Apply the prologue to the row held in registers: chunk c (c < nch) holds
 // the 8 elements at off(c).
-template <int NCH, typename Off>
+template <int NCH, int BATCH, typename Off>
 __device__ __forceinline__ void apply_prologue(uint4 (&xr)[NCH], int nch, Off off, int K,
                                                const Prologue& pro, TokStats* ts, int et) {
     if (pro.x2) {
+        // BATCH loads in flight, then their chunks
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-            if (c >= nch) break;
-            xr[c] = swiglu8(xr[c], ld_cg_v4(pro.x2 + off(c)));
+        for (int c0 = 0; c0 < NCH; c0 += BATCH) {
+            uint4 t[BATCH];
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i)
+                if (c0 + i < NCH && c0 + i < nch) t[i] = ld_cg_v4(pro.x2 + off(c0 + i));
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i)
+                if (c0 + i < NCH && c0 + i < nch) xr[c0 + i] = swiglu8(xr[c0 + i], t[i]);
         }
     }
     if (pro.gamma) {
@@ -282,10 +322,16 @@ __device__ __forceinline__ void apply_prologue(uint4 (&xr)[NCH], int nch, Off of
         }
         bar_prep();
         const double r = ts->norm_r;
+        const float r32 = __double2float_rn(r);
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-            if (c >= nch) break;
-            xr[c] = norm8(xr[c], r, ld_ro_v4(pro.gamma + off(c)));
+        for (int c0 = 0; c0 < NCH; c0 += BATCH) {
+            uint4 t[BATCH];
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i)
+                if (c0 + i < NCH && c0 + i < nch) t[i] = ld_ro_v4(pro.gamma + off(c0 + i));
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i)
+                if (c0 + i < NCH && c0 + i < nch) xr[c0 + i] = norm8(xr[c0 + i], r, r32, t[i]);
         }
     }
 }
@@ -321,7 +367,8 @@ __device__ void prep_layer(int K, const uint16_t* x, const uint16_t* gvec, bool 
                 if (c >= nc) break;
                 xr[c] = ld(x + 8 * (et + c * kPrepThreads));
             }
-            apply_prologue(xr, nc, [&](int c) { return 8 * (et + c * kPrepThreads); }, K, pro, ts, et);
+            apply_prologue<kRegChunks, 4>(xr, nc, [&](int c) { return 8 * (et + c * kPrepThreads); }, K,
+                                          pro, ts, et);
 #pragma unroll
             for (int c = 0; c < kRegChunks; ++c) {
                 if (c >= nc) break;
@@ -380,7 +427,7 @@ __device__ void prep_layer(int K, const uint16_t* x, const uint16_t* gvec, bool 
 #pragma unroll
                 for (int v = 0; v < 4; ++v) xr[4 * c + v] = ld(x + e + 8 * v);
             }
-            apply_prologue(xr, 4 * ng,
+            apply_prologue<kRegChunks, 2>(xr, 4 * ng,
                            [&](int c) { return 32 * (et + (c >> 2) * kPrepThreads) + 8 * (c & 3); }, K,
                            pro, ts, et);
 #pragma unroll
