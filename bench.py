@@ -56,9 +56,13 @@ def int8_peak(peaks):
 
 # DRAM bytes (read + write) per packed-weight byte of the chain kernel, from an
 # ncu capture of a shorter chain of the same blocks (traffic grows with the
-# weights streamed); None until that capture has been taken on this kernel.
-CHAIN_TRAFFIC_PER_WEIGHT_BYTE = None
-CHAIN_TRAFFIC_SOURCE = "not yet captured for this kernel"
+# weights streamed): 101,420,800 B read + 3,256,320 B written by one launch over
+# the 2-block stack (101,187,584 weight bytes), cold caches.  Set to None
+# whenever the chain kernel changes, until it is captured again.
+CHAIN_TRAFFIC_PER_WEIGHT_BYTE = (101420800 + 3256320) / 101187584
+CHAIN_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one chain_kernel<0> launch "
+                        "over the 2-block stack (--layers 2, cold caches), scaled to this launch by its "
+                        "weight bytes; summary under profiles/")
 
 
 def load_peaks():
@@ -237,7 +241,8 @@ def chain_stack(blw, synth, dev, form: str, dependent: bool, layers: int = LLAMA
             if j % 7 in (0, 1, 2, 4, 5):
                 d["norm_w"], d["norm_eps"] = norm_w, 1e-5
             if j % 7 == 6:
-                d["src2"] = j - 1          # down reads SwiGLU(gate, up)
+                d["src2"] = j - 1          # down reads SwiGLU(gate, up), evaluated once per
+                d["swiglu_buf"] = torch.empty((K,), dtype=torch.float16, device=dev)   # element
         yo += N
         if s < 0:
             if dependent and prev_x is not None and j % 7 in (1, 2):
@@ -383,6 +388,37 @@ def cpu_baselines(synth):
     return out
 
 
+def run_case(blw, synth, dev, args, peaks):
+    """Small named workloads for kernel profiles (one GPU):
+    ternary_decode_m1   the ternary 7B-shaped stack at M = 1, one bl_ternary_linear
+                        call per layer (args.layers blocks), as a CUDA graph;
+    onebit_decode_m1    the same in OneBit form (ob_linear);
+    onebit_prefill_m256 ob_linear at M = 256 on the 13B up (5120->13824) and down
+                        (13824->5120) layers, as a CUDA graph."""
+    if args.case in ("ternary_decode_m1", "onebit_decode_m1"):
+        form = args.case.split("_")[0]
+        calls, wbytes, _x, _y = decode_stack(blw, synth, dev, form, layers=args.layers)
+        g = capture(lambda: run_calls(blw, calls, form))
+        ms = time_replays(g, args.steps, args.warmup, False, dev)
+        gbs = wbytes / (ms * 1e-3) / 1e9
+        return {"ms_per_step": round(ms, 4), "weight_bytes_per_step": wbytes, "GBs": round(gbs, 1),
+                "hbm_frac": round(gbs / peaks["hbm_gbs"], 4)}
+    calls, ops = [], 0
+    for j, (name, K, N) in enumerate(LLAMA13B_SWEEP):
+        x = synth.activations(256, K, seed=5_000_000 + j, device=dev)
+        w = synth.sign_weights(N, K, seed=5_000_010 + j, device=dev)
+        calls.append(dict(x=x, w=blw.ob_pack_sign(w), g=synth.value_vector(K, seed=5_000_020 + j, device=dev),
+                          h=synth.value_vector(N, seed=5_000_030 + j, device=dev),
+                          y=torch.empty((256, N), dtype=torch.float16, device=dev),
+                          ws=torch.empty((blw.ob_workspace_bytes(256, K, N),), dtype=torch.uint8, device=dev)))
+        del w
+        ops += 2 * 256 * K * N
+    g = capture(lambda: run_calls(blw, calls, "onebit"))
+    ms = time_replays(g, args.steps, args.warmup, False, dev)
+    return {"ms_per_step": round(ms, 4), "int8_equiv_TOPS": round(ops / (ms * 1e-3) / 1e12, 2),
+            "shapes_KxN": [[K, N] for (_, K, N) in LLAMA13B_SWEEP]}
+
+
 def run_prefill(blw, synth, dev, args, dist_on, world, peaks):
     """M=512 on the LLaMA-70B-shaped ternary layers (tcgen05 prefill path)."""
     pcalls = []
@@ -497,6 +533,9 @@ def main():
                     help="blocks in the decode stack (fewer = a small profiling case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the 13B batch sweep")
+    ap.add_argument("--case", default=None,
+                    choices=["ternary_decode_m1", "onebit_decode_m1", "onebit_prefill_m256"],
+                    help="time one small named workload (for profiling) and print its line only")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the M=512 prefill layers (a profiling case)")
     args = ap.parse_args()
@@ -551,6 +590,14 @@ def main():
     build.build()
     peaks = load_peaks()
 
+    if args.case:
+        res = run_case(blw, synth, dev, args, peaks)
+        if rank == 0:
+            print(json.dumps({"case": args.case, **res}), flush=True)
+        if dist_on:
+            torch.distributed.destroy_process_group()
+        return 0
+
     if args.prefill_only:
         res = run_prefill(blw, synth, dev, args, dist_on, world, peaks)
         if rank == 0:
@@ -582,7 +629,7 @@ def main():
                 "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "algorithmic_bytes_per_launch": alg_bytes,
-                "traffic": CHAIN_TRAFFIC_PER_WEIGHT_BYTE * wbytes if CHAIN_TRAFFIC_PER_WEIGHT_BYTE else None,
+                "traffic": round(CHAIN_TRAFFIC_PER_WEIGHT_BYTE * wbytes) if CHAIN_TRAFFIC_PER_WEIGHT_BYTE else None,
                 "traffic_unit": "bytes",
                 "traffic_source": CHAIN_TRAFFIC_SOURCE,
                 "peak_source": peaks["_source"],

@@ -40,7 +40,7 @@ class ChainLayer(ctypes.Structure):
     """bl_chain_layer (include/bitlinear.h)."""
     _fields_ = [("x", _P), ("src", _I), ("K", _I), ("N", _I), ("w", _P), ("w_scale", ctypes.c_float),
                 ("g", _P), ("h", _P), ("y", _P), ("acc_out", _P), ("src2", _I), ("norm_w", _P),
-                ("norm_eps", ctypes.c_float)]
+                ("norm_eps", ctypes.c_float), ("swiglu_buf", _P)]
 
 
 class ChainPlan(ctypes.Structure):
@@ -161,6 +161,10 @@ def ob_svid(W: torch.Tensor, max_iter: int = 1000, tol: float = 1e-12, return_ab
                                     nws, _stream()))
     out = (s1, g, h, sigma.value, iters.value)
     return out + (a, b) if return_ab else out
+
+
+def billm_workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(lib().billm_workspace_bytes(M, K, N))
 
 
 def billm_binarize(W: torch.Tensor, return_alpha64: bool = False):
@@ -285,15 +289,16 @@ class Chain:
     def __init__(self, form: int, layers: list[dict]):
         """layers: dicts with K, N, w (packed, CUDA), y (fp16 [N] or [1, N],
         CUDA), and either x (fp16 [K], CUDA) or src (index of an earlier
-        layer); optional src2 (SwiGLU of the outputs of src and src2), norm_w
-        (fp16 [K] RMSNorm weight) and norm_eps; ternary: w_scale, optional
-        acc_out (int32 [N]); OneBit: g, h."""
+        layer); optional src2 (SwiGLU of the outputs of src and src2) with an
+        optional swiglu_buf (fp16 [K] scratch: the SwiGLU is then evaluated once
+        per element), norm_w (fp16 [K] RMSNorm weight) and norm_eps; ternary:
+        w_scale, optional acc_out (int32 [N]); OneBit: g, h."""
         n = len(layers)
         arr = (ChainLayer * n)()
         self._keep = []
         dev = None
         for j, d in enumerate(layers):
-            ts = [d.get(k) for k in ("x", "w", "g", "h", "y", "acc_out", "norm_w")]
+            ts = [d.get(k) for k in ("x", "w", "g", "h", "y", "acc_out", "norm_w", "swiglu_buf")]
             _need_cuda(*[t for t in ts if t is not None])
             self._keep.extend(t for t in ts if t is not None)
             dev = dev or d["w"].device
@@ -309,6 +314,7 @@ class Chain:
             arr[j].src2 = int(d.get("src2", -1))
             arr[j].norm_w = None if d.get("norm_w") is None else d["norm_w"].data_ptr()
             arr[j].norm_eps = float(d.get("norm_eps", 0.0))
+            arr[j].swiglu_buf = None if d.get("swiglu_buf") is None else d["swiglu_buf"].data_ptr()
         nbytes = int(lib().bl_chain_bytes(n))
         if nbytes == 0:
             raise ValueError("chain length out of range")

@@ -423,8 +423,10 @@ bl_status bl_chain_build(int form, const bl_chain_layer* layers, int n_layers, v
         if (L.norm_w && !(L.norm_eps >= 0.f)) return BL_ERR_SHAPE;
         if ((L.src < 0 && !L.x) || !L.w || !L.y || (form == 1 && (!L.g || !L.h))) return BL_ERR_NULL;
         if ((L.src < 0 && misaligned(L.x)) || misaligned(L.w) || misaligned(L.y) ||
-            misaligned(L.acc_out) || misaligned(L.g) || misaligned(L.h) || misaligned(L.norm_w))
+            misaligned(L.acc_out) || misaligned(L.g) || misaligned(L.h) || misaligned(L.norm_w) ||
+            misaligned(L.swiglu_buf))
             return BL_ERR_ALIGN;
+        if (L.swiglu_buf && L.src2 < 0) return BL_ERR_SHAPE;
     }
     if (chain_bytes < bl::chain_bytes(n_layers)) return BL_ERR_WORKSPACE;
     if (bl_status st = bl::fault_injected()) return st;

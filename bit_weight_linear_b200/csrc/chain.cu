@@ -36,6 +36,14 @@
 // round-robin from a per-layer rotation, so every CTA carries the same share
 // of the whole list.
 //
+// Fused block steps (the BitNet b1.58 page keeps LLaMA's RMSNorm and SwiGLU
+// around BitLinear): a layer's input may be an RMSNorm of its source and/or
+// SwiGLU(y_src, y_src2), applied to the row in registers before the absmax.
+// With a caller buffer the SwiGLU is instead evaluated once per element, in
+// the epilogue of the later of the two sources (whose tiles are then dealt
+// like the earlier one's, so each thread reads the other output it wrote
+// itself), and the layer reads the finished row.
+//
 // Every wait is bounded (2 s): on expiry the kernel sets the device condition
 // word (BL_ERR_TIMEOUT through bl_device_status), and the producer lets every
 // copy it requested land before its CTA can exit.
@@ -71,7 +79,7 @@ constexpr int kBarPrep = 1;                // named barrier of the activation/ep
 constexpr int kMaxBufs = 4;                // activation buffers: layers prepared ahead
 
 // One layer of a chain in device memory (written by bl_chain_build, read-only
-// in the kernel).  384 bytes, 64-byte aligned: the tensor maps come first.
+// in the kernel).  448 bytes, 64-byte aligned: the tensor maps come first.
 struct alignas(64) ChainLayer {
     CUtensorMap tm_main;   // [step][row][64 B] boxes of 16 rows x bsteps steps
     CUtensorMap tm_tail;   // [row][tail B] box of a partial last step
@@ -90,9 +98,15 @@ struct alignas(64) ChainLayer {
     int steps, nfull, tail, ragged, bsteps, nch, ntile, rot;
     int has_dep;           // a later layer reads y: arrive on done[] after the epilogue
     int reuse;             // same input as the previous layer: copy its prepared activations
-    int pad[2];
+    // SwiGLU evaluated in this layer's epilogue, once per element: for each of
+    // its rows n, swi_out[n] = fp16(silu(a) * b) with {a, b} = {y[n], y_q[n]}
+    // (a = this layer's y when swi_self_a).  Layer swi_q has the same rows and
+    // tile deal, so the thread that writes y[n] here wrote y_q[n] there.
+    int swi_q, swi_self_a;
+    uint16_t* swi_out;
+    int xbuf;              // host only: the input is x = a SwiGLU buffer although src >= 0
 };
-static_assert(sizeof(ChainLayer) == 384, "chain layer descriptor size");
+static_assert(sizeof(ChainLayer) == 448, "chain layer descriptor size");
 
 // The per-layer fields every warp role reads, 32 bytes per layer: written by
 // the host next to the descriptors and copied into shared memory at launch.
@@ -109,7 +123,8 @@ struct alignas(16) LayerInfo {
     uint16_t* y;            // output
 };
 static_assert(sizeof(LayerInfo) == 32, "layer info size");
-constexpr uint8_t kInfoRagged = 1, kInfoHasDep = 2, kInfoReuse = 4, kInfoNorm = 8;
+// kInfoXbuf: the input is x although src >= 0 (a SwiGLU evaluated by layer src's epilogue)
+constexpr uint8_t kInfoRagged = 1, kInfoHasDep = 2, kInfoReuse = 4, kInfoNorm = 8, kInfoXbuf = 16;
 
 struct ChainParams {
     const ChainLayer* layers;
@@ -767,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
                     }
                 } else {
                     // the input, g and prologue pointers, loaded before the dependency wait
-                    const uint16_t* x = L.src >= 0 ? tab[L.src].y : L.x;
+                    const uint16_t* x = (L.src >= 0 && !(L.flags & kInfoXbuf)) ? tab[L.src].y : L.x;
                     const uint16_t* gvec = FORM == 1 ? p.layers[j].g : nullptr;
                     Prologue pro;
                     pro.x2 = L.src2 >= 0 ? tab[L.src2].y : nullptr;
@@ -821,6 +836,9 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
             int32_t* acc_out = FORM == 0 ? p.layers[j].acc_out : nullptr;
             const float w_scale = p.layers[j].w_scale;
             const uint16_t* h = FORM == 1 ? p.layers[j].h : nullptr;
+            uint16_t* swi_out = p.layers[j].swi_out;
+            const uint16_t* yq = swi_out ? tab[p.layers[j].swi_q].y : nullptr;
+            const bool self_a = p.layers[j].swi_self_a != 0;
             // one thread waits (asleep) for the contraction; the others in the barrier
             bool got = true;
             if (et == 0) got = tc::mbar_wait(bar_mma + 8 * b, (uint32_t)((j / NB) & 1), p.flags, p.wait_ns);
@@ -833,17 +851,24 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
             for (int o = et; o < T * 16; o += kPrepThreads) {
                 const int k = o >> 4, r = o & 15;
                 const int nrow = (first + k * G) * 16 + r;
+                uint32_t yb;
                 if constexpr (FORM == 0) {
                     const int a = pb[o] - ts->qsum[b];
                     pb[o] = 0;
-                    y[nrow] = __half_as_ushort(__float2half_rn(__fmul_rn(__fmul_rn((float)a, sc), w_scale)));
+                    yb = __half_as_ushort(__float2half_rn(__fmul_rn(__fmul_rn((float)a, sc), w_scale)));
                     if (acc_out) acc_out[nrow] = a;
                 } else {
                     const long long Z = limb_combine(pb[3 * o], pb[3 * o + 1], pb[3 * o + 2], ts->xsum[b]);
                     pb[3 * o] = pb[3 * o + 1] = pb[3 * o + 2] = 0;
                     const float z = __fmul_rn(sc, (float)Z);
                     const float hv = __half2float(__ushort_as_half(h[nrow]));
-                    y[nrow] = __half_as_ushort(__float2half_rn(__fmul_rn(z, hv)));
+                    yb = __half_as_ushort(__float2half_rn(__fmul_rn(z, hv)));
+                }
+                y[nrow] = (uint16_t)yb;
+                if (swi_out) {
+                    // this thread wrote y_q[nrow] in layer swi_q's epilogue
+                    const uint32_t other = yq[nrow];
+                    swi_out[nrow] = (uint16_t)(self_a ? swiglu1(yb, other) : swiglu1(other, yb));
                 }
             }
             bar_prep();   // every output of this CTA written, partials cleared
@@ -956,6 +981,27 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
         tiles_before += L.ntile;
         if (in.src >= 0) host[(size_t)in.src].has_dep = 1;
         if (in.src2 >= 0) host[(size_t)in.src2].has_dep = 1;
+        L.swi_q = -1;
+        if (in.src2 >= 0 && in.swiglu_buf) {
+            // evaluate the SwiGLU in the epilogue of the later of the two sources,
+            // whose tiles are then dealt like the earlier one's; this layer reads
+            // the finished input from swiglu_buf (unless that layer already
+            // evaluates another SwiGLU)
+            const int pi = in.src > in.src2 ? in.src : in.src2;
+            const int qi = in.src > in.src2 ? in.src2 : in.src;
+            ChainLayer& P = host[(size_t)pi];
+            const int self_a = pi == in.src;
+            if (!P.swi_out || (P.swi_out == in.swiglu_buf && P.swi_q == qi && P.swi_self_a == self_a)) {
+                P.swi_out = in.swiglu_buf;
+                P.swi_q = qi;
+                P.swi_self_a = self_a;
+                P.rot = host[(size_t)qi].rot;
+                L.src = pi;
+                L.src2 = -1;
+                L.x = in.swiglu_buf;
+                L.xbuf = 1;
+            }
+        }
         // the same prepared input as the layer before: same source(s), same
         // prologue, same g (OneBit)
         if (j > 0 && in.K == layers[j - 1].K && in.src == layers[j - 1].src &&
@@ -1004,9 +1050,10 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
         I.bsteps = (uint8_t)L.bsteps;
         I.nch = (uint8_t)L.nch;
         I.flags = (uint8_t)((L.ragged ? kInfoRagged : 0) | (L.has_dep ? kInfoHasDep : 0) |
-                            (L.reuse ? kInfoReuse : 0) | (L.norm_w ? kInfoNorm : 0));
+                            (L.reuse ? kInfoReuse : 0) | (L.norm_w ? kInfoNorm : 0) |
+                            (L.xbuf ? kInfoXbuf : 0));
         I.src2 = (int16_t)L.src2;
-        I.x = L.src < 0 ? L.x : nullptr;
+        I.x = (L.src < 0 || L.xbuf) ? L.x : nullptr;
         I.y = L.y;
     }
     ChainSmem m;

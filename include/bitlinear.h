@@ -315,6 +315,13 @@ typedef struct {
                               fp16((x * r) * norm_w), r = 1/sqrt(sum x^2/K + eps),
                               the sum of squares exact, the rest in fp64 */
     float norm_eps;        /* eps of that RMSNorm */
+    uint16_t *swiglu_buf;  /* NULL, or (with src2 >= 0) a caller-owned fp16 [K]
+                              device buffer: the SwiGLU is then evaluated once per
+                              element, in the epilogue of the later of layers src
+                              and src2, and stored here for this layer to read
+                              (with NULL every CTA evaluates the whole row).  Same
+                              results either way.  The chain writes it during
+                              every run; give each SwiGLU layer its own buffer. */
 } bl_chain_layer;
 
 typedef struct {           /* filled by bl_chain_build; pass unchanged to bl_chain_run */

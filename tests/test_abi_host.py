@@ -169,7 +169,10 @@ def test_chain_build_rejects_bad_layers(L):
     arr[0].N = arr[1].K = 18048
     arr[1].norm_w, arr[1].src2 = 0x20000, -1
     assert L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None) == 2
-    arr[1].norm_w = None                            # unfused, the same row is fine
+    arr[1].norm_w = None
+    arr[1].swiglu_buf = 0x30000                     # a SwiGLU buffer without src2
+    assert L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None) == 2
+    arr[1].swiglu_buf = None                        # unfused, the same row is fine
     r = L.bl_chain_build(0, arr, n, buf, nb, ctypes.byref(plan), None)
     assert r != 2
 

@@ -186,13 +186,17 @@ EPS = float(np.float32(1e-5))
 def test_chain_fused_llama7b_blocks_bit_exact(blw, oref):
     """Four LLaMA-7B blocks with RMSNorm and SwiGLU fused into the chain: every
     layer's accumulators and outputs equal the oracle's RMSNorm / SwiGLU /
-    BitLinear applied to the GPU's own inputs, bit for bit."""
+    BitLinear applied to the GPU's own inputs, bit for bit.  Blocks 0 and 2
+    evaluate SwiGLU once per element in up's epilogue (swiglu_buf, checked
+    against the oracle's SwiGLU too); blocks 1 and 3 in every CTA."""
     blocks = 4
     shapes = [(K, N) for _ in range(blocks) for (_, K, N) in BLOCK_7B]
     plan = fused_block_layers(blocks)
     layers, host = ternary_chain(blw, shapes, [s for s, _, _ in plan], seed=640_000)
     for j, (d, (_, s2, norm)) in enumerate(zip(layers, plan)):
         d["src2"] = s2
+        if s2 >= 0 and (j // 7) % 2 == 0:
+            d["swiglu_buf"] = torch.full((d["K"],), float("nan"), dtype=torch.float16, device="cuda")
         if norm:
             # q, k, v (and gate, up) share one RMSNorm weight: prepared once
             d["norm_w"] = synth.norm_weight(d["K"], seed=641_000 + (j // 7) * 2 + (j % 7 >= 4)).cuda()
@@ -210,6 +214,8 @@ def test_chain_fused_llama7b_blocks_bit_exact(blw, oref):
     for j, (d, w) in enumerate(zip(layers, host)):
         xin = _fused_input(oref, layers, d)
         assert np.isfinite(xin.astype(np.float32)).all(), j
+        if "swiglu_buf" in d:
+            assert np.array_equal(d["swiglu_buf"].cpu().numpy().view(np.uint16), xin.view(np.uint16)), j
         y_ref, acc_ref = oref.ternary_linear(xin[None, :], oref.pack_ternary(w.numpy()), d["w_scale"],
                                              parallel=True)
         assert np.array_equal(d["acc_out"].cpu().numpy(), acc_ref[0]), j
@@ -232,8 +238,10 @@ def test_chain_fused_prologue_edge_rows(blw, oref):
     x2[1::7] = -60000.0
     layers[2]["x"].copy_(x2.half())
     layers[2]["w_scale"] = 0.002
-    layers[4]["src2"] = 3                   # SwiGLU(y2, y3)
-    layers[5]["src2"] = 2                   # SwiGLU(y3, y2), then RMSNorm
+    layers[4]["src2"] = 3                   # SwiGLU(y2, y3), evaluated in layer 3's epilogue
+    layers[5]["src2"] = 2                   # SwiGLU(y3, y2), then RMSNorm: layer 3 already
+    for d in layers[4:]:                    # evaluates the other order, so every CTA does this one
+        d["swiglu_buf"] = torch.empty((1024,), dtype=torch.float16, device="cuda")
     layers[5]["norm_w"], layers[5]["norm_eps"] = synth.norm_weight(1024, seed=650_102).cuda(), EPS
     blw.Chain(0, layers).run()
     torch.cuda.synchronize()
@@ -257,6 +265,8 @@ def test_chain_fused_onebit_block(blw, oref):
     nw = [synth.norm_weight(4096, seed=660_100 + i).cuda() for i in range(2)]
     for j, (d, (_, s2, norm)) in enumerate(zip(layers, plan)):
         d["src2"] = s2
+        if s2 >= 0:
+            d["swiglu_buf"] = torch.empty((d["K"],), dtype=torch.float16, device="cuda")
         if norm:
             d["norm_w"], d["norm_eps"] = nw[j >= 4], EPS
     blw.Chain(1, layers).run()
