@@ -65,8 +65,8 @@ WsLayout ws_layout(int form, int M, int K, int N) {
     l.split = l.rsum + align_up((size_t)M * (form == 0 ? sizeof(int32_t) : sizeof(long long)));
     l.split_bytes = 0;
     l.n_ctr = 0;
-    const int min_m = form == 0 ? bl::kTernaryPrefillMinM : bl::kOnebitPrefillMinM;
-    if (M >= min_m) l.split_bytes = bl::prefill_split_bytes(form, M, K, N, &l.n_ctr);
+    const bool prefill = form == 0 ? M >= bl::kTernaryPrefillMinM : bl::onebit_prefill(M, N);
+    if (prefill) l.split_bytes = bl::prefill_split_bytes(form, M, K, N, &l.n_ctr);
     l.total = l.split + align_up(l.split_bytes);
     return l;
 }
@@ -268,7 +268,7 @@ static bl_status onebit_forward(const uint16_t* x, int M, int K, int N, const ui
     unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + l.split);
     cudaError_t e = bl::launch_prep_onebit(x, g, M, K, planes, step, ts, s, ctr, l.n_ctr);
     if (e != cudaSuccess) return BL_ERR_CUDA;
-    if (M >= bl::kOnebitPrefillMinM) {
+    if (bl::onebit_prefill(M, N)) {
         e = bl::launch_onebit_prefill(s1, planes, step, ts, h, M, K, N, y, flags, s, ws + l.split,
                                       l.split_bytes, zf);
     } else {

@@ -190,11 +190,13 @@ private:
 constexpr int kStreamFusedMaxM = 8;
 constexpr int kStreamFusedMaxMOnebit = 2;
 
-// Token counts at or above which the tensor-core prefill kernel is used
-// (measured crossovers on 13B-shaped layers: ternary M = 16 runs 26 % faster
-// there than in the prepared streamed kernel; OneBit M = 8 up to 56 % faster,
-// while OneBit M = 4 was still faster streamed on the 13824-long rows).
+// Token counts at which the tensor-core prefill kernel is used (measured
+// crossovers on 13B-shaped layers: ternary M = 16 runs 26 % faster there than
+// in the prepared streamed kernel).
 constexpr int kTernaryPrefillMinM = 9;
-constexpr int kOnebitPrefillMinM = 5;
+// OneBit calls take the tensor-core path from 4 tokens, and at 3 tokens on
+// layers of more than 16384 rows, where the streamed plan is slower (measured
+// on the 13B-shaped layers and the BiLLM layer's stacked planes).
+inline bool onebit_prefill(int M, int N) { return M >= 4 || (M == 3 && N > 16384); }
 
 }  // namespace bl

@@ -290,7 +290,7 @@ def test_ternary_prefill_balanced_round(blw, oref, M, K, N):
 # Large layers are checked on 128 sampled weight rows (first and last
 # included, so every tile is likely hit), small ones whole.
 SMALL_M_TERNARY = [(9, 13824, 5120), (16, 13824, 5120), (12, 4096, 4096), (9, 2048, 1024)]
-SMALL_M_ONEBIT = [(5, 13824, 5120), (8, 13824, 5120), (8, 5120, 13824)]
+SMALL_M_ONEBIT = [(3, 13824, 5120), (4, 5120, 13824), (5, 13824, 5120), (8, 13824, 5120), (8, 5120, 13824)]
 
 
 def _sample_rows(N, seed):
