@@ -56,10 +56,10 @@ def int8_peak(peaks):
 
 # DRAM bytes (read + write) per packed-weight byte of the chain kernel, from an
 # ncu capture of a shorter chain of the same blocks (traffic grows with the
-# weights streamed): 101,420,800 B read + 3,256,320 B written by one launch over
-# the 2-block stack (101,187,584 weight bytes), cold caches.  Set to None
-# whenever the chain kernel changes, until it is captured again.
-CHAIN_TRAFFIC_PER_WEIGHT_BYTE = (101420800 + 3256320) / 101187584
+# weights streamed): the DRAM bytes read + written by one launch over the
+# 2-block stack divided by its 101,187,584 weight bytes, cold caches.  None
+# whenever the chain kernel has changed since the last capture.
+CHAIN_TRAFFIC_PER_WEIGHT_BYTE = None
 CHAIN_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one chain_kernel<0> launch "
                         "over the 2-block stack (--layers 2, cold caches), scaled to this launch by its "
                         "weight bytes; summary under profiles/")

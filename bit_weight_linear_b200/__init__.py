@@ -46,7 +46,7 @@ class ChainLayer(ctypes.Structure):
 class ChainPlan(ctypes.Structure):
     """bl_chain_plan (include/bitlinear.h)."""
     _fields_ = [("form", _I), ("n_layers", _I), ("sm_count", _I), ("kmax", _I), ("slots", _I),
-                ("smem_bytes", _I)]
+                ("smem_bytes", _I), ("fused", _I)]
 ABI = {
     "bl_status_string": ([_I], ctypes.c_char_p),
     "bl_abi_version": ([], _I),

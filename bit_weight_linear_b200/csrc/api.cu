@@ -436,7 +436,7 @@ bl_status bl_chain_build(int form, const bl_chain_layer* layers, int n_layers, v
 bl_status bl_chain_run(const bl_chain_plan* plan, const void* chain, bl_stream_t stream) {
     if (!plan || !chain) return BL_ERR_NULL;
     if ((plan->form != 0 && plan->form != 1) || plan->n_layers <= 0 ||
-        plan->n_layers > kMaxChainLayers)
+        plan->n_layers > kMaxChainLayers || (plan->fused != 0 && plan->fused != 1))
         return BL_ERR_SHAPE;
     if ((reinterpret_cast<uintptr_t>(chain) & 255u) != 0) return BL_ERR_ALIGN;
     if (bl_status st = bl::fault_injected()) return st;

@@ -217,8 +217,7 @@ __device__ __forceinline__ uint32_t swiglu1(uint32_t ah, uint32_t bh) {
     return f != 0xffffffffu ? f : swiglu1_f64(a, b);
 }
 
-// out of line: the chunk loops that call it are unrolled
-__device__ __noinline__ uint4 swiglu8(uint4 a, uint4 b) {
+__device__ __forceinline__ uint4 swiglu8(uint4 a, uint4 b) {
     const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
     uint32_t o[4];
 #pragma unroll
@@ -270,7 +269,7 @@ __device__ __forceinline__ uint32_t norm1(uint32_t xh, double r, float r32, uint
     return f != 0xffffffffu ? f : norm1_f64(x, r, gm);
 }
 
-__device__ __noinline__ uint4 norm8(uint4 a, double r, float r32, uint4 gq) {
+__device__ __forceinline__ uint4 norm8(uint4 a, double r, float r32, uint4 gq) {
     const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {gq.x, gq.y, gq.z, gq.w};
     uint32_t o[4];
 #pragma unroll
@@ -362,7 +361,7 @@ constexpr int kRegChunks = 10;
 // (OneBit re-reads g, a parameter, for the products).  Longer rows: two passes
 // over x (the second from L1 or L2).  `cg`: x is another CTA's output, read
 // through L2.
-template <int FORM>
+template <int FORM, bool FUSED>
 __device__ void prep_layer(int K, const uint16_t* x, const uint16_t* gvec, bool cg, const Prologue& pro,
                            uint8_t* act, int astride, TokStats* ts, int b, int et) {
     const int pw = et >> 5, lane = et & 31;
@@ -382,8 +381,9 @@ __device__ void prep_layer(int K, const uint16_t* x, const uint16_t* gvec, bool 
                 if (c >= nc) break;
                 xr[c] = ld(x + 8 * (et + c * kPrepThreads));
             }
-            apply_prologue<kRegChunks, 4>(xr, nc, [&](int c) { return 8 * (et + c * kPrepThreads); }, K,
-                                          pro, ts, et);
+            if constexpr (FUSED)
+                apply_prologue<kRegChunks, 4>(xr, nc, [&](int c) { return 8 * (et + c * kPrepThreads); }, K,
+                                              pro, ts, et);
 #pragma unroll
             for (int c = 0; c < kRegChunks; ++c) {
                 if (c >= nc) break;
@@ -442,7 +442,8 @@ __device__ void prep_layer(int K, const uint16_t* x, const uint16_t* gvec, bool 
 #pragma unroll
                 for (int v = 0; v < 4; ++v) xr[4 * c + v] = ld(x + e + 8 * v);
             }
-            apply_prologue<kRegChunks, 2>(xr, 4 * ng,
+            if constexpr (FUSED)
+                apply_prologue<kRegChunks, 2>(xr, 4 * ng,
                            [&](int c) { return 32 * (et + (c >> 2) * kPrepThreads) + 8 * (c & 3); }, K,
                            pro, ts, et);
 #pragma unroll
@@ -508,7 +509,10 @@ __device__ void prep_layer(int K, const uint16_t* x, const uint16_t* gvec, bool 
     }
 }
 
-template <int FORM>
+// FUSED: the chain has a layer with a prologue or a SwiGLU buffer.  Chains
+// without one run an instantiation that holds none of that code (its mere
+// presence cost the plain chain 5-15 % in register allocation and scheduling).
+template <int FORM, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p) {
     using F = DF<FORM>;
     constexpr int COLS = F::kCPT;          // activation columns of the single token
@@ -813,7 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
                             break;
                         }
                     }
-                    prep_layer<FORM>(K, x, gvec, L.src >= 0, pro, act, p.astride, ts, b, et);
+                    prep_layer<FORM, FUSED>(K, x, gvec, L.src >= 0, pro, act, p.astride, ts, b, et);
                 }
                 // zeros from K to a whole step in every row (a partial last step's
                 // lanes past the row end multiply them)
@@ -836,7 +840,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
             int32_t* acc_out = FORM == 0 ? p.layers[j].acc_out : nullptr;
             const float w_scale = p.layers[j].w_scale;
             const uint16_t* h = FORM == 1 ? p.layers[j].h : nullptr;
-            uint16_t* swi_out = p.layers[j].swi_out;
+            uint16_t* swi_out = FUSED ? p.layers[j].swi_out : nullptr;
             const uint16_t* yq = swi_out ? tab[p.layers[j].swi_q].y : nullptr;
             const bool self_a = p.layers[j].swi_self_a != 0;
             // one thread waits (asleep) for the contraction; the others in the barrier
@@ -865,7 +869,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
                     yb = __half_as_ushort(__float2half_rn(__fmul_rn(z, hv)));
                 }
                 y[nrow] = (uint16_t)yb;
-                if (swi_out) {
+                if (FUSED && swi_out) {
                     // this thread wrote y_q[nrow] in layer swi_q's epilogue
                     const uint32_t other = yq[nrow];
                     swi_out[nrow] = (uint16_t)(self_a ? swiglu1(yb, other) : swiglu1(other, yb));
@@ -921,10 +925,10 @@ bool chain_smem(int form, int kmax, int n, ChainSmem& m) {
     return false;
 }
 
-template <int FORM>
+template <int FORM, bool FUSED>
 cudaError_t launch_chain(const ChainParams& p, int smem, cudaStream_t s) {
     static KernelAttrs kattrs;
-    if (cudaError_t e = kattrs.ensure(chain_kernel<FORM>, kDecodeMaxSmem)) return e;
+    if (cudaError_t e = kattrs.ensure(chain_kernel<FORM, FUSED>, kDecodeMaxSmem)) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(device_sm_count());
     cfg.blockDim = dim3(kThreads);
@@ -936,7 +940,7 @@ cudaError_t launch_chain(const ChainParams& p, int smem, cudaStream_t s) {
     attrs[0].val.cooperative = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, chain_kernel<FORM>, p);
+    return cudaLaunchKernelEx(&cfg, chain_kernel<FORM, FUSED>, p);
 }
 
 }  // namespace
@@ -958,6 +962,7 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
     std::vector<ChainLayer> host((size_t)n);
     std::vector<LayerInfo> info((size_t)n);
     int kmax = 0;
+    bool fused = false;
     long long tiles_before = 0;
     for (int j = 0; j < n; ++j) {
         const bl_chain_layer& in = layers[j];
@@ -982,6 +987,7 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
         if (in.src >= 0) host[(size_t)in.src].has_dep = 1;
         if (in.src2 >= 0) host[(size_t)in.src2].has_dep = 1;
         L.swi_q = -1;
+        if (in.src2 >= 0 || in.norm_w) fused = true;
         if (in.src2 >= 0 && in.swiglu_buf) {
             // evaluate the SwiGLU in the epilogue of the later of the two sources,
             // whose tiles are then dealt like the earlier one's; this layer reads
@@ -1067,6 +1073,7 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
         cudaStreamSynchronize(s) != cudaSuccess)
         return BL_ERR_CUDA;
     plan->form = form;
+    plan->fused = fused ? 1 : 0;
     plan->n_layers = n;
     plan->sm_count = G;
     plan->kmax = kmax;
@@ -1101,7 +1108,9 @@ bl_status chain_run(const bl_chain_plan* plan, const void* chain, unsigned int* 
     p.wait_ns = kWaitNs;
     // the completion counters start at zero on every run
     if (cudaMemsetAsync(p.done, 0, (size_t)n * 4, s) != cudaSuccess) return BL_ERR_CUDA;
-    const cudaError_t e = plan->form == 0 ? launch_chain<0>(p, m.total, s) : launch_chain<1>(p, m.total, s);
+    const cudaError_t e =
+        plan->form == 0 ? (plan->fused ? launch_chain<0, true>(p, m.total, s) : launch_chain<0, false>(p, m.total, s))
+                        : (plan->fused ? launch_chain<1, true>(p, m.total, s) : launch_chain<1, false>(p, m.total, s));
     return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }
 

@@ -331,6 +331,7 @@ typedef struct {           /* filled by bl_chain_build; pass unchanged to bl_cha
     int kmax;              /* largest K of the chain */
     int slots;             /* weight-ring slots per CTA */
     int smem_bytes;        /* shared memory per CTA */
+    int fused;             /* 1: some layer has an RMSNorm or SwiGLU prologue */
 } bl_chain_plan;
 
 /* Device bytes of the chain buffer for n_layers layers, 1 <= n_layers <= 2048
