@@ -154,6 +154,12 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned int* p) {
     return v;
 }
 
+// Bring a read-only fp16 row (an RMSNorm weight) into L1 ahead of use: one
+// prefetch per 128-byte line, spread over the activation threads.
+__device__ __forceinline__ void prefetch_row_l1(const uint16_t* v, int K, int et, int nthreads) {
+    for (int e = 64 * et; e < K; e += 64 * nthreads) asm volatile("prefetch.global.L1 [%0];" ::"l"(v + e));
+}
+
 // 16-byte load through L2 only (another CTA's output, after an acquire).
 __device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
     uint4 v;
@@ -176,7 +182,6 @@ struct TokStats {
     uint32_t red[3][kPrepWarps];
     int redi[3][kPrepWarps];
     unsigned long long ss[kPrepWarps][2];   // RMSNorm: per-warp exact sums of squares
-    double norm_r;                          // RMSNorm: 1 / sqrt(mean square + eps)
 };
 
 // ---- fused prologues of a layer's input (the BitNet b1.58 page keeps LLaMA's
@@ -324,18 +329,17 @@ __device__ __forceinline__ void apply_prologue(uint4 (&xr)[NCH], int nch, Off of
             ts->ss[pw][1] = lo;
         }
         bar_prep();
-        if (et == 0) {
-            unsigned long long H = 0, Lo = 0;
-            for (int w = 0; w < kPrepWarps; ++w) {
-                const unsigned long long nlo = Lo + ts->ss[w][1];
-                H += ts->ss[w][0] + (nlo < Lo ? 1ull : 0ull);
-                Lo = nlo;
-            }
-            const double ssq = ldexp(u128_to_double(H, Lo), -48);
-            ts->norm_r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ssq, (double)K), pro.eps)));
+        // every thread forms the same r from the warps' exact partial sums (no
+        // second barrier to broadcast it)
+        unsigned long long H = 0, Lo = 0;
+#pragma unroll
+        for (int w = 0; w < kPrepWarps; ++w) {
+            const unsigned long long nlo = Lo + ts->ss[w][1];
+            H += ts->ss[w][0] + (nlo < Lo ? 1ull : 0ull);
+            Lo = nlo;
         }
-        bar_prep();
-        const double r = ts->norm_r;
+        const double ssq = ldexp(u128_to_double(H, Lo), -48);
+        const double r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ssq, (double)K), pro.eps)));
         const float r32 = __double2float_rn(r);
 #pragma unroll
         for (int c0 = 0; c0 < NCH; c0 += BATCH) {
@@ -792,6 +796,9 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const ChainParams p)
                     pro.x2 = L.src2 >= 0 ? tab[L.src2].y : nullptr;
                     pro.gamma = (L.flags & kInfoNorm) ? p.layers[j].norm_w : nullptr;
                     pro.eps = (double)p.layers[j].norm_eps;
+                    // the weight is read after the row's sum of squares: fetch it
+                    // while the producing layer finishes
+                    if (FUSED && pro.gamma) prefetch_row_l1(pro.gamma, K, et, kPrepThreads);
                     if (L.src >= 0) {
                         // wait until every CTA has finished the producing layer(s)
                         bool got = true;
@@ -894,7 +901,7 @@ struct ChainSmem {
     int S, NB, astride, off_act, off_part, off_tok, off_bar, off_tab, total;
 };
 
-bool chain_smem(int form, int kmax, int n, ChainSmem& m) {
+bool chain_smem(int form, int kmax, int n, ChainSmem& m, int s_req = 0, bool buffers_first = false) {
     const int cols = form == 0 ? 1 : 3;
     // rows padded to a whole step (256 / 512 k), +16 bytes between rows
     m.astride = (kmax + 511) / 512 * 512 + 16;
@@ -917,8 +924,22 @@ bool chain_smem(int form, int kmax, int n, ChainSmem& m) {
         m.total = off;
         return off <= kDecodeMaxSmem;
     };
-    // the most ring slots first (bytes in flight set the streaming rate), then
-    // the most activation buffers
+    // s_req > 0: that many slots (with the most buffers that fit).  Otherwise
+    // the most ring slots first (bytes in flight, which also carry the next
+    // layers' weights across a dependency), then the most activation buffers;
+    // or, with buffers_first, the most buffers first: a chain whose layers
+    // mostly read given inputs can prepare up to four layers ahead.
+    if (s_req > 0) {
+        for (int NB = kMaxBufs; NB >= 2; --NB)
+            if (layout(NB, s_req)) return true;
+        return false;
+    }
+    if (buffers_first) {
+        for (int NB = kMaxBufs; NB >= 2; --NB)
+            for (int S = kMaxSlots; S >= 3; --S)
+                if (layout(NB, S)) return true;
+        return false;
+    }
     for (int S = kMaxSlots; S >= 3; --S)
         for (int NB = kMaxBufs; NB >= 2; --NB)
             if (layout(NB, S)) return true;
@@ -1063,7 +1084,10 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
         I.y = L.y;
     }
     ChainSmem m;
-    if (!chain_smem(form, kmax, n, m)) return BL_ERR_SHAPE;
+    // layers reading a given input (no dependency) can be prepared far ahead
+    int given = 0;
+    for (int j = 0; j < n; ++j) given += layers[j].src < 0;
+    if (!chain_smem(form, kmax, n, m, 0, 2 * given > n)) return BL_ERR_SHAPE;
     if (bytes < chain_bytes(n)) return BL_ERR_WORKSPACE;
     char* cb = static_cast<char*>(chain);
     if (cudaMemcpyAsync(cb, host.data(), (size_t)n * sizeof(ChainLayer), cudaMemcpyHostToDevice,
@@ -1085,7 +1109,8 @@ bl_status chain_build(int form, const bl_chain_layer* layers, int n, void* chain
 bl_status chain_run(const bl_chain_plan* plan, const void* chain, unsigned int* flags,
                     cudaStream_t s) {
     ChainSmem m;
-    if (!chain_smem(plan->form, plan->kmax, plan->n_layers, m) || m.S != plan->slots ||
+    if (plan->slots < 3 || plan->slots > kMaxSlots ||
+        !chain_smem(plan->form, plan->kmax, plan->n_layers, m, plan->slots) || m.S != plan->slots ||
         m.total != plan->smem_bytes)
         return BL_ERR_SHAPE;
     if (device_sm_count() != plan->sm_count) return BL_ERR_SHAPE;
