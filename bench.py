@@ -59,7 +59,7 @@ def int8_peak(peaks):
 # weights streamed): the DRAM bytes read + written by one launch over the
 # 2-block stack divided by its 101,187,584 weight bytes, cold caches.  None
 # whenever the chain kernel has changed since the last capture.
-CHAIN_TRAFFIC_PER_WEIGHT_BYTE = None
+CHAIN_TRAFFIC_PER_WEIGHT_BYTE = (101250560 + 3626496) / 101187584
 CHAIN_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one chain_kernel<0> launch "
                         "over the 2-block stack (--layers 2, cold caches), scaled to this launch by its "
                         "weight bytes; summary under profiles/")
