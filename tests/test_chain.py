@@ -278,3 +278,26 @@ def test_chain_fused_onebit_block(blw, oref):
                                   parallel=True)
         y = d["y"].cpu().numpy().astype(np.float64)
         assert np.max(np.abs(y - z_ref[0])) <= OB_TOL * np.max(np.abs(z_ref[0])), j
+
+
+def test_chain_swiglu_buffer_either_order(blw, oref):
+    """SwiGLU evaluated once per element in the producing epilogue, with the
+    gate as the later layer (SwiGLU(y_later, y_earlier)) and as the earlier
+    one, on OneBit-free ternary layers of different widths; the buffers hold
+    exactly the oracle's SwiGLU of the GPU's outputs."""
+    shapes = [(512, 1536), (512, 1536), (1536, 256), (1536, 256)]
+    layers, host = ternary_chain(blw, shapes, [-1, -1, 1, 0], seed=670_000)
+    layers[2]["src2"] = 0          # SwiGLU(y1, y0): the producer (layer 1) is the gate
+    layers[3]["src2"] = 1          # SwiGLU(y0, y1): layer 1 already evaluates the other order
+    for d in layers[2:]:
+        d["swiglu_buf"] = torch.full((1536,), float("nan"), dtype=torch.float16, device="cuda")
+    blw.Chain(0, layers).run()
+    torch.cuda.synchronize()
+    assert blw.bl_device_status() == 0
+    h = oref.swiglu(layers[1]["y"].cpu().numpy(), layers[0]["y"].cpu().numpy())
+    assert np.array_equal(layers[2]["swiglu_buf"].cpu().numpy().view(np.uint16), h.view(np.uint16))
+    for j, (d, w) in enumerate(zip(layers, host)):
+        xin = _fused_input(oref, layers, d)
+        y_ref, acc_ref = oref.ternary_linear(xin[None, :], oref.pack_ternary(w.numpy()), d["w_scale"])
+        assert np.array_equal(d["acc_out"].cpu().numpy(), acc_ref[0]), j
+        assert np.array_equal(d["y"].cpu().numpy().view(np.uint16), y_ref[0].view(np.uint16)), j
