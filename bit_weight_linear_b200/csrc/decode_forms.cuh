@@ -1,5 +1,5 @@
 // decode_forms.cuh -- per-form constants and small helpers shared by the
-// decode-shaped kernels (decode.cu, stream.cu).
+// decode-shaped kernels (stream.cu, chain.cu).
 //
 // Packed weight words: ternary 16 codes of 2 bits (code = t + 1), sign 32 bits
 // (1 = +1).  The byte-SIMD unpack (w >> shift*j) & mask yields, in register j,
