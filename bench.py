@@ -636,9 +636,10 @@ def main():
                 "note": "launch duration = timed region / steps (one chain kernel and one "
                         f"{4 * n_layers}-byte counter memset per step)"}
 
-    # ---- e2e: host buffers.  Every step uploads the step's given input from pinned host memory
-    # and downloads every layer's output, inside the timed region.  Two device buffer sets (two
-    # chains, two graphs) alternate, so step i+1's upload and step i-1's download overlap step i.
+    # ---- e2e: host buffers through the C ABI.  Every step is one bl_chain_run_host call: the
+    # step's given input copied from pinned host memory, the chain, and every layer's output
+    # copied back, all inside the timed region.  Two chains over two device buffer sets run on two
+    # streams in turn, so one step's copies overlap the neighbouring step's kernel.
     xin = x_all.cpu().pin_memory()
     youts = [torch.empty(y_all.shape, dtype=torch.float16).pin_memory() for _ in range(2)]
     x_all2, y_all2 = torch.empty_like(x_all), torch.empty_like(y_all)
@@ -650,37 +651,19 @@ def main():
     layers2 = [dict(d, y=rebased(d["y"], y_all, y_all2),
                     **({"x": rebased(d["x"], x_all, x_all2)} if "x" in d else {})) for d in chain_layers]
     chain2 = blw.Chain(0, layers2)
-    g2 = capture(chain2.run)
-    sets = [(x_all, y_all, g), (x_all2, y_all2, g2)]
+    sets = [(chain, x_all, y_all), (chain2, x_all2, y_all2)]
     comp = torch.cuda.current_stream()
-    upl, dnl = torch.cuda.Stream(), torch.cuda.Stream()  # uploads and downloads do not queue behind each other
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
 
     def e2e_run(n):
-        done = [None, None]      # last graph on each set (its inputs consumed)
-        fetched = [None, None]   # last download of each set's outputs
+        for st in streams:
+            st.wait_stream(comp)
         for i in range(n):
-            xs, ys, gi = sets[i % 2]
-            with torch.cuda.stream(upl):
-                if done[i % 2] is not None:
-                    upl.wait_event(done[i % 2])
-                xs.copy_(xin, non_blocking=True)
-                up = torch.cuda.Event()
-                up.record(upl)
-            comp.wait_event(up)
-            if fetched[i % 2] is not None:
-                comp.wait_event(fetched[i % 2])
-            gi.replay()
-            ev = torch.cuda.Event()
-            ev.record(comp)
-            done[i % 2] = ev
-            with torch.cuda.stream(dnl):
-                dnl.wait_event(ev)
-                youts[i % 2].copy_(ys, non_blocking=True)
-                dn = torch.cuda.Event()
-                dn.record(dnl)
-            fetched[i % 2] = dn
-        comp.wait_stream(upl)
-        comp.wait_stream(dnl)
+            ch, xs, ys = sets[i % 2]
+            with torch.cuda.stream(streams[i % 2]):
+                ch.run_host([(xin, xs)], [(ys, youts[i % 2])])
+        for st in streams:
+            comp.wait_stream(st)
 
     e2e_run(args.warmup)
     barrier(dist_on)
@@ -689,8 +672,6 @@ def main():
     e1 = torch.cuda.Event(enable_timing=True)
     e2e_steps = max(10, args.steps // 4)
     e0.record(comp)
-    upl.wait_stream(comp)
-    dnl.wait_stream(comp)
     e2e_run(e2e_steps)
     e1.record(comp)
     torch.cuda.synchronize()
@@ -701,8 +682,9 @@ def main():
     e2e = {"value": round(wbytes * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
            "h2d_bytes_per_step": xin.numel() * 2, "d2h_bytes_per_step": youts[0].numel() * 2,
            "ms_per_step": round(e2e_ms, 4),
-           "overlap": "double-buffered: uploads/downloads of neighbouring steps overlap the launch"}
-    del g2, chain2, layers2, x_all2, y_all2
+           "call": "bl_chain_run_host (host buffers; one H2D copy, the chain, one D2H copy per step)",
+           "overlap": "two chains on two streams in turn: one step's copies overlap the other's kernel"}
+    del chain2, layers2, x_all2, y_all2
     del g, chain, chain_layers, x_all, y_all
     torch.cuda.synchronize()
     torch.cuda.empty_cache()

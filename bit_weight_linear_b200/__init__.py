@@ -43,6 +43,11 @@ class ChainLayer(ctypes.Structure):
                 ("norm_eps", ctypes.c_float), ("swiglu_buf", _P)]
 
 
+class Copy(ctypes.Structure):
+    """bl_copy (include/bitlinear.h)."""
+    _fields_ = [("src", _P), ("dst", _P), ("bytes", _SZ)]
+
+
 class ChainPlan(ctypes.Structure):
     """bl_chain_plan (include/bitlinear.h)."""
     _fields_ = [("form", _I), ("n_layers", _I), ("sm_count", _I), ("kmax", _I), ("slots", _I),
@@ -66,6 +71,7 @@ ABI = {
     "billm_workspace_bytes": ([_I, _I, _I], _SZ),
     "billm_linear": ([_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P], _I),
     "billm_binarize": ([_P, _I, _I, _P, _P, _P, _P, _P], _I),
+    "bl_chain_run_host": ([_P, _P, _P, _I, _P, _I, _P], _I),
     "bl_chain_bytes": ([_I], _SZ),
     "bl_chain_build": ([_I, _P, _I, _P, _SZ, _P, _P], _I),
     "bl_chain_run": ([_P, _P, _P], _I),
@@ -327,6 +333,25 @@ class Chain:
         """One decode step over the chain on torch's current stream."""
         _check("bl_chain_run", lib().bl_chain_run(ctypes.byref(self.plan), _ptr(self.buf),
                                                   _stream()))
+
+    def run_host(self, inputs, outputs):
+        """One decode step with host buffers on torch's current stream: inputs
+        are (host tensor, device tensor) pairs copied to the device first,
+        outputs (device tensor, host tensor) pairs copied back after the run.
+        Host tensors should be pinned; nothing is synchronised."""
+        for h, d in list(inputs) + [(h, d) for d, h in outputs]:
+            if h.is_cuda or not d.is_cuda or not h.is_contiguous() or not d.is_contiguous():
+                raise ValueError("run_host takes contiguous (host, device) tensor pairs")
+            if h.numel() * h.element_size() != d.numel() * d.element_size():
+                raise ValueError("host and device buffers differ in size")
+        ins = (Copy * max(1, len(inputs)))()
+        for i, (h, d) in enumerate(inputs):
+            ins[i] = Copy(h.data_ptr(), d.data_ptr(), h.numel() * h.element_size())
+        outs = (Copy * max(1, len(outputs)))()
+        for i, (d, h) in enumerate(outputs):
+            outs[i] = Copy(d.data_ptr(), h.data_ptr(), d.numel() * d.element_size())
+        _check("bl_chain_run_host", lib().bl_chain_run_host(ctypes.byref(self.plan), _ptr(self.buf), ins,
+                                                            len(inputs), outs, len(outputs), _stream()))
 
 
 def bl_device_status() -> int:

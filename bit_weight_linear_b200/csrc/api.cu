@@ -433,16 +433,45 @@ bl_status bl_chain_build(int form, const bl_chain_layer* layers, int n_layers, v
     return bl::chain_build(form, layers, n_layers, chain, chain_bytes, plan, cs(stream));
 }
 
-bl_status bl_chain_run(const bl_chain_plan* plan, const void* chain, bl_stream_t stream) {
+static bl_status check_chain_plan(const bl_chain_plan* plan, const void* chain) {
     if (!plan || !chain) return BL_ERR_NULL;
     if ((plan->form != 0 && plan->form != 1) || plan->n_layers <= 0 ||
         plan->n_layers > kMaxChainLayers || (plan->fused != 0 && plan->fused != 1))
         return BL_ERR_SHAPE;
     if ((reinterpret_cast<uintptr_t>(chain) & 255u) != 0) return BL_ERR_ALIGN;
+    return BL_OK;
+}
+
+bl_status bl_chain_run(const bl_chain_plan* plan, const void* chain, bl_stream_t stream) {
+    if (bl_status st = check_chain_plan(plan, chain)) return st;
     if (bl_status st = bl::fault_injected()) return st;
     unsigned int* flags = device_flags();
     if (!flags) return BL_ERR_CUDA;
     return bl::chain_run(plan, chain, flags, cs(stream));
+}
+
+bl_status bl_chain_run_host(const bl_chain_plan* plan, const void* chain, const bl_copy* in,
+                            int n_in, const bl_copy* out, int n_out, bl_stream_t stream) {
+    if (bl_status st = check_chain_plan(plan, chain)) return st;
+    if (n_in < 0 || n_out < 0) return BL_ERR_SHAPE;
+    if ((n_in > 0 && !in) || (n_out > 0 && !out)) return BL_ERR_NULL;
+    for (int i = 0; i < n_in; ++i)
+        if (in[i].bytes && (!in[i].src || !in[i].dst)) return BL_ERR_NULL;
+    for (int i = 0; i < n_out; ++i)
+        if (out[i].bytes && (!out[i].src || !out[i].dst)) return BL_ERR_NULL;
+    if (bl_status st = bl::fault_injected()) return st;
+    unsigned int* flags = device_flags();
+    if (!flags) return BL_ERR_CUDA;
+    for (int i = 0; i < n_in; ++i)
+        if (in[i].bytes && cudaMemcpyAsync(in[i].dst, in[i].src, in[i].bytes, cudaMemcpyHostToDevice,
+                                           cs(stream)) != cudaSuccess)
+            return BL_ERR_CUDA;
+    if (bl_status st = bl::chain_run(plan, chain, flags, cs(stream))) return st;
+    for (int i = 0; i < n_out; ++i)
+        if (out[i].bytes && cudaMemcpyAsync(out[i].dst, out[i].src, out[i].bytes, cudaMemcpyDeviceToHost,
+                                            cs(stream)) != cudaSuccess)
+            return BL_ERR_CUDA;
+    return BL_OK;
 }
 
 bl_status bl_debug_stall_next_launch(unsigned long long wait_limit_ns) {

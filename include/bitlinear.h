@@ -357,6 +357,28 @@ bl_status bl_chain_build(int form, const bl_chain_layer *layers, int n_layers, v
  */
 bl_status bl_chain_run(const bl_chain_plan *plan, const void *chain, bl_stream_t stream);
 
+/* One host<->device copy of bl_chain_run_host: `bytes` bytes between a host
+ * buffer (pinned, for the copy to be asynchronous) and a device buffer. */
+typedef struct {
+    const void *src;       /* host (inputs) or device (outputs) */
+    void *dst;             /* device (inputs) or host (outputs) */
+    size_t bytes;
+} bl_copy;
+
+/*
+ * bl_chain_run_host -- one decode step with host buffers, all on `stream`:
+ * copy each of the n_in inputs from host to the device buffers the chain reads
+ * (its layers' given x), run the chain as bl_chain_run does, then copy each of
+ * the n_out outputs (layers' y) back to host memory.  One cudaMemcpyAsync per
+ * copy; nothing is synchronised (wait on `stream` before reading the outputs).
+ * Steps on two streams over two chains (each with its own buffers) overlap one
+ * step's copies with the other's kernel.  Errors: as bl_chain_run, plus
+ * BL_ERR_NULL for a copy with bytes > 0 and a NULL pointer, BL_ERR_SHAPE for
+ * negative counts.
+ */
+bl_status bl_chain_run_host(const bl_chain_plan *plan, const void *chain, const bl_copy *in,
+                            int n_in, const bl_copy *out, int n_out, bl_stream_t stream);
+
 /*
  * bl_prefill_plan -- diagnostic: how the tensor-core (prefill) path would run
  * a call of this shape on a device with `sm_count` SMs (form 0 = ternary,

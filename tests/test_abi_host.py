@@ -215,3 +215,23 @@ def test_billm_rejects_bad_arguments(L):
     assert L.billm_binarize(A, 32, 100, A, A, None, None, None) == 2
     assert L.billm_binarize(A, 32, 128, None, A, None, None, None) == 1
     assert L.billm_binarize(A, 32, 128, A, A, ctypes.c_void_p(0x10008), None, None) == 3
+
+
+def test_chain_run_host_rejects_bad_arguments(L):
+    """bl_chain_run_host validates the plan and every copy before any CUDA call."""
+    import bit_weight_linear_b200 as blw
+    plan = blw.ChainPlan()
+    plan.form, plan.n_layers, plan.fused = 0, 1, 0
+    buf = ctypes.c_void_p(0x100000)
+    cp = (blw.Copy * 1)()
+    cp[0] = blw.Copy(0x10000, 0x20000, 64)
+    assert L.bl_chain_run_host(None, buf, cp, 1, cp, 1, None) == 1
+    assert L.bl_chain_run_host(ctypes.byref(plan), ctypes.c_void_p(0x100010), cp, 1, cp, 1, None) == 3
+    assert L.bl_chain_run_host(ctypes.byref(plan), buf, cp, -1, cp, 1, None) == 2
+    assert L.bl_chain_run_host(ctypes.byref(plan), buf, None, 1, cp, 1, None) == 1
+    bad = (blw.Copy * 1)()
+    bad[0] = blw.Copy(None, 0x20000, 64)
+    assert L.bl_chain_run_host(ctypes.byref(plan), buf, bad, 1, cp, 1, None) == 1
+    assert L.bl_chain_run_host(ctypes.byref(plan), buf, cp, 1, bad, 1, None) == 1
+    plan.fused = 2
+    assert L.bl_chain_run_host(ctypes.byref(plan), buf, cp, 1, cp, 1, None) == 2

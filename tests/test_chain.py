@@ -301,3 +301,25 @@ def test_chain_swiglu_buffer_either_order(blw, oref):
         y_ref, acc_ref = oref.ternary_linear(xin[None, :], oref.pack_ternary(w.numpy()), d["w_scale"])
         assert np.array_equal(d["acc_out"].cpu().numpy(), acc_ref[0]), j
         assert np.array_equal(d["y"].cpu().numpy().view(np.uint16), y_ref[0].view(np.uint16)), j
+
+
+def test_chain_run_host_matches_device_run(blw):
+    """bl_chain_run_host: the given input copied from pinned host memory, the
+    chain, every output copied back, on one stream; identical to run() on the
+    same input."""
+    shapes = [(1024, 512), (512, 256)]
+    layers, _ = ternary_chain(blw, shapes, [-1, 0], seed=680_000)
+    ch = blw.Chain(0, layers)
+    ch.run()
+    torch.cuda.synchronize()
+    ref = [d["y"].cpu() for d in layers]
+    xin = layers[0]["x"].cpu().pin_memory()
+    layers[0]["x"].zero_()
+    outs = [torch.zeros(d["y"].shape, dtype=torch.float16).pin_memory() for d in layers]
+    for d in layers:
+        d["y"].zero_()
+    ch.run_host([(xin, layers[0]["x"])], [(d["y"], o) for d, o in zip(layers, outs)])
+    torch.cuda.current_stream().synchronize()
+    assert blw.bl_device_status() == 0
+    for o, r in zip(outs, ref):
+        assert torch.equal(o.view(torch.int16), r.view(torch.int16))
