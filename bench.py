@@ -1,20 +1,24 @@
 #!/usr/bin/env python
 """Benchmark of the extreme-low-bit linear layer forward on B200.
 
-Headline workload (one "step"): the M=1 decode pass over a LLaMA-7B-shaped
+Headline workload (one "step"): the M=1 decode step over a LLaMA-7B-shaped
 stack of ternary BitLinear layers -- 32 blocks x (q, k, v, o: 4096->4096;
-gate, up: 4096->11008; down: 11008->4096) = 224 calls of ``bl_ternary_linear``,
-each quantising its own fp16 input token to int8 and contracting it with
-2-bit packed weights (1,619,001,344 weight bytes per step, far above the
-126 MB L2, so no flush is needed between steps).  The step is captured once
-as a CUDA graph and replayed.
+gate, up: 4096->11008; down: 11008->4096) = 224 layers with a decode step's
+dependencies, run as ONE decode-chain launch (bl_chain_run: each layer
+quantises its fp16 input token to int8 and contracts it with 2-bit packed
+weights; 1,619,001,344 weight bytes per step, far above the 126 MB L2, so no
+flush is needed between steps).  The step is captured once as a CUDA graph and
+replayed.  The e2e figure runs the same step through bl_chain_run_host (host
+buffers, copies inside the timed region).
 
 Metric: effective packed-weight GB/s at M=1 (and, in the ``prefill`` object,
 int8 TOPS at M=512 on LLaMA-70B-shaped layers), each with its roofline
-fraction.  The ``onebit_decode`` object repeats the headline workload with the
-OneBit layer (1-bit signs, fp16 g and h).
+fraction.  Extra objects: the same stack without dependencies, with RMSNorm
+and SwiGLU fused, in OneBit form, as separate per-layer calls; the SVID of a
+4096x4096 layer; single-layer and batch sweeps (BitLinear, OneBit, BiLLM).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+       python bench.py --case NAME   (one small workload, for ncu profiles)
 Multi-GPU (torchrun): independent replicas, no collective on the data path.
 """
 from __future__ import annotations
@@ -35,9 +39,6 @@ sys.path.insert(0, ROOT)
 LLAMA7B_BLOCK = [("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
                  ("gate", 4096, 11008), ("up", 4096, 11008), ("down", 11008, 4096)]  # (name, K, N)
 LLAMA7B_LAYERS = 32
-# the same block with the projections that share an input fused into one call each
-LLAMA7B_BLOCK_FUSED = [("qkv", 4096, 3 * 4096), ("o", 4096, 4096), ("gate+up", 4096, 2 * 11008),
-                       ("down", 11008, 4096)]
 LLAMA13B_SWEEP = [("up", 5120, 13824), ("down", 13824, 5120)]   # (name, K, N)
 SWEEP_M = [1, 4, 16, 64, 256, 1024]
 LLAMA70B_PREFILL = [("qkvo-like", 8192, 8192), ("gate/up", 8192, 28672), ("down", 28672, 8192)]
