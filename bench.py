@@ -621,7 +621,7 @@ def main():
     time.sleep(0.3)
     clocks.stop()
     n_layers = len(chain_layers)
-    value = wbytes * world / (ms * 1e-3) / 1e9
+    value = whole_job_rate(wbytes, world, ms) / 1e9
 
     # roofline of the one kernel of the step: the persistent chain kernel
     alg_bytes = wbytes + in_b + out_b
