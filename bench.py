@@ -685,7 +685,7 @@ def main():
            "ms_per_step": round(e2e_ms, 4),
            "call": "bl_chain_run_host (host buffers; one H2D copy, the chain, one D2H copy per step)",
            "overlap": "two chains on two streams in turn: one step's copies overlap the other's kernel"}
-    del chain2, layers2, x_all2, y_all2
+    del sets, streams, chain2, layers2, x_all2, y_all2
     del g, chain, chain_layers, x_all, y_all
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
